@@ -1,0 +1,17 @@
+"""CPU oracle (test infrastructure only; see ``w4a16_oracle``)."""
+from .w4a16_oracle import (  # noqa: F401
+    GROUP,
+    QuantRangeError,
+    awq_alpha_grid,
+    awq_scale_search,
+    awq_scales,
+    channel_mean_abs,
+    dequantize,
+    fp16_round_up,
+    gemm,
+    gemm_entries,
+    pack_nibbles,
+    quantize_pack,
+    quantize_rtn,
+    unpack_nibbles,
+)
