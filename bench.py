@@ -1,0 +1,421 @@
+"""Benchmark of the W4A16 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+Workloads (synthetic, seeded; see weight_only_int4_06_b200/synth.py):
+  decode       (default) single-token decode through 7B-class layers: M=1,
+               (K,N) in (4096,4096), (4096,12288), (4096,11008), (11008,4096); one step = one
+               w4_gemm per shape
+  small_batch  M in {4,8,16,32} x 70B-class (K,N); one step = every (M, shape) once
+  prefill      M in {512,2048,4096} x (K,N) in (4096,11008), (4096,4096), (8192,28672)
+  quantize     w4_quantize_pack of the four 7B-class weight matrices
+  awq          awq_scale_search on X_calib [65536,4096], W [4096,4096], 20 alphas
+
+Timing: every step is captured once in a CUDA graph; W warm-up steps run first, then exactly K
+steps are timed with CUDA events on the launching stream between barriers and device
+synchronisations.  Weight-streaming workloads cycle through enough distinct weight buffers that
+the bytes touched between two uses of a buffer exceed 3x the L2 size, so every step reads HBM.
+Under torchrun every rank runs its own replica (no collective on the data path) and the
+reported time is the maximum over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from weight_only_int4_06_b200 import synth  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def gemm_bytes(M, K, N):
+    """Algorithmic HBM bytes of one w4_gemm: packed W, fp16 scales, u8 zeros, X and Y."""
+    return N * K // 2 + N * (K // 128) * 3 + 2 * M * K + 2 * M * N
+
+
+# ---------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"w4_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+            os.unlink(self.path)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        load = [v for v in sm if smax and v > 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------- distributed
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() and dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------- workloads
+def decode_cases():
+    return [(1, K, N) for (K, N) in synth.DECODE_7B_SHAPES], 2, "decode GEMV, 7B-class layer shapes"
+
+
+def small_batch_cases():
+    return ([(M, K, N) for (K, N) in synth.SMALL_BATCH_70B_SHAPES for M in synth.SMALL_BATCH_MS], 3,
+            "small-batch decode, 70B-class shapes")
+
+
+def prefill_cases():
+    return ([(M, K, N) for (K, N) in synth.PREFILL_SHAPES for M in synth.PREFILL_MS], 4,
+            "prefill, compute-bound")
+
+
+class GemmWorkload:
+    """Device-resident inputs for a list of (M, K, N) layers, with rotating weight copies."""
+
+    def __init__(self, cases, case_id, l2_bytes):
+        import torch
+        from weight_only_int4_06_b200 import w4a16 as B
+        self.B = B
+        self.cases = cases
+        step_w = sum(N * K // 2 + N * (K // 128) * 3 for (M, K, N) in cases)
+        self.n_sets = max(1, min(16, int(np.ceil(3 * l2_bytes / max(step_w, 1))) + 1))
+        self.layers = []
+        for (M, K, N) in cases:
+            X, W = synth.layer_case(case_id, M, K, N)
+            Xd = torch.from_numpy(X).cuda()
+            Wd = torch.from_numpy(W).cuda()
+            packed, scales, zeros = B.w4_quantize_pack(Wd)
+            copies = [(packed, scales, zeros)]
+            for c in range(1, self.n_sets):
+                copies.append((packed.clone(), scales.clone(), zeros.clone()))
+            del Wd
+            Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+            need = B.w4_gemm_workspace_size(M, N, K)
+            ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+            self.layers.append(dict(M=M, K=K, N=N, X=Xd, Xh=torch.from_numpy(X).pin_memory(),
+                                    copies=copies, Y=Y, ws=ws))
+        torch.cuda.synchronize()
+        self.bytes_per_step = sum(gemm_bytes(M, K, N) for (M, K, N) in cases)
+        self.flops_per_step = sum(2 * M * K * N for (M, K, N) in cases)
+        self.launches_per_step = len(cases)
+
+    def run_step(self, step, only=None):
+        s = step % self.n_sets
+        for i, L in enumerate(self.layers):
+            if only is not None and i != only:
+                continue
+            p, sc, z = L["copies"][s]
+            self.B.w4_gemm(L["X"], p, sc, z, out=L["Y"], workspace=L["ws"])
+
+    def run_step_host(self, step):
+        """The same step through the public API with host (pinned) activations and results."""
+        s = step % self.n_sets
+        outs = []
+        for L in self.layers:
+            p, sc, z = L["copies"][s]
+            outs.append(self.B.w4_gemm(L["Xh"], p, sc, z))
+        return outs
+
+    def h2d_d2h_bytes(self):
+        return (sum(2 * M * K for (M, K, N) in self.cases), sum(2 * M * N for (M, K, N) in self.cases))
+
+
+def capture(fn, n_steps, first_step=0):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for i in range(n_steps):
+                fn(first_step + i)
+    torch.cuda.current_stream().wait_stream(s)
+    return g
+
+
+def time_graph(g, world, stream=None):
+    import torch
+    barrier(world)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream() if stream is None else stream
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    g.replay()
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier(world)
+    return e0.elapsed_time(e1)  # ms
+
+
+def oracle_cpu_baseline(cases, case_id, budget_s=20.0):
+    """The CPU oracle as it stands, on a bounded sample of the same step."""
+    import oracle
+    t_total = 0.0
+    done = 0
+    per_case = []
+    for (M, K, N) in cases:
+        X, W = synth.layer_case(case_id, M, K, N)
+        p, s, z = oracle.quantize_pack(W)
+        Msub = min(M, 16)
+        t0 = time.perf_counter()
+        oracle.gemm(X[:Msub], p, s, z)
+        dt = time.perf_counter() - t0
+        per_case.append((M, K, N, Msub, dt))
+        t_total += dt * (M / Msub)
+        done += 1
+        if t_total > budget_s:
+            break
+    frac = done / len(cases)
+    cores = len(os.sched_getaffinity(0))
+    return {"value_us_per_step": t_total / frac * 1e6, "cores": cores,
+            "sample": (f"{done} of {len(cases)} layers of one step"
+                       + (", activation rows capped at 16 and scaled by M/16" if any(c[0] > 16 for c in cases) else "")
+                       + "; oracle = numpy dequantise + fp64 matmul (OpenBLAS threads)")}
+
+
+def run_gemm_bench(args, rank, world, local, kind):
+    import torch
+    cases, case_id, desc = {"decode": decode_cases, "small_batch": small_batch_cases,
+                            "prefill": prefill_cases}[kind]()
+    peaks = load_peaks()
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    wl = GemmWorkload(cases, case_id, l2)
+    K_steps, W_steps = args.steps, args.warmup
+
+    # warm-up (eager once, then graphed)
+    for i in range(2):
+        wl.run_step(i)
+    torch.cuda.synchronize()
+    g_warm = capture(wl.run_step, W_steps, 0)
+    g_timed = capture(wl.run_step, K_steps, W_steps)
+    g_warm.replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        t_end = time.time() + 1.0
+        while time.time() < t_end:   # keep the GPU busy while the sampler settles
+            g_warm.replay()
+        torch.cuda.synchronize()
+    ms = time_graph(g_timed, world)
+    clocks = sampler.stop() if sampler else None
+    ms = max_over_ranks(ms, world)
+    ms_per_step = ms / K_steps
+
+    # per-layer times (same protocol, one layer at a time)
+    per_layer = []
+    for i, L in enumerate(wl.layers):
+        reps = max(W_steps, 20)
+        gi = capture(lambda s, i=i: wl.run_step(s, only=i), reps, 0)
+        gi.replay()
+        t = time_graph(gi, world) / reps
+        t = max_over_ranks(t, world)
+        b = gemm_bytes(L["M"], L["K"], L["N"])
+        fl = 2 * L["M"] * L["K"] * L["N"]
+        per_layer.append({"M": L["M"], "K": L["K"], "N": L["N"], "us": round(t * 1e3, 3),
+                          "GBps": round(b / (t * 1e-3) / 1e9, 1),
+                          "TFLOPs": round(fl / (t * 1e-3) / 1e12, 2),
+                          "hbm_frac": round(b / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)})
+
+    # end to end through the public API with host buffers
+    h2d, d2h = wl.h2d_d2h_bytes()
+    e2e_steps = min(K_steps, 50)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        wl.run_step_host(i)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+
+    compute_bound = kind == "prefill"
+    if compute_bound:
+        achieved = wl.flops_per_step / (ms_per_step * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                "frac": round(achieved / peak, 4), "traffic": None}
+    else:
+        achieved = wl.bytes_per_step / (ms_per_step * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": None}
+    roof["peak_source"] = peaks["source"]
+    roof["kernel"] = "skinny_kernel (mma.sync split-K cluster GEMV)" if not compute_bound else "w4 GEMM"
+
+    out = {
+        "metric": "W4A16 GEMM us & % roofline (HBM GB/s at M<=16, TFLOP/s at M>=512)",
+        "value": round(ms_per_step * 1e3, 3),
+        "unit": "us/step",
+        "n_gpus": world,
+        "steps": K_steps,
+        "warmup": W_steps,
+        "ms_per_step": round(ms_per_step, 6),
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16",
+        "data": "synthetic",
+        "config": {"workload": desc, "layers": [list(c) for c in cases], "group": 128,
+                   "weight_buffer_sets": wl.n_sets,
+                   "l2": f"cold: {wl.n_sets} rotating weight-buffer sets, >=3x L2 between reuses",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": roof,
+        "layers": per_layer,
+        "e2e": {"value": round(e2e_ms * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": wl.launches_per_step * K_steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_cpu_baseline(cases, case_id)
+        out["cpu_baseline"] = {"value": round(cb["value_us_per_step"], 1), "unit": "us/step",
+                               "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"]}
+    return out
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle timed on a bounded sample of the same workload."""
+    if rank != 0:
+        return None
+    kind = args.workload
+    cases, case_id, desc = {"decode": decode_cases, "small_batch": small_batch_cases,
+                            "prefill": prefill_cases}.get(kind, decode_cases)()
+    vals = []
+    cb = None
+    for _ in range(args.warmup + args.steps):
+        cb = oracle_cpu_baseline(cases, case_id, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+        vals.append(cb["value_us_per_step"])
+    v = statistics.median(vals[args.warmup:]) if len(vals) > args.warmup else vals[-1]
+    return {
+        "impl": "reference",
+        "metric": "W4A16 GEMM us & % roofline (HBM GB/s at M<=16, TFLOP/s at M>=512)",
+        "value": round(v, 1), "unit": "us/step", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(v / 1e3, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": desc, "layers": [list(c) for c in cases], "group": 128},
+        "cpu_baseline": {"value": round(v, 1), "unit": "us/step", "cores": cb["cores"],
+                         "kind": "oracle", "sample": cb["sample"]},
+        "e2e": {"value": round(v, 1), "unit": "us/step", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "small_batch", "prefill"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args)
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+    else:
+        out = run_gemm_bench(args, rank, world, local, args.workload)
+    if rank == 0 and out is not None:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

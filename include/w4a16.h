@@ -1,0 +1,178 @@
+/*
+ * libw4a16 -- group-wise INT4 weight-only quantisation and the W4A16 matmul on B200 (sm_100a).
+ *
+ * C ABI.  Every entry point takes plain pointers and sizes; no PyTorch or CUDA types appear in
+ * the signatures (a stream is passed as an opaque `void*` holding a cudaStream_t; NULL means the
+ * legacy default stream).
+ *
+ * Conventions shared by all entry points
+ * --------------------------------------
+ *  - Layouts: every matrix is dense row-major with no padding between rows.
+ *      X  [M, K]    fp16 (IEEE binary16 bit patterns in uint16_t)  activations
+ *      W  [N, K]    fp16                                           weights
+ *      packed [N, K/8] uint32: 8 four-bit codes per word, the code of the lowest k in the lowest
+ *                   nibble (word j of row n holds k = 8j .. 8j+7)
+ *      scales [N, K/group] fp16; zeros [N, K/group] uint8 (values 0..15)
+ *      Y  [M, N]    fp16
+ *    Group g of row n covers k in [group*g, group*g + group).  Dequantised weight:
+ *    w[n,k] = (q[n,k] - zeros[n, k/group]) * scales[n, k/group].
+ *  - Memory: all array pointers are DEVICE pointers owned by the caller (except the outputs of
+ *    the *_workspace_size queries and w4_status_string, which are host memory).  The library
+ *    never allocates or frees memory.  Work is enqueued asynchronously on `stream`; the only
+ *    call that synchronises is w4_check_device_status.
+ *  - Validation happens on the host before any launch; a rejected call enqueues nothing.
+ *      W4_ERR_NULL         a required pointer is NULL
+ *      W4_ERR_SHAPE        a size is negative, K % group != 0, N % 8 != 0, or a size exceeds the
+ *                          library's limits (every dimension < 2^31, every matrix < 2^40 elements)
+ *      W4_ERR_UNSUPPORTED  group != 128, or n_alpha outside 1..64
+ *      W4_ERR_ALIGN        X, W, packed, Y or act_scale is not 16-byte aligned
+ *      W4_ERR_WORKSPACE    ws_bytes is smaller than the size the matching query returns
+ *      W4_ERR_CUDA         a CUDA launch or query failed (the CUDA error is left for the caller
+ *                          to read with cudaGetLastError)
+ *    Device-side conditions cannot be seen at launch time; kernels record them in a per-device
+ *    status word that w4_check_device_status reads:
+ *      W4_ERR_RANGE        a group's fp16 scale overflowed (|W * act_scale| too large for fp16);
+ *                          the outputs of that call are unspecified
+ *      W4_ERR_DEVICE_TIMEOUT  a bounded wait inside a kernel gave up; that kernel's outputs are
+ *                          unspecified and the context stays usable
+ *  - Results are deterministic: the same inputs give bit-identical outputs (no floating-point
+ *    atomics; every reduction has a fixed order).
+ *  - Thread safety: calls may come from several host threads; the only shared state is the
+ *    per-device status word.
+ *
+ * Sources.  The method is described by the pages "GPTQ, AWQ and the rules of post-training
+ * quantization" (sections "The problem both methods solve" and "AWQ: find the one percent that
+ * matters"), "AutoGPTQ vs The Stack v2" (per-group quantisation with scales and zero points,
+ * group size typically 128), "AutoAWQ vs The Stack v2" (INT4 storage, FP16 compute, weights
+ * dequantised on the fly inside fused GEMM/GEMV kernels, picked by batch size) and "When to Use
+ * AWQ vs GPTQ" (section "Practical Usage": w_bit 4, q_group_size 128).
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    W4_OK = 0,
+    W4_ERR_NULL = 1,
+    W4_ERR_SHAPE = 2,
+    W4_ERR_ALIGN = 3,
+    W4_ERR_UNSUPPORTED = 4,
+    W4_ERR_WORKSPACE = 5,
+    W4_ERR_CUDA = 6,
+    W4_ERR_DEVICE_TIMEOUT = 7,
+    W4_ERR_RANGE = 8
+} w4_status;
+
+/* Kernel families of w4_gemm_ex (w4_gemm picks one per shape). */
+typedef enum {
+    W4_VARIANT_AUTO = 0,
+    W4_VARIANT_SKINNY = 1, /* warp-level tensor-core GEMV / skinny GEMM, split-K over a cluster */
+    W4_VARIANT_TC = 2      /* tcgen05/TMEM tensor-core GEMM with dequantisation in the smem path */
+} w4_variant;
+
+/*
+ * w4_quantize_pack -- round-to-nearest group quantisation of W * diag(act_scale) and packing.
+ *
+ * Follows "GPTQ, AWQ and the rules of post-training quantization", section "The problem both
+ * methods solve" (round each weight to the nearest level of a small integer format) and
+ * "AutoGPTQ vs The Stack v2" (one scale and one zero point per group of 128 along K).
+ * For each row n and group g, with v_k = W[n,k] * act_scale[k] (one fp32 multiply; v_k = W[n,k]
+ * when act_scale is NULL):
+ *     lo = min(0, min v), hi = max(0, max v)              (fp32)
+ *     s32 = (hi - lo) / 15                                (fp32, IEEE round to nearest)
+ *     s16 = s32 rounded to fp16 toward +infinity          (1.0 when hi == lo)
+ *     z   = clamp(rint(-lo / s16), 0, 15)                 (rint: round half to even)
+ *     q_k = clamp(rint(v_k / s16) + z, 0, 15)
+ * Every step is one correctly rounded fp32 operation, so results are bit-identical to any
+ * IEEE implementation of the same steps.
+ *
+ *   W          [N, K] fp16, device, 16-byte aligned.
+ *   act_scale  [K] fp32, device, 16-byte aligned, or NULL.  AWQ use: quantise W*diag(s) here and
+ *              feed X*diag(1/s) to w4_gemm (or fold 1/s into the producer of X).
+ *   packed     [N, K/8] uint32 out, 16-byte aligned.  scales [N, K/group] fp16 out.
+ *   zeros      [N, K/group] uint8 out.   group must be 128.
+ * N == 0 is a no-op.  Errors: see the conventions above; W4_ERR_RANGE is reported through the
+ * device status word.
+ */
+w4_status w4_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int group,
+                           const float* act_scale, uint32_t* packed, uint16_t* scales,
+                           uint8_t* zeros, void* stream);
+
+/* Bytes of device workspace w4_gemm / w4_gemm_ex need for this shape (may be 0). */
+w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, size_t* bytes);
+
+/*
+ * w4_gemm -- Y = X . dequant(W)^T with fp16 inputs, fp32 accumulation and fp16 output.
+ *
+ * Follows "AutoAWQ vs The Stack v2" (WQLinear blurb: INT4 weights dequantised on the fly inside
+ * the matmul instead of materialising FP16 weights; a GEMV kernel for single-token decode and a
+ * GEMM kernel for batches, chosen by batch size).  The dequantised weights are
+ * w = (q - z) * s16 as above.
+ *
+ *   X [M, K] fp16, packed/scales/zeros as produced by w4_quantize_pack, Y [M, N] fp16 out.
+ *   ws / ws_bytes: device workspace of at least w4_gemm_workspace_size bytes (may be NULL when
+ *   that size is 0).  M == 0 or N == 0 is a no-op; K == 0 writes Y = 0.
+ * The skinny family computes sum_k x_k (q_k - z) exactly per group on tensor cores in fp32 and
+ * scales each group's partial sum by s16 in fp32; the TC family rounds each dequantised weight
+ * once to fp16 before the fp32-accumulating MMA.  Both round Y once to fp16.
+ */
+w4_status w4_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                  const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y, void* ws,
+                  size_t ws_bytes, void* stream);
+
+/* w4_gemm with an explicit kernel family (W4_VARIANT_AUTO behaves exactly like w4_gemm). */
+w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                     const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y,
+                     void* ws, size_t ws_bytes, int variant, void* stream);
+
+/* Bytes of device workspace awq_scale_search needs for this problem. */
+w4_status awq_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha,
+                             size_t* bytes);
+
+/*
+ * awq_scale_search -- the AWQ activation-aware per-channel scale search on one linear layer.
+ *
+ * Follows "GPTQ, AWQ and the rules of post-training quantization", section "AWQ: find the one
+ * percent that matters": the scale of input channel j is the average activation magnitude
+ * raised to a power alpha, alpha is chosen by a grid search over [0, 1], and the layer keeps
+ * its function when W's channel j is multiplied by s_j and X's channel j divided by s_j.
+ *     m_j      = (1/T) sum_t |X[t,j]|                        (exact sum, rounded once to fp64)
+ *     alpha_i  = i / n_alpha, i = 0 .. n_alpha-1
+ *     s_ij     = max(m_j, 1e-6)^alpha_i / sqrt(max_j(.) * min_j(.))   (fp64, then rounded to fp32)
+ *     Wq_i     = dequant(quant(W * diag(s_i)))              (exactly w4_quantize_pack's quantiser)
+ *     MSE_i    = mean over (t, n) of ((X diag(1/s_i)) Wq_i^T - X W^T)^2
+ *     best     = lowest i among the minima of MSE_i
+ * On the device MSE_i is evaluated as sum_{t,n} (X E_i^T)^2 / (T N) with
+ * E_i = Wq_i diag(1/s_i) - W rounded to fp16, fp32 tensor-core accumulation and an fp64
+ * fixed-order reduction.
+ *
+ *   X [T, K] fp16 calibration activations; W [N, K] fp16.
+ *   mse [n_alpha] fp64 out, best_idx [1] int32 out, best_s [K] fp32 out (all device memory).
+ *   ws: device workspace of at least awq_workspace_size bytes.
+ * T must be >= 1 and N >= 8.  Errors: see the conventions above.
+ */
+w4_status awq_scale_search(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K,
+                           int group, int n_alpha, double* mse, int32_t* best_idx, float* best_s,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * w4_check_device_status -- synchronise `stream`, then read and clear the current device's
+ * status word.  Returns W4_OK, W4_ERR_RANGE, W4_ERR_DEVICE_TIMEOUT, or W4_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+w4_status w4_check_device_status(void* stream);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char* w4_status_string(w4_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

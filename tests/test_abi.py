@@ -1,0 +1,102 @@
+"""The C-ABI library loads, exports every symbol include/w4a16.h declares, and rejects bad
+arguments on the host before touching the GPU (CPU only: no compute call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from weight_only_int4_06_b200 import w4a16 as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a16.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(B.LIB_PATH):
+        from weight_only_int4_06_b200 import build_lib
+        build_lib.build()
+    return B.lib()
+
+
+def test_header_declares_expected_api():
+    names = declared_functions()
+    for n in ("w4_quantize_pack", "w4_gemm", "w4_gemm_ex", "w4_gemm_workspace_size",
+              "awq_scale_search", "awq_workspace_size", "w4_check_device_status", "w4_status_string"):
+        assert n in names, n
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_functions():
+        assert hasattr(L, n), n
+        assert n in B.SIGNATURES, n
+
+
+def test_status_strings(L):
+    for code in range(9):
+        s = B.w4_status_string(code)
+        assert isinstance(s, str) and s
+    assert B.w4_status_string(99) == "unknown status"
+
+
+P = ctypes.c_void_p
+GOOD = P(1 << 20)        # never dereferenced: every call below is rejected on the host
+BAD_ALIGN = P((1 << 20) + 2)
+
+
+def test_quantize_pack_rejects(L):
+    q = L.w4_quantize_pack
+    assert q(GOOD, 8, 256, 64, None, GOOD, GOOD, GOOD, None) == 4        # group != 128
+    assert q(GOOD, 8, 200, 128, None, GOOD, GOOD, GOOD, None) == 2       # K % 128
+    assert q(GOOD, 12, 256, 128, None, GOOD, GOOD, GOOD, None) == 2      # N % 8
+    assert q(GOOD, -8, 256, 128, None, GOOD, GOOD, GOOD, None) == 2      # negative
+    assert q(None, 8, 256, 128, None, GOOD, GOOD, GOOD, None) == 1       # null W
+    assert q(GOOD, 8, 256, 128, None, None, GOOD, GOOD, None) == 1       # null packed
+    assert q(BAD_ALIGN, 8, 256, 128, None, GOOD, GOOD, GOOD, None) == 3  # misaligned W
+    assert q(GOOD, 8, 256, 128, BAD_ALIGN, GOOD, GOOD, GOOD, None) == 3  # misaligned act_scale
+    assert q(GOOD, 0, 256, 128, None, None, None, None, None) == 0       # empty: no-op
+    assert q(GOOD, 1 << 31, 256, 128, None, GOOD, GOOD, GOOD, None) == 2 # too large
+
+
+def test_gemm_rejects(L):
+    g = L.w4_gemm_ex
+    args = lambda **kw: [kw.get("X", GOOD), kw.get("M", 4), kw.get("N", 16), kw.get("K", 256),
+                         kw.get("p", GOOD), GOOD, GOOD, kw.get("group", 128), kw.get("Y", GOOD),
+                         None, 0, kw.get("variant", 0), None]
+    assert g(*args(group=32)) == 4
+    assert g(*args(variant=7)) == 4
+    assert g(*args(K=100)) == 2
+    assert g(*args(N=12)) == 2
+    assert g(*args(M=-1)) == 2
+    assert g(*args(X=None)) == 1
+    assert g(*args(p=None)) == 1
+    assert g(*args(Y=None)) == 1
+    assert g(*args(X=BAD_ALIGN)) == 3
+    assert g(*args(Y=BAD_ALIGN)) == 3
+    assert g(*args(M=0)) == 0
+    assert g(*args(N=0)) == 0
+
+
+def test_workspace_queries(L):
+    n = ctypes.c_size_t(123)
+    assert L.w4_gemm_workspace_size(1, 4096, 4096, 128, ctypes.byref(n)) == 0
+    assert L.w4_gemm_workspace_size(1, 4096, 4000, 128, ctypes.byref(n)) == 2
+    assert L.w4_gemm_workspace_size(1, 4096, 4096, 64, ctypes.byref(n)) == 4
+    assert L.w4_gemm_workspace_size(1, 4096, 4096, 128, None) == 1
+    assert L.awq_workspace_size(256, 64, 512, 128, 0, ctypes.byref(n)) == 4
+    assert L.awq_workspace_size(256, 64, 500, 128, 20, ctypes.byref(n)) == 2
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        B.lib()

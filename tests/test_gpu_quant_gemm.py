@@ -1,0 +1,199 @@
+"""GPU parity: w4_quantize_pack bit-exact against the CPU oracle, w4_gemm within
+|Y - Y_ref| <= 5e-3 (|Y_ref| + rms(Y_ref)) elementwise, on the workloads' seeded inputs.
+
+Every input and expected value comes from the seeded generators and the oracle; the GEMM
+tests feed the library the oracle's own packed weights."""
+import hashlib
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_only_int4_06_b200 import synth
+from weight_only_int4_06_b200 import w4a16 as B
+
+pytestmark = pytest.mark.gpu
+
+TOL = 5e-3
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def gpu_quant(W, act=None):
+    a = None if act is None else dev(np.asarray(act, np.float32))
+    p, s, z = B.w4_quantize_pack(dev(W), a)
+    st = B.w4_check_device_status()
+    return p.cpu().numpy().view(np.uint32), s.cpu().numpy(), z.cpu().numpy(), st
+
+
+def assert_quant_equal(W, act=None):
+    p, s, z, st = gpu_quant(W, act)
+    assert st == 0, B.STATUS_NAMES[st]
+    po, so, zo = oracle.quantize_pack(W, act)
+    assert np.array_equal(s.view(np.uint16), so.view(np.uint16)), "scales differ"
+    assert np.array_equal(z, zo), "zeros differ"
+    assert np.array_equal(p, po), "packed codes differ"
+    return p, s, z
+
+
+def gpu_gemm(X, packed, scales, zeros, variant=B.VARIANT_AUTO):
+    Y = B.w4_gemm(dev(X), dev(packed.view(np.int32)), dev(scales), dev(zeros), variant=variant)
+    assert B.w4_check_device_status() == 0
+    return Y.cpu().numpy()
+
+
+def assert_close(Y, Yref, what=""):
+    Y = Y.astype(np.float64)
+    rms = float(np.sqrt(np.mean(Yref ** 2))) if Yref.size else 0.0
+    err = np.abs(Y - Yref)
+    bound = TOL * (np.abs(Yref) + rms)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError(f"{what}: {bad.sum()} of {err.size} outside tolerance; worst at {i}: "
+                             f"got {Y[i]}, ref {Yref[i]}, bound {bound[i]}")
+    assert np.isfinite(Y).all()
+
+
+# ------------------------------------------------------------------ quantiser
+def test_quant_single_layer_matches_oracle_and_golden():
+    _, W = synth.single_layer_case()
+    p, s, z = assert_quant_equal(W)
+    golden = {}
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "single_layer_seed0.txt")
+    for line in open(path):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.split("=", 1)
+            golden[k.strip()] = v.strip()
+    assert hashlib.sha256(p.astype("<u4").tobytes()).hexdigest() == golden["packed_sha256"]
+    assert hashlib.sha256(s.astype("<f2").tobytes()).hexdigest() == golden["scales_sha256"]
+    assert hashlib.sha256(z.tobytes()).hexdigest() == golden["zeros_sha256"]
+
+
+@pytest.mark.parametrize("N,K", [(8, 128), (24, 384), (40, 1152), (16, 11008), (264, 512)])
+def test_quant_ragged_shapes(N, K):
+    X, W = synth.layer_case(11, 1, K, N)
+    assert_quant_equal(W)
+    act = np.exp(np.random.default_rng([N, K]).standard_normal(K)).astype(np.float32)
+    assert_quant_equal(W, act)
+
+
+def test_quant_special_groups():
+    K = 512
+    W = np.zeros((16, K), np.float16)
+    W[1, :] = 0.5                                   # constant group rows
+    W[2, :] = np.abs(synth.layer_case(12, 1, K, 16)[1][2])    # all >= 0
+    W[3, :] = -np.abs(synth.layer_case(12, 1, K, 16)[1][3])   # all <= 0
+    W[4, 37] = 0.75                                 # single nonzero
+    W[5, 300] = -0.75
+    W[6, :] = ((np.arange(K) % 128 - 64) / 64.0).astype(np.float16)  # ramps
+    W[7, :] = np.float16(1e-7)                      # subnormal-size values
+    W[8, ::2] = np.float16(60000.0)                 # near the top of the fp16 range
+    W[8, 1::2] = np.float16(-60000.0)
+    assert_quant_equal(W)
+
+
+def test_quant_range_overflow_is_reported():
+    W = np.zeros((8, 128), np.float16)
+    W[0, 0], W[0, 1] = 60000.0, -60000.0
+    _, _, _, st = gpu_quant(W, np.full(128, 16.0, np.float32))
+    assert st == 8  # W4_ERR_RANGE
+    assert B.w4_check_device_status() == 0  # cleared by the read
+    with pytest.raises(oracle.QuantRangeError):
+        oracle.quantize_pack(W, np.full(128, 16.0, np.float32))
+
+
+@pytest.mark.parametrize("K,N", list(synth.DECODE_7B_SHAPES) + [(28672, 8192)])
+def test_quant_full_size(K, N):
+    _, W = synth.layer_case(2, 1, K, N)
+    assert_quant_equal(W)
+
+
+# ------------------------------------------------------------------ gemm
+def oracle_case(case_id, M, K, N):
+    X, W = synth.layer_case(case_id, M, K, N)
+    p, s, z = oracle.quantize_pack(W)
+    return X, p, s, z
+
+
+def test_gemm_single_layer():
+    X, W = synth.single_layer_case()
+    p, s, z = oracle.quantize_pack(W)
+    Y = gpu_gemm(X, p, s, z)
+    assert_close(Y, oracle.gemm(X, p, s, z), "512x512")
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 7, 8, 9, 13, 16, 17, 24, 31, 32, 33, 40])
+def test_gemm_m_sweep_ragged(M):
+    X, p, s, z = oracle_case(21, M, 384, 136)
+    assert_close(gpu_gemm(X, p, s, z), oracle.gemm(X, p, s, z), f"M={M}")
+
+
+@pytest.mark.parametrize("K,N", [(128, 8), (128, 520), (1152, 264), (4096, 136), (11008, 40),
+                                 (28672, 16), (2048, 4096)])
+@pytest.mark.parametrize("M", [1, 4, 16, 32])
+def test_gemm_split_shapes(M, K, N):
+    X, p, s, z = oracle_case(22, M, K, N)
+    assert_close(gpu_gemm(X, p, s, z, B.VARIANT_SKINNY), oracle.gemm(X, p, s, z), f"{M}x{K}x{N}")
+
+
+@pytest.mark.parametrize("K,N", synth.DECODE_7B_SHAPES)
+def test_gemm_decode_7b_full(K, N):
+    X, p, s, z = oracle_case(2, 1, K, N)
+    assert_close(gpu_gemm(X, p, s, z), oracle.gemm(X, p, s, z), f"decode {K}x{N}")
+
+
+@pytest.mark.parametrize("K,N", synth.SMALL_BATCH_70B_SHAPES)
+def test_gemm_small_batch_70b_full(K, N):
+    for M in synth.SMALL_BATCH_MS:
+        X, p, s, z = oracle_case(3, M, K, N)
+        assert_close(gpu_gemm(X, p, s, z), oracle.gemm(X, p, s, z), f"M={M} {K}x{N}")
+
+
+@pytest.mark.parametrize("M", synth.PREFILL_MS)
+@pytest.mark.parametrize("K,N", synth.PREFILL_SHAPES)
+def test_gemm_prefill_sampled(M, K, N):
+    X, p, s, z = oracle_case(4, M, K, N)
+    Y = gpu_gemm(X, p, s, z)
+    r = np.random.default_rng([M, K, N])
+    rows = np.concatenate([r.integers(0, M, 1500), [0, M - 1, M - 1]])
+    cols = np.concatenate([r.integers(0, N, 1500), [0, N - 1, 0]])
+    ref = oracle.gemm_entries(X, p, s, z, rows, cols)
+    # tolerance uses the rms of the sampled reference values
+    assert_close(Y[rows, cols], ref, f"prefill M={M} {K}x{N}")
+
+
+def test_gemm_deterministic():
+    X, p, s, z = oracle_case(23, 16, 8192, 1024)
+    Y1 = gpu_gemm(X, p, s, z)
+    Y2 = gpu_gemm(X, p, s, z)
+    assert np.array_equal(Y1.view(np.uint16), Y2.view(np.uint16))
+
+
+def test_gemm_empty_and_k0():
+    Y = torch.full((3, 16), 7.0, dtype=torch.float16, device="cuda")
+    X = torch.zeros((3, 0), dtype=torch.float16, device="cuda")
+    p = torch.zeros((16, 0), dtype=torch.int32, device="cuda")
+    s = torch.zeros((16, 0), dtype=torch.float16, device="cuda")
+    z = torch.zeros((16, 0), dtype=torch.uint8, device="cuda")
+    B.w4_gemm(X, p, s, z, out=Y)
+    torch.cuda.synchronize()
+    assert torch.all(Y == 0)
+    X = torch.zeros((0, 128), dtype=torch.float16, device="cuda")
+    p = torch.zeros((16, 16), dtype=torch.int32, device="cuda")
+    s = torch.zeros((16, 1), dtype=torch.float16, device="cuda")
+    z = torch.zeros((16, 1), dtype=torch.uint8, device="cuda")
+    assert B.w4_gemm(X, p, s, z).shape == (0, 16)
+
+
+def test_gemm_host_buffers_match_device():
+    X, p, s, z = oracle_case(24, 1, 4096, 4096)
+    Yd = gpu_gemm(X, p, s, z)
+    Xh = torch.from_numpy(X).pin_memory()
+    Yh = B.w4_gemm(Xh, dev(p.view(np.int32)), dev(s), dev(z))
+    assert not Yh.is_cuda
+    assert np.array_equal(Yh.numpy().view(np.uint16), Yd.view(np.uint16))

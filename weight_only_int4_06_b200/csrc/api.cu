@@ -1,0 +1,174 @@
+// C-ABI entry points of libw4a16: argument validation, per-shape dispatch and the device status
+// word.  Everything is enqueued on the caller's stream; nothing here allocates device memory.
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace w4 {
+
+// First device-side error of any call since the last w4_check_device_status (one per device).
+__device__ int g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_dev_once[kMaxDevices];
+int g_sm_count[kMaxDevices];
+int* g_status_ptr[kMaxDevices];
+cudaError_t g_dev_err[kMaxDevices];
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+    return dev;
+}
+
+// Per-device set-up, done once per device with that device current.
+bool device_setup(int dev) {
+    std::call_once(g_dev_once[dev], [dev]() {
+        cudaError_t e = cudaDeviceGetAttribute(&g_sm_count[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess) e = cudaGetSymbolAddress((void**)&g_status_ptr[dev], g_device_status);
+        g_dev_err[dev] = e;
+    });
+    return g_dev_err[dev] == cudaSuccess;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+constexpr int64_t kMaxElems = (int64_t)1 << 40;
+
+bool dims_ok(int64_t a, int64_t b) {
+    return a >= 0 && b >= 0 && a < kMaxDim && b < kMaxDim && (a == 0 || b <= kMaxElems / a);
+}
+
+}  // namespace
+
+int device_sm_count() {
+    const int dev = current_device();
+    if (dev < 0 || !device_setup(dev)) return 148;
+    return g_sm_count[dev];
+}
+
+int* device_status_ptr() {
+    const int dev = current_device();
+    if (dev < 0 || !device_setup(dev)) return nullptr;
+    return g_status_ptr[dev];
+}
+
+}  // namespace w4
+
+using namespace w4;
+
+extern "C" {
+
+w4_status w4_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int group,
+                           const float* act_scale, uint32_t* packed, uint16_t* scales,
+                           uint8_t* zeros, void* stream) {
+    if (group != 128) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(N, K) || K % group != 0 || N % 8 != 0) return W4_ERR_SHAPE;
+    if (N == 0 || K == 0) return W4_OK;
+    if (!W || !packed || !scales || !zeros) return W4_ERR_NULL;
+    if (!aligned16(W) || !aligned16(packed) || (act_scale && !aligned16(act_scale))) return W4_ERR_ALIGN;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_quantize_pack(W, N, K, act_scale, packed, scales, zeros, status,
+                                         (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, size_t* bytes) {
+    if (!bytes) return W4_ERR_NULL;
+    if (group != 128) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0)
+        return W4_ERR_SHAPE;
+    *bytes = 0;
+    return W4_OK;
+}
+
+w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                     const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y,
+                     void* ws, size_t ws_bytes, int variant, void* stream) {
+    if (group != 128) return W4_ERR_UNSUPPORTED;
+    if (variant < W4_VARIANT_AUTO || variant > W4_VARIANT_TC) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0)
+        return W4_ERR_SHAPE;
+    size_t need = 0;
+    w4_status st = w4_gemm_workspace_size(M, N, K, group, &need);
+    if (st != W4_OK) return st;
+    if (ws_bytes < need) return W4_ERR_WORKSPACE;
+    if (need > 0 && !ws) return W4_ERR_NULL;
+    if (M == 0 || N == 0) return W4_OK;
+    if (!Y) return W4_ERR_NULL;
+    if (!aligned16(Y)) return W4_ERR_ALIGN;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (K == 0) {
+        return cudaMemsetAsync(Y, 0, (size_t)M * (size_t)N * 2, s) == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+    }
+    if (!X || !packed || !scales || !zeros) return W4_ERR_NULL;
+    if (!aligned16(X) || !aligned16(packed)) return W4_ERR_ALIGN;
+    if (!device_status_ptr()) return W4_ERR_CUDA;
+
+    // Skinny path in chunks of at most 32 activation rows.
+    for (int64_t m0 = 0; m0 < M; m0 += 32) {
+        const int64_t mc = (M - m0) < 32 ? (M - m0) : 32;
+        SkinnyPlan plan;
+        if (!plan_skinny(mc, N, K, &plan)) return W4_ERR_SHAPE;
+        cudaError_t e = launch_skinny(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N, plan, s);
+        if (e != cudaSuccess) return W4_ERR_CUDA;
+    }
+    return W4_OK;
+}
+
+w4_status w4_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                  const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y, void* ws,
+                  size_t ws_bytes, void* stream) {
+    return w4_gemm_ex(X, M, N, K, packed, scales, zeros, group, Y, ws, ws_bytes, W4_VARIANT_AUTO,
+                      stream);
+}
+
+w4_status awq_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha,
+                             size_t* bytes) {
+    if (!bytes) return W4_ERR_NULL;
+    if (group != 128 || n_alpha < 1 || n_alpha > 64) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(T, K) || !dims_ok(N, K) || T < 1 || N < 8 || K < 128 || K % group != 0 || N % 8 != 0)
+        return W4_ERR_SHAPE;
+    *bytes = 0;
+    return W4_ERR_UNSUPPORTED;  // not built yet
+}
+
+w4_status awq_scale_search(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K,
+                           int group, int n_alpha, double* mse, int32_t* best_idx, float* best_s,
+                           void* ws, size_t ws_bytes, void* stream) {
+    (void)X; (void)T; (void)W; (void)N; (void)K; (void)group; (void)n_alpha; (void)mse;
+    (void)best_idx; (void)best_s; (void)ws; (void)ws_bytes; (void)stream;
+    return W4_ERR_UNSUPPORTED;  // not built yet
+}
+
+w4_status w4_check_device_status(void* stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return W4_ERR_CUDA;
+    int* p = device_status_ptr();
+    if (!p) return W4_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return W4_ERR_CUDA;
+    if (v != 0 && cudaMemset(p, 0, sizeof(int)) != cudaSuccess) return W4_ERR_CUDA;
+    return (w4_status)v;
+}
+
+const char* w4_status_string(w4_status status) {
+    switch (status) {
+        case W4_OK: return "ok";
+        case W4_ERR_NULL: return "a required pointer is NULL";
+        case W4_ERR_SHAPE: return "unsupported or inconsistent shape";
+        case W4_ERR_ALIGN: return "pointer is not 16-byte aligned";
+        case W4_ERR_UNSUPPORTED: return "unsupported parameter (group must be 128; n_alpha 1..64)";
+        case W4_ERR_WORKSPACE: return "workspace too small";
+        case W4_ERR_CUDA: return "CUDA launch or query failed";
+        case W4_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
+        case W4_ERR_RANGE: return "fp16 group scale overflow";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

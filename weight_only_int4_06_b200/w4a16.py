@@ -1,0 +1,167 @@
+"""Thin ctypes binding of libw4a16 (argument marshalling only).
+
+The functions carry the C ABI's names.  Tensors are PyTorch tensors (PyTorch supplies device
+memory and streams); every step of the computation runs in the library's CUDA kernels.  There is
+no fallback: if libw4a16.so is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libw4a16.so")
+
+W4_OK = 0
+STATUS_NAMES = {
+    0: "W4_OK", 1: "W4_ERR_NULL", 2: "W4_ERR_SHAPE", 3: "W4_ERR_ALIGN", 4: "W4_ERR_UNSUPPORTED",
+    5: "W4_ERR_WORKSPACE", 6: "W4_ERR_CUDA", 7: "W4_ERR_DEVICE_TIMEOUT", 8: "W4_ERR_RANGE",
+}
+VARIANT_AUTO, VARIANT_SKINNY, VARIANT_TC = 0, 1, 2
+
+# Entry points declared in include/w4a16.h: (name, restype, argtypes)
+_P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "w4_quantize_pack": (_I32, [_P, _I64, _I64, _I32, _P, _P, _P, _P, _P]),
+    "w4_gemm_workspace_size": (_I32, [_I64, _I64, _I64, _I32, ctypes.POINTER(_SZ)]),
+    "w4_gemm": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ, _P]),
+    "w4_gemm_ex": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ, _I32, _P]),
+    "awq_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
+    "awq_scale_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
+    "w4_check_device_status": (_I32, [_P]),
+    "w4_status_string": (ctypes.c_char_p, [_I32]),
+}
+
+_lib = None
+
+
+class W4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)}")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libw4a16 (raises if it has not been built or cannot be loaded)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libw4a16.so not built ({LIB_PATH}); run "
+                               "`python -m weight_only_int4_06_b200.build_lib`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(st: int, where: str):
+    if st != W4_OK:
+        raise W4Error(st, where)
+
+
+def _stream(stream):
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(stream)
+
+
+def _dev(t: torch.Tensor, dtype, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def w4_quantize_pack(W: torch.Tensor, act_scale: torch.Tensor | None = None, group: int = 128,
+                     stream=None):
+    """Returns (packed [N, K/8] int32 (uint32 bits), scales [N, K/group] fp16, zeros [N, K/group] uint8)."""
+    N, K = W.shape
+    G = K // group if group else 0
+    packed = torch.empty((N, K // 8), dtype=torch.int32, device=W.device)
+    scales = torch.empty((N, G), dtype=torch.float16, device=W.device)
+    zeros = torch.empty((N, G), dtype=torch.uint8, device=W.device)
+    a = _dev(act_scale, torch.float32, "act_scale") if act_scale is not None else None
+    st = lib().w4_quantize_pack(_dev(W, torch.float16, "W"), N, K, group, a,
+                                ctypes.c_void_p(packed.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                                ctypes.c_void_p(zeros.data_ptr()), _stream(stream))
+    _check(st, "w4_quantize_pack")
+    return packed, scales, zeros
+
+
+def w4_gemm_workspace_size(M: int, N: int, K: int, group: int = 128) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().w4_gemm_workspace_size(M, N, K, group, ctypes.byref(n)), "w4_gemm_workspace_size")
+    return n.value
+
+
+def w4_gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+            group: int = 128, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+            variant: int = VARIANT_AUTO, stream=None) -> torch.Tensor:
+    """Y = X . dequant(W)^T.  A host (CPU) X is copied to the device and Y copied back."""
+    host = not X.is_cuda
+    if host:
+        dev = packed.device
+        Xd = X.to(dev, non_blocking=True)
+    else:
+        Xd = X
+    M, K = Xd.shape
+    N = packed.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=Xd.device)
+    need = w4_gemm_workspace_size(M, N, K, group)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=Xd.device)
+    ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().w4_gemm_ex(_dev(Xd, torch.float16, "X"), M, N, K, _dev(packed, torch.int32, "packed"),
+                          _dev(scales, torch.float16, "scales"), _dev(zeros, torch.uint8, "zeros"),
+                          group, _dev(out, torch.float16, "Y"), ws_ptr, ws_bytes, variant,
+                          _stream(stream))
+    _check(st, "w4_gemm")
+    if host:
+        return out.to("cpu", non_blocking=False)
+    return out
+
+
+def awq_workspace_size(T: int, N: int, K: int, group: int = 128, n_alpha: int = 20) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().awq_workspace_size(T, N, K, group, n_alpha, ctypes.byref(n)), "awq_workspace_size")
+    return n.value
+
+
+def awq_scale_search(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20, group: int = 128,
+                     workspace: torch.Tensor | None = None, stream=None):
+    """Returns (mse [n_alpha] fp64, best_idx [1] int32, best_s [K] fp32), all on the device."""
+    T, K = X.shape
+    N = W.shape[0]
+    need = awq_workspace_size(T, N, K, group, n_alpha)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
+    mse = torch.empty(n_alpha, dtype=torch.float64, device=X.device)
+    best = torch.empty(1, dtype=torch.int32, device=X.device)
+    best_s = torch.empty(K, dtype=torch.float32, device=X.device)
+    st = lib().awq_scale_search(_dev(X, torch.float16, "X"), T, _dev(W, torch.float16, "W"), N, K,
+                                group, n_alpha, ctypes.c_void_p(mse.data_ptr()),
+                                ctypes.c_void_p(best.data_ptr()), ctypes.c_void_p(best_s.data_ptr()),
+                                ctypes.c_void_p(workspace.data_ptr()),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "awq_scale_search")
+    return mse, best, best_s
+
+
+def w4_check_device_status(stream=None) -> int:
+    return lib().w4_check_device_status(_stream(stream))
+
+
+def w4_status_string(status: int) -> str:
+    return lib().w4_status_string(status).decode()
