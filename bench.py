@@ -159,10 +159,11 @@ def prefill_cases():
 class GemmWorkload:
     """Device-resident inputs for a list of (M, K, N) layers, with rotating weight copies."""
 
-    def __init__(self, cases, case_id, l2_bytes):
+    def __init__(self, cases, case_id, l2_bytes, variant=0):
         import torch
         from weight_only_int4_06_b200 import w4a16 as B
         self.B = B
+        self.variant = variant
         self.cases = cases
         step_w = sum(N * K // 2 + N * (K // 128) * 3 for (M, K, N) in cases)
         self.n_sets = max(1, min(16, int(np.ceil(3 * l2_bytes / max(step_w, 1))) + 1))
@@ -192,7 +193,7 @@ class GemmWorkload:
             if only is not None and i != only:
                 continue
             p, sc, z = L["copies"][s]
-            self.B.w4_gemm(L["X"], p, sc, z, out=L["Y"], workspace=L["ws"])
+            self.B.w4_gemm(L["X"], p, sc, z, out=L["Y"], workspace=L["ws"], variant=self.variant)
 
     def run_step_host(self, step):
         """The same step through the public API with host (pinned) activations and results."""
@@ -261,17 +262,41 @@ def oracle_cpu_baseline(cases, case_id, budget_s=20.0):
                        + "; oracle = numpy dequantise + fp64 matmul (OpenBLAS threads)")}
 
 
-def run_gemm_bench(args, rank, world, local, kind):
+def layer_rows(wl, world, reps, peaks, compute_bound):
+    """Per-layer device time, one layer at a time, same graph protocol."""
+    rows = []
+    for i, L in enumerate(wl.layers):
+        gi = capture(lambda s, i=i: wl.run_step(s, only=i), reps, 0)
+        gi.replay()
+        t = max_over_ranks(time_graph(gi, world) / reps, world)
+        b = gemm_bytes(L["M"], L["K"], L["N"])
+        fl = 2 * L["M"] * L["K"] * L["N"]
+        r = {"M": L["M"], "K": L["K"], "N": L["N"], "us": round(t * 1e3, 3),
+             "GBps": round(b / (t * 1e-3) / 1e9, 1), "TFLOPs": round(fl / (t * 1e-3) / 1e12, 2)}
+        if compute_bound:
+            r["tensor_frac"] = round(fl / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 3)
+        else:
+            r["hbm_frac"] = round(b / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)
+        rows.append(r)
+        del gi
+    return rows
+
+
+def run_gemm_bench(args, rank, world, local, kind, with_extras=True):
     import torch
+    from weight_only_int4_06_b200 import w4a16 as B
     cases, case_id, desc = {"decode": decode_cases, "small_batch": small_batch_cases,
                             "prefill": prefill_cases}[kind]()
+    compute_bound = kind == "prefill"
     peaks = load_peaks()
     props = torch.cuda.get_device_properties(torch.cuda.current_device())
     l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
-    wl = GemmWorkload(cases, case_id, l2)
+    # Decode-time weights are resident and never rewritten between calls: declare them static so
+    # each GEMM may start streaming its weights while the previous kernel drains.
+    variant = B.FLAG_WEIGHTS_STATIC
+    wl = GemmWorkload(cases, case_id, l2, variant=variant)
     K_steps, W_steps = args.steps, args.warmup
 
-    # warm-up (eager once, then graphed)
     for i in range(2):
         wl.run_step(i)
     torch.cuda.synchronize()
@@ -291,23 +316,19 @@ def run_gemm_bench(args, rank, world, local, kind):
     clocks = sampler.stop() if sampler else None
     ms = max_over_ranks(ms, world)
     ms_per_step = ms / K_steps
+    del g_timed, g_warm
 
-    # per-layer times (same protocol, one layer at a time)
-    per_layer = []
-    for i, L in enumerate(wl.layers):
-        reps = max(W_steps, 20)
-        gi = capture(lambda s, i=i: wl.run_step(s, only=i), reps, 0)
-        gi.replay()
-        t = time_graph(gi, world) / reps
-        t = max_over_ranks(t, world)
-        b = gemm_bytes(L["M"], L["K"], L["N"])
-        fl = 2 * L["M"] * L["K"] * L["N"]
-        per_layer.append({"M": L["M"], "K": L["K"], "N": L["N"], "us": round(t * 1e3, 3),
-                          "GBps": round(b / (t * 1e-3) / 1e9, 1),
-                          "TFLOPs": round(fl / (t * 1e-3) / 1e12, 2),
-                          "hbm_frac": round(b / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)})
+    # the same step with plain stream-ordered launches (no early weight streaming)
+    wl.variant = 0
+    g_plain = capture(wl.run_step, K_steps, 0)
+    g_plain.replay()
+    ms_plain = max_over_ranks(time_graph(g_plain, world), world) / K_steps
+    del g_plain
+    wl.variant = variant
 
-    # end to end through the public API with host buffers
+    per_layer = layer_rows(wl, world, max(W_steps, 20), peaks, compute_bound)
+
+    # end to end through the public API with host buffers (pinned X in, Y out, every step)
     h2d, d2h = wl.h2d_d2h_bytes()
     e2e_steps = min(K_steps, 50)
     barrier(world)
@@ -321,19 +342,23 @@ def run_gemm_bench(args, rank, world, local, kind):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
 
-    compute_bound = kind == "prefill"
     if compute_bound:
         achieved = wl.flops_per_step / (ms_per_step * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None}
+                "frac": round(achieved / peak, 4), "traffic": None,
+                "peak_note": "dense bf16 burst (fp16 dense rate is the same on B200)"}
+        kern = "tc_gemm_kernel<DEQ> (tcgen05 + TMEM + TMA)"
     else:
         achieved = wl.bytes_per_step / (ms_per_step * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": None}
+        kern = "skinny_kernel (mma.sync GEMV, cluster split-K)"
     roof["peak_source"] = peaks["source"]
-    roof["kernel"] = "skinny_kernel (mma.sync split-K cluster GEMV)" if not compute_bound else "w4 GEMM"
+    roof["kernel"] = kern
+    roof["algorithmic_bytes_per_step"] = wl.bytes_per_step
+    roof["algorithmic_flops_per_step"] = wl.flops_per_step
 
     out = {
         "metric": "W4A16 GEMM us & % roofline (HBM GB/s at M<=16, TFLOP/s at M>=512)",
@@ -349,21 +374,110 @@ def run_gemm_bench(args, rank, world, local, kind):
         "dtype": "f16",
         "data": "synthetic",
         "config": {"workload": desc, "layers": [list(c) for c in cases], "group": 128,
-                   "weight_buffer_sets": wl.n_sets,
+                   "weights_static_flag": True,
                    "l2": f"cold: {wl.n_sets} rotating weight-buffer sets, >=3x L2 between reuses",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": roof,
+        "plain_launch_us_per_step": round(ms_plain * 1e3, 3),
         "layers": per_layer,
         "e2e": {"value": round(e2e_ms * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": wl.launches_per_step * K_steps,
         "clocks": clocks,
     }
+    del wl
+    torch.cuda.empty_cache()
+    if with_extras and not args.no_rows:
+        out["rows"] = other_rows(args, world, peaks, l2)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = oracle_cpu_baseline(cases, case_id)
         out["cpu_baseline"] = {"value": round(cb["value_us_per_step"], 1), "unit": "us/step",
                                "cores": cb["cores"], "kind": "oracle", "sample": cb["sample"]}
     return out
+
+
+def bench_quantize(world, peaks, l2, reps=10):
+    """w4_quantize_pack on the four 7B-class weight matrices, rotating copies (cold L2)."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    res = []
+    for (K, N) in synth.DECODE_7B_SHAPES:
+        _, W = synth.layer_case(2, 1, K, N)
+        Wd = torch.from_numpy(W).cuda()
+        n_sets = max(2, int(np.ceil(3 * l2 / (W.nbytes))) + 1)
+        Ws = [Wd] + [Wd.clone() for _ in range(n_sets - 1)]
+        outs = [B.w4_quantize_pack(w) for w in Ws]
+        G = K // 128
+        L = B.lib()
+        stream = B._stream(None)
+
+        def step(i):
+            w = Ws[i % n_sets]
+            p, s, z = outs[i % n_sets]
+            L.w4_quantize_pack(B._dev(w, torch.float16, "W"), N, K, 128, None,
+                               B.ctypes.c_void_p(p.data_ptr()), B.ctypes.c_void_p(s.data_ptr()),
+                               B.ctypes.c_void_p(z.data_ptr()), B._stream(None))
+        step(0)
+        g = capture(step, reps, 0)
+        g.replay()
+        t = max_over_ranks(time_graph(g, world) / reps, world)
+        byts = N * K * 2 + N * K // 2 + N * G * 3
+        res.append({"K": K, "N": N, "us": round(t * 1e3, 2), "GBps": round(byts / (t * 1e-3) / 1e9, 1),
+                    "hbm_frac": round(byts / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)})
+        del g, Ws, outs, Wd
+        _ = stream
+    torch.cuda.empty_cache()
+    return {"kernel": "quantize_pack_kernel", "bound": "hbm", "layers": res}
+
+
+def bench_awq(world, peaks, reps=2):
+    """awq_scale_search on X_calib [65536, 4096], W [4096, 4096], 20 alphas."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    X, W = synth.awq_case()
+    Xd = torch.from_numpy(X).cuda()
+    Wd = torch.from_numpy(W).cuda()
+    T, K = X.shape
+    N = W.shape[0]
+    ws = torch.empty(B.awq_workspace_size(T, N, K, 128, 20), dtype=torch.uint8, device="cuda")
+    B.awq_scale_search(Xd, Wd, 20, workspace=ws)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        B.awq_scale_search(Xd, Wd, 20, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    t = max_over_ranks(min(times), world)
+    flops = 20 * 2 * T * K * N
+    tf = flops / (t * 1e-3) / 1e12
+    del Xd, Wd, ws
+    torch.cuda.empty_cache()
+    return {"kernel": "colabs + 20 x (awq_fakequant + tc_gemm_kernel<SSE>) + finalize",
+            "T": T, "K": K, "N": N, "n_alpha": 20, "ms": round(t, 3), "TFLOPs": round(tf, 1),
+            "bound": "tensor", "tensor_frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 3),
+            "flops": flops}
+
+
+def other_rows(args, world, peaks, l2):
+    import torch
+    rows = {}
+    rows["quantize"] = bench_quantize(world, peaks, l2)
+    pre = GemmWorkload(prefill_cases()[0], 4, l2)
+    reps = 10
+    pre.run_step(0)
+    torch.cuda.synchronize()
+    rows["prefill"] = {"kernel": "tc_gemm_kernel<DEQ>", "bound": "tensor",
+                       "layers": layer_rows(pre, world, reps, peaks, True)}
+    del pre
+    torch.cuda.empty_cache()
+    rows["awq"] = bench_awq(world, peaks)
+    return rows
 
 
 def run_reference(args, rank, world):
@@ -399,9 +513,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode",
-                    choices=["decode", "small_batch", "prefill"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "small_batch", "prefill"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true",
+                    help="skip the secondary rows (quantize, prefill, awq) in the JSON line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

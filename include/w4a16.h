@@ -73,7 +73,12 @@ typedef enum {
 typedef enum {
     W4_VARIANT_AUTO = 0,
     W4_VARIANT_SKINNY = 1, /* warp-level tensor-core GEMV / skinny GEMM, split-K over a cluster */
-    W4_VARIANT_TC = 2      /* tcgen05/TMEM tensor-core GEMM with dequantisation in the smem path */
+    W4_VARIANT_TC = 2,     /* tcgen05/TMEM tensor-core GEMM with dequantisation in the smem path */
+    /* Flag, OR-ed into the variant: packed/scales/zeros are not written by any work still in
+     * flight on the stream (static weights).  The call may then use programmatic dependent launch
+     * and start streaming the weights before the preceding kernel on the stream has finished;
+     * X is still read only after that kernel has completed. */
+    W4_FLAG_WEIGHTS_STATIC = 0x100
 } w4_variant;
 
 /*
@@ -126,7 +131,8 @@ w4_status w4_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint
                   const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y, void* ws,
                   size_t ws_bytes, void* stream);
 
-/* w4_gemm with an explicit kernel family (W4_VARIANT_AUTO behaves exactly like w4_gemm). */
+/* w4_gemm with an explicit kernel family, optionally OR-ed with W4_FLAG_WEIGHTS_STATIC
+ * (W4_VARIANT_AUTO alone behaves exactly like w4_gemm).  Unknown values: W4_ERR_UNSUPPORTED. */
 w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                      const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y,
                      void* ws, size_t ws_bytes, int variant, void* stream);

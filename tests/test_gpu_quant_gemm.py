@@ -197,3 +197,27 @@ def test_gemm_host_buffers_match_device():
     Yh = B.w4_gemm(Xh, dev(p.view(np.int32)), dev(s), dev(z))
     assert not Yh.is_cuda
     assert np.array_equal(Yh.numpy().view(np.uint16), Yd.view(np.uint16))
+
+
+# ------------------------------------------------------------------ forced kernel families
+@pytest.mark.parametrize("M,K,N", [(1, 128, 8), (7, 256, 136), (128, 384, 256), (129, 4096, 264),
+                                   (300, 1152, 520), (512, 8192, 1024), (64, 11008, 4096)])
+def test_gemm_tc_ragged(M, K, N):
+    X, p, s, z = oracle_case(25, M, K, N)
+    assert_close(gpu_gemm(X, p, s, z, B.VARIANT_TC), oracle.gemm(X, p, s, z), f"tc {M}x{K}x{N}")
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 4096, 4096), (8, 8192, 1024), (32, 28672, 256)])
+def test_gemm_weights_static_flag_same_bits(M, K, N):
+    """The static-weights launch (programmatic dependent launch) computes the same bits."""
+    X, p, s, z = oracle_case(26, M, K, N)
+    Y0 = gpu_gemm(X, p, s, z, B.VARIANT_AUTO)
+    Y1 = gpu_gemm(X, p, s, z, B.VARIANT_AUTO | B.FLAG_WEIGHTS_STATIC)
+    assert np.array_equal(Y0.view(np.uint16), Y1.view(np.uint16))
+
+
+def test_gemm_tc_deterministic():
+    X, p, s, z = oracle_case(27, 1024, 4096, 2048)
+    Y1 = gpu_gemm(X, p, s, z, B.VARIANT_TC)
+    Y2 = gpu_gemm(X, p, s, z, B.VARIANT_TC)
+    assert np.array_equal(Y1.view(np.uint16), Y2.view(np.uint16))

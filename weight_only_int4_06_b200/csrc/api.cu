@@ -91,7 +91,9 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
                      const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y,
                      void* ws, size_t ws_bytes, int variant, void* stream) {
     if (group != 128) return W4_ERR_UNSUPPORTED;
-    if (variant < W4_VARIANT_AUTO || variant > W4_VARIANT_TC) return W4_ERR_UNSUPPORTED;
+    const bool weights_static = (variant & W4_FLAG_WEIGHTS_STATIC) != 0;
+    const int family = variant & ~W4_FLAG_WEIGHTS_STATIC;
+    if (family < W4_VARIANT_AUTO || family > W4_VARIANT_TC) return W4_ERR_UNSUPPORTED;
     if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0)
         return W4_ERR_SHAPE;
     size_t need = 0;
@@ -108,14 +110,21 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     }
     if (!X || !packed || !scales || !zeros) return W4_ERR_NULL;
     if (!aligned16(X) || !aligned16(packed)) return W4_ERR_ALIGN;
-    if (!device_status_ptr()) return W4_ERR_CUDA;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
 
-    // Skinny path in chunks of at most 32 activation rows.
+    const bool use_tc = family == W4_VARIANT_TC || (family == W4_VARIANT_AUTO && M > 32);
+    if (use_tc) {
+        return launch_tc_w4(X, M, N, K, packed, scales, zeros, Y, status, s) == cudaSuccess ? W4_OK
+                                                                                            : W4_ERR_CUDA;
+    }
+    // Skinny path, in chunks of at most 32 activation rows.
     for (int64_t m0 = 0; m0 < M; m0 += 32) {
         const int64_t mc = (M - m0) < 32 ? (M - m0) : 32;
         SkinnyPlan plan;
         if (!plan_skinny(mc, N, K, &plan)) return W4_ERR_SHAPE;
-        cudaError_t e = launch_skinny(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N, plan, s);
+        cudaError_t e = launch_skinny(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N, plan,
+                                      weights_static, s);
         if (e != cudaSuccess) return W4_ERR_CUDA;
     }
     return W4_OK;
@@ -128,22 +137,35 @@ w4_status w4_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint
                       stream);
 }
 
-w4_status awq_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha,
-                             size_t* bytes) {
-    if (!bytes) return W4_ERR_NULL;
+static w4_status awq_check(int64_t T, int64_t N, int64_t K, int group, int n_alpha) {
     if (group != 128 || n_alpha < 1 || n_alpha > 64) return W4_ERR_UNSUPPORTED;
     if (!dims_ok(T, K) || !dims_ok(N, K) || T < 1 || N < 8 || K < 128 || K % group != 0 || N % 8 != 0)
         return W4_ERR_SHAPE;
-    *bytes = 0;
-    return W4_ERR_UNSUPPORTED;  // not built yet
+    return W4_OK;
+}
+
+w4_status awq_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha,
+                             size_t* bytes) {
+    if (!bytes) return W4_ERR_NULL;
+    w4_status st = awq_check(T, N, K, group, n_alpha);
+    if (st != W4_OK) return st;
+    *bytes = awq_layout(T, N, K, n_alpha).bytes;
+    return W4_OK;
 }
 
 w4_status awq_scale_search(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K,
                            int group, int n_alpha, double* mse, int32_t* best_idx, float* best_s,
                            void* ws, size_t ws_bytes, void* stream) {
-    (void)X; (void)T; (void)W; (void)N; (void)K; (void)group; (void)n_alpha; (void)mse;
-    (void)best_idx; (void)best_s; (void)ws; (void)ws_bytes; (void)stream;
-    return W4_ERR_UNSUPPORTED;  // not built yet
+    w4_status st = awq_check(T, N, K, group, n_alpha);
+    if (st != W4_OK) return st;
+    if (ws_bytes < awq_layout(T, N, K, n_alpha).bytes) return W4_ERR_WORKSPACE;
+    if (!X || !W || !mse || !best_idx || !best_s || !ws) return W4_ERR_NULL;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(ws)) return W4_ERR_ALIGN;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_awq(X, T, W, N, K, n_alpha, mse, best_idx, best_s, ws, status,
+                               (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
 w4_status w4_check_device_status(void* stream) {

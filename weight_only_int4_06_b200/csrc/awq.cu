@@ -1,0 +1,253 @@
+// AWQ activation-aware scale search on one linear layer.
+//
+// "GPTQ, AWQ and the rules of post-training quantization", section "AWQ: find the one percent
+// that matters": the scale of input channel j is the average activation magnitude raised to a
+// power alpha; alpha comes from a grid search over [0, 1]; scaling W's channel j by s_j and
+// dividing X's channel j by s_j keeps the layer's function while the quantisation error of the
+// salient channels shrinks.
+//
+// Steps on the device (all on the caller's stream, workspace supplied by the caller):
+//   1. colabs:    c_j = sum_t |X[t, j]| as an exact integer count of 2^-24 units (every fp16 value
+//                 is such a multiple), so the sum is exact and order-independent;
+//                 m_j = c_j * 2^-24 / T, rounded once to fp64.
+//   2. scales:    s_ij = max(m_j, 1e-6)^(i / n_alpha) / sqrt(max_j s * min_j s) in fp64, then
+//                 rounded to fp32 (the value that multiplies W and divides X).
+//   3. per alpha: fake-quantise W * diag(s_i) with exactly the quantiser of w4_quantize_pack and
+//                 emit E_i = (Wq - W * s_i) / s_i rounded to fp16, so that
+//                 (X / s_i) Wq^T - X W^T = X E_i^T;
+//                 then sum_{t,n} (X E_i^T)^2 with the tcgen05 GEMM (sum-of-squares epilogue,
+//                 one fp64 partial per 128x256 tile).
+//   4. finalize:  MSE_i = (fixed-order fp64 sum of the partials) / (T N); best = lowest index
+//                 among the minima; best_s = s_best.
+#include "common.cuh"
+#include "internal.h"
+#include "quant_rtn.cuh"
+
+namespace w4 {
+
+// |x| of an fp16 value as an integer number of 2^-24 units (exact; at most 2^41).
+__device__ __forceinline__ uint64_t abs_units(uint32_t h) {
+    const uint32_t b = h & 0x7FFFu;
+    const uint32_t e = b >> 10, m = b & 0x3FFu;
+    return e == 0 ? (uint64_t)m : ((uint64_t)(m | 0x400u) << (e - 1));
+}
+
+constexpr int CA_ROWS = 256;  // rows of X per CTA
+
+__global__ void __launch_bounds__(256) colabs_kernel(const uint4* __restrict__ X, int64_t T, int K,
+                                                     unsigned long long* __restrict__ colsum) {
+    const int chunks = K >> 3;  // 8 fp16 per 16-byte chunk
+    const int ch = blockIdx.x * blockDim.x + threadIdx.x;
+    if (ch >= chunks) return;
+    const int64_t r0 = (int64_t)blockIdx.y * CA_ROWS;
+    const int64_t r1 = min(T, r0 + CA_ROWS);
+    uint64_t acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int64_t r = r0;
+    for (; r + 4 <= r1; r += 4) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = ldg_stream(X + (r + u) * chunks + ch);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                acc[2 * i] += abs_units(w[i] & 0xFFFFu);
+                acc[2 * i + 1] += abs_units(w[i] >> 16);
+            }
+        }
+    }
+    for (; r < r1; ++r) {
+        const uint4 v = ldg_stream(X + r * chunks + ch);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc[2 * i] += abs_units(w[i] & 0xFFFFu);
+            acc[2 * i + 1] += abs_units(w[i] >> 16);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) atomicAdd(colsum + ch * 8 + i, (unsigned long long)acc[i]);  // exact
+}
+
+// One CTA per alpha.  Block-wide max/min with a fixed reduction tree.
+__global__ void __launch_bounds__(1024) awq_scales_kernel(const unsigned long long* __restrict__ colsum,
+                                                          int64_t T, int K, int n_alpha, float* __restrict__ s_all) {
+    __shared__ double smax[32], smin[32];
+    __shared__ double norm;
+    const int i = blockIdx.x;
+    const double alpha = (double)i / (double)n_alpha;
+    const double inv_units = 5.9604644775390625e-08;  // 2^-24
+    double mx = 0.0, mn = 1.0e308;
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+        const double m = (double)colsum[j] * inv_units / (double)T;
+        const double s = pow(fmax(m, 1e-6), alpha);
+        mx = fmax(mx, s);
+        mn = fmin(mn, s);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+        mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    }
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) { smax[w] = mx; smin[w] = mn; }
+    __syncthreads();
+    if (w == 0) {
+        const int nw = blockDim.x >> 5;
+        mx = l < nw ? smax[l] : 0.0;
+        mn = l < nw ? smin[l] : 1.0e308;
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+            mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            mn = fmin(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        }
+        if (l == 0) norm = sqrt(mx * mn);
+    }
+    __syncthreads();
+    const double nv = norm;
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+        const double m = (double)colsum[j] * inv_units / (double)T;
+        const double s = pow(fmax(m, 1e-6), alpha) / nv;
+        s_all[(int64_t)i * K + j] = __double2float_rn(s);
+    }
+}
+
+// E = (Wq - W*s) / s in fp16 for one alpha; the codes are those of w4_quantize_pack(W, s).
+__global__ void __launch_bounds__(256) awq_fakequant_kernel(const uint4* __restrict__ W, const float* __restrict__ s,
+                                                            int64_t n_groups, int G, uint4* __restrict__ E,
+                                                            int* status) {
+    const int lane = threadIdx.x & 31;
+    const int sub = lane >> 4, l16 = lane & 15;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t n_pairs = (n_groups + 1) >> 1;
+    for (int64_t pair = warp; pair < n_pairs; pair += nwarps) {
+        const int64_t f = 2 * pair + sub;
+        const bool valid = f < n_groups;
+        float v[8], a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { v[i] = 0.0f; a[i] = 1.0f; }
+        if (valid) {
+            const uint4 raw = ldg_stream(W + f * 16 + l16);
+            const int64_t k0 = (f % G) * 128 + 8 * l16;
+            const float4 a0 = __ldg(reinterpret_cast<const float4*>(s + k0));
+            const float4 a1 = __ldg(reinterpret_cast<const float4*>(s + k0) + 1);
+            a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
+            a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+            load8_scaled(raw, a, v);
+        }
+        float mn = v[0], mx = v[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) { mn = fminf(mn, v[i]); mx = fmaxf(mx, v[i]); }
+#pragma unroll
+        for (int o = 8; o; o >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        const GroupQuant p = group_params(fminf(mn, 0.0f), fmaxf(mx, 0.0f));
+        if (valid) {
+            uint32_t out[4];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+                float e2[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int q = (int)quant_code(v[i + u], p);
+                    const float wq = (float)(q - p.z) * p.sf;  // exact: |q - z| <= 15, sf has 11 bits
+                    e2[u] = __fdiv_rn(__fsub_rn(wq, v[i + u]), a[i + u]);
+                }
+                out[i / 2] = pack_half2(e2[0], e2[1]);
+            }
+            E[f * 16 + l16] = make_uint4(out[0], out[1], out[2], out[3]);
+            if (l16 == 0 && p.overflow) record_status(status, W4_ERR_RANGE);
+        }
+    }
+}
+
+// Fixed-order reduction of the per-tile partials, argmin, and the chosen scales.
+__global__ void __launch_bounds__(256) awq_finalize_kernel(const double* __restrict__ part, int n_part, int n_alpha,
+                                                           double denom, const float* __restrict__ s_all, int K,
+                                                           double* __restrict__ mse, int32_t* __restrict__ best_idx,
+                                                           float* __restrict__ best_s) {
+    __shared__ double red[256];
+    __shared__ double vals[64];
+    __shared__ int best_sh;
+    for (int i = 0; i < n_alpha; ++i) {
+        double acc = 0.0;
+        for (int p = threadIdx.x; p < n_part; p += blockDim.x) acc += part[(int64_t)i * n_part + p];
+        red[threadIdx.x] = acc;
+        __syncthreads();
+        for (int w = 128; w; w >>= 1) {
+            if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) vals[i] = red[0] / denom;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+        int b = 0;
+        for (int i = 0; i < n_alpha; ++i) {
+            mse[i] = vals[i];
+            if (vals[i] < vals[b]) b = i;
+        }
+        *best_idx = b;
+        best_sh = b;
+    }
+    __syncthreads();
+    const int b = best_sh;
+    for (int j = threadIdx.x; j < K; j += blockDim.x) best_s[j] = s_all[(int64_t)b * K + j];
+}
+
+// ------------------------------------------------------------------------------------ host side
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+AwqLayout awq_layout(int64_t T, int64_t N, int64_t K, int n_alpha) {
+    AwqLayout L;
+    L.n_part = tc_sse_partials(T, N);
+    size_t off = 0;
+    L.colsum = off; off = align256(off + (size_t)K * 8);
+    L.s_all = off; off = align256(off + (size_t)n_alpha * K * 4);
+    L.E = off; off = align256(off + (size_t)N * K * 2);
+    L.part = off; off = align256(off + (size_t)n_alpha * L.n_part * 8);
+    L.bytes = off;
+    return L;
+}
+
+cudaError_t launch_awq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int n_alpha,
+                       double* mse, int32_t* best_idx, float* best_s, void* ws, int* status, cudaStream_t stream) {
+    const AwqLayout L = awq_layout(T, N, K, n_alpha);
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    auto* colsum = reinterpret_cast<unsigned long long*>(base + L.colsum);
+    float* s_all = reinterpret_cast<float*>(base + L.s_all);
+    uint16_t* E = reinterpret_cast<uint16_t*>(base + L.E);
+    double* part = reinterpret_cast<double*>(base + L.part);
+
+    cudaError_t e = cudaMemsetAsync(colsum, 0, (size_t)K * 8, stream);
+    if (e != cudaSuccess) return e;
+    {
+        const int chunks = (int)(K / 8);
+        dim3 grid((chunks + 255) / 256, (unsigned)((T + CA_ROWS - 1) / CA_ROWS));
+        colabs_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(X), T, (int)K, colsum);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    awq_scales_kernel<<<n_alpha, 1024, 0, stream>>>(colsum, T, (int)K, n_alpha, s_all);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int64_t G = K / 128;
+    const int64_t n_groups = N * G;
+    const int64_t want = ((n_groups + 1) / 2 + 7) / 8;
+    const int64_t cap = (int64_t)device_sm_count() * 8;
+    const int fq_blocks = (int)(want < cap ? want : cap);
+    for (int i = 0; i < n_alpha; ++i) {
+        awq_fakequant_kernel<<<fq_blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(W), s_all + (int64_t)i * K,
+                                                             n_groups, (int)G, reinterpret_cast<uint4*>(E), status);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_tc_sse(X, T, E, N, K, part + (int64_t)i * L.n_part, status, stream);
+        if (e != cudaSuccess) return e;
+    }
+    awq_finalize_kernel<<<1, 256, 0, stream>>>(part, L.n_part, n_alpha, (double)T * (double)N, s_all, (int)K, mse,
+                                               best_idx, best_s);
+    return cudaGetLastError();
+}
+
+}  // namespace w4

@@ -62,11 +62,13 @@ __device__ __forceinline__ size_t sk_xs_bytes(int gps) {
     return a > b ? a : b;
 }
 
+constexpr int SK_MAX_SPLITS = 16;
+
 template <int NT, int MINB>
 __global__ void __launch_bounds__(SK_THREADS, MINB)
     skinny_kernel(const __half* __restrict__ X, int M, int N, int K, const uint4* __restrict__ packed4,
-                  const __half* __restrict__ scales, const uint8_t* __restrict__ zeros,
-                  __half* __restrict__ Y, int splits, int gps) {
+                  const unsigned short* __restrict__ scales, const uint8_t* __restrict__ zeros,
+                  __half* __restrict__ Y, int splits, int gps, int weights_early) {
     constexpr int MT = 8 * NT;
     extern __shared__ __align__(16) unsigned char smem[];
     const int G = K >> 7;
@@ -79,52 +81,69 @@ __global__ void __launch_bounds__(SK_THREADS, MINB)
 
     __half* Xs = reinterpret_cast<__half*>(smem);
     float* Part = reinterpret_cast<float*>(smem);  // reuses the activation area after the main loop
-    float* Ss = reinterpret_cast<float*>(smem + sk_xs_bytes<NT>(gps));
-    uint8_t* Zs = reinterpret_cast<uint8_t*>(Ss + SK_BN * gps);
 
     const int ra = warp * 16 + g8, rb = ra + 8;
     const bool va = n0 + ra < N, vb = n0 + rb < N;
     const int64_t row4 = K >> 5;  // 16-byte chunks per packed row
     const uint4* pa = packed4 + (int64_t)(n0 + ra) * row4 + gb * 4 + c;
     const uint4* pb = packed4 + (int64_t)(n0 + rb) * row4 + gb * 4 + c;
+    const unsigned short* sca = scales + (int64_t)(n0 + ra) * G + gb;
+    const unsigned short* scb = scales + (int64_t)(n0 + rb) * G + gb;
+    const uint8_t* zpa = zeros + (int64_t)(n0 + ra) * G + gb;
+    const uint8_t* zpb = zeros + (int64_t)(n0 + rb) * G + gb;
 
-    // Put the first groups of W in flight before anything else.
+    // W, scales and zero points of the first SK_PD groups go in flight first.  Weights are only
+    // read ahead of the preceding kernel when the caller declared them static.
+    if (!weights_early) pdl_wait();
     uint4 wa[SK_PD], wb[SK_PD];
+    uint32_t ma[SK_PD], mb[SK_PD];  // scale bits | zero << 16
 #pragma unroll
     for (int s = 0; s < SK_PD; ++s) {
         wa[s] = make_uint4(0u, 0u, 0u, 0u);
         wb[s] = make_uint4(0u, 0u, 0u, 0u);
+        ma[s] = 0u;
+        mb[s] = 0u;
         if (s < ng) {
-            if (va) wa[s] = ldg_stream(pa + s * 4);
-            if (vb) wb[s] = ldg_stream(pb + s * 4);
+            if (va) {
+                wa[s] = ldg_stream(pa + s * 4);
+                ma[s] = (uint32_t)__ldg(sca + s) | ((uint32_t)__ldg(zpa + s) << 16);
+            }
+            if (vb) {
+                wb[s] = ldg_stream(pb + s * 4);
+                mb[s] = (uint32_t)__ldg(scb + s) | ((uint32_t)__ldg(zpb + s) << 16);
+            }
         }
     }
+    if (weights_early) pdl_wait();  // activations may come from the preceding kernel
 
-    // Stage this split's activations (rows >= M are zero), 8-k chunks permuted to (0,4,1,5,2,6,3,7).
+    // Stage this split's activations (rows >= M are zero), 8-k chunks permuted to
+    // (0,4,1,5,2,6,3,7); four loads per thread are in flight before any store.
     const int cpr = ng * 16;
-    for (int i = tid; i < MT * cpr; i += SK_THREADS) {
-        const int m = i / cpr, ch = i - m * cpr;
-        uint4 r = make_uint4(0u, 0u, 0u, 0u);
-        if (m < M) r = ldg_cached(X + (int64_t)m * K + gb * 128 + ch * 8);
-        uint4 p;
-        p.x = __byte_perm(r.x, r.z, 0x5410);
-        p.y = __byte_perm(r.x, r.z, 0x7632);
-        p.z = __byte_perm(r.y, r.w, 0x5410);
-        p.w = __byte_perm(r.y, r.w, 0x7632);
-        *reinterpret_cast<uint4*>(Xs + m * RSh + sk_swz(ch) * 8) = p;
-    }
-    // Stage this tile's scales (as fp32) and zero points.
-    for (int i = tid; i < SK_BN * ng; i += SK_THREADS) {
-        const int r = i / ng, gi = i - r * ng;
-        const int n = n0 + r;
-        float s = 0.0f;
-        uint8_t z = 0;
-        if (n < N) {
-            s = __half2float(scales[(int64_t)n * G + gb + gi]);
-            z = zeros[(int64_t)n * G + gb + gi];
+    const int total = MT * cpr;
+    for (int base = tid; base < total; base += 4 * SK_THREADS) {
+        uint4 r[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * SK_THREADS;
+            r[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < total) {
+                const int m = i / cpr, ch = i - m * cpr;
+                if (m < M) r[u] = ldg_cached(X + (int64_t)m * K + gb * 128 + ch * 8);
+            }
         }
-        Ss[r * gps + gi] = s;
-        Zs[r * gps + gi] = z;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * SK_THREADS;
+            if (i < total) {
+                const int m = i / cpr, ch = i - m * cpr;
+                uint4 p;
+                p.x = __byte_perm(r[u].x, r[u].z, 0x5410);
+                p.y = __byte_perm(r[u].x, r[u].z, 0x7632);
+                p.z = __byte_perm(r[u].y, r[u].w, 0x5410);
+                p.w = __byte_perm(r[u].y, r[u].w, 0x7632);
+                *reinterpret_cast<uint4*>(Xs + m * RSh + sk_swz(ch) * 8) = p;
+            }
+        }
     }
     __syncthreads();
 
@@ -141,12 +160,21 @@ __global__ void __launch_bounds__(SK_THREADS, MINB)
             const int gi = g0 + s;
             if (gi < ng) {
                 const uint4 A = wa[s], B = wb[s];
-                if (gi + SK_PD < ng) {
-                    if (va) wa[s] = ldg_stream(pa + (gi + SK_PD) * 4);
-                    if (vb) wb[s] = ldg_stream(pb + (gi + SK_PD) * 4);
+                const uint32_t mA = ma[s], mB = mb[s];
+                const int gn = gi + SK_PD;
+                if (gn < ng) {
+                    if (va) {
+                        wa[s] = ldg_stream(pa + gn * 4);
+                        ma[s] = (uint32_t)__ldg(sca + gn) | ((uint32_t)__ldg(zpa + gn) << 16);
+                    }
+                    if (vb) {
+                        wb[s] = ldg_stream(pb + gn * 4);
+                        mb[s] = (uint32_t)__ldg(scb + gn) | ((uint32_t)__ldg(zpb + gn) << 16);
+                    }
                 }
-                const float sa = Ss[ra * gps + gi], sb = Ss[rb * gps + gi];
-                const uint32_t za = Zs[ra * gps + gi], zb = Zs[rb * gps + gi];
+                const float sa = __half2float(__ushort_as_half((unsigned short)(mA & 0xFFFFu)));
+                const float sb = __half2float(__ushort_as_half((unsigned short)(mB & 0xFFFFu)));
+                const uint32_t za = mA >> 16, zb = mB >> 16;
                 const uint32_t zla = (0x6400u + za) * 0x10001u, zha = (0xD400u | (za << 4)) * 0x10001u;
                 const uint32_t zlb = (0x6400u + zb) * 0x10001u, zhb = (0xD400u | (zb << 4)) * 0x10001u;
                 const uint32_t wA[4] = {A.x, A.y, A.z, A.w};
@@ -179,6 +207,7 @@ __global__ void __launch_bounds__(SK_THREADS, MINB)
             }
         }
     }
+    pdl_launch_dependents();  // the next kernel may start streaming its weights now
 
     __syncthreads();  // every warp is done with Xs before Part overwrites it
 #pragma unroll
@@ -205,8 +234,14 @@ __global__ void __launch_bounds__(SK_THREADS, MINB)
         const int nr = r1 - r0;
         for (int i = tid; i < M * nr; i += SK_THREADS) {
             const int m = i / nr, r = r0 + (i - m * nr);
+            float v[SK_MAX_SPLITS];
+#pragma unroll
+            for (int s = 0; s < SK_MAX_SPLITS; ++s)
+                v[s] = s < splits ? cluster.map_shared_rank(Part, s)[m * SK_BN + r] : 0.0f;
             float sum = 0.0f;
-            for (int s = 0; s < splits; ++s) sum += cluster.map_shared_rank(Part, s)[m * SK_BN + r];
+#pragma unroll
+            for (int s = 0; s < SK_MAX_SPLITS; ++s)
+                if (s < splits) sum += v[s];  // split order: deterministic
             if (n0 + r < N) Y[(int64_t)m * N + n0 + r] = __float2half_rn(sum);
         }
         cluster.sync();  // keep this CTA's partials alive until every peer has read them
@@ -218,7 +253,7 @@ static size_t skinny_smem_bytes(int mt, int gps) {
     const size_t xs_a = (size_t)mt * (gps * 128 + 8) * 2;
     const size_t xs_b = (size_t)mt * SK_BN * 4;
     const size_t xs = xs_a > xs_b ? xs_a : xs_b;
-    return xs + (size_t)SK_BN * gps * 4 + (size_t)SK_BN * gps + 16;
+    return xs + 16;
 }
 
 bool plan_skinny(int64_t M, int64_t N, int64_t K, SkinnyPlan* plan) {
@@ -253,7 +288,7 @@ bool plan_skinny(int64_t M, int64_t N, int64_t K, SkinnyPlan* plan) {
 template <int NT, int MINB>
 static cudaError_t launch_nt(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                              const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
-                             uint16_t* Y, const SkinnyPlan& p, cudaStream_t stream) {
+                             uint16_t* Y, const SkinnyPlan& p, bool weights_static, cudaStream_t stream) {
     auto kern = skinny_kernel<NT, MINB>;
     // Kernel attributes are set once per device (never inside a stream capture).
     static std::once_flag once[64];
@@ -272,26 +307,36 @@ static cudaError_t launch_nt(const uint16_t* X, int64_t M, int64_t N, int64_t K,
     cfg.blockDim = dim3(SK_THREADS, 1, 1);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = (unsigned)p.splits;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    unsigned na = 0;
+    if (p.splits > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 1;
+        attr[na].val.clusterDim.y = (unsigned)p.splits;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (weights_static) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = p.splits > 1 ? 1 : 0;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const __half*>(X), (int)M, (int)N, (int)K,
                               reinterpret_cast<const uint4*>(packed),
-                              reinterpret_cast<const __half*>(scales), zeros,
-                              reinterpret_cast<__half*>(Y), p.splits, p.gps);
+                              reinterpret_cast<const unsigned short*>(scales), zeros,
+                              reinterpret_cast<__half*>(Y), p.splits, p.gps, weights_static ? 1 : 0);
 }
 
 cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
-                          uint16_t* Y, const SkinnyPlan& plan, cudaStream_t stream) {
+                          uint16_t* Y, const SkinnyPlan& plan, bool weights_static,
+                          cudaStream_t stream) {
     switch (plan.mt) {
-        case 8: return launch_nt<1, 2>(X, M, N, K, packed, scales, zeros, Y, plan, stream);
-        case 16: return launch_nt<2, 2>(X, M, N, K, packed, scales, zeros, Y, plan, stream);
-        default: return launch_nt<4, 1>(X, M, N, K, packed, scales, zeros, Y, plan, stream);
+        case 8: return launch_nt<1, 2>(X, M, N, K, packed, scales, zeros, Y, plan, weights_static, stream);
+        case 16: return launch_nt<2, 2>(X, M, N, K, packed, scales, zeros, Y, plan, weights_static, stream);
+        default: return launch_nt<4, 1>(X, M, N, K, packed, scales, zeros, Y, plan, weights_static, stream);
     }
 }
 

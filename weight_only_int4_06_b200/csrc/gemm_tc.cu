@@ -1,0 +1,368 @@
+// Tensor-core W4A16 GEMM for prefill-sized M (tcgen05 + TMEM + TMA, sm_100a).
+//
+// "AutoAWQ vs The Stack v2" (WQLinear blurb): the batch GEMM variant dequantises INT4 weights on
+// the fly instead of materialising FP16 weights.  Prefill is a dense contraction, so it runs on
+// the 5th-generation tensor cores:
+//
+//   D[m, n] = sum_k X[m, k] * What[n, k],  What = (q - z) * s16 rounded once to fp16.
+//
+// One CTA computes a 128 (rows of X) x 256 (rows of W) tile, fp32 accumulator in TMEM
+// (256 columns), K in steps of 64 through a STAGES-deep shared-memory ring:
+//   warp 0      TMA producer: X tile (128 x 64 fp16, 128-byte swizzle) and the packed W tile
+//               (256 rows x 32 bytes) per stage; plain (non-multicast) tile loads.
+//   warp 1      one elected thread issues tcgen05.mma (M=128, N=256, K=16) x 4 per stage and
+//               commits each stage back to the producer.
+//   warp 2      allocates / frees TMEM.
+//   warps 4-11  dequantise: each thread turns one packed row (64 codes) into 64 fp16 weights in
+//               the UMMA K-major 128-byte-swizzle layout, then runs the epilogue (TMEM -> fp16 Y).
+// A second mode (for the AWQ search) loads an fp16 B operand with TMA instead of dequantising and
+// replaces the store by a per-tile sum of squares.
+//
+// Every mbarrier wait is bounded; on timeout the kernel records W4_ERR_DEVICE_TIMEOUT, stops
+// issuing work, drains what it issued and frees TMEM before it exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace w4 {
+
+constexpr int TC_BM = 128;
+constexpr int TC_BN = 256;
+constexpr int TC_BK = 64;
+constexpr int TC_STAGES = 4;
+constexpr int TC_THREADS = 384;
+constexpr int TC_DEQ_THREADS = 256;
+constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 2;  // 16 KB
+constexpr uint32_t TC_B_BYTES = TC_BN * TC_BK * 2;  // 32 KB
+constexpr uint32_t TC_P_BYTES = TC_BN * TC_BK / 2;  // 8 KB of packed codes
+constexpr uint32_t TC_TMEM_COLS = 256;
+constexpr int TC_GROUP_M = 8;  // raster: CTAs in flight share X and W tiles through L2
+
+template <bool DEQ>
+struct TcSmem {
+    static constexpr uint32_t kStage = TC_A_BYTES + TC_B_BYTES + (DEQ ? TC_P_BYTES : 0);
+    static constexpr uint32_t kBarOff = kStage * TC_STAGES;
+    static constexpr uint32_t kBytes = kBarOff + 256 + 1024;  // barriers + slack for 1 KB alignment
+};
+
+__device__ __forceinline__ void tc_tile_coords(int t, int m_tiles, int n_tiles, int& mt, int& nt) {
+    const int per_group = TC_GROUP_M * n_tiles;
+    const int group = t / per_group;
+    const int first_m = group * TC_GROUP_M;
+    const int gm = min(TC_GROUP_M, m_tiles - first_m);
+    const int r = t - group * per_group;
+    mt = first_m + r % gm;
+    nt = r / gm;
+}
+
+template <bool DEQ, bool SSE>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __half* __restrict__ scales, const uint8_t* __restrict__ zeros,
+                   __half* __restrict__ Y, double* __restrict__ sse_part, int M, int N, int K,
+                   int m_tiles, int n_tiles, int* status) {
+    using L = TcSmem<DEQ>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                           ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    auto a_addr = [&](int s) { return sbase + s * L::kStage; };
+    auto b_addr = [&](int s) { return sbase + s * L::kStage + TC_A_BYTES; };
+    auto p_addr = [&](int s) { return sbase + s * L::kStage + TC_A_BYTES + TC_B_BYTES; };
+    const uint32_t bar0 = sbase + L::kBarOff;
+    auto full_bar = [&](int s) { return bar0 + 8 * s; };
+    auto deq_bar = [&](int s) { return bar0 + 8 * (TC_STAGES + s); };
+    auto empty_bar = [&](int s) { return bar0 + 8 * (2 * TC_STAGES + s); };
+    const uint32_t accum_bar = bar0 + 8 * (3 * TC_STAGES);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * (3 * TC_STAGES + 1));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBarOff + 8 * (3 * TC_STAGES + 1) + 8);
+    double* red = reinterpret_cast<double*>(smem + L::kBarOff + 128);  // 8 doubles for the SSE epilogue
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int mt, nt;
+    tc_tile_coords(blockIdx.x, m_tiles, n_tiles, mt, nt);
+    const int m0 = mt * TC_BM, n0 = nt * TC_BN;
+    const int nk = K / TC_BK;
+    const int G = K >> 7;
+
+    if (tid == 0) {
+        for (int s = 0; s < TC_STAGES; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(deq_bar(s), TC_DEQ_THREADS / 32);
+            mbar_init(empty_bar(s), 1);
+        }
+        mbar_init(accum_bar, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(tmem_slot), TC_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_d = *tmem_slot;
+
+    auto fail = [&]() {
+        *abort_flag = 1;
+        record_status(status, W4_ERR_DEVICE_TIMEOUT);
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint32_t tx = TC_A_BYTES + (DEQ ? TC_P_BYTES : TC_B_BYTES);
+            int issued = 0;
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % TC_STAGES;
+                const uint32_t ph = (kb / TC_STAGES) & 1;
+                if (!mbar_wait_bounded(empty_bar(s), ph ^ 1, abort_flag)) { fail(); break; }
+                mbar_arrive_expect_tx(full_bar(s), tx);
+                tma_load_2d(a_addr(s), &tmA, kb * TC_BK, m0, full_bar(s));
+                if (DEQ) tma_load_2d(p_addr(s), &tmB, kb * (TC_BK / 8), n0, full_bar(s));
+                else tma_load_2d(b_addr(s), &tmB, kb * TC_BK, n0, full_bar(s));
+                ++issued;
+            }
+            // Never leave with tile loads in flight: wait (bounded) for the last stages issued.
+            for (int kb = issued - TC_STAGES; kb < issued; ++kb) {
+                if (kb < 0) continue;
+                mbar_wait_bounded(full_bar(kb % TC_STAGES), (kb / TC_STAGES) & 1, nullptr, 200000000ull);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_f16_f32(TC_BM, TC_BN);
+            bool ok = true;
+            for (int kb = 0; kb < nk && ok; ++kb) {
+                const int s = kb % TC_STAGES;
+                const uint32_t ph = (kb / TC_STAGES) & 1;
+                if (!mbar_wait_bounded(full_bar(s), ph, abort_flag)) { fail(); ok = false; break; }
+                if (DEQ && !mbar_wait_bounded(deq_bar(s), ph, abort_flag)) { fail(); ok = false; break; }
+                tc_fence_after();
+                const uint64_t ad = sw128_kmajor_desc(a_addr(s));
+                const uint64_t bd = sw128_kmajor_desc(b_addr(s));
+#pragma unroll
+                for (int j = 0; j < TC_BK / 16; ++j) {
+                    // +32 bytes along K per MMA inside the 128-byte swizzled row
+                    mma_f16_ss(tmem_d, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+                }
+                tc_commit(empty_bar(s));
+            }
+            tc_commit(accum_bar);  // fires once every MMA issued above has completed
+        }
+    } else if (warp >= 4) {
+        const int d = tid - 128;  // 0..255
+        if (DEQ) {
+            // -------------------------------------------------------- dequantisation
+            const int r = d;  // tile row (row of W)
+            const int n = n0 + r;
+            const bool nvalid = n < N;
+            uint32_t s2 = 0, zl = 0, zh = 0;
+            const uint32_t b_row = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % TC_STAGES;
+                const uint32_t ph = (kb / TC_STAGES) & 1;
+                if ((kb & 1) == 0) {  // a new group of 128 every second stage
+                    const int g = kb >> 1;
+                    __half sc = __float2half_rn(0.0f);
+                    uint32_t z = 0;
+                    if (nvalid) {
+                        sc = scales[(int64_t)n * G + g];
+                        z = zeros[(int64_t)n * G + g];
+                    }
+                    const uint32_t sb = (uint32_t)__half_as_ushort(sc);
+                    s2 = sb | (sb << 16);
+                    zl = (0x6400u + z) * 0x10001u;
+                    zh = (0xD400u | (z << 4)) * 0x10001u;
+                }
+                if (!mbar_wait_bounded(full_bar(s), ph, abort_flag)) { fail(); break; }
+                const unsigned char* prow = smem + (p_addr(s) - sbase) + r * 32;
+                const uint4 w0 = *reinterpret_cast<const uint4*>(prow);
+                const uint4 w1 = *reinterpret_cast<const uint4*>(prow + 16);
+                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                unsigned char* brow = smem + (b_addr(s) - sbase) + b_row;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t w = words[c];
+                    uint32_t lo0 = hsub2_u32(lop3_and_or(w, 0x000F000Fu, 0x64006400u), zl);           // n0,n4
+                    uint32_t hi0 = hfma2_u32(lop3_and_or(w, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zh); // n1,n5
+                    const uint32_t w8 = w >> 8;
+                    uint32_t lo1 = hsub2_u32(lop3_and_or(w8, 0x000F000Fu, 0x64006400u), zl);          // n2,n6
+                    uint32_t hi1 = hfma2_u32(lop3_and_or(w8, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zh);// n3,n7
+                    lo0 = hmul2_u32(lo0, s2);
+                    hi0 = hmul2_u32(hi0, s2);
+                    lo1 = hmul2_u32(lo1, s2);
+                    hi1 = hmul2_u32(hi1, s2);
+                    uint4 o;
+                    o.x = __byte_perm(lo0, hi0, 0x5410);  // k0, k1
+                    o.y = __byte_perm(lo1, hi1, 0x5410);  // k2, k3
+                    o.z = __byte_perm(lo0, hi0, 0x7632);  // k4, k5
+                    o.w = __byte_perm(lo1, hi1, 0x7632);  // k6, k7
+                    *reinterpret_cast<uint4*>(brow + ((c ^ (r & 7)) << 4)) = o;
+                }
+                fence_proxy_async_shared();  // generic-proxy writes -> visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(deq_bar(s));
+            }
+        }
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;            // TMEM lane quarter this warp may access
+        const int half = (warp - 4) >> 2;  // which 128 of the 256 accumulator columns
+        // not cut short by the abort flag: TMEM is freed only after every issued MMA completed
+        const bool ok = mbar_wait_bounded(accum_bar, 0, nullptr, 4000000000ull);
+        if (!ok) fail();
+        tc_fence_after();
+        const int m = m0 + q * 32 + lane;
+        double sq = 0.0;
+        if (ok && !*abort_flag) {
+#pragma unroll 1
+            for (int cc = 0; cc < 128; cc += 32) {
+                const int col = half * 128 + cc;
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)col, v);
+                tmem_wait_ld();
+                if (SSE) {
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float f = __uint_as_float(v[i]);
+                        acc = fmaf(f, f, acc);
+                    }
+                    sq += (double)acc;
+                } else if (m < M) {
+                    const int nb = n0 + col;
+                    __half* yrow = Y + (int64_t)m * N + nb;
+                    if (nb + 32 <= N) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            uint4 o;
+                            o.x = pack_half2(__uint_as_float(v[i + 0]), __uint_as_float(v[i + 1]));
+                            o.y = pack_half2(__uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+                            o.z = pack_half2(__uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
+                            o.w = pack_half2(__uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
+                            *reinterpret_cast<uint4*>(yrow + i) = o;
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (nb + i < N) yrow[i] = __float2half_rn(__uint_as_float(v[i]));
+                    }
+                }
+            }
+        }
+        if (SSE) {
+            // rows beyond M read zeros from TMA fill, so they add nothing
+#pragma unroll
+            for (int o = 16; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+            if (lane == 0) red[warp - 4] = sq;
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (SSE && tid == 0) {
+        double t = 0.0;
+        for (int i = 0; i < 8; ++i) t += red[i];
+        sse_part[(int64_t)mt * n_tiles + nt] = t;
+    }
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem_d, TC_TMEM_COLS);
+    }
+}
+
+// ------------------------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, []() {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
+                        uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle swz) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * elem_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <bool DEQ, bool SSE>
+static cudaError_t set_tc_attrs() {
+    static std::once_flag once[64];
+    static cudaError_t err[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [&]() {
+        err[dev] = cudaFuncSetAttribute(tc_gemm_kernel<DEQ, SSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)TcSmem<DEQ>::kBytes);
+    });
+    return err[dev];
+}
+
+cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                         const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,
+                         cudaStream_t stream) {
+    CUtensorMap ta, tb;
+    if (!make_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, TC_BK, TC_BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_map_2d(&tb, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)(K / 8), (uint64_t)N, TC_BK / 8,
+                     TC_BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    cudaError_t e = set_tc_attrs<true, false>();
+    if (e != cudaSuccess) return e;
+    const int m_tiles = (int)((M + TC_BM - 1) / TC_BM);
+    const int n_tiles = (int)((N + TC_BN - 1) / TC_BN);
+    tc_gemm_kernel<true, false><<<m_tiles * n_tiles, TC_THREADS, TcSmem<true>::kBytes, stream>>>(
+        ta, tb, reinterpret_cast<const __half*>(scales), zeros, reinterpret_cast<__half*>(Y), nullptr, (int)M,
+        (int)N, (int)K, m_tiles, n_tiles, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64_t N, int64_t K,
+                          double* sse_part, int* status, cudaStream_t stream) {
+    CUtensorMap ta, tb;
+    if (!make_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)T, TC_BK, TC_BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!make_map_2d(&tb, E, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)N, TC_BK, TC_BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    cudaError_t e = set_tc_attrs<false, true>();
+    if (e != cudaSuccess) return e;
+    const int m_tiles = (int)((T + TC_BM - 1) / TC_BM);
+    const int n_tiles = (int)((N + TC_BN - 1) / TC_BN);
+    tc_gemm_kernel<false, true><<<m_tiles * n_tiles, TC_THREADS, TcSmem<false>::kBytes, stream>>>(
+        ta, tb, nullptr, nullptr, nullptr, sse_part, (int)T, (int)N, (int)K, m_tiles, n_tiles, status);
+    return cudaGetLastError();
+}
+
+int tc_sse_partials(int64_t T, int64_t N) {
+    return (int)(((T + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN));
+}
+
+}  // namespace w4

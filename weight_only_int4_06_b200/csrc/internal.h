@@ -25,8 +25,30 @@ struct SkinnyPlan {
     size_t smem;   // dynamic shared memory per CTA
 };
 bool plan_skinny(int64_t M, int64_t N, int64_t K, SkinnyPlan* plan);
+// weights_static: packed/scales/zeros are not written by work still in flight on the stream, so
+// the kernel is launched with programmatic dependent launch and starts streaming them before the
+// preceding kernel has finished (activations are read only after it has).
 cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
-                          uint16_t* Y, const SkinnyPlan& plan, cudaStream_t stream);
+                          uint16_t* Y, const SkinnyPlan& plan, bool weights_static,
+                          cudaStream_t stream);
+
+// tcgen05 GEMM (gemm_tc.cu).
+cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                         const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,
+                         cudaStream_t stream);
+cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64_t N, int64_t K,
+                          double* sse_part, int* status, cudaStream_t stream);
+int tc_sse_partials(int64_t T, int64_t N);
+
+// AWQ search (awq.cu).  Workspace layout (byte offsets, 256-byte aligned).
+struct AwqLayout {
+    size_t colsum, s_all, E, part, bytes;
+    int n_part;
+};
+AwqLayout awq_layout(int64_t T, int64_t N, int64_t K, int n_alpha);
+cudaError_t launch_awq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int n_alpha,
+                       double* mse, int32_t* best_idx, float* best_s, void* ws, int* status,
+                       cudaStream_t stream);
 
 }  // namespace w4

@@ -20,6 +20,7 @@ STATUS_NAMES = {
     5: "W4_ERR_WORKSPACE", 6: "W4_ERR_CUDA", 7: "W4_ERR_DEVICE_TIMEOUT", 8: "W4_ERR_RANGE",
 }
 VARIANT_AUTO, VARIANT_SKINNY, VARIANT_TC = 0, 1, 2
+FLAG_WEIGHTS_STATIC = 0x100
 
 # Entry points declared in include/w4a16.h: (name, restype, argtypes)
 _P, _I64, _I32, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
