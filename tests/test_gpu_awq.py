@@ -24,8 +24,8 @@ def check_against_oracle(X, W, n_alpha=20):
     mse_o, best_o, s_o, s_all = oracle.awq_scale_search(X, W, n_alpha)
     rel = np.abs(mse_g - mse_o) / mse_o
     assert np.all(rel <= 1e-3), f"max rel err {rel.max():.3g} at alpha {np.argmax(rel)}"
-    order = np.argsort(mse_o)
-    near_tie = (mse_o[order[1]] - mse_o[order[0]]) <= 2e-3 * mse_o[order[0]]
+    order = np.argsort(mse_o, kind="stable")
+    near_tie = n_alpha > 1 and (mse_o[order[1]] - mse_o[order[0]]) <= 2e-3 * mse_o[order[0]]
     if near_tie:
         assert best_g in (int(order[0]), int(order[1]))
     else:

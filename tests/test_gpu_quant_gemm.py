@@ -107,6 +107,32 @@ def test_quant_range_overflow_is_reported():
         oracle.quantize_pack(W, np.full(128, 16.0, np.float32))
 
 
+def test_quant_exact_midpoints():
+    """Elements exactly at (n + 1/2) s16 (ties, rounded half to even) and one fp16 ulp either side."""
+    rows = []
+    for s in (0.0625, 0.046875, 0.001953125, 3.0, 0.75):
+        for sign in (1.0, -1.0):
+            base = np.array([15 * s] + [(n + 0.5) * s for n in range(15)] + [0.0], np.float64) * sign
+            h = base.astype(np.float16)
+            assert np.all(h.astype(np.float64) == base)   # exactly representable
+            up = np.nextafter(h, np.float16(np.inf))
+            dn = np.nextafter(h, np.float16(-np.inf))
+            vals = np.concatenate([h, up[1:16], dn[1:16]])
+            row = np.zeros(128, np.float16)
+            row[:vals.size] = vals
+            rows.append(row)
+    W = np.stack(rows)
+    W = np.concatenate([W, np.zeros(((-len(W)) % 8, 128), np.float16)])
+    assert_quant_equal(W)
+
+
+def test_quant_wide_act_scale_sweep():
+    """16.7M quotients with fp32 activation scales spanning 2^-10 .. 2^10."""
+    _, W = synth.layer_case(13, 1, 4096, 4096)
+    act = np.exp2(np.random.default_rng(13).uniform(-10, 10, 4096)).astype(np.float32)
+    assert_quant_equal(W, act)
+
+
 @pytest.mark.parametrize("K,N", list(synth.DECODE_7B_SHAPES) + [(28672, 8192)])
 def test_quant_full_size(K, N):
     _, W = synth.layer_case(2, 1, K, N)

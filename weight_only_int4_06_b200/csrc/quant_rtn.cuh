@@ -19,10 +19,24 @@ namespace w4 {
 
 struct GroupQuant {
     float sf;      // s16 as fp32
+    float rcp;     // 1 / sf rounded to nearest (correctly rounded reciprocal)
     int z;         // zero point 0..15
     __half s16;    // fp16 scale
     bool overflow; // s16 is +inf
 };
+
+// Correctly rounded a / b from the correctly rounded reciprocal y = RN(1/b), by Markstein's
+// correction step (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Develop. 34(1), 1990): with q0 = RN(a*y) within one ulp of
+// a/b, the remainder r = a - b*q0 is exact in one fma and RN(q0 + r*y) is the correctly rounded
+// quotient.  Valid here because b is a positive normal fp32 value (an fp16 scale), a is finite
+// and |a / b| < 2^24, so nothing over- or underflows.  An exact binary quotient is never a
+// rounding midpoint, so the result is unique and equals IEEE division.
+__device__ __forceinline__ float div_rn_from_rcp(float a, float b, float y) {
+    const float q0 = __fmul_rn(a, y);
+    const float r = __fmaf_rn(-q0, b, a);
+    return __fmaf_rn(r, y, q0);
+}
 
 __device__ __forceinline__ GroupQuant group_params(float lo, float hi) {
     GroupQuant p;
@@ -31,14 +45,16 @@ __device__ __forceinline__ GroupQuant group_params(float lo, float hi) {
     if (d == 0.0f) s = __float2half_rn(1.0f);
     p.s16 = s;
     p.sf = __half2float(s);
+    p.rcp = __frcp_rn(p.sf);
     p.overflow = isinf(p.sf);
     const int z = __float2int_rn(__fdiv_rn(-lo, p.sf));
     p.z = min(max(z, 0), 15);
     return p;
 }
 
+// q = clamp(rint(v / s16) + z, 0, 15) with v / s16 the correctly rounded fp32 quotient.
 __device__ __forceinline__ uint32_t quant_code(float v, const GroupQuant& p) {
-    const int q = __float2int_rn(__fdiv_rn(v, p.sf)) + p.z;
+    const int q = __float2int_rn(div_rn_from_rcp(v, p.sf, p.rcp)) + p.z;
     return (uint32_t)min(max(q, 0), 15);
 }
 

@@ -13,6 +13,51 @@
 namespace w4 {
 
 template <bool HAS_SCALE>
+__device__ __forceinline__ void quantize_group_slice(const uint4 raw, int64_t f, bool valid, int l16, int G,
+                                                     const float* __restrict__ act,
+                                                     uint32_t* __restrict__ packed, __half* __restrict__ scales,
+                                                     uint8_t* __restrict__ zeros, int* status) {
+    float v[8];
+    if (valid) {
+        if (HAS_SCALE) {
+            const int64_t k0 = (f % G) * 128 + 8 * l16;
+            const float4 a0 = __ldg(reinterpret_cast<const float4*>(act + k0));
+            const float4 a1 = __ldg(reinterpret_cast<const float4*>(act + k0) + 1);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            load8_scaled(raw, a, v);
+        } else {
+            load8_scaled(raw, nullptr, v);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    }
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+        mn = fminf(mn, v[i]);
+        mx = fmaxf(mx, v[i]);
+    }
+#pragma unroll
+    for (int o = 8; o; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const GroupQuant p = group_params(fminf(mn, 0.0f), fmaxf(mx, 0.0f));
+    if (valid) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) word |= quant_code(v[i], p) << (4 * i);
+        packed[f * 16 + l16] = word;
+        if (l16 == 0) {
+            scales[f] = p.s16;
+            zeros[f] = (uint8_t)p.z;
+            if (p.overflow) record_status(status, W4_ERR_RANGE);
+        }
+    }
+}
+
+template <bool HAS_SCALE>
 __global__ void __launch_bounds__(256) quantize_pack_kernel(
     const uint4* __restrict__ W, const float* __restrict__ act, int64_t n_groups, int G,
     uint32_t* __restrict__ packed, __half* __restrict__ scales, uint8_t* __restrict__ zeros,
@@ -24,48 +69,17 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t n_pairs = (n_groups + 1) >> 1;
 
-    for (int64_t pair = warp; pair < n_pairs; pair += nwarps) {
-        const int64_t f = 2 * pair + sub;
-        const bool valid = f < n_groups;
-        float v[8];
-        if (valid) {
-            const uint4 raw = ldg_stream(W + f * 16 + l16);
-            if (HAS_SCALE) {
-                const int64_t k0 = (f % G) * 128 + 8 * l16;
-                const float4 a0 = __ldg(reinterpret_cast<const float4*>(act + k0));
-                const float4 a1 = __ldg(reinterpret_cast<const float4*>(act + k0) + 1);
-                const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                load8_scaled(raw, a, v);
-            } else {
-                load8_scaled(raw, nullptr, v);
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[i] = 0.0f;
-        }
-        float mn = v[0], mx = v[0];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) {
-            mn = fminf(mn, v[i]);
-            mx = fmaxf(mx, v[i]);
-        }
-#pragma unroll
-        for (int o = 8; o; o >>= 1) {
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
-        const GroupQuant p = group_params(fminf(mn, 0.0f), fmaxf(mx, 0.0f));
-        if (valid) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) word |= quant_code(v[i], p) << (4 * i);
-            packed[f * 16 + l16] = word;
-            if (l16 == 0) {
-                scales[f] = p.s16;
-                zeros[f] = (uint8_t)p.z;
-                if (p.overflow) record_status(status, W4_ERR_RANGE);
-            }
-        }
+    // Two pairs per iteration, both loads in flight before either is processed.
+    for (int64_t pair = warp; pair < n_pairs; pair += 2 * nwarps) {
+        const int64_t f0 = 2 * pair + sub;
+        const int64_t f1 = 2 * (pair + nwarps) + sub;
+        const bool v0 = f0 < n_groups, v1 = f1 < n_groups;
+        uint4 r0 = make_uint4(0u, 0u, 0u, 0u), r1 = make_uint4(0u, 0u, 0u, 0u);
+        if (v0) r0 = ldg_stream(W + f0 * 16 + l16);
+        if (v1) r1 = ldg_stream(W + f1 * 16 + l16);
+        quantize_group_slice<HAS_SCALE>(r0, f0, v0, l16, G, act, packed, scales, zeros, status);
+        if (pair + nwarps < n_pairs)  // warp-uniform
+            quantize_group_slice<HAS_SCALE>(r1, f1, v1, l16, G, act, packed, scales, zeros, status);
     }
 }
 
