@@ -74,6 +74,7 @@ typedef enum {
     W4_VARIANT_AUTO = 0,
     W4_VARIANT_SKINNY = 1, /* warp-level tensor-core GEMV / skinny GEMM, split-K over a cluster */
     W4_VARIANT_TC = 2,     /* tcgen05/TMEM tensor-core GEMM with dequantisation in the smem path */
+    W4_VARIANT_GEMV = 3,   /* persistent TMA-fed GEMV, one activation row at a time (decode) */
     /* Flag, OR-ed into the variant: packed/scales/zeros are not written by any work still in
      * flight on the stream (static weights).  The call may then use programmatic dependent launch
      * and start streaming the weights before the preceding kernel on the stream has finished;

@@ -233,6 +233,20 @@ def test_gemm_tc_ragged(M, K, N):
     assert_close(gpu_gemm(X, p, s, z, B.VARIANT_TC), oracle.gemm(X, p, s, z), f"tc {M}x{K}x{N}")
 
 
+@pytest.mark.parametrize("M,K,N", [(1, 128, 8), (1, 384, 24), (1, 1152, 136), (1, 4096, 4104),
+                                   (1, 11008, 40), (1, 28672, 264), (3, 2048, 520), (1, 8192, 28672)])
+def test_gemm_gemv_ragged(M, K, N):
+    X, p, s, z = oracle_case(28, M, K, N)
+    assert_close(gpu_gemm(X, p, s, z, B.VARIANT_GEMV), oracle.gemm(X, p, s, z), f"gemv {M}x{K}x{N}")
+
+
+def test_gemm_gemv_outlier_heavy_activations():
+    """Large activations stress the offset removal (raw operands carry a 1024 offset)."""
+    X, p, s, z = oracle_case(29, 1, 4096, 1024)
+    X = (X.astype(np.float32) * 40).astype(np.float16)
+    assert_close(gpu_gemm(X, p, s, z, B.VARIANT_GEMV), oracle.gemm(X, p, s, z), "gemv x40")
+
+
 @pytest.mark.parametrize("M,K,N", [(1, 4096, 4096), (8, 8192, 1024), (32, 28672, 256)])
 def test_gemm_weights_static_flag_same_bits(M, K, N):
     """The static-weights launch (programmatic dependent launch) computes the same bits."""

@@ -93,7 +93,7 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     if (group != 128) return W4_ERR_UNSUPPORTED;
     const bool weights_static = (variant & W4_FLAG_WEIGHTS_STATIC) != 0;
     const int family = variant & ~W4_FLAG_WEIGHTS_STATIC;
-    if (family < W4_VARIANT_AUTO || family > W4_VARIANT_TC) return W4_ERR_UNSUPPORTED;
+    if (family < W4_VARIANT_AUTO || family > W4_VARIANT_GEMV) return W4_ERR_UNSUPPORTED;
     if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0)
         return W4_ERR_SHAPE;
     size_t need = 0;
@@ -117,6 +117,17 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     if (use_tc) {
         return launch_tc_w4(X, M, N, K, packed, scales, zeros, Y, status, s) == cudaSuccess ? W4_OK
                                                                                             : W4_ERR_CUDA;
+    }
+    const bool gemv_fits = gemv_stream_smem(K) <= 200 * 1024;
+    if (family == W4_VARIANT_GEMV && !gemv_fits) return W4_ERR_SHAPE;
+    if (family == W4_VARIANT_GEMV || (family == W4_VARIANT_AUTO && M == 1 && gemv_fits)) {
+        // one activation row at a time (single-token decode has M == 1)
+        for (int64_t m = 0; m < M; ++m) {
+            cudaError_t e = launch_gemv_stream(X + m * K, N, K, packed, scales, zeros, Y + m * N,
+                                               weights_static, status, s);
+            if (e != cudaSuccess) return W4_ERR_CUDA;
+        }
+        return W4_OK;
     }
     // Skinny path, in chunks of at most 32 activation rows.
     for (int64_t m0 = 0; m0 < M; m0 += 32) {

@@ -6,11 +6,12 @@
 //
 //   D[m, n] = sum_k X[m, k] * What[n, k],  What = (q - z) * s16 rounded once to fp16.
 //
-// One CTA computes a 128 (rows of X) x 256 (rows of W) tile, fp32 accumulator in TMEM
-// (256 columns), K in steps of 64 through a STAGES-deep shared-memory ring:
-//   warp 0      TMA producer: X tile (128 x 64 fp16, 128-byte swizzle) and the packed W tile
+// One CTA computes an (MT x 128) (rows of X) x 256 (rows of W) tile: MT fp32 accumulators of
+// 128 x 256 in TMEM (256 columns each) share one dequantised W tile, so with MT = 2 every
+// dequantised weight feeds two MMAs.  K advances in steps of 64 through a shared-memory ring:
+//   warp 0      TMA producer: X tile (MT*128 x 64 fp16, 128-byte swizzle) and the packed W tile
 //               (256 rows x 32 bytes) per stage; plain (non-multicast) tile loads.
-//   warp 1      one elected thread issues tcgen05.mma (M=128, N=256, K=16) x 4 per stage and
+//   warp 1      one elected thread issues MT x 4 tcgen05.mma (M=128, N=256, K=16) per stage and
 //               commits each stage back to the producer.
 //   warp 2      allocates / frees TMEM.
 //   warps 4-11  dequantise: each thread turns one packed row (64 codes) into 64 fp16 weights in
@@ -31,23 +32,24 @@
 
 namespace w4 {
 
-constexpr int TC_BM = 128;
 constexpr int TC_BN = 256;
 constexpr int TC_BK = 64;
-constexpr int TC_STAGES = 4;
 constexpr int TC_THREADS = 384;
 constexpr int TC_DEQ_THREADS = 256;
-constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 2;  // 16 KB
+constexpr uint32_t TC_A1_BYTES = 128 * TC_BK * 2;   // 16 KB per 128-row X tile
 constexpr uint32_t TC_B_BYTES = TC_BN * TC_BK * 2;  // 32 KB
 constexpr uint32_t TC_P_BYTES = TC_BN * TC_BK / 2;  // 8 KB of packed codes
-constexpr uint32_t TC_TMEM_COLS = 256;
 constexpr int TC_GROUP_M = 8;  // raster: CTAs in flight share X and W tiles through L2
 
-template <bool DEQ>
-struct TcSmem {
-    static constexpr uint32_t kStage = TC_A_BYTES + TC_B_BYTES + (DEQ ? TC_P_BYTES : 0);
-    static constexpr uint32_t kBarOff = kStage * TC_STAGES;
+template <bool DEQ, int MT>
+struct TcCfg {
+    static constexpr int kBM = 128 * MT;
+    static constexpr uint32_t kA = TC_A1_BYTES * MT;
+    static constexpr uint32_t kStage = kA + TC_B_BYTES + (DEQ ? TC_P_BYTES : 0);
+    static constexpr int kStages = (MT == 1) ? 4 : 3;
+    static constexpr uint32_t kBarOff = kStage * kStages;
     static constexpr uint32_t kBytes = kBarOff + 256 + 1024;  // barriers + slack for 1 KB alignment
+    static constexpr uint32_t kTmemCols = 256 * MT;
 };
 
 __device__ __forceinline__ void tc_tile_coords(int t, int m_tiles, int n_tiles, int& mt, int& nt) {
@@ -60,38 +62,39 @@ __device__ __forceinline__ void tc_tile_coords(int t, int m_tiles, int n_tiles, 
     nt = r / gm;
 }
 
-template <bool DEQ, bool SSE>
+template <bool DEQ, bool SSE, int MT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __half* __restrict__ scales, const uint8_t* __restrict__ zeros,
                    __half* __restrict__ Y, double* __restrict__ sse_part, int M, int N, int K,
                    int m_tiles, int n_tiles, int* status) {
-    using L = TcSmem<DEQ>;
+    using C = TcCfg<DEQ, MT>;
+    constexpr int S = C::kStages;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                            ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    auto a_addr = [&](int s) { return sbase + s * L::kStage; };
-    auto b_addr = [&](int s) { return sbase + s * L::kStage + TC_A_BYTES; };
-    auto p_addr = [&](int s) { return sbase + s * L::kStage + TC_A_BYTES + TC_B_BYTES; };
-    const uint32_t bar0 = sbase + L::kBarOff;
+    auto a_addr = [&](int s) { return sbase + s * C::kStage; };
+    auto b_addr = [&](int s) { return sbase + s * C::kStage + C::kA; };
+    auto p_addr = [&](int s) { return sbase + s * C::kStage + C::kA + TC_B_BYTES; };
+    const uint32_t bar0 = sbase + C::kBarOff;
     auto full_bar = [&](int s) { return bar0 + 8 * s; };
-    auto deq_bar = [&](int s) { return bar0 + 8 * (TC_STAGES + s); };
-    auto empty_bar = [&](int s) { return bar0 + 8 * (2 * TC_STAGES + s); };
-    const uint32_t accum_bar = bar0 + 8 * (3 * TC_STAGES);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBarOff + 8 * (3 * TC_STAGES + 1));
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBarOff + 8 * (3 * TC_STAGES + 1) + 8);
-    double* red = reinterpret_cast<double*>(smem + L::kBarOff + 128);  // 8 doubles for the SSE epilogue
+    auto deq_bar = [&](int s) { return bar0 + 8 * (S + s); };
+    auto empty_bar = [&](int s) { return bar0 + 8 * (2 * S + s); };
+    const uint32_t accum_bar = bar0 + 8 * (3 * S);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kBarOff + 8 * (3 * S + 1));
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kBarOff + 8 * (3 * S + 1) + 8);
+    double* red = reinterpret_cast<double*>(smem + C::kBarOff + 128);  // 8 doubles for the SSE epilogue
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int mt, nt;
     tc_tile_coords(blockIdx.x, m_tiles, n_tiles, mt, nt);
-    const int m0 = mt * TC_BM, n0 = nt * TC_BN;
+    const int m0 = mt * C::kBM, n0 = nt * TC_BN;
     const int nk = K / TC_BK;
     const int G = K >> 7;
 
     if (tid == 0) {
-        for (int s = 0; s < TC_STAGES; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(deq_bar(s), TC_DEQ_THREADS / 32);
             mbar_init(empty_bar(s), 1);
@@ -103,7 +106,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         prefetch_tmap(&tmB);
     }
     if (warp == 2) {
-        tmem_alloc(smem_u32(tmem_slot), TC_TMEM_COLS);
+        tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -119,11 +122,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint32_t tx = TC_A_BYTES + (DEQ ? TC_P_BYTES : TC_B_BYTES);
+            const uint32_t tx = C::kA + (DEQ ? TC_P_BYTES : TC_B_BYTES);
             int issued = 0;
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % TC_STAGES;
-                const uint32_t ph = (kb / TC_STAGES) & 1;
+                const int s = kb % S;
+                const uint32_t ph = (kb / S) & 1;
                 if (!mbar_wait_bounded(empty_bar(s), ph ^ 1, abort_flag)) { fail(); break; }
                 mbar_arrive_expect_tx(full_bar(s), tx);
                 tma_load_2d(a_addr(s), &tmA, kb * TC_BK, m0, full_bar(s));
@@ -132,28 +135,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 ++issued;
             }
             // Never leave with tile loads in flight: wait (bounded) for the last stages issued.
-            for (int kb = issued - TC_STAGES; kb < issued; ++kb) {
+            for (int kb = issued - S; kb < issued; ++kb) {
                 if (kb < 0) continue;
-                mbar_wait_bounded(full_bar(kb % TC_STAGES), (kb / TC_STAGES) & 1, nullptr, 200000000ull);
+                mbar_wait_bounded(full_bar(kb % S), (kb / S) & 1, nullptr, 200000000ull);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16_f32(TC_BM, TC_BN);
+            constexpr uint32_t idesc = idesc_f16_f32(128, TC_BN);
             bool ok = true;
             for (int kb = 0; kb < nk && ok; ++kb) {
-                const int s = kb % TC_STAGES;
-                const uint32_t ph = (kb / TC_STAGES) & 1;
+                const int s = kb % S;
+                const uint32_t ph = (kb / S) & 1;
                 if (!mbar_wait_bounded(full_bar(s), ph, abort_flag)) { fail(); ok = false; break; }
                 if (DEQ && !mbar_wait_bounded(deq_bar(s), ph, abort_flag)) { fail(); ok = false; break; }
                 tc_fence_after();
-                const uint64_t ad = sw128_kmajor_desc(a_addr(s));
                 const uint64_t bd = sw128_kmajor_desc(b_addr(s));
 #pragma unroll
                 for (int j = 0; j < TC_BK / 16; ++j) {
-                    // +32 bytes along K per MMA inside the 128-byte swizzled row
-                    mma_f16_ss(tmem_d, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+#pragma unroll
+                    for (int t = 0; t < MT; ++t) {
+                        const uint64_t ad = sw128_kmajor_desc(a_addr(s) + t * TC_A1_BYTES);
+                        // +32 bytes along K per MMA inside the 128-byte swizzled row
+                        mma_f16_ss(tmem_d + t * 256, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+                    }
                 }
                 tc_commit(empty_bar(s));
             }
@@ -169,8 +175,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             uint32_t s2 = 0, zl = 0, zh = 0;
             const uint32_t b_row = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % TC_STAGES;
-                const uint32_t ph = (kb / TC_STAGES) & 1;
+                const int s = kb % S;
+                const uint32_t ph = (kb / S) & 1;
                 if ((kb & 1) == 0) {  // a new group of 128 every second stage
                     const int g = kb >> 1;
                     __half sc = __float2half_rn(0.0f);
@@ -193,11 +199,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const uint32_t w = words[c];
-                    uint32_t lo0 = hsub2_u32(lop3_and_or(w, 0x000F000Fu, 0x64006400u), zl);           // n0,n4
-                    uint32_t hi0 = hfma2_u32(lop3_and_or(w, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zh); // n1,n5
+                    uint32_t lo0 = hsub2_u32(lop3_and_or(w, 0x000F000Fu, 0x64006400u), zl);            // n0,n4
+                    uint32_t hi0 = hfma2_u32(lop3_and_or(w, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zh);  // n1,n5
                     const uint32_t w8 = w >> 8;
-                    uint32_t lo1 = hsub2_u32(lop3_and_or(w8, 0x000F000Fu, 0x64006400u), zl);          // n2,n6
-                    uint32_t hi1 = hfma2_u32(lop3_and_or(w8, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zh);// n3,n7
+                    uint32_t lo1 = hsub2_u32(lop3_and_or(w8, 0x000F000Fu, 0x64006400u), zl);           // n2,n6
+                    uint32_t hi1 = hfma2_u32(lop3_and_or(w8, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zh); // n3,n7
                     lo0 = hmul2_u32(lo0, s2);
                     hi0 = hmul2_u32(hi0, s2);
                     lo1 = hmul2_u32(lo1, s2);
@@ -215,29 +221,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
         }
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;            // TMEM lane quarter this warp may access
-        const int half = (warp - 4) >> 2;  // which 128 of the 256 accumulator columns
+        // warp (4 + 4*slot + q) reads TMEM lanes [32q, 32q + 32) (the quarter it may access):
+        // MT == 1: columns [128*slot, 128*slot + 128) of the single accumulator;
+        // MT == 2: all 256 columns of accumulator `slot`.
+        const int q = warp & 3;
+        const int slot = (warp - 4) >> 2;
+        const int acc = MT == 1 ? 0 : slot;
+        const int c_begin = MT == 1 ? slot * 128 : 0;
+        const int c_count = MT == 1 ? 128 : 256;
         // not cut short by the abort flag: TMEM is freed only after every issued MMA completed
         const bool ok = mbar_wait_bounded(accum_bar, 0, nullptr, 4000000000ull);
         if (!ok) fail();
         tc_fence_after();
-        const int m = m0 + q * 32 + lane;
+        const int m = m0 + acc * 128 + q * 32 + lane;
         double sq = 0.0;
         if (ok && !*abort_flag) {
 #pragma unroll 1
-            for (int cc = 0; cc < 128; cc += 32) {
-                const int col = half * 128 + cc;
+            for (int cc = 0; cc < c_count; cc += 32) {
+                const int col = c_begin + cc;
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)col, v);
+                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256 + col), v);
                 tmem_wait_ld();
                 if (SSE) {
-                    float acc = 0.0f;
+                    float a = 0.0f;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const float f = __uint_as_float(v[i]);
-                        acc = fmaf(f, f, acc);
+                        a = fmaf(f, f, a);
                     }
-                    sq += (double)acc;
+                    sq += (double)a;
                 } else if (m < M) {
                     const int nb = n0 + col;
                     __half* yrow = Y + (int64_t)m * N + nb;
@@ -276,7 +288,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     if (warp == 2) {
         tc_fence_after();
-        tmem_dealloc(tmem_d, TC_TMEM_COLS);
+        tmem_dealloc(tmem_d, C::kTmemCols);
     }
 }
 
@@ -294,7 +306,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
+bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
                         uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
                         CUtensorMapSwizzle swz) {
     auto enc = tensor_map_encoder();
@@ -308,7 +320,7 @@ static bool make_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
     return r == CUDA_SUCCESS;
 }
 
-template <bool DEQ, bool SSE>
+template <bool DEQ, bool SSE, int MT>
 static cudaError_t set_tc_attrs() {
     static std::once_flag once[64];
     static cudaError_t err[64];
@@ -317,52 +329,58 @@ static cudaError_t set_tc_attrs() {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&]() {
-        err[dev] = cudaFuncSetAttribute(tc_gemm_kernel<DEQ, SSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)TcSmem<DEQ>::kBytes);
+        err[dev] = cudaFuncSetAttribute(tc_gemm_kernel<DEQ, SSE, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)TcCfg<DEQ, MT>::kBytes);
     });
     return err[dev];
 }
 
-cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                         const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,
-                         cudaStream_t stream) {
+template <bool DEQ, bool SSE, int MT>
+static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int64_t N, int64_t K,
+                             const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, double* sse_part,
+                             int* status, cudaStream_t stream) {
+    using C = TcCfg<DEQ, MT>;
     CUtensorMap ta, tb;
-    if (!make_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, TC_BK, TC_BM,
+    if (!make_tensor_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, TC_BK, C::kBM,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (!make_map_2d(&tb, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)(K / 8), (uint64_t)N, TC_BK / 8,
-                     TC_BN, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    cudaError_t e = set_tc_attrs<true, false>();
+    const bool okb =
+        DEQ ? make_tensor_map_2d(&tb, Bop, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)(K / 8), (uint64_t)N, TC_BK / 8,
+                          TC_BN, CU_TENSOR_MAP_SWIZZLE_NONE)
+            : make_tensor_map_2d(&tb, Bop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)N, TC_BK, TC_BN,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!okb) return cudaErrorInvalidValue;
+    cudaError_t e = set_tc_attrs<DEQ, SSE, MT>();
     if (e != cudaSuccess) return e;
-    const int m_tiles = (int)((M + TC_BM - 1) / TC_BM);
+    const int m_tiles = (int)((M + C::kBM - 1) / C::kBM);
     const int n_tiles = (int)((N + TC_BN - 1) / TC_BN);
-    tc_gemm_kernel<true, false><<<m_tiles * n_tiles, TC_THREADS, TcSmem<true>::kBytes, stream>>>(
-        ta, tb, reinterpret_cast<const __half*>(scales), zeros, reinterpret_cast<__half*>(Y), nullptr, (int)M,
+    tc_gemm_kernel<DEQ, SSE, MT><<<m_tiles * n_tiles, TC_THREADS, C::kBytes, stream>>>(
+        ta, tb, reinterpret_cast<const __half*>(scales), zeros, reinterpret_cast<__half*>(Y), sse_part, (int)M,
         (int)N, (int)K, m_tiles, n_tiles, status);
     return cudaGetLastError();
 }
 
+// 256-row tiles once M is large enough to fill them; 128-row tiles otherwise.
+static int tc_mt(int64_t M) { return M > 128 ? 2 : 1; }
+
+cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                         const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,
+                         cudaStream_t stream) {
+    if (tc_mt(M) == 2)
+        return launch_tc<true, false, 2>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
+    return launch_tc<true, false, 1>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
+}
+
 cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64_t N, int64_t K,
                           double* sse_part, int* status, cudaStream_t stream) {
-    CUtensorMap ta, tb;
-    if (!make_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)T, TC_BK, TC_BM,
-                     CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    if (!make_map_2d(&tb, E, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)N, TC_BK, TC_BN,
-                     CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
-    cudaError_t e = set_tc_attrs<false, true>();
-    if (e != cudaSuccess) return e;
-    const int m_tiles = (int)((T + TC_BM - 1) / TC_BM);
-    const int n_tiles = (int)((N + TC_BN - 1) / TC_BN);
-    tc_gemm_kernel<false, true><<<m_tiles * n_tiles, TC_THREADS, TcSmem<false>::kBytes, stream>>>(
-        ta, tb, nullptr, nullptr, nullptr, sse_part, (int)T, (int)N, (int)K, m_tiles, n_tiles, status);
-    return cudaGetLastError();
+    if (tc_mt(T) == 2)
+        return launch_tc<false, true, 2>(X, T, E, N, K, nullptr, nullptr, nullptr, sse_part, status, stream);
+    return launch_tc<false, true, 1>(X, T, E, N, K, nullptr, nullptr, nullptr, sse_part, status, stream);
 }
 
 int tc_sse_partials(int64_t T, int64_t N) {
-    return (int)(((T + TC_BM - 1) / TC_BM) * ((N + TC_BN - 1) / TC_BN));
+    const int64_t bm = 128 * tc_mt(T);
+    return (int)(((T + bm - 1) / bm) * ((N + TC_BN - 1) / TC_BN));
 }
 
 }  // namespace w4

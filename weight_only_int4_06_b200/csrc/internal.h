@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <cuda.h>
+
 #include "w4a16.h"
 
 namespace w4 {
@@ -33,6 +35,12 @@ cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           uint16_t* Y, const SkinnyPlan& plan, bool weights_static,
                           cudaStream_t stream);
 
+// Single-token decode GEMV, persistent TMA-fed (gemv_stream.cu).
+cudaError_t launch_gemv_stream(const uint16_t* X, int64_t N, int64_t K, const uint32_t* packed,
+                               const uint16_t* scales, const uint8_t* zeros, uint16_t* Y,
+                               bool weights_static, int* status, cudaStream_t stream);
+size_t gemv_stream_smem(int64_t K);
+
 // tcgen05 GEMM (gemm_tc.cu).
 cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                          const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,
@@ -40,6 +48,10 @@ cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, con
 cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64_t N, int64_t K,
                           double* sse_part, int* status, cudaStream_t stream);
 int tc_sse_partials(int64_t T, int64_t N);
+// 2-D tensor map (TMA descriptor) over a row-major matrix, through the driver entry point.
+bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
+                        uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle swz);
 
 // AWQ search (awq.cu).  Workspace layout (byte offsets, 256-byte aligned).
 struct AwqLayout {
