@@ -174,18 +174,24 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const bool nvalid = n < N;
             uint32_t s2 = 0, zl = 0, zh = 0;
             const uint32_t b_row = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128);
+            const unsigned short* srow = reinterpret_cast<const unsigned short*>(scales) + (int64_t)n * G;
+            const uint8_t* zrow = zeros + (int64_t)n * G;
+            // scale/zero of the next group are fetched one group (two stages) ahead
+            uint32_t sc_next = 0, z_next = 0;
+            if (nvalid) {
+                sc_next = __ldg(srow);
+                z_next = __ldg(zrow);
+            }
             for (int kb = 0; kb < nk; ++kb) {
                 const int s = kb % S;
                 const uint32_t ph = (kb / S) & 1;
                 if ((kb & 1) == 0) {  // a new group of 128 every second stage
                     const int g = kb >> 1;
-                    __half sc = __float2half_rn(0.0f);
-                    uint32_t z = 0;
-                    if (nvalid) {
-                        sc = scales[(int64_t)n * G + g];
-                        z = zeros[(int64_t)n * G + g];
+                    const uint32_t sb = sc_next, z = z_next;
+                    if (nvalid && g + 1 < G) {
+                        sc_next = __ldg(srow + g + 1);
+                        z_next = __ldg(zrow + g + 1);
                     }
-                    const uint32_t sb = (uint32_t)__half_as_ushort(sc);
                     s2 = sb | (sb << 16);
                     zl = (0x6400u + z) * 0x10001u;
                     zh = (0xD400u | (z << 4)) * 0x10001u;

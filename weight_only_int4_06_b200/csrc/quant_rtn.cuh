@@ -38,23 +38,36 @@ __device__ __forceinline__ float div_rn_from_rcp(float a, float b, float y) {
     return __fmaf_rn(r, y, q0);
 }
 
+// rint (round half to even) of an fp32 value with |x| < 2^22: adding 1.5 * 2^23 moves x into the
+// binade [2^23, 2^24) whose spacing is 1, so the IEEE round-to-nearest-even of the addition is
+// the rounding of x; the integer is the difference of the bit patterns (both in that binade).
+__device__ __forceinline__ int rint_small(float x) {
+    const float t = __fadd_rn(x, 12582912.0f);  // 1.5 * 2^23 (even, so ties keep x's parity rule)
+    return __float_as_int(t) - 0x4B400000;      // bit pattern of 1.5 * 2^23
+}
+
 __device__ __forceinline__ GroupQuant group_params(float lo, float hi) {
     GroupQuant p;
     const float d = __fsub_rn(hi, lo);
-    __half s = __float2half_ru(__fdiv_rn(d, 15.0f));
+    __half s = __float2half_ru(div_rn_from_rcp(d, 15.0f, __frcp_rn(15.0f)));  // d / 15, IEEE-exact
     if (d == 0.0f) s = __float2half_rn(1.0f);
     p.s16 = s;
     p.sf = __half2float(s);
     p.rcp = __frcp_rn(p.sf);
     p.overflow = isinf(p.sf);
-    const int z = __float2int_rn(__fdiv_rn(-lo, p.sf));
+    if (p.overflow) {  // codes are unspecified then; keep every intermediate finite
+        p.sf = 1.0f;
+        p.rcp = 1.0f;
+    }
+    const int z = rint_small(div_rn_from_rcp(-lo, p.sf, p.rcp));  // -lo / s16 in [0, 15 + 2^-20]
     p.z = min(max(z, 0), 15);
     return p;
 }
 
-// q = clamp(rint(v / s16) + z, 0, 15) with v / s16 the correctly rounded fp32 quotient.
+// q = clamp(rint(v / s16) + z, 0, 15) with v / s16 the correctly rounded fp32 quotient
+// (|v / s16| <= 15 + 2^-20 because the 16 levels span the zero-inclusive range).
 __device__ __forceinline__ uint32_t quant_code(float v, const GroupQuant& p) {
-    const int q = __float2int_rn(div_rn_from_rcp(v, p.sf, p.rcp)) + p.z;
+    const int q = rint_small(div_rn_from_rcp(v, p.sf, p.rcp)) + p.z;
     return (uint32_t)min(max(q, 0), 15);
 }
 
