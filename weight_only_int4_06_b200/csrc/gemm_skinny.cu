@@ -96,21 +96,22 @@ __global__ void __launch_bounds__(SK_THREADS, MINB)
     // read ahead of the preceding kernel when the caller declared them static.
     if (!weights_early) pdl_wait();
     uint4 wa[SK_PD], wb[SK_PD];
-    uint32_t ma[SK_PD], mb[SK_PD];  // scale bits | zero << 16
+    unsigned short sra[SK_PD], srb[SK_PD];  // raw scale bits, untouched until used
+    uint8_t zra[SK_PD], zrb[SK_PD];          // raw zero points
 #pragma unroll
     for (int s = 0; s < SK_PD; ++s) {
         wa[s] = make_uint4(0u, 0u, 0u, 0u);
         wb[s] = make_uint4(0u, 0u, 0u, 0u);
-        ma[s] = 0u;
-        mb[s] = 0u;
+        sra[s] = 0; zra[s] = 0;
+        srb[s] = 0; zrb[s] = 0;
         if (s < ng) {
             if (va) {
                 wa[s] = ldg_stream(pa + s * 4);
-                ma[s] = (uint32_t)__ldg(sca + s) | ((uint32_t)__ldg(zpa + s) << 16);
+                sra[s] = __ldg(sca + s); zra[s] = __ldg(zpa + s);
             }
             if (vb) {
                 wb[s] = ldg_stream(pb + s * 4);
-                mb[s] = (uint32_t)__ldg(scb + s) | ((uint32_t)__ldg(zpb + s) << 16);
+                srb[s] = __ldg(scb + s); zrb[s] = __ldg(zpb + s);
             }
         }
     }
@@ -160,21 +161,21 @@ __global__ void __launch_bounds__(SK_THREADS, MINB)
             const int gi = g0 + s;
             if (gi < ng) {
                 const uint4 A = wa[s], B = wb[s];
-                const uint32_t mA = ma[s], mB = mb[s];
+                const unsigned short rsa = sra[s], rsb = srb[s];
+                const uint32_t za = zra[s], zb = zrb[s];
                 const int gn = gi + SK_PD;
                 if (gn < ng) {
                     if (va) {
                         wa[s] = ldg_stream(pa + gn * 4);
-                        ma[s] = (uint32_t)__ldg(sca + gn) | ((uint32_t)__ldg(zpa + gn) << 16);
+                        sra[s] = __ldg(sca + gn); zra[s] = __ldg(zpa + gn);
                     }
                     if (vb) {
                         wb[s] = ldg_stream(pb + gn * 4);
-                        mb[s] = (uint32_t)__ldg(scb + gn) | ((uint32_t)__ldg(zpb + gn) << 16);
+                        srb[s] = __ldg(scb + gn); zrb[s] = __ldg(zpb + gn);
                     }
                 }
-                const float sa = __half2float(__ushort_as_half((unsigned short)(mA & 0xFFFFu)));
-                const float sb = __half2float(__ushort_as_half((unsigned short)(mB & 0xFFFFu)));
-                const uint32_t za = mA >> 16, zb = mB >> 16;
+                const float sa = __half2float(__ushort_as_half(rsa));
+                const float sb = __half2float(__ushort_as_half(rsb));
                 const uint32_t zla = (0x6400u + za) * 0x10001u, zha = (0xD400u | (za << 4)) * 0x10001u;
                 const uint32_t zlb = (0x6400u + zb) * 0x10001u, zhb = (0xD400u | (zb << 4)) * 0x10001u;
                 const uint32_t wA[4] = {A.x, A.y, A.z, A.w};
@@ -335,7 +336,7 @@ cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           cudaStream_t stream) {
     switch (plan.mt) {
         case 8: return launch_nt<1, 2>(X, M, N, K, packed, scales, zeros, Y, plan, weights_static, stream);
-        case 16: return launch_nt<2, 2>(X, M, N, K, packed, scales, zeros, Y, plan, weights_static, stream);
+        case 16: return launch_nt<2, 1>(X, M, N, K, packed, scales, zeros, Y, plan, weights_static, stream);
         default: return launch_nt<4, 1>(X, M, N, K, packed, scales, zeros, Y, plan, weights_static, stream);
     }
 }

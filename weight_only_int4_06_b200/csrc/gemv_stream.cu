@@ -152,22 +152,32 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     const bool xlane = g8 == 0;  // only B column 0 (the single activation row) is nonzero
 
     // Scale and zero point of unit v (tile t0 + v / NC, group (v % NC) * 8 + warp) for this
-    // thread's two rows, packed as scale bits | zero << 16; fetched GV_PF units ahead.
-    auto meta_load = [&](int v, uint32_t& ma, uint32_t& mb) {
-        ma = 0u;
-        mb = 0u;
+    // thread's two rows, fetched GV_PF units ahead.  The loaded values stay untouched in their
+    // own registers until they are used, so no instruction waits on them early.
+    auto meta_load = [&](int v, unsigned short& sa, unsigned short& sb, uint8_t& za, uint8_t& zb) {
+        sa = 0;
+        sb = 0;
+        za = 0;
+        zb = 0;
         if (v < n_units) {
             const int t = t0 + v / NC, gi = (v % NC) * GV_CWARPS + warp;
             if (gi < G) {
                 const int na = t * 16 + g8, nb = na + 8;
-                if (na < N) ma = (uint32_t)__ldg(scales + (int64_t)na * G + gi) | ((uint32_t)__ldg(zeros + (int64_t)na * G + gi) << 16);
-                if (nb < N) mb = (uint32_t)__ldg(scales + (int64_t)nb * G + gi) | ((uint32_t)__ldg(zeros + (int64_t)nb * G + gi) << 16);
+                if (na < N) {
+                    sa = __ldg(scales + (int64_t)na * G + gi);
+                    za = __ldg(zeros + (int64_t)na * G + gi);
+                }
+                if (nb < N) {
+                    sb = __ldg(scales + (int64_t)nb * G + gi);
+                    zb = __ldg(zeros + (int64_t)nb * G + gi);
+                }
             }
         }
     };
-    uint32_t pa[GV_PF], pb[GV_PF];
+    unsigned short psa[GV_PF], psb[GV_PF];
+    uint8_t pza[GV_PF], pzb[GV_PF];
 #pragma unroll
-    for (int p = 0; p < GV_PF; ++p) meta_load(p, pa[p], pb[p]);
+    for (int p = 0; p < GV_PF; ++p) meta_load(p, psa[p], psb[p], pza[p], pzb[p]);
 
     float acc_a = 0.0f, acc_b = 0.0f;
     for (int u0 = 0; u0 < n_units; u0 += GV_PF) {
@@ -175,8 +185,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         for (int p = 0; p < GV_PF; ++p) {
             const int u = u0 + p;
             if (u >= n_units) break;  // uniform across the CTA
-            const uint32_t ma = pa[p], mb = pb[p];
-            meta_load(u + GV_PF, pa[p], pb[p]);
+            const unsigned short sa = psa[p], sb = psb[p];
+            const uint32_t za = pza[p], zb = pzb[p];
+            meta_load(u + GV_PF, psa[p], psb[p], pza[p], pzb[p]);
             const int s = u % GV_STAGES;
             const uint32_t ph = (u / GV_STAGES) & 1;
             const int t = t0 + u / NC, kc = u % NC;
@@ -210,10 +221,10 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
                               lop3_and_or(b8, 0x00F000F0u, 0x64006400u), xf.z, xf.w);
                 }
                 const float2 cs = corr[gi];
-                const float ra = (c0[0] + c1[0]) - fmaf((float)(ma >> 16), cs.y, cs.x);
-                const float rb = (c0[2] + c1[2]) - fmaf((float)(mb >> 16), cs.y, cs.x);
-                acc_a = fmaf(__half2float(__ushort_as_half((unsigned short)(ma & 0xFFFFu))), ra, acc_a);
-                acc_b = fmaf(__half2float(__ushort_as_half((unsigned short)(mb & 0xFFFFu))), rb, acc_b);
+                const float ra = (c0[0] + c1[0]) - fmaf((float)za, cs.y, cs.x);
+                const float rb = (c0[2] + c1[2]) - fmaf((float)zb, cs.y, cs.x);
+                acc_a = fmaf(__half2float(__ushort_as_half(sa)), ra, acc_a);
+                acc_b = fmaf(__half2float(__ushort_as_half(sb)), rb, acc_b);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty_bar(s));
