@@ -169,6 +169,33 @@ w4_status awq_scale_search(const uint16_t* X, int64_t T, const uint16_t* W, int6
                            void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * awq_scale_search_noalloc -- awq_scale_search for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart to this call; it exists for integration.  Some callers cannot
+ * call cudaMalloc or any allocating routine: a plugin inside an inference engine that owns all
+ * device memory, a service held to a fixed memory budget, or a latency-critical path that must
+ * not risk the implicit device synchronisation an allocation can cause.  This entry point takes
+ * the same arguments as awq_scale_search minus the workspace: its scratch is one array of
+ * W4_NOALLOC_SCRATCH_BYTES compiled into the library, which every GPU that loads the library
+ * holds until the process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ *   - Limit: problems whose awq_workspace_size exceeds W4_NOALLOC_SCRATCH_BYTES are rejected
+ *     with W4_ERR_WORKSPACE before anything is enqueued (e.g. T = 4096, K = N = 2048 fits;
+ *     K = N = 4096 does not).
+ *   - The first call on each device looks up that device's copy of the scratch array
+ *     (cudaGetSymbolAddress, with the device current); make that first call before any stream
+ *     capture on the device.
+ *   - Every call shares the one array and leaves its contents behind; the call clears what must
+ *     start at zero itself.  Calls whose work overlaps on the GPU (for example on two streams)
+ *     race on the array and give wrong results: serialise them.
+ * Results are the same as awq_scale_search's on the same inputs.
+ */
+#define W4_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+w4_status awq_scale_search_noalloc(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N,
+                                   int64_t K, int group, int n_alpha, double* mse,
+                                   int32_t* best_idx, float* best_s, void* stream);
+
+/*
  * w4_check_device_status -- synchronise `stream`, then read and clear the current device's
  * status word.  Returns W4_OK, W4_ERR_RANGE, W4_ERR_DEVICE_TIMEOUT, or W4_ERR_CUDA if the
  * synchronisation itself failed.

@@ -31,6 +31,7 @@ SIGNATURES = {
     "w4_gemm_ex": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ, _I32, _P]),
     "awq_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_scale_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
+    "awq_scale_search_noalloc": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P]),
     "w4_check_device_status": (_I32, [_P]),
     "w4_status_string": (ctypes.c_char_p, [_I32]),
 }
@@ -157,6 +158,24 @@ def awq_scale_search(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20, group:
                                 ctypes.c_void_p(workspace.data_ptr()),
                                 workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "awq_scale_search")
+    return mse, best, best_s
+
+
+def awq_scale_search_noalloc(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20, group: int = 128,
+                             stream=None):
+    """awq_scale_search without a workspace: the library's built-in scratch array is used instead
+    (for callers that cannot allocate device memory).  The outputs are allocated here only for
+    convenience; a caller that cannot allocate passes its own buffers to the C entry point."""
+    T, K = X.shape
+    N = W.shape[0]
+    mse = torch.empty(n_alpha, dtype=torch.float64, device=X.device)
+    best = torch.empty(1, dtype=torch.int32, device=X.device)
+    best_s = torch.empty(K, dtype=torch.float32, device=X.device)
+    st = lib().awq_scale_search_noalloc(_dev(X, torch.float16, "X"), T, _dev(W, torch.float16, "W"), N, K,
+                                        group, n_alpha, ctypes.c_void_p(mse.data_ptr()),
+                                        ctypes.c_void_p(best.data_ptr()), ctypes.c_void_p(best_s.data_ptr()),
+                                        _stream(stream))
+    _check(st, "awq_scale_search_noalloc")
     return mse, best, best_s
 
 
