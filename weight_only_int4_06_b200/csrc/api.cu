@@ -118,12 +118,14 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
         return launch_tc_w4(X, M, N, K, packed, scales, zeros, Y, status, s) == cudaSuccess ? W4_OK
                                                                                             : W4_ERR_CUDA;
     }
-    const bool gemv_fits = gemv_stream_smem(K) <= 200 * 1024;
+    const int64_t gemv_rows = M < 8 ? M : 8;
+    const bool gemv_fits = gemv_stream_smem(gemv_rows, K) <= 227 * 1024;
     if (family == W4_VARIANT_GEMV && !gemv_fits) return W4_ERR_SHAPE;
-    if (family == W4_VARIANT_GEMV || (family == W4_VARIANT_AUTO && M == 1 && gemv_fits)) {
-        // one activation row at a time (single-token decode has M == 1)
-        for (int64_t m = 0; m < M; ++m) {
-            cudaError_t e = launch_gemv_stream(X + m * K, N, K, packed, scales, zeros, Y + m * N,
+    if (family == W4_VARIANT_GEMV || (family == W4_VARIANT_AUTO && M <= 8 && gemv_fits)) {
+        // up to 8 activation rows per launch (token-by-token decode has M == 1)
+        for (int64_t m0 = 0; m0 < M; m0 += 8) {
+            const int64_t mc = (M - m0) < 8 ? (M - m0) : 8;
+            cudaError_t e = launch_gemv_stream(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N,
                                                weights_static, status, s);
             if (e != cudaSuccess) return W4_ERR_CUDA;
         }

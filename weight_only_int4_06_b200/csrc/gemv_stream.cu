@@ -1,6 +1,6 @@
-// Single-token decode GEMV (M = 1): y = dequant(W) x, streamed at HBM rate.
+// Decode GEMV / skinny GEMM for M <= 8: Y = X dequant(W)^T, streamed at HBM rate.
 //
-// "AutoAWQ vs The Stack v2" (WQLinear blurb): the GEMV kernel serves single-token generation,
+// "AutoAWQ vs The Stack v2" (WQLinear blurb): the GEMV kernel serves token-by-token generation,
 // where the layer is bound by memory traffic and weight reuse is minimal.  The traffic is the
 // packed weights (0.5 B/weight) plus 3 B of scale and zero point per group of 128.
 //
@@ -8,18 +8,22 @@
 //  * Persistent: one CTA per SM; CTA c owns a contiguous range of 16-row tiles over the whole K,
 //    so every output is finished inside one CTA (no split-K workspace, no cluster barrier).
 //  * A producer warp streams the packed tile through a GV_STAGES-deep shared-memory ring with
-//    TMA (16 rows x 1024 k = 8 KB per stage), so each SM keeps ~64 KB of weights in flight no
-//    matter how long the consumers take for one stage.  With static weights it starts before
-//    the preceding kernel has finished (programmatic dependent launch).
-//  * Eight consumer warps take one group of 128 each per stage and run mma.sync m16n8k16 with the
-//    16 weight rows as the A operand.  Dequantisation is one LOP3 per two weights: the operands
-//    are the raw fp16 values 1024+q (low nibble of a byte) and 1024+16q (high nibble); the
-//    activations that meet high nibbles are staged pre-multiplied by 1/16, and the constant
-//    offsets and the zero point are removed per group in fp32 with the exact activation sums
+//    TMA (16 rows x 2048 k = 16 KB per stage), so each SM keeps ~96 KB of weights in flight no
+//    matter how long one stage takes.  With static weights it starts before the preceding kernel
+//    has finished (programmatic dependent launch).
+//  * Sixteen consumer warps take one group of 128 each per stage and run mma.sync m16n8k16 with
+//    the 16 weight rows as the A operand and the (up to 8) activation rows as B.  Dequantisation
+//    is one LOP3 per two weights: the operands are the raw fp16 values 1024+q (low nibble of a
+//    byte) and 1024+16q (high nibble); activations that meet high nibbles are staged pre-multiplied
+//    by 1/16, and the constant offsets and the zero point are removed per group in fp32 with the
+//    exact activation sums
 //        sum_k x_k (q_k - z) = raw - 1024 (Sl + Sh') - z (Sl + 16 Sh'),
 //    Sl = sum of x over low-nibble slots, Sh' = sum of the staged x/16 over high-nibble slots
 //    (both summed exactly in fp64).  The group's fp16 scale then multiplies that sum in fp32.
-//  * Partial sums of the eight warps are added in warp order in shared memory (deterministic).
+//  * The activations are staged once per CTA with each 8-k chunk as
+//    [x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16], so one 16-byte shared load yields the B
+//    fragments of the two MMAs that consume one packed word.
+//  * Partial sums of the sixteen warps are added in warp order in shared memory (deterministic).
 #include <mutex>
 
 #include "common.cuh"
@@ -28,24 +32,25 @@
 
 namespace w4 {
 
-constexpr int GV_CWARPS = 8;                      // consumer warps (one group each per stage)
+constexpr int GV_CWARPS = 16;                     // consumer warps (one group each per stage)
 constexpr int GV_THREADS = 32 * (GV_CWARPS + 1);  // + one producer warp
 constexpr int GV_KC = 128 * GV_CWARPS;            // k per stage
-constexpr uint32_t GV_STAGE_BYTES = 16 * GV_KC / 2;  // 8 KB of packed codes
-constexpr int GV_STAGES = 8;
-constexpr int GV_PF = 8;  // units of metadata prefetched ahead
+constexpr uint32_t GV_STAGE_BYTES = 16 * GV_KC / 2;  // 16 KB of packed codes
+constexpr int GV_STAGES = 6;
+constexpr int GV_PF = 4;  // units of metadata prefetched ahead
+constexpr int GV_MAXM = 8;
 
 struct GvLayout {
     uint32_t ring, xs, corr, red, bars, total;
 };
 
-__host__ __device__ inline GvLayout gv_layout(int K) {
+__host__ __device__ inline GvLayout gv_layout(int M, int K) {
     GvLayout L;
     L.ring = 0;
     L.xs = GV_STAGES * GV_STAGE_BYTES;
-    L.corr = L.xs + (uint32_t)K * 2;                            // float2 per group
-    L.red = L.corr + (uint32_t)(K / 128) * 8;                   // 2 x 8 warps x 16 floats
-    L.bars = (L.red + 2 * GV_CWARPS * 16 * 4 + 7) & ~7u;
+    L.corr = L.xs + (uint32_t)M * (uint32_t)K * 2;               // float2 [G][8]
+    L.red = L.corr + (uint32_t)(K / 128) * GV_MAXM * 8;         // 2 x warps x 16 rows x 8 cols
+    L.bars = L.red + 2 * GV_CWARPS * 16 * GV_MAXM * 4;
     L.total = L.bars + 2 * GV_STAGES * 8 + 8;
     return L;
 }
@@ -57,12 +62,13 @@ __device__ __forceinline__ void gv_named_barrier() {
 __global__ void __launch_bounds__(GV_THREADS, 1)
     gemv_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __half* __restrict__ X,
                        const unsigned short* __restrict__ scales, const uint8_t* __restrict__ zeros,
-                       __half* __restrict__ Y, int N, int K, int n_tiles, int weights_early, int* status) {
+                       __half* __restrict__ Y, int M, int N, int K, int n_tiles, int weights_early,
+                       int* status) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // TMA destinations need an aligned base: round up (the launch reserves 1 KB of slack)
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                            ~uintptr_t(1023));
-    const GvLayout L = gv_layout(K);
+    const GvLayout L = gv_layout(M, K);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = K >> 7;
@@ -90,10 +96,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         if (lane == 0) {
             prefetch_tmap(&tmW);
             if (!weights_early) pdl_wait();
-            int issued = 0;
+            int issued = 0, t = t0, kc = 0, s = 0;
+            uint32_t ph = 0;
             for (int u = 0; u < n_units; ++u) {
-                const int s = u % GV_STAGES;
-                const uint32_t ph = (u / GV_STAGES) & 1;
                 // The ring is full: from here on progress depends on the consumers, who first
                 // wait for the preceding kernel; start the bounded waits only after that point.
                 if (u == GV_STAGES && weights_early) pdl_wait();
@@ -102,10 +107,11 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
                     record_status(status, W4_ERR_DEVICE_TIMEOUT);
                     break;
                 }
-                const int t = t0 + u / NC, kc = u % NC;
                 mbar_arrive_expect_tx(full_bar(s), GV_STAGE_BYTES);
                 tma_load_2d(sbase + L.ring + s * GV_STAGE_BYTES, &tmW, kc * (GV_KC / 8), t * 16, full_bar(s));
                 ++issued;
+                if (++kc == NC) { kc = 0; ++t; }
+                if (++s == GV_STAGES) { s = 0; ph ^= 1; }
             }
             for (int u = issued - GV_STAGES; u < issued; ++u)  // no loads in flight at exit
                 if (u >= 0) mbar_wait_bounded(full_bar(u % GV_STAGES), (u / GV_STAGES) & 1, nullptr, 200000000ull);
@@ -114,15 +120,14 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     }
 
     // ---------------------------------------------------------------- consumers
-    // Stage x: every 8-k chunk as [x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16] (the B fragments
-    // of two MMAs), then the exact per-group sums that remove the operand offsets.
-    pdl_wait();  // x may be produced by the preceding kernel
+    pdl_wait();  // the activations may be produced by the preceding kernel
     __half* xs = reinterpret_cast<__half*>(smem + L.xs);
     const __half2 sixteenth = __float2half2_rn(0.0625f);
-    for (int i = tid; i < K / 8; i += 32 * GV_CWARPS) {
-        const uint4 r = ldg_cached(X + (int64_t)i * 8);
+    const int cpr = K / 8;  // 8-k chunks per activation row
+    for (int i = tid; i < M * cpr; i += 32 * GV_CWARPS) {
+        const uint4 r = ldg_cached(X + (int64_t)i * 8);  // rows are contiguous: chunk i of row i / cpr
         uint4 p;
-        p.x = __byte_perm(r.x, r.z, 0x5410);  // x0, x4
+        p.x = __byte_perm(r.x, r.z, 0x5410);         // x0, x4
         uint32_t h = __byte_perm(r.x, r.z, 0x7632);  // x1, x5
         __half2 hh = __hmul2(*reinterpret_cast<__half2*>(&h), sixteenth);
         p.y = *reinterpret_cast<uint32_t*>(&hh);
@@ -134,63 +139,60 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     }
     gv_named_barrier();
     float2* corr = reinterpret_cast<float2*>(smem + L.corr);
-    for (int g = tid; g < G; g += 32 * GV_CWARPS) {
+    for (int idx = tid; idx < G * GV_MAXM; idx += 32 * GV_CWARPS) {
+        const int g = idx / GV_MAXM, m = idx % GV_MAXM;
         double lo = 0.0, hi = 0.0;  // exact: at most 128 fp16 values
-        const __half* xg = xs + g * 128;
-        for (int i = 0; i < 128; i += 8) {
-            lo += (double)__half2float(xg[i + 0]) + (double)__half2float(xg[i + 1]) +
-                  (double)__half2float(xg[i + 4]) + (double)__half2float(xg[i + 5]);
-            hi += (double)__half2float(xg[i + 2]) + (double)__half2float(xg[i + 3]) +
-                  (double)__half2float(xg[i + 6]) + (double)__half2float(xg[i + 7]);
+        if (m < M) {
+            const __half* xg = xs + (int64_t)m * K + g * 128;
+            for (int i = 0; i < 128; i += 8) {
+                lo += (double)__half2float(xg[i + 0]) + (double)__half2float(xg[i + 1]) +
+                      (double)__half2float(xg[i + 4]) + (double)__half2float(xg[i + 5]);
+                hi += (double)__half2float(xg[i + 2]) + (double)__half2float(xg[i + 3]) +
+                      (double)__half2float(xg[i + 6]) + (double)__half2float(xg[i + 7]);
+            }
         }
-        corr[g] = make_float2((float)(1024.0 * (lo + hi)), (float)(lo + 16.0 * hi));
+        corr[idx] = make_float2((float)(1024.0 * (lo + hi)), (float)(lo + 16.0 * hi));
     }
     gv_named_barrier();
 
     const int g8 = lane >> 2, c = lane & 3;
     float* red = reinterpret_cast<float*>(smem + L.red);
-    const bool xlane = g8 == 0;  // only B column 0 (the single activation row) is nonzero
+    const bool xlane = g8 < M;  // B column g8 holds activation row g8
+    const __half* xrow = xs + (int64_t)(xlane ? g8 : 0) * K;
+    const unsigned short* srow = scales + (int64_t)(t0 * 16 + g8) * G;
+    const uint8_t* zrow = zeros + (int64_t)(t0 * 16 + g8) * G;
 
-    // Scale and zero point of unit v (tile t0 + v / NC, group (v % NC) * 8 + warp) for this
-    // thread's two rows, fetched GV_PF units ahead.  The loaded values stay untouched in their
-    // own registers until they are used, so no instruction waits on them early.
-    auto meta_load = [&](int v, unsigned short& sa, unsigned short& sb, uint8_t& za, uint8_t& zb) {
-        sa = 0;
-        sb = 0;
-        za = 0;
-        zb = 0;
-        if (v < n_units) {
-            const int t = t0 + v / NC, gi = (v % NC) * GV_CWARPS + warp;
+    // Metadata of the unit GV_PF ahead: (tile, chunk) tracked incrementally, raw loads kept in
+    // their own registers until use.
+    int pf_t = t0, pf_kc = 0;
+    auto meta_load = [&](unsigned short& sa, unsigned short& sb, uint8_t& za, uint8_t& zb) {
+        sa = 0; sb = 0; za = 0; zb = 0;
+        if (pf_t < t1) {
+            const int gi = pf_kc * GV_CWARPS + warp;
             if (gi < G) {
-                const int na = t * 16 + g8, nb = na + 8;
-                if (na < N) {
-                    sa = __ldg(scales + (int64_t)na * G + gi);
-                    za = __ldg(zeros + (int64_t)na * G + gi);
-                }
-                if (nb < N) {
-                    sb = __ldg(scales + (int64_t)nb * G + gi);
-                    zb = __ldg(zeros + (int64_t)nb * G + gi);
-                }
+                const int na = pf_t * 16 + g8;
+                const int64_t off = (int64_t)(pf_t - t0) * 16 * G + gi;
+                if (na < N) { sa = __ldg(srow + off); za = __ldg(zrow + off); }
+                if (na + 8 < N) { sb = __ldg(srow + off + 8 * G); zb = __ldg(zrow + off + 8 * G); }
             }
+            if (++pf_kc == NC) { pf_kc = 0; ++pf_t; }
         }
     };
     unsigned short psa[GV_PF], psb[GV_PF];
     uint8_t pza[GV_PF], pzb[GV_PF];
 #pragma unroll
-    for (int p = 0; p < GV_PF; ++p) meta_load(p, psa[p], psb[p], pza[p], pzb[p]);
+    for (int p = 0; p < GV_PF; ++p) meta_load(psa[p], psb[p], pza[p], pzb[p]);
 
-    float acc_a = 0.0f, acc_b = 0.0f;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // rows (g8, g8+8) x cols (2c, 2c+1)
+    int t = t0, kc = 0, s = 0;
+    uint32_t ph = 0;
     for (int u0 = 0; u0 < n_units; u0 += GV_PF) {
 #pragma unroll
         for (int p = 0; p < GV_PF; ++p) {
-            const int u = u0 + p;
-            if (u >= n_units) break;  // uniform across the CTA
+            if (u0 + p >= n_units) break;  // uniform across the CTA
             const unsigned short sa = psa[p], sb = psb[p];
             const uint32_t za = pza[p], zb = pzb[p];
-            meta_load(u + GV_PF, psa[p], psb[p], pza[p], pzb[p]);
-            const int s = u % GV_STAGES;
-            const uint32_t ph = (u / GV_STAGES) & 1;
-            const int t = t0 + u / NC, kc = u % NC;
+            meta_load(psa[p], psb[p], pza[p], pzb[p]);
             const int gi = kc * GV_CWARPS + warp;
             // After a timeout every wait is skipped but the control flow (and every barrier) stays
             // the same, so no warp is left behind at a barrier.
@@ -201,69 +203,82 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
                 ok = false;
             }
             if (ok && gi < G) {
-                const unsigned char* st = smem + L.ring + s * GV_STAGE_BYTES;
-                const uint4 A = *reinterpret_cast<const uint4*>(st + g8 * (GV_KC / 2) + warp * 64 + c * 16);
-                const uint4 B = *reinterpret_cast<const uint4*>(st + (g8 + 8) * (GV_KC / 2) + warp * 64 + c * 16);
+                const unsigned char* st = smem + L.ring + s * GV_STAGE_BYTES + warp * 64 + c * 16;
+                const uint4 A = *reinterpret_cast<const uint4*>(st + g8 * (GV_KC / 2));
+                const uint4 B = *reinterpret_cast<const uint4*>(st + (g8 + 8) * (GV_KC / 2));
                 const uint32_t wA[4] = {A.x, A.y, A.z, A.w};
                 const uint32_t wB[4] = {B.x, B.y, B.z, B.w};
-                float c0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, c1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                const __half* xg = xrow + gi * 128 + c * 32;
+                float cc[4][4];  // four independent accumulation chains, one per packed word
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) cc[j][e] = 0.0f;
                     const uint32_t a = wA[j], b = wB[j], a8 = a >> 8, b8 = b >> 8;
                     uint4 xf = make_uint4(0u, 0u, 0u, 0u);
-                    if (xlane) xf = *reinterpret_cast<const uint4*>(xs + gi * 128 + c * 32 + j * 8);
-                    float(&cc)[4] = (j & 1) ? c1 : c0;  // two independent accumulation chains
-                    mma_16816(cc, lop3_and_or(a, 0x000F000Fu, 0x64006400u), lop3_and_or(b, 0x000F000Fu, 0x64006400u),
-                              lop3_and_or(a, 0x00F000F0u, 0x64006400u), lop3_and_or(b, 0x00F000F0u, 0x64006400u),
-                              xf.x, xf.y);
-                    mma_16816(cc, lop3_and_or(a8, 0x000F000Fu, 0x64006400u),
+                    if (xlane) xf = *reinterpret_cast<const uint4*>(xg + j * 8);
+                    mma_16816(cc[j], lop3_and_or(a, 0x000F000Fu, 0x64006400u),
+                              lop3_and_or(b, 0x000F000Fu, 0x64006400u), lop3_and_or(a, 0x00F000F0u, 0x64006400u),
+                              lop3_and_or(b, 0x00F000F0u, 0x64006400u), xf.x, xf.y);
+                    mma_16816(cc[j], lop3_and_or(a8, 0x000F000Fu, 0x64006400u),
                               lop3_and_or(b8, 0x000F000Fu, 0x64006400u), lop3_and_or(a8, 0x00F000F0u, 0x64006400u),
                               lop3_and_or(b8, 0x00F000F0u, 0x64006400u), xf.z, xf.w);
                 }
-                const float2 cs = corr[gi];
-                const float ra = (c0[0] + c1[0]) - fmaf((float)za, cs.y, cs.x);
-                const float rb = (c0[2] + c1[2]) - fmaf((float)zb, cs.y, cs.x);
-                acc_a = fmaf(__half2float(__ushort_as_half(sa)), ra, acc_a);
-                acc_b = fmaf(__half2float(__ushort_as_half(sb)), rb, acc_b);
+                const float4 cs = *reinterpret_cast<const float4*>(corr + gi * GV_MAXM + 2 * c);  // cols 2c, 2c+1
+                const float fza = (float)za, fzb = (float)zb;
+                const float fsa = __half2float(__ushort_as_half(sa)), fsb = __half2float(__ushort_as_half(sb));
+                const float r0 = (cc[0][0] + cc[1][0]) + (cc[2][0] + cc[3][0]);
+                const float r1 = (cc[0][1] + cc[1][1]) + (cc[2][1] + cc[3][1]);
+                const float r2 = (cc[0][2] + cc[1][2]) + (cc[2][2] + cc[3][2]);
+                const float r3 = (cc[0][3] + cc[1][3]) + (cc[2][3] + cc[3][3]);
+                acc[0] = fmaf(fsa, r0 - fmaf(fza, cs.y, cs.x), acc[0]);  // row g8,   col 2c
+                acc[1] = fmaf(fsa, r1 - fmaf(fza, cs.w, cs.z), acc[1]);  // row g8,   col 2c+1
+                acc[2] = fmaf(fsb, r2 - fmaf(fzb, cs.y, cs.x), acc[2]);  // row g8+8, col 2c
+                acc[3] = fmaf(fsb, r3 - fmaf(fzb, cs.w, cs.z), acc[3]);  // row g8+8, col 2c+1
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty_bar(s));
-            if (kc == NC - 1) {
-                // tile done: lanes with c == 0 hold column 0 for rows g8 (acc_a) and g8 + 8 (acc_b)
-                float* rt = red + ((t - t0) & 1) * (GV_CWARPS * 16);
-                if (c == 0) {
-                    rt[warp * 16 + g8] = acc_a;
-                    rt[warp * 16 + g8 + 8] = acc_b;
-                }
+            if (++s == GV_STAGES) { s = 0; ph ^= 1; }
+            if (++kc == NC) {
+                // tile done: combine the sixteen warps' partial sums in warp order
+                float* rt = red + ((t - t0) & 1) * (GV_CWARPS * 16 * GV_MAXM);
+                float* mine = rt + warp * (16 * GV_MAXM);
+                mine[g8 * GV_MAXM + 2 * c] = acc[0];
+                mine[g8 * GV_MAXM + 2 * c + 1] = acc[1];
+                mine[(g8 + 8) * GV_MAXM + 2 * c] = acc[2];
+                mine[(g8 + 8) * GV_MAXM + 2 * c + 1] = acc[3];
                 gv_named_barrier();
-                if (warp == 0 && lane < 16) {
+                for (int o = tid; o < 16 * M; o += 32 * GV_CWARPS) {
+                    const int row = o % 16, m = o / 16;
                     float sum = 0.0f;
 #pragma unroll
-                    for (int w = 0; w < GV_CWARPS; ++w) sum += rt[w * 16 + lane];  // warp order
-                    const int n = t * 16 + lane;
-                    if (n < N) Y[n] = __float2half_rn(sum);
+                    for (int w = 0; w < GV_CWARPS; ++w) sum += rt[w * (16 * GV_MAXM) + row * GV_MAXM + m];
+                    const int n = t * 16 + row;
+                    if (n < N) Y[(int64_t)m * N + n] = __float2half_rn(sum);
                 }
-                acc_a = 0.0f;
-                acc_b = 0.0f;
+                acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+                kc = 0;
+                ++t;
             }
         }
     }
 }
 
 // ------------------------------------------------------------------------------------ host side
-size_t gemv_stream_smem(int64_t K) {
-    if (K > 65536) return SIZE_MAX;  // the activation row is staged whole in shared memory
-    return (size_t)gv_layout((int)K).total + 1024;
+size_t gemv_stream_smem(int64_t M, int64_t K) {
+    if (M < 1 || M > GV_MAXM || K > 65536) return SIZE_MAX;  // activations are staged whole
+    return (size_t)gv_layout((int)M, (int)K).total + 1024;
 }
 
-cudaError_t launch_gemv_stream(const uint16_t* X, int64_t N, int64_t K, const uint32_t* packed,
+cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                                const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, bool weights_static,
                                int* status, cudaStream_t stream) {
     CUtensorMap tm;
     if (!make_tensor_map_2d(&tm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)(K / 8), (uint64_t)N,
                             GV_KC / 8, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    const size_t smem = gemv_stream_smem(K);
+    const size_t smem = gemv_stream_smem(M, K);
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
     int dev = 0;
@@ -290,7 +305,7 @@ cudaError_t launch_gemv_stream(const uint16_t* X, int64_t N, int64_t K, const ui
     cfg.numAttrs = weights_static ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, gemv_stream_kernel, tm, reinterpret_cast<const __half*>(X),
                               reinterpret_cast<const unsigned short*>(scales), zeros, reinterpret_cast<__half*>(Y),
-                              (int)N, (int)K, n_tiles, weights_static ? 1 : 0, status);
+                              (int)M, (int)N, (int)K, n_tiles, weights_static ? 1 : 0, status);
 }
 
 }  // namespace w4

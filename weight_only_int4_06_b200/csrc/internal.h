@@ -35,11 +35,11 @@ cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           uint16_t* Y, const SkinnyPlan& plan, bool weights_static,
                           cudaStream_t stream);
 
-// Single-token decode GEMV, persistent TMA-fed (gemv_stream.cu).
-cudaError_t launch_gemv_stream(const uint16_t* X, int64_t N, int64_t K, const uint32_t* packed,
+// Decode GEMV for M <= 8, persistent TMA-fed (gemv_stream.cu).
+cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                                const uint16_t* scales, const uint8_t* zeros, uint16_t* Y,
                                bool weights_static, int* status, cudaStream_t stream);
-size_t gemv_stream_smem(int64_t K);
+size_t gemv_stream_smem(int64_t M, int64_t K);  // SIZE_MAX when the shape cannot use the kernel
 
 // tcgen05 GEMM (gemm_tc.cu).
 cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
