@@ -8,10 +8,10 @@
 //  * Persistent: one CTA per SM; CTA c owns a contiguous range of 16-row tiles over the whole K,
 //    so every output is finished inside one CTA (no split-K workspace, no cluster barrier).
 //  * A producer warp streams the packed tile through a GV_STAGES-deep shared-memory ring with
-//    TMA (16 rows x 2048 k = 16 KB per stage), so each SM keeps ~96 KB of weights in flight no
-//    matter how long one stage takes.  With static weights it starts before the preceding kernel
-//    has finished (programmatic dependent launch).
-//  * Sixteen consumer warps take one group of 128 each per stage and run mma.sync m16n8k16 with
+//    TMA: one stage is 16 rows x 4096 k (32 KB; for K = 4096 the whole tile, one contiguous
+//    block of HBM).  With static weights it starts before the preceding kernel has finished
+//    (programmatic dependent launch).
+//  * Sixteen consumer warps take two groups of 128 each per stage and run mma.sync m16n8k16 with
 //    the 16 weight rows as the A operand and the (up to 8) activation rows as B.  Dequantisation
 //    is one LOP3 per two weights: the operands are the raw fp16 values 1024+q (low nibble of a
 //    byte) and 1024+16q (high nibble); activations that meet high nibbles are staged pre-multiplied
@@ -19,11 +19,14 @@
 //    exact activation sums
 //        sum_k x_k (q_k - z) = raw - 1024 (Sl + Sh') - z (Sl + 16 Sh'),
 //    Sl = sum of x over low-nibble slots, Sh' = sum of the staged x/16 over high-nibble slots
-//    (both summed exactly in fp64).  The group's fp16 scale then multiplies that sum in fp32.
+//    (both exact integer sums of 2^-24 units).  The group's fp16 scale then multiplies that sum
+//    in fp32.
 //  * The activations are staged once per CTA with each 8-k chunk as
 //    [x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16], so one 16-byte shared load yields the B
 //    fragments of the two MMAs that consume one packed word.
-//  * Partial sums of the sixteen warps are added in warp order in shared memory (deterministic).
+//  * At the end of a tile every warp parks its partial sums in shared memory; the last warp to
+//    finish the tile (a shared counter) adds the sixteen partials in warp order and writes Y, so
+//    no warp waits for the others (deterministic, no CTA-wide barrier in the main loop).
 #include <mutex>
 
 #include "common.cuh"
@@ -32,31 +35,66 @@
 
 namespace w4 {
 
-constexpr int GV_CWARPS = 16;                     // consumer warps (one group each per stage)
-constexpr int GV_THREADS = 32 * (GV_CWARPS + 1);  // + one producer warp
-constexpr int GV_KC = 128 * GV_CWARPS;            // k per stage
-constexpr uint32_t GV_STAGE_BYTES = 16 * GV_KC / 2;  // 16 KB of packed codes
-constexpr int GV_STAGES = 6;
-constexpr int GV_PF = 4;  // units of metadata prefetched ahead
+constexpr int GV_CWARPS = 16;                        // consumer warps
+constexpr int GV_GPW = 2;                            // groups per warp per stage
+constexpr int GV_THREADS = 32 * (GV_CWARPS + 1);     // + one producer warp
+constexpr int GV_SG = GV_CWARPS * GV_GPW;            // groups per stage (32)
+constexpr int GV_ROWB = GV_SG * 64;                  // bytes of one row in a stage (2 KB)
+constexpr uint32_t GV_STAGE_BYTES = 16 * GV_ROWB;    // 32 KB of packed codes
+constexpr int GV_STAGES = 4;
 constexpr int GV_MAXM = 8;
+constexpr int GV_TSLOTS = GV_STAGES + 2;             // tiles whose partials may be pending at once
 
 struct GvLayout {
-    uint32_t ring, xs, corr, red, bars, total;
+    uint32_t ring, xs, corr, red, cnt, bars, total;
 };
 
 __host__ __device__ inline GvLayout gv_layout(int M, int K) {
     GvLayout L;
     L.ring = 0;
     L.xs = GV_STAGES * GV_STAGE_BYTES;
-    L.corr = L.xs + (uint32_t)M * (uint32_t)K * 2;               // float2 [G][8]
-    L.red = L.corr + (uint32_t)(K / 128) * GV_MAXM * 8;         // 2 x warps x 16 rows x 8 cols
-    L.bars = L.red + 2 * GV_CWARPS * 16 * GV_MAXM * 4;
+    L.corr = L.xs + (uint32_t)M * (uint32_t)(K + 8) * 2;                 // float2 [G][8]
+    L.red = L.corr + (uint32_t)(K / 128) * GV_MAXM * 8;                 // [slot][warp][16][M] fp32
+    L.cnt = L.red + (uint32_t)GV_TSLOTS * GV_CWARPS * 16 * (uint32_t)M * 4;
+    L.bars = (L.cnt + GV_TSLOTS * 4 + 7) & ~7u;
     L.total = L.bars + 2 * GV_STAGES * 8 + 8;
     return L;
 }
 
+// 16-byte chunk swizzle of a staged activation row (row stride padded to 16 mod 128 bytes):
+// makes the B-fragment loads of a warp bank-conflict free for up to 8 activation rows.
+__device__ __forceinline__ int gv_swz(int ch) { return ch ^ ((ch >> 2) & 2); }
+
+// An fp16 value as a signed integer number of 2^-24 units (exact; |value| <= 2^40 units).
+__device__ __forceinline__ long long half_units(uint32_t h) {
+    const uint32_t e = (h >> 10) & 0x1Fu, m = h & 0x3FFu;
+    const long long mag = e == 0 ? (long long)m : ((long long)(m | 0x400u) << (e - 1));
+    return (h & 0x8000u) ? -mag : mag;
+}
+
 __device__ __forceinline__ void gv_named_barrier() {
     asm volatile("bar.sync 1, %0;" ::"n"(32 * GV_CWARPS) : "memory");
+}
+
+// One group (16 rows x 128 k) of the current stage: raw MMA sums for this thread's C fragment.
+__device__ __forceinline__ void gv_group_mma(const uint4 A, const uint4 B, const __half* xg, const int (&xoff)[4],
+                                             bool xlane, float (&r)[4]) {
+    float c0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, c1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const uint32_t wA[4] = {A.x, A.y, A.z, A.w};
+    const uint32_t wB[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t a = wA[j], b = wB[j], a8 = a >> 8, b8 = b >> 8;
+        uint4 xf = make_uint4(0u, 0u, 0u, 0u);
+        if (xlane) xf = *reinterpret_cast<const uint4*>(xg + xoff[j]);
+        float(&cc)[4] = (j & 1) ? c1 : c0;  // two independent accumulation chains
+        mma_16816(cc, lop3_and_or(a, 0x000F000Fu, 0x64006400u), lop3_and_or(b, 0x000F000Fu, 0x64006400u),
+                  lop3_and_or(a, 0x00F000F0u, 0x64006400u), lop3_and_or(b, 0x00F000F0u, 0x64006400u), xf.x, xf.y);
+        mma_16816(cc, lop3_and_or(a8, 0x000F000Fu, 0x64006400u), lop3_and_or(b8, 0x000F000Fu, 0x64006400u),
+                  lop3_and_or(a8, 0x00F000F0u, 0x64006400u), lop3_and_or(b8, 0x00F000F0u, 0x64006400u), xf.z, xf.w);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) r[e] = c0[e] + c1[e];
 }
 
 __global__ void __launch_bounds__(GV_THREADS, 1)
@@ -72,19 +110,21 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = K >> 7;
-    const int NC = (G + GV_CWARPS - 1) / GV_CWARPS;  // stages per tile
+    const int NC = (G + GV_SG - 1) / GV_SG;  // stages per tile
     const int t0 = (int)(((int64_t)blockIdx.x * n_tiles) / gridDim.x);
     const int t1 = (int)(((int64_t)(blockIdx.x + 1) * n_tiles) / gridDim.x);
     const int n_units = (t1 - t0) * NC;
     auto full_bar = [&](int s) { return sbase + L.bars + 8 * s; };
     auto empty_bar = [&](int s) { return sbase + L.bars + 8 * (GV_STAGES + s); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bars + 16 * GV_STAGES);
+    int* cnt = reinterpret_cast<int*>(smem + L.cnt);
 
     if (tid == 0) {
         for (int s = 0; s < GV_STAGES; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), GV_CWARPS);
         }
+        for (int i = 0; i < GV_TSLOTS; ++i) cnt[i] = 0;
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -108,7 +148,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
                     break;
                 }
                 mbar_arrive_expect_tx(full_bar(s), GV_STAGE_BYTES);
-                tma_load_2d(sbase + L.ring + s * GV_STAGE_BYTES, &tmW, kc * (GV_KC / 8), t * 16, full_bar(s));
+                tma_load_2d(sbase + L.ring + s * GV_STAGE_BYTES, &tmW, kc * (GV_ROWB / 8), t * 16, full_bar(s));
                 ++issued;
                 if (++kc == NC) { kc = 0; ++t; }
                 if (++s == GV_STAGES) { s = 0; ph ^= 1; }
@@ -120,12 +160,19 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     }
 
     // ---------------------------------------------------------------- consumers
+    // Stage the activations and, in the same pass, the exact per-group sums that remove the
+    // operand offsets: every fp16 value (and every staged x/16) is an integer number of 2^-24
+    // units, so the sums are exact 64-bit integer additions.  The 16 chunks of one group sit in
+    // 16 consecutive lanes, which reduce them with shuffles.
     pdl_wait();  // the activations may be produced by the preceding kernel
     __half* xs = reinterpret_cast<__half*>(smem + L.xs);
+    float2* corr = reinterpret_cast<float2*>(smem + L.corr);
     const __half2 sixteenth = __float2half2_rn(0.0625f);
     const int cpr = K / 8;  // 8-k chunks per activation row
-    for (int i = tid; i < M * cpr; i += 32 * GV_CWARPS) {
-        const uint4 r = ldg_cached(X + (int64_t)i * 8);  // rows are contiguous: chunk i of row i / cpr
+    const int RS = K + 8;   // staged row stride in halves (16 bytes of padding)
+    for (int i = tid; i < M * cpr; i += 32 * GV_CWARPS) {  // uniform trip count per 16-lane half
+        const int m = i / cpr, ch = i - m * cpr;
+        const uint4 r = ldg_cached(X + (int64_t)i * 8);  // rows are contiguous
         uint4 p;
         p.x = __byte_perm(r.x, r.z, 0x5410);         // x0, x4
         uint32_t h = __byte_perm(r.x, r.z, 0x7632);  // x1, x5
@@ -135,131 +182,129 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         h = __byte_perm(r.y, r.w, 0x7632);    // x3, x7
         hh = __hmul2(*reinterpret_cast<__half2*>(&h), sixteenth);
         p.w = *reinterpret_cast<uint32_t*>(&hh);
-        *reinterpret_cast<uint4*>(xs + (int64_t)i * 8) = p;
-    }
-    gv_named_barrier();
-    float2* corr = reinterpret_cast<float2*>(smem + L.corr);
-    for (int idx = tid; idx < G * GV_MAXM; idx += 32 * GV_CWARPS) {
-        const int g = idx / GV_MAXM, m = idx % GV_MAXM;
-        double lo = 0.0, hi = 0.0;  // exact: at most 128 fp16 values
-        if (m < M) {
-            const __half* xg = xs + (int64_t)m * K + g * 128;
-            for (int i = 0; i < 128; i += 8) {
-                lo += (double)__half2float(xg[i + 0]) + (double)__half2float(xg[i + 1]) +
-                      (double)__half2float(xg[i + 4]) + (double)__half2float(xg[i + 5]);
-                hi += (double)__half2float(xg[i + 2]) + (double)__half2float(xg[i + 3]) +
-                      (double)__half2float(xg[i + 6]) + (double)__half2float(xg[i + 7]);
-            }
+        *reinterpret_cast<uint4*>(xs + (int64_t)m * RS + gv_swz(ch) * 8) = p;
+        long long lo = half_units(p.x & 0xFFFFu) + half_units(p.x >> 16) + half_units(p.z & 0xFFFFu) +
+                       half_units(p.z >> 16);
+        long long hi = half_units(p.y & 0xFFFFu) + half_units(p.y >> 16) + half_units(p.w & 0xFFFFu) +
+                       half_units(p.w >> 16);
+        const unsigned half_mask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;  // both halves may differ
+#pragma unroll
+        for (int o = 8; o; o >>= 1) {
+            lo += __shfl_xor_sync(half_mask, lo, o);
+            hi += __shfl_xor_sync(half_mask, hi, o);
         }
-        corr[idx] = make_float2((float)(1024.0 * (lo + hi)), (float)(lo + 16.0 * hi));
+        if ((ch & 15) == 0)  // C = 1024 (Sl + Sh'), S = Sl + 16 Sh', one rounding each
+            corr[(ch >> 4) * GV_MAXM + m] =
+                make_float2(__ll2float_rn(lo + hi) * 0x1p-14f, __ll2float_rn(lo + 16 * hi) * 0x1p-24f);
     }
+    for (int idx = tid; idx < G * GV_MAXM; idx += 32 * GV_CWARPS)  // activation rows >= M
+        if (idx % GV_MAXM >= M) corr[idx] = make_float2(0.0f, 0.0f);
     gv_named_barrier();
 
     const int g8 = lane >> 2, c = lane & 3;
     float* red = reinterpret_cast<float*>(smem + L.red);
     const bool xlane = g8 < M;  // B column g8 holds activation row g8
-    const __half* xrow = xs + (int64_t)(xlane ? g8 : 0) * K;
-    const unsigned short* srow = scales + (int64_t)(t0 * 16 + g8) * G;
-    const uint8_t* zrow = zeros + (int64_t)(t0 * 16 + g8) * G;
+    const __half* xrow = xs + (int64_t)(xlane ? g8 : 0) * RS;
+    int xoff[4];  // swizzled offset (halves) of word j's chunk within a group, for this lane
+#pragma unroll
+    for (int j = 0; j < 4; ++j) xoff[j] = gv_swz(c * 4 + j) * 8;
 
-    // Metadata of the unit GV_PF ahead: (tile, chunk) tracked incrementally, raw loads kept in
-    // their own registers until use.
-    int pf_t = t0, pf_kc = 0;
-    auto meta_load = [&](unsigned short& sa, unsigned short& sb, uint8_t& za, uint8_t& zb) {
-        sa = 0; sb = 0; za = 0; zb = 0;
-        if (pf_t < t1) {
-            const int gi = pf_kc * GV_CWARPS + warp;
+    // this thread's W bytes inside a stage: row g8 / g8 + 8, group (warp + 16 e), 16 bytes at 16 c
+    const uint32_t wofs = (uint32_t)(g8 * GV_ROWB + warp * 64 + c * 16);
+    int s = 0, kc = 0, t = t0;
+    uint32_t ph = 0;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // rows (g8, g8+8) x cols (2c, 2c+1)
+    bool dead = false;
+    // Scale and zero point of this thread's two rows for the warp's two groups of unit (tt, kk),
+    // fetched one unit ahead; the loaded values are not touched until they are used.
+    auto meta_fetch = [&](int tt, int kk, unsigned short (&sv)[4], uint8_t (&zv)[4]) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { sv[i] = 0; zv[i] = 0; }
+        if (tt >= t1) return;
+        const int gA = kk * GV_SG + warp, na = tt * 16 + g8;
+        const int64_t mo = (int64_t)na * G;
+        const bool ra_ok = na < N, rb_ok = na + 8 < N;
+#pragma unroll
+        for (int e = 0; e < GV_GPW; ++e) {
+            const int gi = gA + e * GV_CWARPS;
             if (gi < G) {
-                const int na = pf_t * 16 + g8;
-                const int64_t off = (int64_t)(pf_t - t0) * 16 * G + gi;
-                if (na < N) { sa = __ldg(srow + off); za = __ldg(zrow + off); }
-                if (na + 8 < N) { sb = __ldg(srow + off + 8 * G); zb = __ldg(zrow + off + 8 * G); }
+                if (ra_ok) { sv[2 * e] = __ldg(scales + mo + gi); zv[2 * e] = __ldg(zeros + mo + gi); }
+                if (rb_ok) { sv[2 * e + 1] = __ldg(scales + mo + 8 * G + gi); zv[2 * e + 1] = __ldg(zeros + mo + 8 * G + gi); }
             }
-            if (++pf_kc == NC) { pf_kc = 0; ++pf_t; }
         }
     };
-    unsigned short psa[GV_PF], psb[GV_PF];
-    uint8_t pza[GV_PF], pzb[GV_PF];
+    unsigned short s_nx[4];
+    uint8_t z_nx[4];
+    meta_fetch(t0, 0, s_nx, z_nx);
+    for (int u = 0; u < n_units; ++u) {
+        const int gA = kc * GV_SG + warp;
+        unsigned short sv[4];  // [group e][row]: e * 2 + (0: row g8, 1: row g8 + 8)
+        uint8_t zv[4];
 #pragma unroll
-    for (int p = 0; p < GV_PF; ++p) meta_load(psa[p], psb[p], pza[p], pzb[p]);
-
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // rows (g8, g8+8) x cols (2c, 2c+1)
-    int t = t0, kc = 0, s = 0;
-    uint32_t ph = 0;
-    for (int u0 = 0; u0 < n_units; u0 += GV_PF) {
+        for (int i = 0; i < 4; ++i) { sv[i] = s_nx[i]; zv[i] = z_nx[i]; }
+        if (kc + 1 < NC) meta_fetch(t, kc + 1, s_nx, z_nx);
+        else meta_fetch(t + 1, 0, s_nx, z_nx);
+        // After a timeout every wait is skipped; the loop still runs to the end.
+        if (!dead && !mbar_wait_bounded(full_bar(s), ph, abort_flag)) {
+            *abort_flag = 1;
+            record_status(status, W4_ERR_DEVICE_TIMEOUT);
+            dead = true;
+        }
+        if (!dead) {
+            const unsigned char* st = smem + L.ring + s * GV_STAGE_BYTES + wofs;
 #pragma unroll
-        for (int p = 0; p < GV_PF; ++p) {
-            if (u0 + p >= n_units) break;  // uniform across the CTA
-            const unsigned short sa = psa[p], sb = psb[p];
-            const uint32_t za = pza[p], zb = pzb[p];
-            meta_load(psa[p], psb[p], pza[p], pzb[p]);
-            const int gi = kc * GV_CWARPS + warp;
-            // After a timeout every wait is skipped but the control flow (and every barrier) stays
-            // the same, so no warp is left behind at a barrier.
-            bool ok = !*abort_flag;
-            if (ok && !mbar_wait_bounded(full_bar(s), ph, abort_flag)) {
-                *abort_flag = 1;
-                record_status(status, W4_ERR_DEVICE_TIMEOUT);
-                ok = false;
-            }
-            if (ok && gi < G) {
-                const unsigned char* st = smem + L.ring + s * GV_STAGE_BYTES + warp * 64 + c * 16;
-                const uint4 A = *reinterpret_cast<const uint4*>(st + g8 * (GV_KC / 2));
-                const uint4 B = *reinterpret_cast<const uint4*>(st + (g8 + 8) * (GV_KC / 2));
-                const uint32_t wA[4] = {A.x, A.y, A.z, A.w};
-                const uint32_t wB[4] = {B.x, B.y, B.z, B.w};
-                const __half* xg = xrow + gi * 128 + c * 32;
-                float cc[4][4];  // four independent accumulation chains, one per packed word
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) cc[j][e] = 0.0f;
-                    const uint32_t a = wA[j], b = wB[j], a8 = a >> 8, b8 = b >> 8;
-                    uint4 xf = make_uint4(0u, 0u, 0u, 0u);
-                    if (xlane) xf = *reinterpret_cast<const uint4*>(xg + j * 8);
-                    mma_16816(cc[j], lop3_and_or(a, 0x000F000Fu, 0x64006400u),
-                              lop3_and_or(b, 0x000F000Fu, 0x64006400u), lop3_and_or(a, 0x00F000F0u, 0x64006400u),
-                              lop3_and_or(b, 0x00F000F0u, 0x64006400u), xf.x, xf.y);
-                    mma_16816(cc[j], lop3_and_or(a8, 0x000F000Fu, 0x64006400u),
-                              lop3_and_or(b8, 0x000F000Fu, 0x64006400u), lop3_and_or(a8, 0x00F000F0u, 0x64006400u),
-                              lop3_and_or(b8, 0x00F000F0u, 0x64006400u), xf.z, xf.w);
+            for (int e = 0; e < GV_GPW; ++e) {
+                const int gi = gA + e * GV_CWARPS;
+                if (gi < G) {
+                    const uint4 A = *reinterpret_cast<const uint4*>(st + e * (GV_CWARPS * 64));
+                    const uint4 B = *reinterpret_cast<const uint4*>(st + e * (GV_CWARPS * 64) + 8 * GV_ROWB);
+                    float r[4];
+                    gv_group_mma(A, B, xrow + gi * 128, xoff, xlane, r);
+                    const float4 cs = *reinterpret_cast<const float4*>(corr + gi * GV_MAXM + 2 * c);
+                    const float fza = (float)zv[2 * e], fzb = (float)zv[2 * e + 1];
+                    const float fsa = __half2float(__ushort_as_half(sv[2 * e]));
+                    const float fsb = __half2float(__ushort_as_half(sv[2 * e + 1]));
+                    acc[0] = fmaf(fsa, r[0] - fmaf(fza, cs.y, cs.x), acc[0]);  // row g8,   col 2c
+                    acc[1] = fmaf(fsa, r[1] - fmaf(fza, cs.w, cs.z), acc[1]);  // row g8,   col 2c+1
+                    acc[2] = fmaf(fsb, r[2] - fmaf(fzb, cs.y, cs.x), acc[2]);  // row g8+8, col 2c
+                    acc[3] = fmaf(fsb, r[3] - fmaf(fzb, cs.w, cs.z), acc[3]);  // row g8+8, col 2c+1
                 }
-                const float4 cs = *reinterpret_cast<const float4*>(corr + gi * GV_MAXM + 2 * c);  // cols 2c, 2c+1
-                const float fza = (float)za, fzb = (float)zb;
-                const float fsa = __half2float(__ushort_as_half(sa)), fsb = __half2float(__ushort_as_half(sb));
-                const float r0 = (cc[0][0] + cc[1][0]) + (cc[2][0] + cc[3][0]);
-                const float r1 = (cc[0][1] + cc[1][1]) + (cc[2][1] + cc[3][1]);
-                const float r2 = (cc[0][2] + cc[1][2]) + (cc[2][2] + cc[3][2]);
-                const float r3 = (cc[0][3] + cc[1][3]) + (cc[2][3] + cc[3][3]);
-                acc[0] = fmaf(fsa, r0 - fmaf(fza, cs.y, cs.x), acc[0]);  // row g8,   col 2c
-                acc[1] = fmaf(fsa, r1 - fmaf(fza, cs.w, cs.z), acc[1]);  // row g8,   col 2c+1
-                acc[2] = fmaf(fsb, r2 - fmaf(fzb, cs.y, cs.x), acc[2]);  // row g8+8, col 2c
-                acc[3] = fmaf(fsb, r3 - fmaf(fzb, cs.w, cs.z), acc[3]);  // row g8+8, col 2c+1
             }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));
+        if (++s == GV_STAGES) { s = 0; ph ^= 1; }
+        if (++kc == NC) {
+            // tile done: park this warp's partials; the last warp of the tile adds all sixteen
+            const int slot = (t - t0) % GV_TSLOTS;
+            float* rs = red + (size_t)slot * (GV_CWARPS * 16 * M);
+            float* mine = rs + warp * (16 * M);
+            const int m0 = 2 * c, m1 = 2 * c + 1;
+            if (m0 < M) { mine[g8 * M + m0] = acc[0]; mine[(g8 + 8) * M + m0] = acc[2]; }
+            if (m1 < M) { mine[g8 * M + m1] = acc[1]; mine[(g8 + 8) * M + m1] = acc[3]; }
             __syncwarp();
-            if (lane == 0) mbar_arrive(empty_bar(s));
-            if (++s == GV_STAGES) { s = 0; ph ^= 1; }
-            if (++kc == NC) {
-                // tile done: combine the sixteen warps' partial sums in warp order
-                float* rt = red + ((t - t0) & 1) * (GV_CWARPS * 16 * GV_MAXM);
-                float* mine = rt + warp * (16 * GV_MAXM);
-                mine[g8 * GV_MAXM + 2 * c] = acc[0];
-                mine[g8 * GV_MAXM + 2 * c + 1] = acc[1];
-                mine[(g8 + 8) * GV_MAXM + 2 * c] = acc[2];
-                mine[(g8 + 8) * GV_MAXM + 2 * c + 1] = acc[3];
-                gv_named_barrier();
-                for (int o = tid; o < 16 * M; o += 32 * GV_CWARPS) {
-                    const int row = o % 16, m = o / 16;
+            int last = 0;
+            if (lane == 0) {
+                __threadfence_block();
+                last = atomicAdd(&cnt[slot], 1) == GV_CWARPS - 1;
+            }
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence_block();
+                for (int o = lane; o < 16 * M; o += 32) {
                     float sum = 0.0f;
 #pragma unroll
-                    for (int w = 0; w < GV_CWARPS; ++w) sum += rt[w * (16 * GV_MAXM) + row * GV_MAXM + m];
+                    for (int w = 0; w < GV_CWARPS; ++w) sum += rs[w * (16 * M) + o];  // warp order
+                    const int row = o / M, m = o - row * M;
                     const int n = t * 16 + row;
                     if (n < N) Y[(int64_t)m * N + n] = __float2half_rn(sum);
                 }
-                acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
-                kc = 0;
-                ++t;
+                __syncwarp();
+                if (lane == 0) cnt[slot] = 0;
             }
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+            kc = 0;
+            ++t;
         }
     }
 }
@@ -273,9 +318,9 @@ size_t gemv_stream_smem(int64_t M, int64_t K) {
 cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                                const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, bool weights_static,
                                int* status, cudaStream_t stream) {
-    CUtensorMap tm;
-    if (!make_tensor_map_2d(&tm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)(K / 8), (uint64_t)N,
-                            GV_KC / 8, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+    CUtensorMap tm;  // packed rows as 8-byte elements: a 256-element box is 2 KB (4096 k) of a row
+    if (!make_tensor_map_2d(&tm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)(K / 16), (uint64_t)N,
+                            GV_ROWB / 8, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     const size_t smem = gemv_stream_smem(M, K);
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
