@@ -74,7 +74,8 @@ typedef enum {
     W4_VARIANT_AUTO = 0,
     W4_VARIANT_SKINNY = 1, /* warp-level tensor-core GEMV / skinny GEMM, split-K over a cluster */
     W4_VARIANT_TC = 2,     /* tcgen05/TMEM tensor-core GEMM with dequantisation in the smem path */
-    W4_VARIANT_GEMV = 3,   /* persistent TMA-fed GEMV, one activation row at a time (decode) */
+    W4_VARIANT_GEMV = 3,   /* persistent TMA-fed mma.sync GEMV, up to 8 activation rows per launch */
+    W4_VARIANT_GEMV_TC = 4, /* tcgen05 GEMV, weights as a TMEM operand, up to 8 rows per launch */
     /* Flag, OR-ed into the variant: packed/scales/zeros are not written by any work still in
      * flight on the stream (static weights).  The call may then use programmatic dependent launch
      * and start streaming the weights before the preceding kernel on the stream has finished;

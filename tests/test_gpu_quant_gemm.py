@@ -240,6 +240,20 @@ def test_gemm_gemv_ragged(M, K, N):
     assert_close(gpu_gemm(X, p, s, z, B.VARIANT_GEMV), oracle.gemm(X, p, s, z), f"gemv {M}x{K}x{N}")
 
 
+@pytest.mark.parametrize("M,K,N", [(1, 128, 8), (1, 384, 24), (1, 1152, 136), (1, 4096, 4104),
+                                   (1, 11008, 40), (2, 2048, 520), (5, 4096, 264), (8, 1536, 1032),
+                                   (1, 4096, 12288), (1, 11008, 4096), (12, 512, 136)])
+def test_gemm_gemv_tc_ragged(M, K, N):
+    X, p, s, z = oracle_case(30, M, K, N)
+    assert_close(gpu_gemm(X, p, s, z, B.VARIANT_GEMV_TC), oracle.gemm(X, p, s, z), f"gemv_tc {M}x{K}x{N}")
+
+
+def test_gemm_gemv_tc_outlier_heavy_activations():
+    X, p, s, z = oracle_case(31, 3, 4096, 1024)
+    X = (X.astype(np.float32) * 40).astype(np.float16)
+    assert_close(gpu_gemm(X, p, s, z, B.VARIANT_GEMV_TC), oracle.gemm(X, p, s, z), "gemv_tc x40")
+
+
 def test_gemm_gemv_outlier_heavy_activations():
     """Large activations stress the offset removal (raw operands carry a 1024 offset)."""
     X, p, s, z = oracle_case(29, 1, 4096, 1024)

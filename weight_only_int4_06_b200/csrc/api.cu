@@ -93,7 +93,7 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     if (group != 128) return W4_ERR_UNSUPPORTED;
     const bool weights_static = (variant & W4_FLAG_WEIGHTS_STATIC) != 0;
     const int family = variant & ~W4_FLAG_WEIGHTS_STATIC;
-    if (family < W4_VARIANT_AUTO || family > W4_VARIANT_GEMV) return W4_ERR_UNSUPPORTED;
+    if (family < W4_VARIANT_AUTO || family > W4_VARIANT_GEMV_TC) return W4_ERR_UNSUPPORTED;
     if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0)
         return W4_ERR_SHAPE;
     size_t need = 0;
@@ -117,6 +117,18 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     if (use_tc) {
         return launch_tc_w4(X, M, N, K, packed, scales, zeros, Y, status, s) == cudaSuccess ? W4_OK
                                                                                             : W4_ERR_CUDA;
+    }
+    GemvTcPlan gtp;
+    const bool gemv_tc_ok = M <= 8 && plan_gemv_tc(M, N, K, &gtp);
+    if (family == W4_VARIANT_GEMV_TC && !plan_gemv_tc(M < 8 ? M : 8, N, K, &gtp)) return W4_ERR_SHAPE;
+    if (family == W4_VARIANT_GEMV_TC || (family == W4_VARIANT_AUTO && gemv_tc_ok)) {
+        for (int64_t m0 = 0; m0 < M; m0 += 8) {  // up to 8 activation rows per launch
+            const int64_t mc = (M - m0) < 8 ? (M - m0) : 8;
+            cudaError_t e = launch_gemv_tc(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N, gtp,
+                                           weights_static, status, s);
+            if (e != cudaSuccess) return W4_ERR_CUDA;
+        }
+        return W4_OK;
     }
     const int64_t gemv_rows = M < 8 ? M : 8;
     const bool gemv_fits = gemv_stream_smem(gemv_rows, K) <= 227 * 1024;

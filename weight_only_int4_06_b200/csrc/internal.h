@@ -41,6 +41,18 @@ cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t 
                                bool weights_static, int* status, cudaStream_t stream);
 size_t gemv_stream_smem(int64_t M, int64_t K);  // SIZE_MAX when the shape cannot use the kernel
 
+// Decode GEMV for M <= 8 on tcgen05 with the weights as a TMEM operand (gemv_tc.cu).
+struct GemvTcPlan {
+    int splits;   // K splits = cluster size (1..16)
+    int gps;      // groups of 128 per split (<= 12)
+    int n_tiles;  // 128-row tiles
+    size_t smem;  // dynamic shared memory per CTA
+};
+bool plan_gemv_tc(int64_t M, int64_t N, int64_t K, GemvTcPlan* plan);
+cudaError_t launch_gemv_tc(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                           const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, const GemvTcPlan& plan,
+                           bool weights_static, int* status, cudaStream_t stream);
+
 // tcgen05 GEMM (gemm_tc.cu).
 cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                          const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,

@@ -19,7 +19,7 @@ STATUS_NAMES = {
     0: "W4_OK", 1: "W4_ERR_NULL", 2: "W4_ERR_SHAPE", 3: "W4_ERR_ALIGN", 4: "W4_ERR_UNSUPPORTED",
     5: "W4_ERR_WORKSPACE", 6: "W4_ERR_CUDA", 7: "W4_ERR_DEVICE_TIMEOUT", 8: "W4_ERR_RANGE",
 }
-VARIANT_AUTO, VARIANT_SKINNY, VARIANT_TC, VARIANT_GEMV = 0, 1, 2, 3
+VARIANT_AUTO, VARIANT_SKINNY, VARIANT_TC, VARIANT_GEMV, VARIANT_GEMV_TC = 0, 1, 2, 3, 4
 FLAG_WEIGHTS_STATIC = 0x100
 
 # Entry points declared in include/w4a16.h: (name, restype, argtypes)
