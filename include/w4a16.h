@@ -74,7 +74,9 @@ typedef enum {
     W4_VARIANT_AUTO = 0,
     W4_VARIANT_SKINNY = 1, /* warp-level tensor-core GEMV / skinny GEMM, split-K over a cluster */
     W4_VARIANT_TC = 2,     /* tcgen05/TMEM tensor-core GEMM with dequantisation in the smem path */
-    W4_VARIANT_GEMV = 3,   /* persistent TMA-fed mma.sync GEMV, up to 8 activation rows per launch */
+    W4_VARIANT_GEMV = 3,   /* persistent TMA-fed mma.sync GEMV, up to 8 activation rows per launch;
+                            * needs 16-byte aligned scales and zeros (else W4_ERR_ALIGN; w4_gemm
+                            * then uses the skinny family) */
     W4_VARIANT_GEMV_TC = 4, /* tcgen05 GEMV, weights as a TMEM operand, up to 8 rows per launch */
     /* Flag, OR-ed into the variant: packed/scales/zeros are not written by any work still in
      * flight on the stream (static weights).  The call may then use programmatic dependent launch

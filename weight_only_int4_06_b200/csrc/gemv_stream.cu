@@ -46,18 +46,28 @@ constexpr int GV_MAXM = 8;
 constexpr int GV_TSLOTS = GV_STAGES + 2;             // tiles whose partials may be pending at once
 
 struct GvLayout {
-    uint32_t ring, xs, corr, red, cnt, bars, total;
+    uint32_t ring, meta, mslot, nmslot, xs, corr, red, cnt, bars, total;
 };
 
+// A tile's metadata (16 rows x G scales, then 16 rows x G zero points) is one contiguous block of
+// each array, so it travels as two bulk copies into a per-tile slot of 48 G bytes.  The producer
+// runs at most GV_STAGES stages ahead of the slowest consumer, so ceil(GV_STAGES / stages per
+// tile) + 1 slots let it refill a slot without waiting.
 __host__ __device__ inline GvLayout gv_layout(int M, int K) {
     GvLayout L;
+    const uint32_t G = (uint32_t)(K / 128);
+    const uint32_t NC = (G + GV_SG - 1) / GV_SG;
+    const uint32_t need = (GV_STAGES + NC - 1) / NC + 1;
     L.ring = 0;
-    L.xs = GV_STAGES * GV_STAGE_BYTES;
+    L.meta = GV_STAGES * GV_STAGE_BYTES;
+    L.mslot = 48u * G;
+    L.nmslot = need < (uint32_t)GV_TSLOTS ? need : (uint32_t)GV_TSLOTS;
+    L.xs = L.meta + L.nmslot * L.mslot;
     L.corr = L.xs + (uint32_t)M * (uint32_t)(K + 8) * 2;                 // float2 [G][8]
-    L.red = L.corr + (uint32_t)(K / 128) * GV_MAXM * 8;                 // [slot][warp][16][M] fp32
+    L.red = L.corr + G * GV_MAXM * 8;                                   // [slot][warp][16][M] fp32
     L.cnt = L.red + (uint32_t)GV_TSLOTS * GV_CWARPS * 16 * (uint32_t)M * 4;
-    L.bars = (L.cnt + GV_TSLOTS * 4 + 7) & ~7u;
-    L.total = L.bars + 2 * GV_STAGES * 8 + 8;
+    L.bars = (L.cnt + GV_TSLOTS * 4 + 7) & ~7u;                          // full, empty, meta_empty
+    L.total = L.bars + (2 * GV_STAGES + GV_TSLOTS) * 8 + 8;
     return L;
 }
 
@@ -116,7 +126,9 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     const int n_units = (t1 - t0) * NC;
     auto full_bar = [&](int s) { return sbase + L.bars + 8 * s; };
     auto empty_bar = [&](int s) { return sbase + L.bars + 8 * (GV_STAGES + s); };
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bars + 16 * GV_STAGES);
+    auto meta_empty = [&](int slot) { return sbase + L.bars + 8 * (2 * GV_STAGES + slot); };
+    const int nms = (int)L.nmslot;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bars + 8 * (2 * GV_STAGES + GV_TSLOTS));
     int* cnt = reinterpret_cast<int*>(smem + L.cnt);
 
     if (tid == 0) {
@@ -125,6 +137,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
             mbar_init(empty_bar(s), GV_CWARPS);
         }
         for (int i = 0; i < GV_TSLOTS; ++i) cnt[i] = 0;
+        for (int i = 0; i < nms; ++i) mbar_init(meta_empty(i), GV_CWARPS);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -136,21 +149,35 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         if (lane == 0) {
             prefetch_tmap(&tmW);
             if (!weights_early) pdl_wait();
-            int issued = 0, t = t0, kc = 0, s = 0;
+            int issued = 0, ti = 0, kc = 0, s = 0;
             uint32_t ph = 0;
             for (int u = 0; u < n_units; ++u) {
                 // The ring is full: from here on progress depends on the consumers, who first
                 // wait for the preceding kernel; start the bounded waits only after that point.
                 if (u == GV_STAGES && weights_early) pdl_wait();
-                if (!mbar_wait_bounded(empty_bar(s), ph ^ 1, abort_flag)) {
+                const int t = t0 + ti, slot = ti % nms;
+                if ((kc == 0 && !mbar_wait_bounded(meta_empty(slot), ((ti / nms) & 1) ^ 1, abort_flag)) ||
+                    !mbar_wait_bounded(empty_bar(s), ph ^ 1, abort_flag)) {
                     *abort_flag = 1;
                     record_status(status, W4_ERR_DEVICE_TIMEOUT);
                     break;
                 }
-                mbar_arrive_expect_tx(full_bar(s), GV_STAGE_BYTES);
+                uint32_t sb = 0, zb = 0;
+                const int64_t mofs = (int64_t)t * 16 * G;  // first metadata entry of the tile
+                if (kc == 0) {  // the tile's metadata rides on its first stage
+                    const int rows = N - t * 16 < 16 ? N - t * 16 : 16;  // 8 or 16 (N % 8 == 0)
+                    sb = (uint32_t)(rows * 2 * G);
+                    zb = (uint32_t)(rows * G) & ~15u;
+                    if (zb != (uint32_t)(rows * G))  // 8 trailing zero points (8 rows, odd G): plain copy
+                        *reinterpret_cast<uint2*>(smem + L.meta + slot * L.mslot + 32 * G + zb) =
+                            *reinterpret_cast<const uint2*>(zeros + mofs + zb);
+                }
+                mbar_arrive_expect_tx(full_bar(s), GV_STAGE_BYTES + sb + zb);
                 tma_load_2d(sbase + L.ring + s * GV_STAGE_BYTES, &tmW, kc * (GV_ROWB / 8), t * 16, full_bar(s));
+                if (sb) bulk_load_1d(sbase + L.meta + slot * L.mslot, scales + mofs, sb, full_bar(s));
+                if (zb) bulk_load_1d(sbase + L.meta + slot * L.mslot + 32 * G, zeros + mofs, zb, full_bar(s));
                 ++issued;
-                if (++kc == NC) { kc = 0; ++t; }
+                if (++kc == NC) { kc = 0; ++ti; }
                 if (++s == GV_STAGES) { s = 0; ph ^= 1; }
             }
             for (int u = issued - GV_STAGES; u < issued; ++u)  // no loads in flight at exit
@@ -215,41 +242,17 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     uint32_t ph = 0;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // rows (g8, g8+8) x cols (2c, 2c+1)
     bool dead = false;
-    // Scale and zero point of this thread's two rows for the warp's two groups of unit (tt, kk),
-    // fetched one unit ahead; the loaded values are not touched until they are used.
-    auto meta_fetch = [&](int tt, int kk, unsigned short (&sv)[4], uint8_t (&zv)[4]) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { sv[i] = 0; zv[i] = 0; }
-        if (tt >= t1) return;
-        const int gA = kk * GV_SG + warp, na = tt * 16 + g8;
-        const int64_t mo = (int64_t)na * G;
-        const bool ra_ok = na < N, rb_ok = na + 8 < N;
-#pragma unroll
-        for (int e = 0; e < GV_GPW; ++e) {
-            const int gi = gA + e * GV_CWARPS;
-            if (gi < G) {
-                if (ra_ok) { sv[2 * e] = __ldg(scales + mo + gi); zv[2 * e] = __ldg(zeros + mo + gi); }
-                if (rb_ok) { sv[2 * e + 1] = __ldg(scales + mo + 8 * G + gi); zv[2 * e + 1] = __ldg(zeros + mo + 8 * G + gi); }
-            }
-        }
-    };
-    unsigned short s_nx[4];
-    uint8_t z_nx[4];
-    meta_fetch(t0, 0, s_nx, z_nx);
     for (int u = 0; u < n_units; ++u) {
         const int gA = kc * GV_SG + warp;
-        unsigned short sv[4];  // [group e][row]: e * 2 + (0: row g8, 1: row g8 + 8)
-        uint8_t zv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) { sv[i] = s_nx[i]; zv[i] = z_nx[i]; }
-        if (kc + 1 < NC) meta_fetch(t, kc + 1, s_nx, z_nx);
-        else meta_fetch(t + 1, 0, s_nx, z_nx);
         // After a timeout every wait is skipped; the loop still runs to the end.
         if (!dead && !mbar_wait_bounded(full_bar(s), ph, abort_flag)) {
             *abort_flag = 1;
             record_status(status, W4_ERR_DEVICE_TIMEOUT);
             dead = true;
         }
+        const int mslot = (t - t0) % nms;
+        const unsigned short* msc = reinterpret_cast<const unsigned short*>(smem + L.meta + mslot * L.mslot);
+        const uint8_t* mzp = smem + L.meta + mslot * L.mslot + 32 * G;
         if (!dead) {
             const unsigned char* st = smem + L.ring + s * GV_STAGE_BYTES + wofs;
 #pragma unroll
@@ -261,9 +264,10 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
                     float r[4];
                     gv_group_mma(A, B, xrow + gi * 128, xoff, xlane, r);
                     const float4 cs = *reinterpret_cast<const float4*>(corr + gi * GV_MAXM + 2 * c);
-                    const float fza = (float)zv[2 * e], fzb = (float)zv[2 * e + 1];
-                    const float fsa = __half2float(__ushort_as_half(sv[2 * e]));
-                    const float fsb = __half2float(__ushort_as_half(sv[2 * e + 1]));
+                    // rows g8 + 8 of a half tile (N % 16 == 8) hold stale values; never stored
+                    const float fza = (float)mzp[g8 * G + gi], fzb = (float)mzp[(g8 + 8) * G + gi];
+                    const float fsa = __half2float(__ushort_as_half(msc[g8 * G + gi]));
+                    const float fsb = __half2float(__ushort_as_half(msc[(g8 + 8) * G + gi]));
                     acc[0] = fmaf(fsa, r[0] - fmaf(fza, cs.y, cs.x), acc[0]);  // row g8,   col 2c
                     acc[1] = fmaf(fsa, r[1] - fmaf(fza, cs.w, cs.z), acc[1]);  // row g8,   col 2c+1
                     acc[2] = fmaf(fsb, r[2] - fmaf(fzb, cs.y, cs.x), acc[2]);  // row g8+8, col 2c
@@ -289,6 +293,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
                 last = atomicAdd(&cnt[slot], 1) == GV_CWARPS - 1;
             }
             last = __shfl_sync(0xffffffffu, last, 0);
+            if (lane == 0) mbar_arrive(meta_empty(mslot));  // this warp is done with the tile's metadata
             if (last) {
                 __threadfence_block();
                 for (int o = lane; o < 16 * M; o += 32) {
