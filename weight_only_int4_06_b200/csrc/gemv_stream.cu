@@ -9,8 +9,9 @@
 //    so every output is finished inside one CTA (no split-K workspace, no cluster barrier).
 //  * A producer warp streams the packed tile through a GV_STAGES-deep shared-memory ring with
 //    TMA: one stage is 16 rows x 4096 k (32 KB; for K = 4096 the whole tile, one contiguous
-//    block of HBM).  With static weights it starts before the preceding kernel has finished
-//    (programmatic dependent launch).
+//    block of HBM).  A tile's scales and zero points are one contiguous block of each array and
+//    ride on the tile's first stage as two bulk copies.  With static weights the producer starts
+//    before the preceding kernel has finished (programmatic dependent launch).
 //  * Sixteen consumer warps take two groups of 128 each per stage and run mma.sync m16n8k16 with
 //    the 16 weight rows as the A operand and the (up to 8) activation rows as B.  Dequantisation
 //    is one LOP3 per two weights: the operands are the raw fp16 values 1024+q (low nibble of a
@@ -23,10 +24,13 @@
 //    in fp32.
 //  * The activations are staged once per CTA with each 8-k chunk as
 //    [x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16], so one 16-byte shared load yields the B
-//    fragments of the two MMAs that consume one packed word.
-//  * At the end of a tile every warp parks its partial sums in shared memory; the last warp to
-//    finish the tile (a shared counter) adds the sixteen partials in warp order and writes Y, so
-//    no warp waits for the others (deterministic, no CTA-wide barrier in the main loop).
+//    fragments of the two MMAs that consume one packed word.  Lanes whose B column is not an
+//    activation row read a block of zeros instead (no predication in the inner loop).
+//  * At the end of a tile every consumer warp parks its partial sums in a shared slot and moves
+//    on; a reducer warp adds the sixteen partials in warp order (deterministic) and writes Y, so
+//    the stage ring never waits for a reduction.
+//  * The kernel is instantiated per activation-row bound MT (1, 2, 4, 8): columns >= MT of the
+//    MMA fragments are never folded or parked.
 #include <mutex>
 
 #include "common.cuh"
@@ -37,23 +41,24 @@ namespace w4 {
 
 constexpr int GV_CWARPS = 16;                        // consumer warps
 constexpr int GV_GPW = 2;                            // groups per warp per stage
-constexpr int GV_THREADS = 32 * (GV_CWARPS + 1);     // + one producer warp
+constexpr int GV_PWARP = GV_CWARPS;                  // producer warp
+constexpr int GV_RWARP = GV_CWARPS + 1;              // reducer warp
+constexpr int GV_THREADS = 32 * (GV_CWARPS + 2);
 constexpr int GV_SG = GV_CWARPS * GV_GPW;            // groups per stage (32)
 constexpr int GV_ROWB = GV_SG * 64;                  // bytes of one row in a stage (2 KB)
 constexpr uint32_t GV_STAGE_BYTES = 16 * GV_ROWB;    // 32 KB of packed codes
 constexpr int GV_STAGES = 4;
 constexpr int GV_MAXM = 8;
-constexpr int GV_TSLOTS = GV_STAGES + 2;             // tiles whose partials may be pending at once
+constexpr int GV_TSLOTS = 6;                         // tiles whose partials may be pending at once
 
 struct GvLayout {
-    uint32_t ring, meta, mslot, nmslot, xs, corr, red, cnt, bars, total;
+    uint32_t ring, meta, mslot, nmslot, xs, xzero, corr, red, bars, total;
 };
 
-// A tile's metadata (16 rows x G scales, then 16 rows x G zero points) is one contiguous block of
-// each array, so it travels as two bulk copies into a per-tile slot of 48 G bytes.  The producer
-// runs at most GV_STAGES stages ahead of the slowest consumer, so ceil(GV_STAGES / stages per
-// tile) + 1 slots let it refill a slot without waiting.
-__host__ __device__ inline GvLayout gv_layout(int M, int K) {
+// A tile's metadata (16 rows x G scales, then 16 rows x G zero points) lands in a per-tile slot
+// of 48 G bytes.  The producer runs at most GV_STAGES stages ahead of the slowest consumer, so
+// ceil(GV_STAGES / stages per tile) + 1 slots let it refill a slot without waiting.
+__host__ __device__ inline GvLayout gv_layout(int MT, int M, int K) {
     GvLayout L;
     const uint32_t G = (uint32_t)(K / 128);
     const uint32_t NC = (G + GV_SG - 1) / GV_SG;
@@ -63,11 +68,12 @@ __host__ __device__ inline GvLayout gv_layout(int M, int K) {
     L.mslot = 48u * G;
     L.nmslot = need < (uint32_t)GV_TSLOTS ? need : (uint32_t)GV_TSLOTS;
     L.xs = L.meta + L.nmslot * L.mslot;
-    L.corr = L.xs + (uint32_t)M * (uint32_t)(K + 8) * 2;                 // float2 [G][8]
-    L.red = L.corr + G * GV_MAXM * 8;                                   // [slot][warp][16][M] fp32
-    L.cnt = L.red + (uint32_t)GV_TSLOTS * GV_CWARPS * 16 * (uint32_t)M * 4;
-    L.bars = (L.cnt + GV_TSLOTS * 4 + 7) & ~7u;                          // full, empty, meta_empty
-    L.total = L.bars + (2 * GV_STAGES + GV_TSLOTS) * 8 + 8;
+    L.xzero = L.xs + (uint32_t)M * (uint32_t)(K + 8) * 2;               // one group of zeros
+    L.corr = L.xzero + 256;                                             // float2 [G][8]
+    L.red = L.corr + G * GV_MAXM * 8;                                   // [slot][warp][16][MT] fp32
+    L.bars = L.red + (uint32_t)GV_TSLOTS * GV_CWARPS * 16 * (uint32_t)MT * 4;
+    // full, empty [GV_STAGES]; meta_empty, tile_full, red_empty [GV_TSLOTS]; abort flag
+    L.total = L.bars + (2 * GV_STAGES + 3 * GV_TSLOTS) * 8 + 8;
     return L;
 }
 
@@ -88,15 +94,14 @@ __device__ __forceinline__ void gv_named_barrier() {
 
 // One group (16 rows x 128 k) of the current stage: raw MMA sums for this thread's C fragment.
 __device__ __forceinline__ void gv_group_mma(const uint4 A, const uint4 B, const __half* xg, const int (&xoff)[4],
-                                             bool xlane, float (&r)[4]) {
+                                             float (&r)[4]) {
     float c0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, c1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     const uint32_t wA[4] = {A.x, A.y, A.z, A.w};
     const uint32_t wB[4] = {B.x, B.y, B.z, B.w};
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const uint32_t a = wA[j], b = wB[j], a8 = a >> 8, b8 = b >> 8;
-        uint4 xf = make_uint4(0u, 0u, 0u, 0u);
-        if (xlane) xf = *reinterpret_cast<const uint4*>(xg + xoff[j]);
+        const uint4 xf = *reinterpret_cast<const uint4*>(xg + xoff[j]);
         float(&cc)[4] = (j & 1) ? c1 : c0;  // two independent accumulation chains
         mma_16816(cc, lop3_and_or(a, 0x000F000Fu, 0x64006400u), lop3_and_or(b, 0x000F000Fu, 0x64006400u),
                   lop3_and_or(a, 0x00F000F0u, 0x64006400u), lop3_and_or(b, 0x00F000F0u, 0x64006400u), xf.x, xf.y);
@@ -107,6 +112,7 @@ __device__ __forceinline__ void gv_group_mma(const uint4 A, const uint4 B, const
     for (int e = 0; e < 4; ++e) r[e] = c0[e] + c1[e];
 }
 
+template <int MT>
 __global__ void __launch_bounds__(GV_THREADS, 1)
     gemv_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __half* __restrict__ X,
                        const unsigned short* __restrict__ scales, const uint8_t* __restrict__ zeros,
@@ -116,7 +122,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     // TMA destinations need an aligned base: round up (the launch reserves 1 KB of slack)
     unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                            ~uintptr_t(1023));
-    const GvLayout L = gv_layout(M, K);
+    const GvLayout L = gv_layout(MT, M, K);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = K >> 7;
@@ -124,39 +130,44 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     const int t0 = (int)(((int64_t)blockIdx.x * n_tiles) / gridDim.x);
     const int t1 = (int)(((int64_t)(blockIdx.x + 1) * n_tiles) / gridDim.x);
     const int n_units = (t1 - t0) * NC;
-    auto full_bar = [&](int s) { return sbase + L.bars + 8 * s; };
-    auto empty_bar = [&](int s) { return sbase + L.bars + 8 * (GV_STAGES + s); };
-    auto meta_empty = [&](int slot) { return sbase + L.bars + 8 * (2 * GV_STAGES + slot); };
     const int nms = (int)L.nmslot;
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bars + 8 * (2 * GV_STAGES + GV_TSLOTS));
-    int* cnt = reinterpret_cast<int*>(smem + L.cnt);
+    const uint32_t bar0 = sbase + L.bars;
+    auto full_bar = [&](int s) { return bar0 + 8 * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8 * (GV_STAGES + s); };
+    auto meta_empty = [&](int i) { return bar0 + 8 * (2 * GV_STAGES + i); };
+    auto tile_full = [&](int i) { return bar0 + 8 * (2 * GV_STAGES + GV_TSLOTS + i); };
+    auto red_empty = [&](int i) { return bar0 + 8 * (2 * GV_STAGES + 2 * GV_TSLOTS + i); };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.bars + 8 * (2 * GV_STAGES + 3 * GV_TSLOTS));
+    float* red = reinterpret_cast<float*>(smem + L.red);
 
     if (tid == 0) {
         for (int s = 0; s < GV_STAGES; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), GV_CWARPS);
         }
-        for (int i = 0; i < GV_TSLOTS; ++i) cnt[i] = 0;
-        for (int i = 0; i < nms; ++i) mbar_init(meta_empty(i), GV_CWARPS);
+        for (int i = 0; i < GV_TSLOTS; ++i) {
+            mbar_init(meta_empty(i), GV_CWARPS);
+            mbar_init(tile_full(i), 32 * GV_CWARPS);  // every consumer lane arrives after parking
+            mbar_init(red_empty(i), 1);
+        }
         *abort_flag = 0;
         fence_mbarrier_init();
     }
     __syncthreads();
     pdl_launch_dependents();  // the next kernel may claim SM space and start its own weight stream
 
-    if (warp == GV_CWARPS) {
+    if (warp == GV_PWARP) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&tmW);
             if (!weights_early) pdl_wait();
-            int issued = 0, ti = 0, kc = 0, s = 0;
-            uint32_t ph = 0;
+            int issued = 0, t = t0, kc = 0, s = 0, ms = 0;
+            uint32_t ph = 0, mph = 0;
             for (int u = 0; u < n_units; ++u) {
                 // The ring is full: from here on progress depends on the consumers, who first
                 // wait for the preceding kernel; start the bounded waits only after that point.
                 if (u == GV_STAGES && weights_early) pdl_wait();
-                const int t = t0 + ti, slot = ti % nms;
-                if ((kc == 0 && !mbar_wait_bounded(meta_empty(slot), ((ti / nms) & 1) ^ 1, abort_flag)) ||
+                if ((kc == 0 && !mbar_wait_bounded(meta_empty(ms), mph ^ 1, abort_flag)) ||
                     !mbar_wait_bounded(empty_bar(s), ph ^ 1, abort_flag)) {
                     *abort_flag = 1;
                     record_status(status, W4_ERR_DEVICE_TIMEOUT);
@@ -164,24 +175,59 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
                 }
                 uint32_t sb = 0, zb = 0;
                 const int64_t mofs = (int64_t)t * 16 * G;  // first metadata entry of the tile
+                const uint32_t mdst = L.meta + ms * L.mslot;
                 if (kc == 0) {  // the tile's metadata rides on its first stage
                     const int rows = N - t * 16 < 16 ? N - t * 16 : 16;  // 8 or 16 (N % 8 == 0)
                     sb = (uint32_t)(rows * 2 * G);
                     zb = (uint32_t)(rows * G) & ~15u;
                     if (zb != (uint32_t)(rows * G))  // 8 trailing zero points (8 rows, odd G): plain copy
-                        *reinterpret_cast<uint2*>(smem + L.meta + slot * L.mslot + 32 * G + zb) =
+                        *reinterpret_cast<uint2*>(smem + mdst + 32 * G + zb) =
                             *reinterpret_cast<const uint2*>(zeros + mofs + zb);
                 }
                 mbar_arrive_expect_tx(full_bar(s), GV_STAGE_BYTES + sb + zb);
                 tma_load_2d(sbase + L.ring + s * GV_STAGE_BYTES, &tmW, kc * (GV_ROWB / 8), t * 16, full_bar(s));
-                if (sb) bulk_load_1d(sbase + L.meta + slot * L.mslot, scales + mofs, sb, full_bar(s));
-                if (zb) bulk_load_1d(sbase + L.meta + slot * L.mslot + 32 * G, zeros + mofs, zb, full_bar(s));
+                if (sb) bulk_load_1d(sbase + mdst, scales + mofs, sb, full_bar(s));
+                if (zb) bulk_load_1d(sbase + mdst + 32 * G, zeros + mofs, zb, full_bar(s));
                 ++issued;
-                if (++kc == NC) { kc = 0; ++ti; }
+                if (++kc == NC) {
+                    kc = 0;
+                    ++t;
+                    if (++ms == nms) { ms = 0; mph ^= 1; }
+                }
                 if (++s == GV_STAGES) { s = 0; ph ^= 1; }
             }
             for (int u = issued - GV_STAGES; u < issued; ++u)  // no loads in flight at exit
                 if (u >= 0) mbar_wait_bounded(full_bar(u % GV_STAGES), (u / GV_STAGES) & 1, nullptr, 200000000ull);
+        }
+        return;
+    }
+
+    if (warp == GV_RWARP) {
+        // ------------------------------------------------------------ reducer: Y, in warp order
+        pdl_wait();  // Y may be read by the preceding kernel
+        int rs = 0;
+        uint32_t rph = 0;
+        for (int t = t0; t < t1; ++t) {
+            if (!mbar_wait_bounded(tile_full(rs), rph, abort_flag)) {
+                *abort_flag = 1;
+                record_status(status, W4_ERR_DEVICE_TIMEOUT);
+                break;
+            }
+            const float* rsl = red + (size_t)rs * (GV_CWARPS * 16 * MT);
+#pragma unroll
+            for (int o0 = 0; o0 < 16 * MT; o0 += 32) {
+                const int o = o0 + lane, row = o / MT, m = o - row * MT;
+                const int n = t * 16 + row;
+                if (o < 16 * MT && m < M && n < N) {
+                    float sum = 0.0f;
+#pragma unroll
+                    for (int w = 0; w < GV_CWARPS; ++w) sum += rsl[w * (16 * MT) + o];
+                    Y[(int64_t)m * N + n] = __float2half_rn(sum);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(red_empty(rs));
+            if (++rs == GV_TSLOTS) { rs = 0; rph ^= 1; }
         }
         return;
     }
@@ -224,54 +270,63 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
             corr[(ch >> 4) * GV_MAXM + m] =
                 make_float2(__ll2float_rn(lo + hi) * 0x1p-14f, __ll2float_rn(lo + 16 * hi) * 0x1p-24f);
     }
-    for (int idx = tid; idx < G * GV_MAXM; idx += 32 * GV_CWARPS)  // activation rows >= M
-        if (idx % GV_MAXM >= M) corr[idx] = make_float2(0.0f, 0.0f);
+    if (tid < 16) reinterpret_cast<uint4*>(smem + L.xzero)[tid] = make_uint4(0u, 0u, 0u, 0u);
+    // corr entries of activation rows >= M stay unset: they only feed columns that are never stored
     gv_named_barrier();
 
     const int g8 = lane >> 2, c = lane & 3;
-    float* red = reinterpret_cast<float*>(smem + L.red);
-    const bool xlane = g8 < M;  // B column g8 holds activation row g8
-    const __half* xrow = xs + (int64_t)(xlane ? g8 : 0) * RS;
+    // B column g8 holds activation row g8; other lanes read one group of zeros at every k
+    const bool xlane = g8 < M;
+    const __half* xbase = xlane ? xs + (int64_t)g8 * RS : reinterpret_cast<const __half*>(smem + L.xzero);
+    const int xstride = xlane ? 128 : 0;
     int xoff[4];  // swizzled offset (halves) of word j's chunk within a group, for this lane
 #pragma unroll
     for (int j = 0; j < 4; ++j) xoff[j] = gv_swz(c * 4 + j) * 8;
+    const int moa = g8 * G, mob = (g8 + 8) * G;  // this thread's two rows in a metadata slot
 
     // this thread's W bytes inside a stage: row g8 / g8 + 8, group (warp + 16 e), 16 bytes at 16 c
     const uint32_t wofs = (uint32_t)(g8 * GV_ROWB + warp * 64 + c * 16);
-    int s = 0, kc = 0, t = t0;
-    uint32_t ph = 0;
+    int s = 0, kc = 0, ms = 0, rs = 0;
+    uint32_t ph = 0, rph = 0;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // rows (g8, g8+8) x cols (2c, 2c+1)
     bool dead = false;
     for (int u = 0; u < n_units; ++u) {
-        const int gA = kc * GV_SG + warp;
         // After a timeout every wait is skipped; the loop still runs to the end.
         if (!dead && !mbar_wait_bounded(full_bar(s), ph, abort_flag)) {
             *abort_flag = 1;
             record_status(status, W4_ERR_DEVICE_TIMEOUT);
             dead = true;
         }
-        const int mslot = (t - t0) % nms;
-        const unsigned short* msc = reinterpret_cast<const unsigned short*>(smem + L.meta + mslot * L.mslot);
-        const uint8_t* mzp = smem + L.meta + mslot * L.mslot + 32 * G;
         if (!dead) {
             const unsigned char* st = smem + L.ring + s * GV_STAGE_BYTES + wofs;
+            const unsigned short* msc = reinterpret_cast<const unsigned short*>(smem + L.meta + ms * L.mslot);
+            const uint8_t* mzp = smem + L.meta + ms * L.mslot + 32 * G;
+            const int gA = kc * GV_SG + warp;
+            // groups gA and gA + 16; the last stage of a tile may hold fewer than 32 groups
+            const int ng = gA + GV_CWARPS < G ? 2 : (gA < G ? 1 : 0);
 #pragma unroll
             for (int e = 0; e < GV_GPW; ++e) {
-                const int gi = gA + e * GV_CWARPS;
-                if (gi < G) {
+                if (e < ng) {
+                    const int gi = gA + e * GV_CWARPS;
                     const uint4 A = *reinterpret_cast<const uint4*>(st + e * (GV_CWARPS * 64));
                     const uint4 B = *reinterpret_cast<const uint4*>(st + e * (GV_CWARPS * 64) + 8 * GV_ROWB);
                     float r[4];
-                    gv_group_mma(A, B, xrow + gi * 128, xoff, xlane, r);
-                    const float4 cs = *reinterpret_cast<const float4*>(corr + gi * GV_MAXM + 2 * c);
-                    // rows g8 + 8 of a half tile (N % 16 == 8) hold stale values; never stored
-                    const float fza = (float)mzp[g8 * G + gi], fzb = (float)mzp[(g8 + 8) * G + gi];
-                    const float fsa = __half2float(__ushort_as_half(msc[g8 * G + gi]));
-                    const float fsb = __half2float(__ushort_as_half(msc[(g8 + 8) * G + gi]));
-                    acc[0] = fmaf(fsa, r[0] - fmaf(fza, cs.y, cs.x), acc[0]);  // row g8,   col 2c
-                    acc[1] = fmaf(fsa, r[1] - fmaf(fza, cs.w, cs.z), acc[1]);  // row g8,   col 2c+1
-                    acc[2] = fmaf(fsb, r[2] - fmaf(fzb, cs.y, cs.x), acc[2]);  // row g8+8, col 2c
-                    acc[3] = fmaf(fsb, r[3] - fmaf(fzb, cs.w, cs.z), acc[3]);  // row g8+8, col 2c+1
+                    gv_group_mma(A, B, xbase + gi * xstride, xoff, r);
+                    // rows g8 + 8 of a half tile (N % 16 == 8) hold stale metadata; never stored
+                    const float fza = (float)mzp[moa + gi], fzb = (float)mzp[mob + gi];
+                    const float fsa = __half2float(__ushort_as_half(msc[moa + gi]));
+                    const float fsb = __half2float(__ushort_as_half(msc[mob + gi]));
+                    if (MT == 1) {
+                        const float2 cs = corr[gi * GV_MAXM + 2 * c];
+                        acc[0] = fmaf(fsa, r[0] - fmaf(fza, cs.y, cs.x), acc[0]);  // row g8,   col 2c
+                        acc[2] = fmaf(fsb, r[2] - fmaf(fzb, cs.y, cs.x), acc[2]);  // row g8+8, col 2c
+                    } else {
+                        const float4 cs = *reinterpret_cast<const float4*>(corr + gi * GV_MAXM + 2 * c);
+                        acc[0] = fmaf(fsa, r[0] - fmaf(fza, cs.y, cs.x), acc[0]);  // row g8,   col 2c
+                        acc[1] = fmaf(fsa, r[1] - fmaf(fza, cs.w, cs.z), acc[1]);  // row g8,   col 2c+1
+                        acc[2] = fmaf(fsb, r[2] - fmaf(fzb, cs.y, cs.x), acc[2]);  // row g8+8, col 2c
+                        acc[3] = fmaf(fsb, r[3] - fmaf(fzb, cs.w, cs.z), acc[3]);  // row g8+8, col 2c+1
+                    }
                 }
             }
         }
@@ -279,56 +334,37 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         if (lane == 0) mbar_arrive(empty_bar(s));
         if (++s == GV_STAGES) { s = 0; ph ^= 1; }
         if (++kc == NC) {
-            // tile done: park this warp's partials; the last warp of the tile adds all sixteen
-            const int slot = (t - t0) % GV_TSLOTS;
-            float* rs = red + (size_t)slot * (GV_CWARPS * 16 * M);
-            float* mine = rs + warp * (16 * M);
-            const int m0 = 2 * c, m1 = 2 * c + 1;
-            if (m0 < M) { mine[g8 * M + m0] = acc[0]; mine[(g8 + 8) * M + m0] = acc[2]; }
-            if (m1 < M) { mine[g8 * M + m1] = acc[1]; mine[(g8 + 8) * M + m1] = acc[3]; }
-            __syncwarp();
-            int last = 0;
-            if (lane == 0) {
-                __threadfence_block();
-                last = atomicAdd(&cnt[slot], 1) == GV_CWARPS - 1;
+            // tile done: release its metadata, park this warp's partials for the reducer
+            if (lane == 0) mbar_arrive(meta_empty(ms));
+            if (++ms == nms) ms = 0;
+            if (!dead && !mbar_wait_bounded(red_empty(rs), rph ^ 1, abort_flag)) {
+                *abort_flag = 1;
+                record_status(status, W4_ERR_DEVICE_TIMEOUT);
+                dead = true;
             }
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (lane == 0) mbar_arrive(meta_empty(mslot));  // this warp is done with the tile's metadata
-            if (last) {
-                __threadfence_block();
-                for (int o = lane; o < 16 * M; o += 32) {
-                    float sum = 0.0f;
-#pragma unroll
-                    for (int w = 0; w < GV_CWARPS; ++w) sum += rs[w * (16 * M) + o];  // warp order
-                    const int row = o / M, m = o - row * M;
-                    const int n = t * 16 + row;
-                    if (n < N) Y[(int64_t)m * N + n] = __float2half_rn(sum);
-                }
-                __syncwarp();
-                if (lane == 0) cnt[slot] = 0;
-            }
+            float* mine = red + (size_t)rs * (GV_CWARPS * 16 * MT) + warp * (16 * MT);
+            if (2 * c < MT) { mine[g8 * MT + 2 * c] = acc[0]; mine[(g8 + 8) * MT + 2 * c] = acc[2]; }
+            if (2 * c + 1 < MT) { mine[g8 * MT + 2 * c + 1] = acc[1]; mine[(g8 + 8) * MT + 2 * c + 1] = acc[3]; }
+            mbar_arrive(tile_full(rs));  // every lane: its own stores are released with it
+            if (++rs == GV_TSLOTS) { rs = 0; rph ^= 1; }
             acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
             kc = 0;
-            ++t;
         }
     }
 }
 
 // ------------------------------------------------------------------------------------ host side
+static int gv_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+
 size_t gemv_stream_smem(int64_t M, int64_t K) {
     if (M < 1 || M > GV_MAXM || K > 65536) return SIZE_MAX;  // activations are staged whole
-    return (size_t)gv_layout((int)M, (int)K).total + 1024;
+    return (size_t)gv_layout(gv_mt(M), (int)M, (int)K).total + 1024;
 }
 
-cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                               const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, bool weights_static,
-                               int* status, cudaStream_t stream) {
-    CUtensorMap tm;  // packed rows as 8-byte elements: a 256-element box is 2 KB (4096 k) of a row
-    if (!make_tensor_map_2d(&tm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)(K / 16), (uint64_t)N,
-                            GV_ROWB / 8, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    const size_t smem = gemv_stream_smem(M, K);
-    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+template <int MT>
+static cudaError_t gv_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                             const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, bool weights_static,
+                             int* status, cudaStream_t stream) {
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
     int dev = 0;
@@ -336,7 +372,7 @@ cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t 
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&]() {
-        attr_err[dev] = cudaFuncSetAttribute(gemv_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err[dev] = cudaFuncSetAttribute(gemv_stream_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              227 * 1024);
     });
     if (attr_err[dev] != cudaSuccess) return attr_err[dev];
@@ -346,16 +382,32 @@ cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3(GV_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = gemv_stream_smem(M, K);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = weights_static ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_stream_kernel, tm, reinterpret_cast<const __half*>(X),
+    return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<MT>, tm, reinterpret_cast<const __half*>(X),
                               reinterpret_cast<const unsigned short*>(scales), zeros, reinterpret_cast<__half*>(Y),
                               (int)M, (int)N, (int)K, n_tiles, weights_static ? 1 : 0, status);
+}
+
+cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                               const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, bool weights_static,
+                               int* status, cudaStream_t stream) {
+    CUtensorMap tm;  // packed rows as 8-byte elements: a 256-element box is 2 KB (4096 k) of a row
+    if (!make_tensor_map_2d(&tm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)(K / 16), (uint64_t)N,
+                            GV_ROWB / 8, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    if (gemv_stream_smem(M, K) > 227 * 1024) return cudaErrorInvalidValue;
+    switch (gv_mt(M)) {
+        case 1: return gv_launch<1>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
+        case 2: return gv_launch<2>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
+        case 4: return gv_launch<4>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
+        default: return gv_launch<8>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
+    }
 }
 
 }  // namespace w4
