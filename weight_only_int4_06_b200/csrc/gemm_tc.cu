@@ -71,8 +71,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     using C = TcCfg<DEQ, MT>;
     constexpr int S = C::kStages;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~uintptr_t(1023));
+    unsigned char* smem = smem_align1024(smem_raw);
     const uint32_t sbase = smem_u32(smem);
     auto a_addr = [&](int s) { return sbase + s * C::kStage; };
     auto b_addr = [&](int s) { return sbase + s * C::kStage + C::kA; };

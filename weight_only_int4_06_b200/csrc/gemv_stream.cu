@@ -120,8 +120,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
                        int* status) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // TMA destinations need an aligned base: round up (the launch reserves 1 KB of slack)
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~uintptr_t(1023));
+    unsigned char* smem = smem_align1024(smem_raw);
     const GvLayout L = gv_layout(MT, M, K);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

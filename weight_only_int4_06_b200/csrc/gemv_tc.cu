@@ -76,8 +76,7 @@ __global__ void __launch_bounds__(GT_THREADS, 2)
                    __half* __restrict__ Y, int M, int N, int K, int splits, int gps, int weights_early,
                    int* status) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~uintptr_t(1023));
+    unsigned char* smem = smem_align1024(smem_raw);
     const GtLayout L = gt_layout(gps);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

@@ -13,6 +13,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
 }
 
+// Dynamic shared memory rounded up to a 1024-byte boundary by pointer arithmetic: a round trip
+// through an integer would hide the address space from the compiler and make every access through
+// the result a generic one (64-bit address math, generic loads).
+__device__ __forceinline__ unsigned char* smem_align1024(unsigned char* raw) {
+    return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
