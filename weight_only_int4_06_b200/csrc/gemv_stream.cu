@@ -17,11 +17,12 @@
 //    is one LOP3 per two weights: the operands are the raw fp16 values 1024+q (low nibble of a
 //    byte) and 1024+16q (high nibble); activations that meet high nibbles are staged pre-multiplied
 //    by 1/16, and the constant offsets and the zero point are removed per group in fp32 with the
-//    exact activation sums
+//    activation sums
 //        sum_k x_k (q_k - z) = raw - 1024 (Sl + Sh') - z (Sl + 16 Sh'),
-//    Sl = sum of x over low-nibble slots, Sh' = sum of the staged x/16 over high-nibble slots
-//    (both exact integer sums of 2^-24 units).  The group's fp16 scale then multiplies that sum
-//    in fp32.
+//    Sl = sum of x over low-nibble slots, Sh' = sum of the staged x/16 over high-nibble slots,
+//    both summed in fp32 in a fixed tree order (deterministic; their rounding is of the same order
+//    as the MMA's own fp32 accumulation of the offset operands).  The group's fp16 scale then
+//    multiplies that sum in fp32.
 //  * The activations are staged once per CTA with each 8-k chunk as
 //    [x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16], so one 16-byte shared load yields the B
 //    fragments of the two MMAs that consume one packed word.  Lanes whose B column is not an
@@ -81,12 +82,13 @@ __host__ __device__ inline GvLayout gv_layout(int MT, int M, int K) {
 // makes the B-fragment loads of a warp bank-conflict free for up to 8 activation rows.
 __device__ __forceinline__ int gv_swz(int ch) { return ch ^ ((ch >> 2) & 2); }
 
-// An fp16 value as a signed integer number of 2^-24 units (exact; |value| <= 2^40 units).
-__device__ __forceinline__ long long half_units(uint32_t h) {
-    const uint32_t e = (h >> 10) & 0x1Fu, m = h & 0x3FFu;
-    const long long mag = e == 0 ? (long long)m : ((long long)(m | 0x400u) << (e - 1));
-    return (h & 0x8000u) ? -mag : mag;
+// Sum of the two fp16 halves of a packed pair, in fp32.
+__device__ __forceinline__ float half2_sum(uint32_t h) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    return f.x + f.y;
 }
+
+constexpr int GV_XILP = 4;  // activation chunks each consumer thread loads before using any
 
 __device__ __forceinline__ void gv_named_barrier() {
     asm volatile("bar.sync 1, %0;" ::"n"(32 * GV_CWARPS) : "memory");
@@ -232,42 +234,51 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     }
 
     // ---------------------------------------------------------------- consumers
-    // Stage the activations and, in the same pass, the exact per-group sums that remove the
-    // operand offsets: every fp16 value (and every staged x/16) is an integer number of 2^-24
-    // units, so the sums are exact 64-bit integer additions.  The 16 chunks of one group sit in
-    // 16 consecutive lanes, which reduce them with shuffles.
+    // Stage the activations and, in the same pass, the per-group sums that remove the operand
+    // offsets.  Each thread first issues all its loads of a round (one memory round trip per
+    // round instead of one per chunk).  The 16 chunks of one group sit in 16 consecutive lanes,
+    // which reduce them with shuffles in a fixed order.
     pdl_wait();  // the activations may be produced by the preceding kernel
     __half* xs = reinterpret_cast<__half*>(smem + L.xs);
     float2* corr = reinterpret_cast<float2*>(smem + L.corr);
     const __half2 sixteenth = __float2half2_rn(0.0625f);
     const int cpr = K / 8;  // 8-k chunks per activation row
     const int RS = K + 8;   // staged row stride in halves (16 bytes of padding)
-    for (int i = tid; i < M * cpr; i += 32 * GV_CWARPS) {  // uniform trip count per 16-lane half
-        const int m = i / cpr, ch = i - m * cpr;
-        const uint4 r = ldg_cached(X + (int64_t)i * 8);  // rows are contiguous
-        uint4 p;
-        p.x = __byte_perm(r.x, r.z, 0x5410);         // x0, x4
-        uint32_t h = __byte_perm(r.x, r.z, 0x7632);  // x1, x5
-        __half2 hh = __hmul2(*reinterpret_cast<__half2*>(&h), sixteenth);
-        p.y = *reinterpret_cast<uint32_t*>(&hh);
-        p.z = __byte_perm(r.y, r.w, 0x5410);  // x2, x6
-        h = __byte_perm(r.y, r.w, 0x7632);    // x3, x7
-        hh = __hmul2(*reinterpret_cast<__half2*>(&h), sixteenth);
-        p.w = *reinterpret_cast<uint32_t*>(&hh);
-        *reinterpret_cast<uint4*>(xs + (int64_t)m * RS + gv_swz(ch) * 8) = p;
-        long long lo = half_units(p.x & 0xFFFFu) + half_units(p.x >> 16) + half_units(p.z & 0xFFFFu) +
-                       half_units(p.z >> 16);
-        long long hi = half_units(p.y & 0xFFFFu) + half_units(p.y >> 16) + half_units(p.w & 0xFFFFu) +
-                       half_units(p.w >> 16);
-        const unsigned half_mask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;  // both halves may differ
+    const int xtot = M * cpr;
+    const unsigned half_mask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;  // the two halves may differ
+    for (int base = 0; base < xtot; base += 32 * GV_CWARPS * GV_XILP) {
+        uint4 raw[GV_XILP];
 #pragma unroll
-        for (int o = 8; o; o >>= 1) {
-            lo += __shfl_xor_sync(half_mask, lo, o);
-            hi += __shfl_xor_sync(half_mask, hi, o);
+        for (int v = 0; v < GV_XILP; ++v) {
+            const int i = base + v * 32 * GV_CWARPS + tid;
+            if (i < xtot) raw[v] = ldg_cached(X + (int64_t)i * 8);  // rows are contiguous
         }
-        if ((ch & 15) == 0)  // C = 1024 (Sl + Sh'), S = Sl + 16 Sh', one rounding each
-            corr[(ch >> 4) * GV_MAXM + m] =
-                make_float2(__ll2float_rn(lo + hi) * 0x1p-14f, __ll2float_rn(lo + 16 * hi) * 0x1p-24f);
+#pragma unroll
+        for (int v = 0; v < GV_XILP; ++v) {
+            const int i = base + v * 32 * GV_CWARPS + tid;
+            if (i >= xtot) break;  // uniform per 16-lane half: xtot is a multiple of 16
+            const int m = i / cpr, ch = i - m * cpr;
+            const uint4 r = raw[v];
+            uint4 p;
+            p.x = __byte_perm(r.x, r.z, 0x5410);         // x0, x4
+            uint32_t h = __byte_perm(r.x, r.z, 0x7632);  // x1, x5
+            __half2 hh = __hmul2(*reinterpret_cast<__half2*>(&h), sixteenth);
+            p.y = *reinterpret_cast<uint32_t*>(&hh);
+            p.z = __byte_perm(r.y, r.w, 0x5410);  // x2, x6
+            h = __byte_perm(r.y, r.w, 0x7632);    // x3, x7
+            hh = __hmul2(*reinterpret_cast<__half2*>(&h), sixteenth);
+            p.w = *reinterpret_cast<uint32_t*>(&hh);
+            *reinterpret_cast<uint4*>(xs + (int64_t)m * RS + gv_swz(ch) * 8) = p;
+            float lo = half2_sum(p.x) + half2_sum(p.z);  // staged low-nibble partners
+            float hi = half2_sum(p.y) + half2_sum(p.w);  // staged high-nibble partners (x/16)
+#pragma unroll
+            for (int o = 8; o; o >>= 1) {
+                lo += __shfl_xor_sync(half_mask, lo, o);
+                hi += __shfl_xor_sync(half_mask, hi, o);
+            }
+            if ((ch & 15) == 0)  // C = 1024 (Sl + Sh'), S = Sl + 16 Sh'
+                corr[(ch >> 4) * GV_MAXM + m] = make_float2(1024.0f * (lo + hi), fmaf(16.0f, hi, lo));
+        }
     }
     if (tid < 16) reinterpret_cast<uint4*>(smem + L.xzero)[tid] = make_uint4(0u, 0u, 0u, 0u);
     // corr entries of activation rows >= M stay unset: they only feed columns that are never stored
