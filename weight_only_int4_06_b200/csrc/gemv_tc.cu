@@ -60,10 +60,9 @@ __host__ __device__ inline GtLayout gt_layout(int gps) {
     return L;
 }
 
-__device__ __forceinline__ long long gt_half_units(uint32_t h) {  // exact multiple of 2^-24
-    const uint32_t e = (h >> 10) & 0x1Fu, m = h & 0x3FFu;
-    const long long mag = e == 0 ? (long long)m : ((long long)(m | 0x400u) << (e - 1));
-    return (h & 0x8000u) ? -mag : mag;
+__device__ __forceinline__ float gt_half2_sum(uint32_t h) {  // sum of the two halves, in fp32
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    return f.x + f.y;
 }
 
 __device__ __forceinline__ void gt_deq_barrier() {
@@ -175,42 +174,7 @@ __global__ void __launch_bounds__(GT_THREADS, 2)
         const int r = q * 32 + lane;  // tile row = TMEM lane
         const int n = n0 + r;
         const int dt = tid - 128;     // 0..255
-        // stage the activations (exact group sums in the same pass) and this row's metadata
-        pdl_wait();
-        const int cpw = ng * 16;  // 8-k chunks in this split
-        const __half2 sixteenth = __float2half2_rn(0.0625f);
-        for (int i = dt; i < 16 * cpw; i += 256) {  // uniform trip count per 16-lane half
-            const int m = i / cpw, ch = i - m * cpw;
-            unsigned char* dst = smem + L.xs + ch * 256 + (m < 8 ? m * 16 : 128 + (m - 8) * 16);
-            uint4 p = make_uint4(0u, 0u, 0u, 0u);
-            if (m < M) {
-                const uint4 v = ldg_cached(X + (int64_t)m * K + (int64_t)gb * 128 + ch * 8);
-                p.x = __byte_perm(v.x, v.z, 0x5410);         // x0, x4
-                uint32_t t = __byte_perm(v.x, v.z, 0x7632);  // x1, x5
-                __half2 hh = __hmul2(*reinterpret_cast<__half2*>(&t), sixteenth);
-                p.y = *reinterpret_cast<uint32_t*>(&hh);
-                p.z = __byte_perm(v.y, v.w, 0x5410);         // x2, x6
-                t = __byte_perm(v.y, v.w, 0x7632);           // x3, x7
-                hh = __hmul2(*reinterpret_cast<__half2*>(&t), sixteenth);
-                p.w = *reinterpret_cast<uint32_t*>(&hh);
-            }
-            *reinterpret_cast<uint4*>(dst) = p;
-            if (m < 8) {  // group sums for the 8 possible activation rows (zero for rows >= M)
-                long long lo = gt_half_units(p.x & 0xFFFFu) + gt_half_units(p.x >> 16) +
-                               gt_half_units(p.z & 0xFFFFu) + gt_half_units(p.z >> 16);
-                long long hi = gt_half_units(p.y & 0xFFFFu) + gt_half_units(p.y >> 16) +
-                               gt_half_units(p.w & 0xFFFFu) + gt_half_units(p.w >> 16);
-                const unsigned half_mask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;
-#pragma unroll
-                for (int o = 8; o; o >>= 1) {
-                    lo += __shfl_xor_sync(half_mask, lo, o);
-                    hi += __shfl_xor_sync(half_mask, hi, o);
-                }
-                if ((ch & 15) == 0)
-                    corr[(ch >> 4) * GT_MAXM + m] =
-                        make_float2(__ll2float_rn(lo + hi) * 0x1p-14f, __ll2float_rn(lo + 16 * hi) * 0x1p-24f);
-            }
-        }
+        // This row's metadata does not depend on the preceding kernel: fetch it first.
         float sv[GT_MAXG / 2], zv[GT_MAXG / 2];  // this row's scale / zero for groups h, h+2, ...
 #pragma unroll
         for (int k = 0; k < GT_MAXG / 2; ++k) {
@@ -222,6 +186,55 @@ __global__ void __launch_bounds__(GT_THREADS, 2)
                 zv[k] = (float)__ldg(zeros + (int64_t)n * G + gb + g);
             }
         }
+        // Stage the activations of this split with the group sums that remove the operand
+        // offsets (fp32, fixed tree order); B rows M..15 are zero.
+        const int cpw = ng * 16;  // 8-k chunks in this split
+        for (int i = dt; i < cpw * (16 - M); i += 256) {
+            const int m = M + i / cpw, ch = i % cpw;
+            *reinterpret_cast<uint4*>(smem + L.xs + ch * 256 + (m < 8 ? m * 16 : 128 + (m - 8) * 16)) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        for (int m = M; m < GT_MAXM; ++m)
+            for (int g = dt; g < ng; g += 256) corr[g * GT_MAXM + m] = make_float2(0.0f, 0.0f);
+        pdl_wait();  // the activations may be produced by the preceding kernel
+        const __half2 sixteenth = __float2half2_rn(0.0625f);
+        const unsigned half_mask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;
+        constexpr int XILP = 2;
+        for (int base = 0; base < M * cpw; base += 256 * XILP) {  // uniform per 16-lane half
+            uint4 raw[XILP];
+#pragma unroll
+            for (int v = 0; v < XILP; ++v) {
+                const int i = base + v * 256 + dt;
+                if (i < M * cpw) raw[v] = ldg_cached(X + (int64_t)(i / cpw) * K + (int64_t)gb * 128 + (i % cpw) * 8);
+            }
+#pragma unroll
+            for (int v = 0; v < XILP; ++v) {
+                const int i = base + v * 256 + dt;
+                if (i >= M * cpw) break;
+                const int m = i / cpw, ch = i - m * cpw;
+                const uint4 r4 = raw[v];
+                uint4 p;
+                p.x = __byte_perm(r4.x, r4.z, 0x5410);         // x0, x4
+                uint32_t t = __byte_perm(r4.x, r4.z, 0x7632);  // x1, x5
+                __half2 hh = __hmul2(*reinterpret_cast<__half2*>(&t), sixteenth);
+                p.y = *reinterpret_cast<uint32_t*>(&hh);
+                p.z = __byte_perm(r4.y, r4.w, 0x5410);         // x2, x6
+                t = __byte_perm(r4.y, r4.w, 0x7632);           // x3, x7
+                hh = __hmul2(*reinterpret_cast<__half2*>(&t), sixteenth);
+                p.w = *reinterpret_cast<uint32_t*>(&hh);
+                *reinterpret_cast<uint4*>(smem + L.xs + ch * 256 + m * 16) = p;  // m < 8
+                float lo = gt_half2_sum(p.x) + gt_half2_sum(p.z);
+                float hi = gt_half2_sum(p.y) + gt_half2_sum(p.w);
+#pragma unroll
+                for (int o = 8; o; o >>= 1) {
+                    lo += __shfl_xor_sync(half_mask, lo, o);
+                    hi += __shfl_xor_sync(half_mask, hi, o);
+                }
+                if ((ch & 15) == 0)  // C = 1024 (Sl + Sh'), S = Sl + 16 Sh'
+                    corr[(ch >> 4) * GT_MAXM + m] = make_float2(1024.0f * (lo + hi), fmaf(16.0f, hi, lo));
+            }
+        }
+        fence_proxy_async_shared();  // staged activations: generic-proxy writes read by the MMA
         gt_deq_barrier();  // x staged (the MMA thread reads it after the first a_full)
 
         float acc[GT_MAXM];
@@ -266,8 +279,6 @@ __global__ void __launch_bounds__(GT_THREADS, 2)
                 const int c = (g & 1) * 4 + cc;
                 c4[cc] = *reinterpret_cast<const uint4*>(row + ((c ^ (r & 7)) << 4));
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(w_empty(s));
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t regs[32];
@@ -290,7 +301,10 @@ __global__ void __launch_bounds__(GT_THREADS, 2)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(a_full(a));
+            if (lane == 0) {
+                mbar_arrive(w_empty(s));  // every lane's stage loads were consumed above
+                mbar_arrive(a_full(a));
+            }
             if (k > 0) fold(g - 2, k - 1);
         }
         if (k > 0) fold(h + 2 * (k - 1), k - 1);
@@ -331,22 +345,21 @@ __global__ void __launch_bounds__(GT_THREADS, 2)
 }
 
 // ------------------------------------------------------------------------------------ host side
+// One wave: at most two CTAs per SM (each fits half an SM), as many (tile, split) CTAs as
+// possible, fewest splits among equals.  Shapes whose splits would exceed GT_MAXG groups each
+// or 16 CTAs per cluster are not planned.
 bool plan_gemv_tc(int64_t M, int64_t N, int64_t K, GemvTcPlan* plan) {
     if (M < 1 || M > GT_MAXM || K < 128 || N < 8) return false;
     const int G = (int)(K / 128);
     const int n_tiles = (int)((N + GT_ROWS - 1) / GT_ROWS);
-    const int slots = 2 * device_sm_count();
-    double best = -1.0;
-    for (int gps = 1; gps <= GT_MAXG; ++gps) {
-        const int S = (G + gps - 1) / gps;
-        if (S > 16) continue;
-        const int g2 = (G + S - 1) / S;  // balanced groups per split for this split count
-        if (g2 != gps) continue;
-        const long ctas = (long)n_tiles * S;
-        const long waves = (ctas + slots - 1) / slots;
-        const double util = (double)ctas / (double)(waves * slots);
-        if (util > best + 1e-9) {
-            best = util;
+    const long slots = 2L * device_sm_count();
+    long best = -1;
+    for (int S = 1; S <= 16 && S <= G; ++S) {
+        const int gps = (G + S - 1) / S;
+        if (gps > GT_MAXG || (long)n_tiles * S > slots) continue;
+        if ((G + gps - 1) / gps != S) continue;  // every split gets at least one group
+        if ((long)n_tiles * S > best) {
+            best = (long)n_tiles * S;
             plan->splits = S;
             plan->gps = gps;
             plan->n_tiles = n_tiles;
