@@ -34,6 +34,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from weight_only_int4_06_b200 import synth  # noqa: E402
+from weight_only_int4_06_b200.ncu_traffic import load_traffic  # noqa: E402
 
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -346,15 +347,19 @@ def run_gemm_bench(args, rank, world, local, kind, with_extras=True):
         achieved = wl.flops_per_step / (ms_per_step * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": None,
+                "frac": round(achieved / peak, 4), "traffic": load_traffic("prefill"),
                 "peak_note": "dense bf16 burst (fp16 dense rate is the same on B200)"}
         kern = "tc_gemm_kernel<DEQ> (tcgen05 + TMEM + TMA)"
     else:
         achieved = wl.bytes_per_step / (ms_per_step * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": None}
-        kern = "skinny_kernel (mma.sync GEMV, cluster split-K)"
+                "frac": round(achieved / peak, 4),
+                "traffic": load_traffic("decode") if kind == "decode" else None}
+        kern = ("gemv_stream_kernel<MT> (persistent TMA ring, mma.sync, metadata by bulk copy)"
+                if kind == "decode" else
+                "gemv_stream_kernel<MT> for M <= 8, skinny_kernel (cluster split-K) above")
+    roof["traffic_unit"] = "DRAM bytes per step (ncu, see profiles/)"
     roof["peak_source"] = peaks["source"]
     roof["kernel"] = kern
     roof["algorithmic_bytes_per_step"] = wl.bytes_per_step
