@@ -312,8 +312,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
             const unsigned short* msc = reinterpret_cast<const unsigned short*>(smem + L.meta + ms * L.mslot);
             const uint8_t* mzp = smem + L.meta + ms * L.mslot + 32 * G;
             const int gA = kc * GV_SG + warp;
-            // groups gA and gA + 16; the last stage of a tile may hold fewer than 32 groups
-            const int ng = gA + GV_CWARPS < G ? 2 : (gA < G ? 1 : 0);
+            // groups gA + GV_CWARPS e; the last stage of a tile may hold fewer than GV_SG groups
+            const int ng = gA >= G ? 0 : min(GV_GPW, (G - gA + GV_CWARPS - 1) / GV_CWARPS);
 #pragma unroll
             for (int e = 0; e < GV_GPW; ++e) {
                 if (e < ng) {
