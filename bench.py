@@ -182,6 +182,7 @@ class GemmWorkload:
             need = B.w4_gemm_workspace_size(M, N, K)
             ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
             self.layers.append(dict(M=M, K=K, N=N, X=Xd, Xh=torch.from_numpy(X).pin_memory(),
+                                    Yh=torch.empty((M, N), dtype=torch.float16).pin_memory(),
                                     copies=copies, Y=Y, ws=ws))
         torch.cuda.synchronize()
         self.bytes_per_step = sum(gemm_bytes(M, K, N) for (M, K, N) in cases)
@@ -197,13 +198,16 @@ class GemmWorkload:
             self.B.w4_gemm(L["X"], p, sc, z, out=L["Y"], workspace=L["ws"], variant=self.variant)
 
     def run_step_host(self, step):
-        """The same step through the public API with host (pinned) activations and results."""
+        """The same step through the public API with host (pinned) activations and results:
+        every layer copies its X in and its Y out on the stream; the step ends when the stream
+        has drained (the results are then readable on the host)."""
+        import torch
         s = step % self.n_sets
-        outs = []
         for L in self.layers:
             p, sc, z = L["copies"][s]
-            outs.append(self.B.w4_gemm(L["Xh"], p, sc, z))
-        return outs
+            self.B.w4_gemm(L["Xh"], p, sc, z, out=L["Yh"])
+        torch.cuda.current_stream().synchronize()
+        return [L["Yh"] for L in self.layers]
 
     def h2d_d2h_bytes(self):
         return (sum(2 * M * K for (M, K, N) in self.cases), sum(2 * M * N for (M, K, N) in self.cases))

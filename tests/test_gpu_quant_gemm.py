@@ -225,6 +225,40 @@ def test_gemm_host_buffers_match_device():
     assert np.array_equal(Yh.numpy().view(np.uint16), Yd.view(np.uint16))
 
 
+def test_gemm_async_pinned_host_out_on_a_side_stream():
+    """Pinned host X and out: copies and kernel are enqueued on the given stream, no sync."""
+    X, p, s, z = oracle_case(26, 3, 4096, 1032)
+    Yd = gpu_gemm(X, p, s, z)
+    Xh = torch.from_numpy(X).pin_memory()
+    out = torch.full((3, 1032), 7.0, dtype=torch.float16).pin_memory()
+    side = torch.cuda.Stream()
+    r = B.w4_gemm(Xh, dev(p.view(np.int32)), dev(s), dev(z), out=out, stream=side)
+    assert r is out
+    side.synchronize()
+    assert np.array_equal(out.numpy().view(np.uint16), Yd.view(np.uint16))
+    with pytest.raises(ValueError):  # a pageable host out is refused
+        B.w4_gemm(Xh, dev(p.view(np.int32)), dev(s), dev(z), out=torch.empty((3, 1032), dtype=torch.float16))
+
+
+def test_gemm_misaligned_metadata_falls_back_or_reports():
+    """The GEMV bulk-copies metadata and needs 16-byte aligned scales/zeros: w4_gemm falls back to
+    the skinny kernel, the explicit GEMV family reports W4_ERR_ALIGN."""
+    X, p, s, z = oracle_case(27, 1, 4096, 264)
+    ref = oracle.gemm(X, p, s, z)
+    sbuf = torch.zeros(s.size + 8, dtype=torch.float16, device="cuda")
+    zbuf = torch.zeros(z.size + 16, dtype=torch.uint8, device="cuda")
+    s_mis = sbuf[1:1 + s.size].view(s.shape)
+    z_mis = zbuf[3:3 + z.size].view(z.shape)
+    s_mis.copy_(dev(s))
+    z_mis.copy_(dev(z))
+    Xd, pd = dev(X), dev(p.view(np.int32))
+    Y = B.w4_gemm(Xd, pd, s_mis, z_mis)
+    assert_close(Y.cpu().numpy(), ref, "auto with misaligned metadata")
+    with pytest.raises(B.W4Error) as e:
+        B.w4_gemm(Xd, pd, s_mis, z_mis, variant=B.VARIANT_GEMV)
+    assert e.value.status == 3  # W4_ERR_ALIGN
+
+
 # ------------------------------------------------------------------ forced kernel families
 @pytest.mark.parametrize("M,K,N", [(1, 128, 8), (7, 256, 136), (128, 384, 256), (129, 4096, 264),
                                    (300, 1152, 520), (512, 8192, 1024), (64, 11008, 4096)])

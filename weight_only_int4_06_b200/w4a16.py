@@ -109,30 +109,58 @@ def w4_gemm_workspace_size(M: int, N: int, K: int, group: int = 128) -> int:
 def w4_gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
             group: int = 128, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
             variant: int = VARIANT_AUTO, stream=None) -> torch.Tensor:
-    """Y = X . dequant(W)^T.  A host (CPU) X is copied to the device and Y copied back."""
+    """Y = X . dequant(W)^T.
+
+    Device X: Y is written to `out` (or a new device tensor) on `stream`; nothing synchronises.
+    Host X (ideally pinned): X is copied to the device on `stream`.  If `out` is a pinned host
+    tensor, Y is copied into it asynchronously on `stream` and the call returns at once (`out` is
+    valid after the stream synchronises); otherwise the call synchronises and returns Y on the host.
+    """
     host = not X.is_cuda
-    if host:
-        dev = packed.device
-        Xd = X.to(dev, non_blocking=True)
-    else:
-        Xd = X
-    M, K = Xd.shape
+    dev = packed.device
+    M, K = X.shape
     N = packed.shape[0]
-    if out is None:
-        out = torch.empty((M, N), dtype=torch.float16, device=Xd.device)
-    need = w4_gemm_workspace_size(M, N, K, group)
-    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
-        workspace = torch.empty(need, dtype=torch.uint8, device=Xd.device)
-    ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
-    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    st = lib().w4_gemm_ex(_dev(Xd, torch.float16, "X"), M, N, K, _dev(packed, torch.int32, "packed"),
-                          _dev(scales, torch.float16, "scales"), _dev(zeros, torch.uint8, "zeros"),
-                          group, _dev(out, torch.float16, "Y"), ws_ptr, ws_bytes, variant,
-                          _stream(stream))
-    _check(st, "w4_gemm")
-    if host:
-        return out.to("cpu", non_blocking=False)
-    return out
+    if stream is None:
+        tstream = torch.cuda.current_stream(dev)
+    elif isinstance(stream, torch.cuda.Stream):
+        tstream = stream
+    else:
+        tstream = torch.cuda.ExternalStream(stream, device=dev)
+    host_out = out is not None and not out.is_cuda
+    if host_out and (not host or not out.is_pinned()):
+        raise ValueError("a host `out` must be pinned and needs a host X")
+    with torch.cuda.stream(tstream):
+        Xd = X.to(dev, non_blocking=True) if host else X
+        Yd = out if (out is not None and not host_out) else torch.empty((M, N), dtype=torch.float16,
+                                                                          device=dev)
+        need = _ws_size(M, N, K, group)
+        if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        st = lib().w4_gemm_ex(_dev(Xd, torch.float16, "X"), M, N, K, _dev(packed, torch.int32, "packed"),
+                              _dev(scales, torch.float16, "scales"), _dev(zeros, torch.uint8, "zeros"),
+                              group, _dev(Yd, torch.float16, "Y"), ws_ptr, ws_bytes, variant,
+                              ctypes.c_void_p(tstream.cuda_stream))
+        _check(st, "w4_gemm")
+        if host_out:
+            if out.dtype != torch.float16 or tuple(out.shape) != (M, N):
+                raise ValueError("out must be float16 [M, N]")
+            out.copy_(Yd, non_blocking=True)
+            return out
+        if host:
+            return Yd.to("cpu", non_blocking=False)
+    return Yd
+
+
+_ws_cache: dict = {}
+
+
+def _ws_size(M: int, N: int, K: int, group: int) -> int:
+    key = (M, N, K, group)
+    if key not in _ws_cache:
+        _ws_cache[key] = w4_gemm_workspace_size(M, N, K, group)
+    return _ws_cache[key]
 
 
 def awq_workspace_size(T: int, N: int, K: int, group: int = 128, n_alpha: int = 20) -> int:
