@@ -74,10 +74,14 @@ def fp16_round_up(x32: np.ndarray) -> np.ndarray:
 # ----------------------------------------------------------------------------
 # Round-to-nearest group quantisation (one row group of 128 along K)
 # ----------------------------------------------------------------------------
-def quantize_rtn(W: np.ndarray, act_scale: np.ndarray | None = None, group: int = GROUP):
+def quantize_rtn(W: np.ndarray, act_scale: np.ndarray | None = None, group: int = GROUP,
+                 clip_ratio: np.ndarray | None = None):
     """Group-wise asymmetric INT4 round-to-nearest quantisation of W (or of W * diag(act_scale)).
 
     W: [N, K] fp16.  act_scale: [K] (cast to fp32) or None.
+    clip_ratio: [N, K/group] fp32 or None.  When given, both ends of each group's zero-inclusive
+    range are multiplied by the ratio (one fp32 multiply each) before the scale and zero point
+    are derived; codes of weights outside the shrunk range saturate at 0 or 15.
     Returns (q [N, K] uint8 codes, scales [N, K/group] fp16, zeros [N, K/group] uint8).
     """
     W = np.asarray(W, dtype=np.float16)
@@ -92,6 +96,10 @@ def quantize_rtn(W: np.ndarray, act_scale: np.ndarray | None = None, group: int 
 
     lo = np.minimum(vg.min(axis=2), np.float32(0))
     hi = np.maximum(vg.max(axis=2), np.float32(0))
+    if clip_ratio is not None:
+        r = np.asarray(clip_ratio, dtype=np.float32).reshape(N, G)
+        lo = lo * r
+        hi = hi * r
     d = hi - lo  # fp32, rounded to nearest
     s32 = d / np.float32(QMAX)  # fp32 IEEE division
     s16 = fp16_round_up(s32)
@@ -227,3 +235,49 @@ def awq_scale_search(X: np.ndarray, W: np.ndarray, n_alpha: int = 20, group: int
         assert Y_q.shape == (T, N)
     best = int(np.argmin(mse))  # first occurrence = lowest index among the minima
     return mse, best, s_all[best].copy(), s_all
+
+
+# ----------------------------------------------------------------------------
+# AWQ clip search: per-group shrinking of the quantisation range
+# ----------------------------------------------------------------------------
+def clip_ratio_grid(n_ratios: int = 10) -> np.ndarray:
+    """Shrink ratios r_j = 1 - j/20, j = 0 .. n_ratios-1 (fp32; 1.0 first)."""
+    return np.array([1.0 - j / 20.0 for j in range(n_ratios)], dtype=np.float64).astype(np.float32)
+
+
+def awq_clip_search(X: np.ndarray, W: np.ndarray, act_scale: np.ndarray | None = None,
+                    n_ratios: int = 10, group: int = GROUP):
+    """Choose, for every (row n, group g), the range shrink ratio with the least output error.
+
+    The layer sees activations X diag(1/a) and quantises W diag(a) (a = act_scale, or 1).  For
+    ratio r_j the group is quantised with its range shrunk by r_j (quantize_rtn's clip_ratio) and
+        err[n, g, j] = sum_t ( sum_{k in g} (X[t,k] / a_k) * (w_hat[n,k] - v[n,k]) )^2
+    with v = W a as the quantiser sees it (fp32) and w_hat = (q - z) * s16 (fp64); the output
+    error of the group's own columns, every group on its own.  best = lowest j among the minima.
+    Returns (err [N, G, R] fp64, best [N, G] int64, packed, scales, zeros) where the last three
+    are the quantisation of W diag(a) with every group's best ratio.
+    """
+    X64 = np.asarray(X).astype(np.float64)
+    W16 = np.asarray(W, dtype=np.float16)
+    N, K = W16.shape
+    G = K // group
+    v = W16.astype(np.float32)
+    if act_scale is not None:
+        a32 = np.asarray(act_scale).astype(np.float32)
+        v = v * a32[None, :]
+        Xs = X64 / a32.astype(np.float64)[None, :]
+    else:
+        Xs = X64
+    v64 = v.astype(np.float64)
+    ratios = clip_ratio_grid(n_ratios)
+    err = np.empty((N, G, n_ratios), dtype=np.float64)
+    for j, r in enumerate(ratios):
+        q, s16, z = quantize_rtn(W16, act_scale, group, np.full((N, G), r, dtype=np.float32))
+        E = dequantize(pack_nibbles(q), s16, z, group) - v64  # [N, K]
+        for g in range(G):
+            cols = slice(g * group, (g + 1) * group)
+            out = Xs[:, cols] @ E[:, cols].T  # [T, N]: the group's contribution to the output error
+            err[:, g, j] = np.sum(out * out, axis=0)
+    best = np.argmin(err, axis=2)  # first occurrence = lowest j among the minima
+    q, s16, z = quantize_rtn(W16, act_scale, group, ratios[best])
+    return err, best, pack_nibbles(q), s16, z
