@@ -473,6 +473,48 @@ def bench_awq(world, peaks, reps=2):
             "flops": flops}
 
 
+FP32_FMA_PER_CLK_PER_SM = 128     # B200 SM: 4 partitions x 32 fp32 FMA lanes
+B200_SMS, B200_MAX_SM_MHZ = 148, 1965
+
+
+def bench_awq_clip(world, peaks, reps=3, n_ratios=10):
+    """awq_clip_search on X_calib [65536, 4096], W [4096, 4096], 10 ratios, with an AWQ scale."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    X, W = synth.awq_case()
+    Xd = torch.from_numpy(X).cuda()
+    Wd = torch.from_numpy(W).cuda()
+    T, K = X.shape
+    N = W.shape[0]
+    a = torch.ones(K, dtype=torch.float32, device="cuda")
+    ws = torch.empty(B.awq_clip_workspace_size(T, N, K, 128, n_ratios), dtype=torch.uint8, device="cuda")
+    B.awq_clip_search(Xd, Wd, a, n_ratios, workspace=ws)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        B.awq_clip_search(Xd, Wd, a, n_ratios, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    t = max_over_ranks(min(times), world)
+    G = K // 128
+    flops = 2 * T * K * 128 + N * G * n_ratios * 2 * 128 * 128  # Gram blocks + quadratic forms
+    tf = flops / (t * 1e-3) / 1e12
+    peak = 2 * FP32_FMA_PER_CLK_PER_SM * B200_SMS * B200_MAX_SM_MHZ * 1e6 / 1e12
+    del Xd, Wd, ws
+    torch.cuda.empty_cache()
+    return {"kernel": "gram_partial + gram_reduce + clip_kernel (fp32 CUDA cores)",
+            "T": T, "K": K, "N": N, "n_ratios": n_ratios, "ms": round(t, 3), "TFLOPs": round(tf, 2),
+            "bound": "alu", "peak_tflops": round(peak, 1),
+            "peak_note": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x 1965 MHz (unit counts and max clock)",
+            "alu_frac": round(tf / peak, 3), "flops": flops}
+
+
 def other_rows(args, world, peaks, l2):
     import torch
     rows = {}
@@ -486,6 +528,7 @@ def other_rows(args, world, peaks, l2):
     del pre
     torch.cuda.empty_cache()
     rows["awq"] = bench_awq(world, peaks)
+    rows["awq_clip"] = bench_awq_clip(world, peaks)
     return rows
 
 

@@ -198,6 +198,38 @@ w4_status awq_scale_search_noalloc(const uint16_t* X, int64_t T, const uint16_t*
                                    int64_t K, int group, int n_alpha, double* mse,
                                    int32_t* best_idx, float* best_s, void* stream);
 
+/* Bytes of device workspace awq_clip_search needs for this problem. */
+w4_status awq_clip_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_ratios,
+                                  size_t* bytes);
+
+/*
+ * awq_clip_search -- AWQ's activation-guided clipping: per (row, group), shrink the quantisation
+ * range when that lowers the layer's output error on calibration data, then quantise.
+ *
+ * Follows "GPTQ, AWQ and the rules of post-training quantization", section "AWQ: find the one
+ * percent that matters" (the layer computes the same function when W's channel j is multiplied
+ * by s_j and X's channel j divided by s_j) and the AutoAWQ pages' "activation-guided clipping",
+ * which give no grid.  Reading: ratio r_j = 1 - j/20 (double, rounded once to fp32),
+ * j = 0 .. n_ratios-1, multiplies both ends of a group's zero-inclusive range (one fp32 multiply
+ * each) before w4_quantize_pack's scale and zero point are derived; codes beyond the shrunk
+ * range saturate.  With v = W * diag(act_scale) and w_hat the dequantised codes under r_j,
+ *     err[n, g, j] = sum_t ( sum_{k in g} (X[t,k] / act_scale[k]) * (w_hat[n,k] - v[n,k]) )^2
+ * (each group's own contribution to the output error), evaluated as e'^T G_g e' with the
+ * group's Gram block G_g = X_g^T X_g in fp32; best = lowest j among the minima.
+ *
+ *   X [T, K] fp16 calibration activations (as the layer receives them before the AWQ scaling);
+ *   W [N, K] fp16; act_scale [K] fp32 (the AWQ scales) or NULL for none; n_ratios 1..10.
+ *   best_idx [N, K/group] uint8 out; err [N, K/group, n_ratios] fp32 out, or NULL;
+ *   packed / scales / zeros out: w4_quantize_pack's format for W * diag(act_scale), each group
+ *   quantised with its chosen ratio (n_ratios == 1 gives w4_quantize_pack's result exactly).
+ *   ws: device workspace of at least awq_clip_workspace_size bytes.
+ * T >= 1.  X, W, packed and act_scale 16-byte aligned.  Errors: see the conventions above.
+ */
+w4_status awq_clip_search(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K,
+                          int group, int n_ratios, const float* act_scale, uint8_t* best_idx,
+                          float* err, uint32_t* packed, uint16_t* scales, uint8_t* zeros,
+                          void* ws, size_t ws_bytes, void* stream);
+
 /*
  * w4_check_device_status -- synchronise `stream`, then read and clear the current device's
  * status word.  Returns W4_OK, W4_ERR_RANGE, W4_ERR_DEVICE_TIMEOUT, or W4_ERR_CUDA if the

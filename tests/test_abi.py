@@ -30,7 +30,8 @@ def L():
 def test_header_declares_expected_api():
     names = declared_functions()
     for n in ("w4_quantize_pack", "w4_gemm", "w4_gemm_ex", "w4_gemm_workspace_size",
-              "awq_scale_search", "awq_workspace_size", "w4_check_device_status", "w4_status_string"):
+              "awq_scale_search", "awq_workspace_size", "awq_clip_search", "awq_clip_workspace_size",
+              "w4_check_device_status", "w4_status_string"):
         assert n in names, n
 
 
@@ -93,6 +94,25 @@ def test_workspace_queries(L):
     assert L.w4_gemm_workspace_size(1, 4096, 4096, 128, None) == 1
     assert L.awq_workspace_size(256, 64, 512, 128, 0, ctypes.byref(n)) == 4
     assert L.awq_workspace_size(256, 64, 500, 128, 20, ctypes.byref(n)) == 2
+    assert L.awq_clip_workspace_size(256, 64, 512, 128, 10, ctypes.byref(n)) == 0 and n.value > 0
+    assert L.awq_clip_workspace_size(256, 64, 512, 128, 11, ctypes.byref(n)) == 4
+    assert L.awq_clip_workspace_size(256, 64, 512, 128, 0, ctypes.byref(n)) == 4
+    assert L.awq_clip_workspace_size(256, 64, 500, 128, 10, ctypes.byref(n)) == 2
+    assert L.awq_clip_workspace_size(0, 64, 512, 128, 10, ctypes.byref(n)) == 2
+
+
+def test_clip_search_rejects(L):
+    P = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(1 << 12)
+    d = P(ctypes.addressof(buf) + (-ctypes.addressof(buf) % 16))
+    args = lambda **kw: [kw.get("X", d), 64, kw.get("W", d), 64, 512, kw.get("group", 128), kw.get("R", 10), None,
+                         kw.get("best", d), None, d, d, d, kw.get("ws", d), kw.get("ws_bytes", 1 << 30), None]
+    assert L.awq_clip_search(*args(R=0)) == 4
+    assert L.awq_clip_search(*args(group=64)) == 4
+    assert L.awq_clip_search(*args(ws_bytes=16)) == 5
+    assert L.awq_clip_search(*args(X=None)) == 1
+    assert L.awq_clip_search(*args(best=None)) == 1
+    assert L.awq_clip_search(*args(W=P(d.value + 2))) == 3
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -194,6 +194,38 @@ w4_status awq_scale_search(const uint16_t* X, int64_t T, const uint16_t* W, int6
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
+static w4_status clip_check(int64_t T, int64_t N, int64_t K, int group, int n_ratios) {
+    if (group != 128 || n_ratios < 1 || n_ratios > 10) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(T, K) || !dims_ok(N, K) || T < 1 || N < 8 || K < 128 || K % group != 0 || N % 8 != 0)
+        return W4_ERR_SHAPE;
+    return W4_OK;
+}
+
+w4_status awq_clip_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_ratios, size_t* bytes) {
+    if (!bytes) return W4_ERR_NULL;
+    w4_status st = clip_check(T, N, K, group, n_ratios);
+    if (st != W4_OK) return st;
+    *bytes = awq_clip_layout(T, N, K, n_ratios).bytes;
+    return W4_OK;
+}
+
+w4_status awq_clip_search(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int group,
+                          int n_ratios, const float* act_scale, uint8_t* best_idx, float* err, uint32_t* packed,
+                          uint16_t* scales, uint8_t* zeros, void* ws, size_t ws_bytes, void* stream) {
+    w4_status st = clip_check(T, N, K, group, n_ratios);
+    if (st != W4_OK) return st;
+    if (ws_bytes < awq_clip_layout(T, N, K, n_ratios).bytes) return W4_ERR_WORKSPACE;
+    if (!X || !W || !best_idx || !packed || !scales || !zeros || !ws) return W4_ERR_NULL;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(packed) || !aligned16(ws) ||
+        (act_scale && !aligned16(act_scale)))
+        return W4_ERR_ALIGN;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_awq_clip(X, T, W, N, K, n_ratios, act_scale, best_idx, err, packed, scales, zeros, ws,
+                                    status, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 w4_status w4_check_device_status(void* stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return W4_ERR_CUDA;
     int* p = device_status_ptr();

@@ -75,4 +75,14 @@ cudaError_t launch_awq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t 
                        double* mse, int32_t* best_idx, float* best_s, void* ws, int* status,
                        cudaStream_t stream);
 
+// AWQ clip search (awq_clip.cu).  Workspace: Gram blocks, then per-split partial Gram blocks.
+struct AwqClipLayout {
+    size_t gram, part, bytes;
+    int splits;
+};
+AwqClipLayout awq_clip_layout(int64_t T, int64_t N, int64_t K, int n_ratios);
+cudaError_t launch_awq_clip(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int n_ratios,
+                            const float* act_scale, uint8_t* best_idx, float* err, uint32_t* packed,
+                            uint16_t* scales, uint8_t* zeros, void* ws, int* status, cudaStream_t stream);
+
 }  // namespace w4

@@ -32,6 +32,8 @@ SIGNATURES = {
     "awq_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_scale_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "awq_scale_search_noalloc": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P]),
+    "awq_clip_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
+    "awq_clip_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "w4_check_device_status": (_I32, [_P]),
     "w4_status_string": (ctypes.c_char_p, [_I32]),
 }
@@ -205,6 +207,39 @@ def awq_scale_search_noalloc(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20
                                         _stream(stream))
     _check(st, "awq_scale_search_noalloc")
     return mse, best, best_s
+
+
+def awq_clip_workspace_size(T: int, N: int, K: int, group: int = 128, n_ratios: int = 10) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().awq_clip_workspace_size(T, N, K, group, n_ratios, ctypes.byref(n)), "awq_clip_workspace_size")
+    return n.value
+
+
+def awq_clip_search(X: torch.Tensor, W: torch.Tensor, act_scale: torch.Tensor | None = None,
+                    n_ratios: int = 10, group: int = 128, with_err: bool = False, workspace=None, stream=None):
+    """AWQ clip search.  Returns (best_idx [N, G] uint8, err [N, G, R] fp32 or None, packed, scales,
+    zeros), all on X's device."""
+    T, K = X.shape
+    N = W.shape[0]
+    G = K // group
+    dev = X.device
+    need = awq_clip_workspace_size(T, N, K, group, n_ratios)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    best = torch.empty((N, G), dtype=torch.uint8, device=dev)
+    err = torch.empty((N, G, n_ratios), dtype=torch.float32, device=dev) if with_err else None
+    packed = torch.empty((N, K // 8), dtype=torch.int32, device=dev)
+    scales = torch.empty((N, G), dtype=torch.float16, device=dev)
+    zeros = torch.empty((N, G), dtype=torch.uint8, device=dev)
+    a = _dev(act_scale, torch.float32, "act_scale") if act_scale is not None else None
+    st = lib().awq_clip_search(_dev(X, torch.float16, "X"), T, _dev(W, torch.float16, "W"), N, K, group,
+                               n_ratios, a, ctypes.c_void_p(best.data_ptr()),
+                               ctypes.c_void_p(err.data_ptr()) if err is not None else None,
+                               ctypes.c_void_p(packed.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                               ctypes.c_void_p(zeros.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "awq_clip_search")
+    return best, err, packed, scales, zeros
 
 
 def w4_check_device_status(stream=None) -> int:
