@@ -183,6 +183,7 @@ class GemmWorkload:
             ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
             self.layers.append(dict(M=M, K=K, N=N, X=Xd, Xh=torch.from_numpy(X).pin_memory(),
                                     Yh=torch.empty((M, N), dtype=torch.float16).pin_memory(),
+                                    xs=torch.empty((M, K), dtype=torch.float16, device="cuda"),
                                     copies=copies, Y=Y, ws=ws))
         torch.cuda.synchronize()
         self.bytes_per_step = sum(gemm_bytes(M, K, N) for (M, K, N) in cases)
@@ -205,7 +206,7 @@ class GemmWorkload:
         s = step % self.n_sets
         for L in self.layers:
             p, sc, z = L["copies"][s]
-            self.B.w4_gemm(L["Xh"], p, sc, z, out=L["Yh"])
+            self.B.w4_gemm_host(L["Xh"], p, sc, z, L["Yh"], L["xs"], L["Y"], workspace=L["ws"])
         torch.cuda.current_stream().synchronize()
         return [L["Yh"] for L in self.layers]
 

@@ -141,6 +141,22 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
                      const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y,
                      void* ws, size_t ws_bytes, int variant, void* stream);
 
+/*
+ * w4_gemm_host -- w4_gemm with X and Y in host memory.
+ *
+ * Enqueues on `stream`: one copy of X_host [M, K] into the caller's device buffer x_dev, the
+ * GEMM of w4_gemm_ex (same `variant`) into the caller's device buffer y_dev [M, N], and one copy
+ * of y_dev into Y_host.  Returns once enqueued; Y_host holds the result when the stream has
+ * drained.  With pinned host buffers both copies are asynchronous; with pageable ones the CUDA
+ * runtime may stage them synchronously.  x_dev and y_dev: 16-byte aligned device memory the
+ * caller owns (the library still allocates nothing).  Errors: as w4_gemm_ex, plus W4_ERR_CUDA if
+ * a copy cannot be enqueued.
+ */
+w4_status w4_gemm_host(const uint16_t* X_host, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                       const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y_host,
+                       uint16_t* x_dev, uint16_t* y_dev, void* ws, size_t ws_bytes, int variant,
+                       void* stream);
+
 /* Bytes of device workspace awq_scale_search needs for this problem. */
 w4_status awq_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha,
                              size_t* bytes);

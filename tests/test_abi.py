@@ -29,7 +29,7 @@ def L():
 
 def test_header_declares_expected_api():
     names = declared_functions()
-    for n in ("w4_quantize_pack", "w4_gemm", "w4_gemm_ex", "w4_gemm_workspace_size",
+    for n in ("w4_quantize_pack", "w4_gemm", "w4_gemm_ex", "w4_gemm_host", "w4_gemm_workspace_size",
               "awq_scale_search", "awq_workspace_size", "awq_clip_search", "awq_clip_workspace_size",
               "w4_check_device_status", "w4_status_string"):
         assert n in names, n

@@ -240,6 +240,21 @@ def test_gemm_async_pinned_host_out_on_a_side_stream():
         B.w4_gemm(Xh, dev(p.view(np.int32)), dev(s), dev(z), out=torch.empty((3, 1032), dtype=torch.float16))
 
 
+def test_gemm_host_entry_point_one_call():
+    """w4_gemm_host: H2D of X, the GEMM and D2H of Y enqueued by one C call on a side stream."""
+    X, p, s, z = oracle_case(28, 5, 1152, 520)
+    Yd = gpu_gemm(X, p, s, z)
+    Xh = torch.from_numpy(X).pin_memory()
+    out = torch.zeros((5, 520), dtype=torch.float16).pin_memory()
+    xs = torch.empty((5, 1152), dtype=torch.float16, device="cuda")
+    ys = torch.empty((5, 520), dtype=torch.float16, device="cuda")
+    side = torch.cuda.Stream()
+    B.w4_gemm_host(Xh, dev(p.view(np.int32)), dev(s), dev(z), out, xs, ys, stream=side)
+    side.synchronize()
+    assert np.array_equal(out.numpy().view(np.uint16), Yd.view(np.uint16))
+    assert_close(out.numpy(), oracle.gemm(X, p, s, z), "w4_gemm_host")
+
+
 def test_gemm_misaligned_metadata_falls_back_or_reports():
     """The GEMV bulk-copies metadata and needs 16-byte aligned scales/zeros: w4_gemm falls back to
     the skinny kernel, the explicit GEMV family reports W4_ERR_ALIGN."""

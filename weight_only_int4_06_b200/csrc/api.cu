@@ -163,6 +163,24 @@ w4_status w4_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint
                       stream);
 }
 
+w4_status w4_gemm_host(const uint16_t* X_host, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                       const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y_host, uint16_t* x_dev,
+                       uint16_t* y_dev, void* ws, size_t ws_bytes, int variant, void* stream) {
+    if (group != 128) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0)
+        return W4_ERR_SHAPE;
+    if (M == 0 || N == 0) return W4_OK;
+    if (!Y_host || !y_dev || (K > 0 && (!X_host || !x_dev))) return W4_ERR_NULL;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (K > 0 && cudaMemcpyAsync(x_dev, X_host, (size_t)M * (size_t)K * 2, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return W4_ERR_CUDA;
+    const w4_status st = w4_gemm_ex(x_dev, M, N, K, packed, scales, zeros, group, y_dev, ws, ws_bytes, variant, stream);
+    if (st != W4_OK) return st;
+    if (cudaMemcpyAsync(Y_host, y_dev, (size_t)M * (size_t)N * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return W4_ERR_CUDA;
+    return W4_OK;
+}
+
 static w4_status awq_check(int64_t T, int64_t N, int64_t K, int group, int n_alpha) {
     if (group != 128 || n_alpha < 1 || n_alpha > 64) return W4_ERR_UNSUPPORTED;
     if (!dims_ok(T, K) || !dims_ok(N, K) || T < 1 || N < 8 || K < 128 || K % group != 0 || N % 8 != 0)

@@ -29,6 +29,7 @@ SIGNATURES = {
     "w4_gemm_workspace_size": (_I32, [_I64, _I64, _I64, _I32, ctypes.POINTER(_SZ)]),
     "w4_gemm": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ, _P]),
     "w4_gemm_ex": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ, _I32, _P]),
+    "w4_gemm_host": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P, _P, _P, _P, _SZ, _I32, _P]),
     "awq_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_scale_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "awq_scale_search_noalloc": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P]),
@@ -153,6 +154,32 @@ def w4_gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: 
         if host:
             return Yd.to("cpu", non_blocking=False)
     return Yd
+
+
+def w4_gemm_host(X_host: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                 out_host: torch.Tensor, x_dev: torch.Tensor, y_dev: torch.Tensor, group: int = 128,
+                 workspace: torch.Tensor | None = None, variant: int = VARIANT_AUTO, stream=None) -> torch.Tensor:
+    """One C-ABI call: copy X_host to x_dev, GEMM into y_dev, copy y_dev to out_host, all enqueued on
+    `stream` (no synchronisation; out_host is valid once the stream has drained).  Host tensors
+    should be pinned; x_dev / y_dev are caller-owned device staging buffers."""
+    M, K = X_host.shape
+    N = packed.shape[0]
+    for t, name, shape in ((X_host, "X_host", (M, K)), (out_host, "out_host", (M, N))):
+        if t.is_cuda or t.dtype != torch.float16 or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise ValueError(f"{name} must be a contiguous float16 host tensor of shape {shape}")
+    if x_dev.numel() < M * K or y_dev.numel() < M * N:
+        raise ValueError("x_dev / y_dev too small")
+    need = _ws_size(M, N, K, group)
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        raise ValueError("workspace too small: see w4_gemm_workspace_size")
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib().w4_gemm_host(X_host.data_ptr(), M, N, K, _dev(packed, torch.int32, "packed"),
+                            _dev(scales, torch.float16, "scales"), _dev(zeros, torch.uint8, "zeros"), group,
+                            out_host.data_ptr(), _dev(x_dev, torch.float16, "x_dev"),
+                            _dev(y_dev, torch.float16, "y_dev"), ws_ptr, ws_bytes, variant, _stream(stream))
+    _check(st, "w4_gemm_host")
+    return out_host
 
 
 _ws_cache: dict = {}
