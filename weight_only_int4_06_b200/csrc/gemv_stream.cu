@@ -7,7 +7,7 @@
 // Design (sm_100a):
 //  * Persistent: one CTA per SM; CTA c owns a contiguous range of 16-row tiles over the whole K,
 //    so every output is finished inside one CTA (no split-K workspace, no cluster barrier).
-//  * A producer warp streams the packed tile through a GV_STAGES-deep shared-memory ring with
+//  * A producer warp streams the packed tile through a shared-memory ring of stages with
 //    TMA: one stage is 16 rows x 4096 k (32 KB; for K = 4096 the whole tile, one contiguous
 //    block of HBM).  A tile's scales and zero points are one contiguous block of each array and
 //    ride on the tile's first stage as two bulk copies.  With static weights the producer starts
@@ -40,15 +40,9 @@
 
 namespace w4 {
 
-constexpr int GV_CWARPS = 16;                        // consumer warps
-constexpr int GV_GPW = 2;                            // groups per warp per stage
-constexpr int GV_PWARP = GV_CWARPS;                  // producer warp
-constexpr int GV_RWARP = GV_CWARPS + 1;              // reducer warp
-constexpr int GV_THREADS = 32 * (GV_CWARPS + 2);
-constexpr int GV_SG = GV_CWARPS * GV_GPW;            // groups per stage (32)
+constexpr int GV_SG = 32;                            // groups per stage
 constexpr int GV_ROWB = GV_SG * 64;                  // bytes of one row in a stage (2 KB)
 constexpr uint32_t GV_STAGE_BYTES = 16 * GV_ROWB;    // 32 KB of packed codes
-constexpr int GV_STAGES = 4;
 constexpr int GV_MAXM = 8;
 constexpr int GV_TSLOTS = 6;                         // tiles whose partials may be pending at once
 
@@ -56,25 +50,42 @@ struct GvLayout {
     uint32_t ring, meta, mslot, nmslot, xs, xzero, corr, red, bars, total;
 };
 
+// Two shapes of CTA: one per SM with 16 consumer warps and a 4-stage ring, or two per SM (each
+// within half an SM's shared memory) with 8 consumer warps and a 2-stage ring.  Two half-SM CTAs
+// let the next kernel's CTAs start streaming on an SM as soon as one of this kernel's finishes.
+template <int CW_, int NS_>
+struct GvCfg {
+    static constexpr int CW = CW_;                 // consumer warps
+    static constexpr int GPW = GV_SG / CW_;        // groups per consumer warp per stage
+    static constexpr int NS = NS_;                 // ring stages
+    static constexpr int PWARP = CW_;              // producer warp
+    static constexpr int RWARP = CW_ + 1;          // reducer warp
+    static constexpr int THREADS = 32 * (CW_ + 2);
+    static constexpr int CTAS_PER_SM = CW_ == 16 ? 1 : 2;
+    static constexpr int SMEM_LIMIT = CTAS_PER_SM == 1 ? 227 * 1024 : 113 * 1024;
+};
+using GvFull = GvCfg<16, 4>;
+using GvHalf = GvCfg<8, 2>;
+
 // A tile's metadata (16 rows x G scales, then 16 rows x G zero points) lands in a per-tile slot
-// of 48 G bytes.  The producer runs at most GV_STAGES stages ahead of the slowest consumer, so
-// ceil(GV_STAGES / stages per tile) + 1 slots let it refill a slot without waiting.
-__host__ __device__ inline GvLayout gv_layout(int MT, int M, int K) {
+// of 48 G bytes.  The producer runs at most NS stages ahead of the slowest consumer, so
+// ceil(NS / stages per tile) + 1 slots let it refill a slot without waiting.
+__host__ __device__ inline GvLayout gv_layout(int MT, int M, int K, int CW, int NS) {
     GvLayout L;
     const uint32_t G = (uint32_t)(K / 128);
     const uint32_t NC = (G + GV_SG - 1) / GV_SG;
-    const uint32_t need = (GV_STAGES + NC - 1) / NC + 1;
+    const uint32_t need = (NS + NC - 1) / NC + 1;
     L.ring = 0;
-    L.meta = GV_STAGES * GV_STAGE_BYTES;
+    L.meta = NS * GV_STAGE_BYTES;
     L.mslot = 48u * G;
     L.nmslot = need < (uint32_t)GV_TSLOTS ? need : (uint32_t)GV_TSLOTS;
     L.xs = L.meta + L.nmslot * L.mslot;
     L.xzero = L.xs + (uint32_t)M * (uint32_t)(K + 8) * 2;               // one group of zeros
     L.corr = L.xzero + 256;                                             // float2 [G][8]
     L.red = L.corr + G * GV_MAXM * 8;                                   // [slot][warp][16][MT] fp32
-    L.bars = L.red + (uint32_t)GV_TSLOTS * GV_CWARPS * 16 * (uint32_t)MT * 4;
-    // full, empty [GV_STAGES]; meta_empty, tile_full, red_empty [GV_TSLOTS]; abort flag
-    L.total = L.bars + (2 * GV_STAGES + 3 * GV_TSLOTS) * 8 + 8;
+    L.bars = L.red + (uint32_t)GV_TSLOTS * CW * 16 * (uint32_t)MT * 4;
+    // full, empty [NS]; meta_empty, tile_full, red_empty [GV_TSLOTS]; abort flag
+    L.total = L.bars + (2 * NS + 3 * GV_TSLOTS) * 8 + 8;
     return L;
 }
 
@@ -90,8 +101,9 @@ __device__ __forceinline__ float half2_sum(uint32_t h) {
 
 constexpr int GV_XILP = 4;  // activation chunks each consumer thread loads before using any
 
+template <int CW>
 __device__ __forceinline__ void gv_named_barrier() {
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * GV_CWARPS) : "memory");
+    asm volatile("bar.sync 1, %0;" ::"n"(32 * CW) : "memory");
 }
 
 // One group (16 rows x 128 k) of the current stage: raw MMA sums for this thread's C fragment.
@@ -114,8 +126,8 @@ __device__ __forceinline__ void gv_group_mma(const uint4 A, const uint4 B, const
     for (int e = 0; e < 4; ++e) r[e] = c0[e] + c1[e];
 }
 
-template <int MT>
-__global__ void __launch_bounds__(GV_THREADS, 1)
+template <int MT, class C>
+__global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
     gemv_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __half* __restrict__ X,
                        const unsigned short* __restrict__ scales, const uint8_t* __restrict__ zeros,
                        __half* __restrict__ Y, int M, int N, int K, int n_tiles, int weights_early,
@@ -123,7 +135,8 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // TMA destinations need an aligned base: round up (the launch reserves 1 KB of slack)
     unsigned char* smem = smem_align1024(smem_raw);
-    const GvLayout L = gv_layout(MT, M, K);
+    constexpr int GV_CWARPS = C::CW, GV_GPW = C::GPW, GV_STAGES = C::NS;
+    const GvLayout L = gv_layout(MT, M, K, GV_CWARPS, GV_STAGES);
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = K >> 7;
@@ -157,7 +170,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     __syncthreads();
     pdl_launch_dependents();  // the next kernel may claim SM space and start its own weight stream
 
-    if (warp == GV_PWARP) {
+    if (warp == C::PWARP) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&tmW);
@@ -203,7 +216,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
         return;
     }
 
-    if (warp == GV_RWARP) {
+    if (warp == C::RWARP) {
         // ------------------------------------------------------------ reducer: Y, in warp order
         pdl_wait();  // Y may be read by the preceding kernel
         int rs = 0;
@@ -282,7 +295,7 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
     }
     if (tid < 16) reinterpret_cast<uint4*>(smem + L.xzero)[tid] = make_uint4(0u, 0u, 0u, 0u);
     // corr entries of activation rows >= M stay unset: they only feed columns that are never stored
-    gv_named_barrier();
+    gv_named_barrier<GV_CWARPS>();
 
     const int g8 = lane >> 2, c = lane & 3;
     // B column g8 holds activation row g8; other lanes read one group of zeros at every k
@@ -366,12 +379,25 @@ __global__ void __launch_bounds__(GV_THREADS, 1)
 // ------------------------------------------------------------------------------------ host side
 static int gv_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
-size_t gemv_stream_smem(int64_t M, int64_t K) {
-    if (M < 1 || M > GV_MAXM || K > 65536) return SIZE_MAX;  // activations are staged whole
-    return (size_t)gv_layout(gv_mt(M), (int)M, (int)K).total + 1024;
+template <class C>
+static size_t gv_smem(int64_t M, int64_t K) {
+    return (size_t)gv_layout(gv_mt(M), (int)M, (int)K, C::CW, C::NS).total + 1024;
 }
 
-template <int MT>
+// The half-SM shape when a tile is one stage (K <= 4096) and it fits half an SM; the full shape
+// otherwise (a shallower ring per CTA costs more than the finer overlap gains once a tile spans
+// several stages).
+static bool gv_use_half(int64_t M, int64_t K) {
+    return K <= GV_SG * 128 && gv_smem<GvHalf>(M, K) <= (size_t)GvHalf::SMEM_LIMIT;
+}
+
+size_t gemv_stream_smem(int64_t M, int64_t K) {
+    if (M < 1 || M > GV_MAXM || K > 65536) return SIZE_MAX;  // activations are staged whole
+    if (gv_use_half(M, K)) return gv_smem<GvHalf>(M, K) * 2;  // two CTAs share the SM
+    return gv_smem<GvFull>(M, K);
+}
+
+template <int MT, class C>
 static cudaError_t gv_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, int64_t N, int64_t K,
                              const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, bool weights_static,
                              int* status, cudaStream_t stream) {
@@ -382,24 +408,26 @@ static cudaError_t gv_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&]() {
-        attr_err[dev] = cudaFuncSetAttribute(gemv_stream_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             227 * 1024);
+        attr_err[dev] = cudaFuncSetAttribute(gemv_stream_kernel<MT, C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM_LIMIT);
     });
     if (attr_err[dev] != cudaSuccess) return attr_err[dev];
     const int n_tiles = (int)((N + 15) / 16);
     const int sms = device_sm_count();
-    const int grid = n_tiles < sms ? n_tiles : sms;
+    const int slots = C::CTAS_PER_SM * sms;
+    const int grid = n_tiles < slots ? n_tiles : slots;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid, 1, 1);
-    cfg.blockDim = dim3(GV_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = gemv_stream_smem(M, K);
+    cfg.blockDim = dim3(C::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = gv_smem<C>(M, K);
+    if (cfg.dynamicSmemBytes > (size_t)C::SMEM_LIMIT) return cudaErrorInvalidValue;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = weights_static ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<MT>, tm, reinterpret_cast<const __half*>(X),
+    return cudaLaunchKernelEx(&cfg, gemv_stream_kernel<MT, C>, tm, reinterpret_cast<const __half*>(X),
                               reinterpret_cast<const unsigned short*>(scales), zeros, reinterpret_cast<__half*>(Y),
                               (int)M, (int)N, (int)K, n_tiles, weights_static ? 1 : 0, status);
 }
@@ -412,11 +440,19 @@ cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t 
                             GV_ROWB / 8, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     if (gemv_stream_smem(M, K) > 227 * 1024) return cudaErrorInvalidValue;
+    const bool half = gv_use_half(M, K);
     switch (gv_mt(M)) {
-        case 1: return gv_launch<1>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
-        case 2: return gv_launch<2>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
-        case 4: return gv_launch<4>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
-        default: return gv_launch<8>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
+#define GV_CASE(MTV)                                                                                     \
+    case MTV:                                                                                            \
+        return half ? gv_launch<MTV, GvHalf>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream) \
+                    : gv_launch<MTV, GvFull>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
+        GV_CASE(1)
+        GV_CASE(2)
+        GV_CASE(4)
+        default:
+            return half ? gv_launch<8, GvHalf>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream)
+                        : gv_launch<8, GvFull>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
+#undef GV_CASE
     }
 }
 
