@@ -120,3 +120,17 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         B.lib()
+
+
+def test_gemm_host_rejects(L):
+    P = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(1 << 12)
+    d = P(ctypes.addressof(buf) + (-ctypes.addressof(buf) % 16))
+    args = lambda **kw: [kw.get("X", d), kw.get("M", 1), 64, kw.get("K", 128), d, d, d, kw.get("group", 128),
+                         kw.get("Y", d), kw.get("xd", d), kw.get("yd", d), None, 0, 0, None]
+    assert L.w4_gemm_host(*args(group=64)) == 4
+    assert L.w4_gemm_host(*args(K=100)) == 2
+    assert L.w4_gemm_host(*args(Y=None)) == 1
+    assert L.w4_gemm_host(*args(xd=None)) == 1
+    assert L.w4_gemm_host(*args(yd=None)) == 1
+    assert L.w4_gemm_host(*args(M=0)) == 0  # empty: nothing enqueued
