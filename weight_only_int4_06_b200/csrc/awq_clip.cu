@@ -231,8 +231,9 @@ __global__ void __launch_bounds__(32 * CL_WARPS) clip_kernel(const __half* __res
 }
 
 // ------------------------------------------------------------------------------------ host side
+// T slices per group: as many as keep all (group, slice) CTAs in one wave of 2 CTAs per SM.
 static int gram_splits(int64_t T, int G, int sms) {
-    const int64_t want = (2L * sms + G - 1) / G;
+    const int64_t want = (2L * sms) / G;
     const int64_t max_by_rows = (T + GR_TT - 1) / GR_TT;
     const int64_t s = want < max_by_rows ? want : max_by_rows;
     return (int)(s < 1 ? 1 : s);
