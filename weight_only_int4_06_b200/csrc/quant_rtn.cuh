@@ -71,6 +71,25 @@ __device__ __forceinline__ uint32_t quant_code(float v, const GroupQuant& p) {
     return (uint32_t)min(max(q, 0), 15);
 }
 
+// Eight codes of an unclipped group packed into one word (lowest k in the lowest nibble).
+// Same codes as quant_code: on the zero-inclusive range rint(v / s16) + z is never below 0
+// (RN and rint are odd-symmetric and monotone, and z = rint(-lo / s16) is never clamped since
+// -lo / s16 <= 15 (1 + 2^-23)), so only the upper clamp remains; z joins the bias of rint_small
+// in one integer add, and nibbles are placed by adds (fields never overlap).  A group whose
+// scale overflowed has unspecified codes (its status is reported); adds keep them inside the
+// group's own words.
+__device__ __forceinline__ uint32_t quant_pack8_rtn(const float (&v)[8], const GroupQuant& p) {
+    const int zoff = p.z - 0x4B400000;  // bit pattern of 1.5 * 2^23, see rint_small
+    uint32_t word = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float t = __fadd_rn(div_rn_from_rcp(v[i], p.sf, p.rcp), 12582912.0f);
+        const int q = min(__float_as_int(t) + zoff, 15);
+        word += (uint32_t)q << (4 * i);
+    }
+    return word;
+}
+
 // Eight consecutive fp16 weights (one 16-byte load) -> fp32, optionally times act_scale.
 __device__ __forceinline__ void load8_scaled(const uint4 raw, const float* a, float (&v)[8]) {
     const __half2* h = reinterpret_cast<const __half2*>(&raw);

@@ -45,10 +45,7 @@ __device__ __forceinline__ void quantize_group_slice(const uint4 raw, int64_t f,
     }
     const GroupQuant p = group_params(fminf(mn, 0.0f), fmaxf(mx, 0.0f));
     if (valid) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) word |= quant_code(v[i], p) << (4 * i);
-        packed[f * 16 + l16] = word;
+        packed[f * 16 + l16] = quant_pack8_rtn(v, p);
         if (l16 == 0) {
             scales[f] = p.s16;
             zeros[f] = (uint8_t)p.z;
