@@ -83,3 +83,26 @@ def test_clip_deterministic():
     r2 = run_gpu(X, W, None, 10)
     for u, v in zip(r1, r2):
         assert np.array_equal(u, v)
+
+
+def test_clip_calibration_full_size_sampled_rows():
+    """The bench's configuration (T = 65536, K = N = 4096, 10 ratios): for sampled rows, the errors
+    of every ratio against the oracle on the full calibration rows, and the codes at the GPU's
+    chosen ratio bit for bit."""
+    X, W = synth.awq_case()
+    Xd, Wd = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
+    best, err, p, s, z = B.awq_clip_search(Xd, Wd, None, 10, with_err=True)
+    assert B.w4_check_device_status() == 0
+    best = best.cpu().numpy().astype(np.int64)
+    assert best.min() >= 0 and best.max() <= 9
+    rows = np.sort(np.random.default_rng(71).choice(W.shape[0], 8, replace=False))
+    err_o, best_o, _, _, _ = oracle.awq_clip_search(X, np.ascontiguousarray(W[rows]), None, 10)
+    err_g = err.cpu().numpy()[rows].astype(np.float64)
+    assert np.all(np.abs(err_g - err_o) <= 1e-3 * err_o + 1e-6 * err_o.max(axis=2, keepdims=True))
+    srt = np.sort(err_o, axis=2)
+    tie = (srt[..., 1] - srt[..., 0]) <= 2e-3 * srt[..., 0]
+    assert np.all((best[rows] == best_o) | tie)
+    q, s2, z2 = oracle.quantize_rtn(np.ascontiguousarray(W[rows]), None, 128, oracle.clip_ratio_grid(10)[best[rows]])
+    assert np.array_equal(p.cpu().numpy().view(np.uint32)[rows], oracle.pack_nibbles(q))
+    assert np.array_equal(s.cpu().numpy().view(np.uint16)[rows], s2.view(np.uint16))
+    assert np.array_equal(z.cpu().numpy()[rows], z2)
