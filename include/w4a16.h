@@ -127,9 +127,13 @@ w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, siz
  *   X [M, K] fp16, packed/scales/zeros as produced by w4_quantize_pack, Y [M, N] fp16 out.
  *   ws / ws_bytes: device workspace of at least w4_gemm_workspace_size bytes (may be NULL when
  *   that size is 0).  M == 0 or N == 0 is a no-op; K == 0 writes Y = 0.
- * The skinny family computes sum_k x_k (q_k - z) exactly per group on tensor cores in fp32 and
- * scales each group's partial sum by s16 in fp32; the TC family rounds each dequantised weight
- * once to fp16 before the fp32-accumulating MMA.  Both round Y once to fp16.
+ * Families (w4_gemm picks by M: GEMV for M <= 8 when its staged activations fit shared memory
+ * and scales/zeros are 16-byte aligned, skinny for M <= 32, TC above):
+ *   - GEMV: tensor-core sums of x with the raw operands 1024+q / 1024+16q, offsets and z removed
+ *     per group with fp32 activation sums (fixed order), times s16 in fp32;
+ *   - skinny: sum_k x_k (q_k - z) exactly per group on tensor cores in fp32, times s16 in fp32;
+ *   - TC: each dequantised weight rounded once to fp16 before the fp32-accumulating MMA.
+ * All accumulate in fp32, round Y once to fp16 and are deterministic (fixed reduction orders).
  */
 w4_status w4_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                   const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y, void* ws,
