@@ -62,9 +62,12 @@ struct GvCfg {
     static constexpr int RWARP = CW_ + 1;          // reducer warp
     static constexpr int THREADS = 32 * (CW_ + 2);
     static constexpr int CTAS_PER_SM = CW_ == 16 ? 1 : 2;
+    static constexpr int ID = CW_ == 16 ? NS_ : 0;  // 4, 3, 2: one CTA per SM; 0: two
     static constexpr int SMEM_LIMIT = CTAS_PER_SM == 1 ? 227 * 1024 : 113 * 1024;
 };
 using GvFull = GvCfg<16, 4>;
+using GvFull3 = GvCfg<16, 3>;  // fewer stages when the staged activations leave too little room
+using GvFull2 = GvCfg<16, 2>;
 using GvHalf = GvCfg<8, 2>;
 
 // A tile's metadata (16 rows x G scales, then 16 rows x G zero points) lands in a per-tile slot
@@ -384,17 +387,26 @@ static size_t gv_smem(int64_t M, int64_t K) {
     return (size_t)gv_layout(gv_mt(M), (int)M, (int)K, C::CW, C::NS).total + 1024;
 }
 
-// The half-SM shape when a tile is one stage (K <= 4096) and it fits half an SM; the full shape
-// otherwise (a shallower ring per CTA costs more than the finer overlap gains once a tile spans
-// several stages).
-static bool gv_use_half(int64_t M, int64_t K) {
-    return K <= GV_SG * 128 && gv_smem<GvHalf>(M, K) <= (size_t)GvHalf::SMEM_LIMIT;
+// The half-SM shape when a tile is one stage (K <= 4096) and it fits half an SM; otherwise the
+// full shape with the deepest ring that fits next to the staged activations (a shallower ring
+// per CTA costs more than the finer overlap gains once a tile spans several stages).  0: none.
+static int gv_pick(int64_t M, int64_t K) {
+    if (M < 1 || M > GV_MAXM || K > 65536) return -1;  // activations are staged whole
+    if (K <= GV_SG * 128 && gv_smem<GvHalf>(M, K) <= (size_t)GvHalf::SMEM_LIMIT) return GvHalf::ID;
+    if (gv_smem<GvFull>(M, K) <= (size_t)GvFull::SMEM_LIMIT) return GvFull::ID;
+    if (gv_smem<GvFull3>(M, K) <= (size_t)GvFull3::SMEM_LIMIT) return GvFull3::ID;
+    if (gv_smem<GvFull2>(M, K) <= (size_t)GvFull2::SMEM_LIMIT) return GvFull2::ID;
+    return -1;
 }
 
 size_t gemv_stream_smem(int64_t M, int64_t K) {
-    if (M < 1 || M > GV_MAXM || K > 65536) return SIZE_MAX;  // activations are staged whole
-    if (gv_use_half(M, K)) return gv_smem<GvHalf>(M, K) * 2;  // two CTAs share the SM
-    return gv_smem<GvFull>(M, K);
+    switch (gv_pick(M, K)) {
+        case GvHalf::ID: return gv_smem<GvHalf>(M, K) * 2;  // two CTAs share the SM
+        case GvFull::ID: return gv_smem<GvFull>(M, K);
+        case GvFull3::ID: return gv_smem<GvFull3>(M, K);
+        case GvFull2::ID: return gv_smem<GvFull2>(M, K);
+        default: return SIZE_MAX;
+    }
 }
 
 template <int MT, class C>
@@ -439,21 +451,25 @@ cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t 
     if (!make_tensor_map_2d(&tm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)(K / 16), (uint64_t)N,
                             GV_ROWB / 8, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    if (gemv_stream_smem(M, K) > 227 * 1024) return cudaErrorInvalidValue;
-    const bool half = gv_use_half(M, K);
-    switch (gv_mt(M)) {
-#define GV_CASE(MTV)                                                                                     \
-    case MTV:                                                                                            \
-        return half ? gv_launch<MTV, GvHalf>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream) \
-                    : gv_launch<MTV, GvFull>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
-        GV_CASE(1)
-        GV_CASE(2)
-        GV_CASE(4)
-        default:
-            return half ? gv_launch<8, GvHalf>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream)
-                        : gv_launch<8, GvFull>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream);
-#undef GV_CASE
+    const int pick = gv_pick(M, K);
+    if (pick < 0) return cudaErrorInvalidValue;
+    const int mt = gv_mt(M);
+#define GV_LAUNCH(MTV, CFG) gv_launch<MTV, CFG>(tm, X, M, N, K, scales, zeros, Y, weights_static, status, stream)
+#define GV_BY_MT(CFG)                                   \
+    switch (mt) {                                       \
+        case 1: return GV_LAUNCH(1, CFG);               \
+        case 2: return GV_LAUNCH(2, CFG);               \
+        case 4: return GV_LAUNCH(4, CFG);               \
+        default: return GV_LAUNCH(8, CFG);              \
     }
+    switch (pick) {
+        case GvHalf::ID: GV_BY_MT(GvHalf)
+        case GvFull::ID: GV_BY_MT(GvFull)
+        case GvFull3::ID: GV_BY_MT(GvFull3)
+        default: GV_BY_MT(GvFull2)
+    }
+#undef GV_BY_MT
+#undef GV_LAUNCH
 }
 
 }  // namespace w4
