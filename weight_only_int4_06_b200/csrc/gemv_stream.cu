@@ -46,6 +46,11 @@ constexpr uint32_t GV_STAGE_BYTES = 16 * GV_ROWB;    // 32 KB of packed codes
 constexpr int GV_MAXM = 8;
 constexpr int GV_TSLOTS = 6;                         // tiles whose partials may be pending at once
 
+// Partial-sum slots of the reducer: two suffice (the reducer adds a tile in far less time than the
+// consumers take for the next one); eight activation rows use two to leave room for the staged
+// activations, fewer rows keep more slack.
+__host__ __device__ constexpr int gv_rslots(int MT) { return MT >= 8 ? 2 : GV_TSLOTS; }
+
 struct GvLayout {
     uint32_t ring, meta, mslot, nmslot, xs, xzero, corr, red, bars, total;
 };
@@ -86,7 +91,7 @@ __host__ __device__ inline GvLayout gv_layout(int MT, int M, int K, int CW, int 
     L.xzero = L.xs + (uint32_t)M * (uint32_t)(K + 8) * 2;               // one group of zeros
     L.corr = L.xzero + 256;                                             // float2 [G][8]
     L.red = L.corr + G * GV_MAXM * 8;                                   // [slot][warp][16][MT] fp32
-    L.bars = L.red + (uint32_t)GV_TSLOTS * CW * 16 * (uint32_t)MT * 4;
+    L.bars = L.red + (uint32_t)gv_rslots(MT) * CW * 16 * (uint32_t)MT * 4;
     // full, empty [NS]; meta_empty, tile_full, red_empty [GV_TSLOTS]; abort flag
     L.total = L.bars + (2 * NS + 3 * GV_TSLOTS) * 8 + 8;
     return L;
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(red_empty(rs));
-            if (++rs == GV_TSLOTS) { rs = 0; rph ^= 1; }
+            if (++rs == gv_rslots(MT)) { rs = 0; rph ^= 1; }
         }
         return;
     }
@@ -372,7 +377,7 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
             if (2 * c < MT) { mine[g8 * MT + 2 * c] = acc[0]; mine[(g8 + 8) * MT + 2 * c] = acc[2]; }
             if (2 * c + 1 < MT) { mine[g8 * MT + 2 * c + 1] = acc[1]; mine[(g8 + 8) * MT + 2 * c + 1] = acc[3]; }
             mbar_arrive(tile_full(rs));  // every lane: its own stores are released with it
-            if (++rs == GV_TSLOTS) { rs = 0; rph ^= 1; }
+            if (++rs == gv_rslots(MT)) { rs = 0; rph ^= 1; }
             acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
             kc = 0;
         }
