@@ -33,3 +33,10 @@ def test_record_is_ignored_once_the_kernel_sources_change(tmp_path, monkeypatch)
     assert T.load_traffic("decode") == 123
     rec.write_text(json.dumps({"dram_bytes_per_step": 123, "source_sha256": "0" * 64}))
     assert T.load_traffic("decode") is None
+
+
+def test_digest_ignores_comments_and_layout_only():
+    a = "int f(int x) {  // one\n  return x + 1; /* two\n lines */ }\n"
+    b = "int f(int x) {\n    return x + 1;\n}  // edited comment\n"
+    c = "int f(int x) { return x + 2; }"
+    assert T.code_only(a) == T.code_only(b) != T.code_only(c)

@@ -5,14 +5,16 @@
 // packed weights (0.5 B/weight) plus 3 B of scale and zero point per group of 128.
 //
 // Design (sm_100a):
-//  * Persistent: one CTA per SM; CTA c owns a contiguous range of 16-row tiles over the whole K,
-//    so every output is finished inside one CTA (no split-K workspace, no cluster barrier).
+//  * Persistent: one CTA per SM (or two half-SM CTAs, see GvCfg); CTA c owns a contiguous range
+//    of 16-row tiles over the whole K, so every output is finished inside one CTA (no split-K
+//    workspace, no cluster barrier).
 //  * A producer warp streams the packed tile through a shared-memory ring of stages with
 //    TMA: one stage is 16 rows x 4096 k (32 KB; for K = 4096 the whole tile, one contiguous
 //    block of HBM).  A tile's scales and zero points are one contiguous block of each array and
 //    ride on the tile's first stage as two bulk copies.  With static weights the producer starts
 //    before the preceding kernel has finished (programmatic dependent launch).
-//  * Sixteen consumer warps take two groups of 128 each per stage and run mma.sync m16n8k16 with
+//  * The consumer warps (16, or 8 in a half-SM CTA) split a stage's 32 groups of 128 between them
+//    (two or four each) and run mma.sync m16n8k16 with
 //    the 16 weight rows as the A operand and the (up to 8) activation rows as B.  Dequantisation
 //    is one LOP3 per two weights: the operands are the raw fp16 values 1024+q (low nibble of a
 //    byte) and 1024+16q (high nibble); activations that meet high nibbles are staged pre-multiplied
@@ -28,7 +30,7 @@
 //    fragments of the two MMAs that consume one packed word.  Lanes whose B column is not an
 //    activation row read a block of zeros instead (no predication in the inner loop).
 //  * At the end of a tile every consumer warp parks its partial sums in a shared slot and moves
-//    on; a reducer warp adds the sixteen partials in warp order (deterministic) and writes Y, so
+//    on; a reducer warp adds the warps' partials in warp order (deterministic) and writes Y, so
 //    the stage ring never waits for a reduction.
 //  * The kernel is instantiated per activation-row bound MT (1, 2, 4, 8): columns >= MT of the
 //    MMA fragments are never folded or parked.

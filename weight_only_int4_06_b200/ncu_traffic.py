@@ -30,11 +30,21 @@ KERNEL_SOURCES = {
 }
 
 
+_COMMENT = re.compile(r"/\*.*?\*/|//[^\n]*", re.S)
+
+
+def code_only(text: str) -> str:
+    """C/C++ source without comments and with whitespace collapsed: what the compiler sees."""
+    return " ".join(_COMMENT.sub(" ", text).split())
+
+
 def source_digest(workload: str) -> str:
+    """Digest of the kernel sources' code (comments and layout excluded, so a record stays valid
+    across comment edits and goes stale on any change to the code)."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES[workload]:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(f.encode() + b"\0" + fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + code_only(fh.read()).encode())
     return h.hexdigest()
 
 
