@@ -281,3 +281,63 @@ def awq_clip_search(X: np.ndarray, W: np.ndarray, act_scale: np.ndarray | None =
     best = np.argmin(err, axis=2)  # first occurrence = lowest j among the minima
     q, s16, z = quantize_rtn(W16, act_scale, group, ratios[best])
     return err, best, pack_nibbles(q), s16, z
+
+
+# ----------------------------------------------------------------------------
+# GPTQ: quantise one column at a time and let the later columns absorb the error
+# ----------------------------------------------------------------------------
+def _group_params_rtn(v32: np.ndarray):
+    """Scale and zero point of quantize_rtn for one group per row: v32 [N, group] fp32."""
+    lo = np.minimum(v32.min(axis=1), np.float32(0))
+    hi = np.maximum(v32.max(axis=1), np.float32(0))
+    d = hi - lo
+    s16 = fp16_round_up(d / np.float32(QMAX))
+    s16[d == 0] = np.float16(1.0)
+    if np.isinf(s16).any():
+        raise QuantRangeError("fp16 group scale overflow")
+    sf = s16.astype(np.float32)
+    z = np.clip(np.rint(-lo / sf), 0, QMAX)
+    return s16, sf, z
+
+
+def gptq_quantize(X: np.ndarray, W: np.ndarray, damp: float = 0.01, group: int = GROUP,
+                  stop_after: int | None = None):
+    """GPTQ on one layer ("GPTQ, AWQ and the rules of post-training quantization", section "GPTQ: pay
+    for the error with the other weights"): columns are quantised in order, and after each one the
+    not-yet-quantised columns are corrected so that the layer's output on the calibration data
+    moves as little as possible.
+
+    H = X^T X (fp64) plus damp * mean(diag H) on the diagonal; U = the upper Cholesky factor of H^-1.
+    For column k: q_k = RTN code of the current W[:, k] with its group's scale and zero point, which
+    are taken (quantize_rtn's rule) from the current, already corrected weights of the group when
+    its first column is reached; e = (W[:, k] - (q_k - z) s) / U[k, k]; W[:, j] -= e U[k, j], j > k.
+    The weights are carried in fp64; the group parameters see them rounded to fp32.
+    stop_after: return after that many columns (for tests), with the corrected W.
+    Returns (packed, scales, zeros, W_corrected fp64).
+    """
+    X64 = np.asarray(X).astype(np.float64)
+    Wc = np.asarray(W, dtype=np.float16).astype(np.float64).copy()
+    N, K = Wc.shape
+    G = K // group
+    H = X64.T @ X64
+    H[np.diag_indices(K)] += damp * np.mean(np.diag(H))
+    Hinv = np.linalg.inv(H)
+    U = np.linalg.cholesky(Hinv).T  # upper: Hinv = U^T U
+    q = np.zeros((N, K), dtype=np.uint8)
+    s16 = np.zeros((N, G), dtype=np.float16)
+    z = np.zeros((N, G), dtype=np.uint8)
+    sf = zg = None
+    ncols = K if stop_after is None else stop_after
+    for k in range(ncols):
+        g = k // group
+        if k % group == 0:
+            s_g, sf, zg = _group_params_rtn(Wc[:, k:k + group].astype(np.float32))
+            s16[:, g] = s_g
+            z[:, g] = zg.astype(np.uint8)
+        v = Wc[:, k].astype(np.float32)
+        qk = np.clip(np.rint(v / sf) + zg, 0, QMAX)
+        q[:, k] = qk.astype(np.uint8)
+        w_hat = (qk.astype(np.float64) - zg.astype(np.float64)) * sf.astype(np.float64)
+        e = (Wc[:, k] - w_hat) / U[k, k]
+        Wc[:, k + 1:] -= np.outer(e, U[k, k + 1:])
+    return pack_nibbles(q), s16, z, Wc
