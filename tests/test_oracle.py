@@ -429,3 +429,34 @@ def test_golden_single_layer_digests():
     mg = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mg)
     assert mg.digests() == _read_golden("single_layer_seed0.txt")
+
+
+def test_unclamped_codes_never_negative():
+    """The GPU packer drops the lower clamp of q = rint(v / s16) + z for the unclipped range: with
+    z = rint(-lo / s16) and rint odd-symmetric, v >= lo gives q >= 0.  Check the unclamped value on
+    adversarial groups: exact ties, subnormals, one-sided, constant and wide ranges."""
+    rng = np.random.default_rng(123)
+    groups = []
+    for _ in range(400):
+        kind = rng.integers(0, 6)
+        if kind == 0:
+            g = rng.standard_normal(128) * 10.0 ** rng.uniform(-6, 3)
+        elif kind == 1:
+            g = np.abs(rng.standard_normal(128)) * 10.0 ** rng.uniform(-6, 3)
+        elif kind == 2:
+            g = -np.abs(rng.standard_normal(128)) * 10.0 ** rng.uniform(-6, 3)
+        elif kind == 3:
+            g = rng.integers(-8, 8, 128) * 2.0 ** rng.integers(-20, 4)  # many exact ties
+        elif kind == 4:
+            g = rng.standard_normal(128) * 6e-8  # fp16 subnormals
+        else:
+            g = np.full(128, rng.standard_normal())
+        groups.append(g)
+    W = np.clip(np.array(groups), -6e4, 6e4).astype(np.float16)
+    q, s, z = O.quantize_rtn(W)
+    v = W.astype(np.float32)
+    sf = s.astype(np.float32)
+    raw = np.rint(v / sf) + z.astype(np.float32)  # the same fp32 steps without the clamp
+    assert raw.min() >= 0
+    assert raw.max() <= 16
+    assert np.array_equal(np.minimum(raw, 15).astype(np.uint8), q)
