@@ -218,6 +218,41 @@ w4_status awq_scale_search_noalloc(const uint16_t* X, int64_t T, const uint16_t*
                                    int64_t K, int group, int n_alpha, double* mse,
                                    int32_t* best_idx, float* best_s, void* stream);
 
+/* Bytes of device workspace awq_scale_search_gram needs for this problem. */
+w4_status awq_gram_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha,
+                                  size_t* bytes);
+
+/*
+ * awq_scale_search_gram -- awq_scale_search with the calibration rows folded into their Gram
+ * matrix first.
+ *
+ * Same search, same arguments, same outputs ("GPTQ, AWQ and the rules of post-training
+ * quantization", section "AWQ: find the one percent that matters").  The output error of a
+ * weight error E is sum_{t,n} (X E^T)[t,n]^2 = sum_n e_n^T (X^T X) e_n, so X is read once to form
+ * G = X^T X (fp16 inputs, fp32 tensor-core accumulation) and each alpha then costs one N x K x K
+ * product instead of a T x N x K one: the faster call once T exceeds about K.  Arithmetic:
+ *     G    = sum over chunks c of X_c^T X_c, X_c = rows [4096 c, 4096 c + 4096) of X: each chunk
+ *            one fp32 tensor-core product, the chunks added in fp64 in chunk order
+ *     d_k  = sqrt(G_kk) rounded to fp32 (1 where channel k is zero in every row)
+ *     G'   = fp16(G_ij / (d_i d_j))          (entries in [-1, 1]; fp16 cannot hold G itself)
+ *     E'_i = fp16(((Wq_i - W diag(s_i)) / s_i) * d)   (Wq_i exactly as in awq_scale_search)
+ *     MSE_i = sum over tiles of sum_{n,k} (E'_i G'^T)[n,k] E'_i[n,k]  / (T N)
+ * with fp32 accumulation inside a tile and an fp64 fixed-order sum over tiles.  The rounding of
+ * G' and E' differs from the direct form's, so MSE_i agrees with awq_scale_search's to about
+ * 1e-5 relative, not bit for bit; best_idx can differ only where two alphas' errors are that
+ * close.  An E' entry beyond the fp16 range (a weight error far larger than the activations'
+ * norm can carry) makes that alpha's MSE infinite and sets W4_ERR_RANGE in the device status.
+ *
+ *   X [T, K] fp16; W [N, K] fp16; mse [n_alpha] fp64, best_idx [1] int32, best_s [K] fp32 out.
+ *   ws: device workspace of at least awq_gram_workspace_size bytes (it holds X^T with T padded
+ *   to whole chunks, one chunk's G in fp32, G in fp64 and G' in fp16: about
+ *   2 T K + 14 K^2 + 2 N K bytes).
+ * T must be >= 1 and N >= 8.  Errors: see the conventions above.
+ */
+w4_status awq_scale_search_gram(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N,
+                                int64_t K, int group, int n_alpha, double* mse, int32_t* best_idx,
+                                float* best_s, void* ws, size_t ws_bytes, void* stream);
+
 /* Bytes of device workspace awq_clip_search needs for this problem. */
 w4_status awq_clip_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_ratios,
                                   size_t* bytes);

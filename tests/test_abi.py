@@ -31,6 +31,7 @@ def test_header_declares_expected_api():
     names = declared_functions()
     for n in ("w4_quantize_pack", "w4_gemm", "w4_gemm_ex", "w4_gemm_host", "w4_gemm_workspace_size",
               "awq_scale_search", "awq_workspace_size", "awq_clip_search", "awq_clip_workspace_size",
+              "awq_scale_search_gram", "awq_gram_workspace_size",
               "w4_check_device_status", "w4_status_string"):
         assert n in names, n
 
@@ -99,6 +100,23 @@ def test_workspace_queries(L):
     assert L.awq_clip_workspace_size(256, 64, 512, 128, 0, ctypes.byref(n)) == 4
     assert L.awq_clip_workspace_size(256, 64, 500, 128, 10, ctypes.byref(n)) == 2
     assert L.awq_clip_workspace_size(0, 64, 512, 128, 10, ctypes.byref(n)) == 2
+    assert L.awq_gram_workspace_size(300, 64, 512, 128, 20, ctypes.byref(n)) == 0
+    assert n.value >= 512 * 320 * 2 + 512 * 512 * 14 + 64 * 512 * 2  # X^T padded to 320 rows, G (fp32, fp64), G', E'
+    assert L.awq_gram_workspace_size(256, 64, 512, 128, 0, ctypes.byref(n)) == 4
+    assert L.awq_gram_workspace_size(256, 60, 512, 128, 20, ctypes.byref(n)) == 2
+
+
+def test_gram_search_rejects(L):
+    P = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(1 << 12)
+    d = P(ctypes.addressof(buf) + (-ctypes.addressof(buf) % 16))
+    args = lambda **kw: [kw.get("X", d), 64, kw.get("W", d), 64, 512, kw.get("group", 128), kw.get("A", 20), d, d,
+                         d, kw.get("ws", d), kw.get("ws_bytes", 1 << 30), None]
+    assert L.awq_scale_search_gram(*args(A=65)) == 4
+    assert L.awq_scale_search_gram(*args(group=64)) == 4
+    assert L.awq_scale_search_gram(*args(ws_bytes=16)) == 5
+    assert L.awq_scale_search_gram(*args(X=None)) == 1
+    assert L.awq_scale_search_gram(*args(W=P(d.value + 2))) == 3
 
 
 def test_clip_search_rejects(L):

@@ -212,6 +212,29 @@ w4_status awq_scale_search(const uint16_t* X, int64_t T, const uint16_t* W, int6
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
+w4_status awq_gram_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha, size_t* bytes) {
+    if (!bytes) return W4_ERR_NULL;
+    w4_status st = awq_check(T, N, K, group, n_alpha);
+    if (st != W4_OK) return st;
+    *bytes = awq_gram_layout(T, N, K, n_alpha).bytes;
+    return W4_OK;
+}
+
+w4_status awq_scale_search_gram(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K,
+                                int group, int n_alpha, double* mse, int32_t* best_idx, float* best_s,
+                                void* ws, size_t ws_bytes, void* stream) {
+    w4_status st = awq_check(T, N, K, group, n_alpha);
+    if (st != W4_OK) return st;
+    if (ws_bytes < awq_gram_layout(T, N, K, n_alpha).bytes) return W4_ERR_WORKSPACE;
+    if (!X || !W || !mse || !best_idx || !best_s || !ws) return W4_ERR_NULL;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(ws)) return W4_ERR_ALIGN;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_awq_gram(X, T, W, N, K, n_alpha, mse, best_idx, best_s, ws, status,
+                                    (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 static w4_status clip_check(int64_t T, int64_t N, int64_t K, int group, int n_ratios) {
     if (group != 128 || n_ratios < 1 || n_ratios > 10) return W4_ERR_UNSUPPORTED;
     if (!dims_ok(T, K) || !dims_ok(N, K) || T < 1 || N < 8 || K < 128 || K % group != 0 || N % 8 != 0)

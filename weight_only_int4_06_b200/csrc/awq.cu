@@ -250,4 +250,210 @@ cudaError_t launch_awq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t 
     return cudaGetLastError();
 }
 
+// ==================================================================================================
+// Gram form of the same search.  sum_{t,n} (X E_i^T)^2 = sum_n e_n^T G e_n with G = X^T X, so the T
+// calibration rows are read once: G on the tensor cores, then per alpha one GEMM over K x K instead
+// of T x K.  G is formed chunk by chunk: each chunk of at most GRAM_CHUNK rows is one fp32
+// tensor-core product (the same accumulation length as the direct form's K-long dot products; one
+// fp32 accumulator over all 65536 rows showed a systematic 4e-4 relative shortfall), and the chunks
+// are summed in fp64 in chunk order.  G carries the squared activations' dynamic range (beyond
+// fp16), so it is scaled symmetrically: d_k = sqrt(G_kk) (1 for a channel that is zero in every
+// row), G' = D^-1 G D^-1 with entries in [-1, 1] in fp16, and E'_i = E_i D in fp16, so that
+// e^T G e = e'^T G' e'.  The per-alpha GEMM E' G'^T has an epilogue that sums (E' G'^T)[n, k] E'[n, k]
+// per tile; MSE_i = (fixed-order sum of the tile partials) / (T N), exactly as in the direct form.
+
+constexpr int TP_TILE = 32;
+constexpr int64_t GRAM_CHUNK = 4096;
+
+// Rows per chunk: all of T (padded to a multiple of 64) when T fits one chunk.
+static int64_t gram_chunk_rows(int64_t T) {
+    const int64_t Tp = (T + 63) / 64 * 64;
+    return Tp < GRAM_CHUNK ? Tp : GRAM_CHUNK;
+}
+
+// XT holds X^T chunk by chunk: chunk c is a [K, L] row-major block of rows t in [cL, cL + L), rows
+// t >= T zero (L % 64 == 0: whole K-steps for the GEMM).
+__global__ void __launch_bounds__(256) transpose_pad_kernel(const unsigned short* __restrict__ X, int64_t T,
+                                                            int K, int64_t L, int64_t Tp,
+                                                            unsigned short* __restrict__ XT) {
+    __shared__ unsigned short tile[TP_TILE][TP_TILE + 1];
+    const int64_t t0 = (int64_t)blockIdx.x * TP_TILE;
+    const int k0 = blockIdx.y * TP_TILE;
+    for (int r = threadIdx.y; r < TP_TILE; r += blockDim.y) {
+        const int64_t t = t0 + r;
+        tile[r][threadIdx.x] = t < T ? X[t * K + k0 + threadIdx.x] : (unsigned short)0;
+    }
+    __syncthreads();
+    const int64_t t = t0 + threadIdx.x;
+    const int64_t c = t / L, tt = t - c * L;
+    for (int r = threadIdx.y; r < TP_TILE; r += blockDim.y)
+        if (t < Tp) XT[(c * K + k0 + r) * L + tt] = tile[threadIdx.x][r];
+}
+
+// G64 = Gc (first chunk) or G64 += Gc, elementwise in fp64.
+__global__ void gram_accumulate_kernel(const float* __restrict__ Gc, int64_t n, bool first, double* __restrict__ G64) {
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+        G64[e] = first ? (double)Gc[e] : G64[e] + (double)Gc[e];
+}
+
+// d_k = sqrt(G_kk) (1 when G_kk is 0) and rd = 1 / d, from the fp64 G rounded once to fp32.
+__global__ void gram_diag_kernel(const double* __restrict__ G64, int K, float* __restrict__ d, float* __restrict__ rd) {
+    const int k = blockIdx.x * blockDim.x + threadIdx.x;
+    if (k >= K) return;
+    const double g = G64[(int64_t)k * K + k];
+    const float dk = g > 0.0 ? __double2float_rn(sqrt(g)) : 1.0f;
+    d[k] = dk;
+    rd[k] = __frcp_rn(dk);
+}
+
+// G' = D^-1 G D^-1 in fp16.
+__global__ void gram_scale_kernel(const double* __restrict__ G64, const float* __restrict__ rd, int K,
+                                  __half* __restrict__ Gp) {
+    const int64_t n = (int64_t)K * K;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
+        const int i = (int)(e / K), j = (int)(e - (int64_t)i * K);
+        Gp[e] = __double2half(G64[e] * (double)rd[i] * (double)rd[j]);
+    }
+}
+
+// E' = ((Wq - W*s) / s) * d in fp16 for one alpha; the codes are those of w4_quantize_pack(W, s).
+__global__ void __launch_bounds__(256) awq_fakequant_scaled_kernel(const uint4* __restrict__ W,
+                                                                   const float* __restrict__ s,
+                                                                   const float* __restrict__ dmul, int64_t n_groups,
+                                                                   int G, uint4* __restrict__ E, int* status) {
+    const int lane = threadIdx.x & 31;
+    const int sub = lane >> 4, l16 = lane & 15;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t n_pairs = (n_groups + 1) >> 1;
+    for (int64_t pair = warp; pair < n_pairs; pair += nwarps) {
+        const int64_t f = 2 * pair + sub;
+        const bool valid = f < n_groups;
+        float v[8], a[8], dm[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { v[i] = 0.0f; a[i] = 1.0f; dm[i] = 1.0f; }
+        if (valid) {
+            const uint4 raw = ldg_stream(W + f * 16 + l16);
+            const int64_t k0 = (f % G) * 128 + 8 * l16;
+            const float4 a0 = __ldg(reinterpret_cast<const float4*>(s + k0));
+            const float4 a1 = __ldg(reinterpret_cast<const float4*>(s + k0) + 1);
+            const float4 d0 = __ldg(reinterpret_cast<const float4*>(dmul + k0));
+            const float4 d1 = __ldg(reinterpret_cast<const float4*>(dmul + k0) + 1);
+            a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
+            a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+            dm[0] = d0.x; dm[1] = d0.y; dm[2] = d0.z; dm[3] = d0.w;
+            dm[4] = d1.x; dm[5] = d1.y; dm[6] = d1.z; dm[7] = d1.w;
+            load8_scaled(raw, a, v);
+        }
+        float mn = v[0], mx = v[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) { mn = fminf(mn, v[i]); mx = fmaxf(mx, v[i]); }
+#pragma unroll
+        for (int o = 8; o; o >>= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        const GroupQuant p = group_params(fminf(mn, 0.0f), fmaxf(mx, 0.0f));
+        if (valid) {
+            uint32_t out[4];
+            bool bad = false;
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+                float e2[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int q = (int)quant_code(v[i + u], p);
+                    const float wq = (float)(q - p.z) * p.sf;  // exact: |q - z| <= 15, sf has 11 bits
+                    e2[u] = __fmul_rn(__fdiv_rn(__fsub_rn(wq, v[i + u]), a[i + u]), dm[i + u]);
+                    if (!(fabsf(e2[u]) <= 65504.0f)) bad = true;  // E' beyond fp16: the MSE would be inf
+                }
+                out[i / 2] = pack_half2(e2[0], e2[1]);
+            }
+            E[f * 16 + l16] = make_uint4(out[0], out[1], out[2], out[3]);
+            if ((l16 == 0 && p.overflow) || bad) record_status(status, W4_ERR_RANGE);
+        }
+    }
+}
+
+AwqGramLayout awq_gram_layout(int64_t T, int64_t N, int64_t K, int n_alpha) {
+    AwqGramLayout L;
+    L.chunk = gram_chunk_rows(T);
+    L.n_chunks = (T + L.chunk - 1) / L.chunk;
+    L.Tp = L.chunk * L.n_chunks;
+    L.n_part = tc_sse_partials(N, K);
+    size_t off = 0;
+    L.colsum = off; off = align256(off + (size_t)K * 8);
+    L.s_all = off; off = align256(off + (size_t)n_alpha * K * 4);
+    L.E = off; off = align256(off + (size_t)N * K * 2);
+    L.part = off; off = align256(off + (size_t)n_alpha * L.n_part * 8);
+    L.XT = off; off = align256(off + (size_t)K * (size_t)L.Tp * 2);
+    L.G = off; off = align256(off + (size_t)K * K * 4);
+    L.G64 = off; off = align256(off + (size_t)K * K * 8);
+    L.Gp = off; off = align256(off + (size_t)K * K * 2);
+    L.d = off; off = align256(off + (size_t)K * 4);
+    L.rd = off; off = align256(off + (size_t)K * 4);
+    L.bytes = off;
+    return L;
+}
+
+cudaError_t launch_awq_gram(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int n_alpha,
+                            double* mse, int32_t* best_idx, float* best_s, void* ws, int* status,
+                            cudaStream_t stream) {
+    const AwqGramLayout L = awq_gram_layout(T, N, K, n_alpha);
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    auto* colsum = reinterpret_cast<unsigned long long*>(base + L.colsum);
+    float* s_all = reinterpret_cast<float*>(base + L.s_all);
+    uint16_t* E = reinterpret_cast<uint16_t*>(base + L.E);
+    double* part = reinterpret_cast<double*>(base + L.part);
+    uint16_t* XT = reinterpret_cast<uint16_t*>(base + L.XT);
+    float* Gc = reinterpret_cast<float*>(base + L.G);
+    double* G64 = reinterpret_cast<double*>(base + L.G64);
+    __half* Gp = reinterpret_cast<__half*>(base + L.Gp);
+    float* d = reinterpret_cast<float*>(base + L.d);
+    float* rd = reinterpret_cast<float*>(base + L.rd);
+
+    cudaError_t e = cudaMemsetAsync(colsum, 0, (size_t)K * 8, stream);
+    if (e != cudaSuccess) return e;
+    {
+        const int chunks = (int)(K / 8);
+        dim3 grid((chunks + 255) / 256, (unsigned)((T + CA_ROWS - 1) / CA_ROWS));
+        colabs_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(X), T, (int)K, colsum);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    awq_scales_kernel<<<n_alpha, 1024, 0, stream>>>(colsum, T, (int)K, n_alpha, s_all);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    transpose_pad_kernel<<<dim3((unsigned)(L.Tp / TP_TILE), (unsigned)(K / TP_TILE)), dim3(TP_TILE, 8), 0, stream>>>(
+        reinterpret_cast<const unsigned short*>(X), T, (int)K, L.chunk, L.Tp, reinterpret_cast<unsigned short*>(XT));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const unsigned ew_blocks = (unsigned)device_sm_count() * 8;
+    for (int64_t c = 0; c < L.n_chunks; ++c) {  // G = sum over chunks of X_c^T X_c
+        const uint16_t* XTc = XT + c * K * L.chunk;
+        e = launch_tc_f32(XTc, K, XTc, K, L.chunk, Gc, status, stream);
+        if (e != cudaSuccess) return e;
+        gram_accumulate_kernel<<<ew_blocks, 256, 0, stream>>>(Gc, K * K, c == 0, G64);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    gram_diag_kernel<<<(unsigned)((K + 255) / 256), 256, 0, stream>>>(G64, (int)K, d, rd);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    gram_scale_kernel<<<ew_blocks, 256, 0, stream>>>(G64, rd, (int)K, Gp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int64_t G = K / 128;
+    const int64_t n_groups = N * G;
+    const int64_t want = ((n_groups + 1) / 2 + 7) / 8;
+    const int64_t cap = (int64_t)device_sm_count() * 8;
+    const int fq_blocks = (int)(want < cap ? want : cap);
+    for (int i = 0; i < n_alpha; ++i) {
+        awq_fakequant_scaled_kernel<<<fq_blocks, 256, 0, stream>>>(
+            reinterpret_cast<const uint4*>(W), s_all + (int64_t)i * K, d, n_groups, (int)G, reinterpret_cast<uint4*>(E),
+            status);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_tc_dot(E, N, reinterpret_cast<const uint16_t*>(Gp), K, K, part + (int64_t)i * L.n_part, status,
+                          stream);
+        if (e != cudaSuccess) return e;
+    }
+    awq_finalize_kernel<<<1, 256, 0, stream>>>(part, L.n_part, n_alpha, (double)T * (double)N, s_all, (int)K, mse,
+                                               best_idx, best_s);
+    return cudaGetLastError();
+}
+
 }  // namespace w4

@@ -16,8 +16,9 @@
 //   warp 2      allocates / frees TMEM.
 //   warps 4-11  dequantise: each thread turns one packed row (64 codes) into 64 fp16 weights in
 //               the UMMA K-major 128-byte-swizzle layout, then runs the epilogue (TMEM -> fp16 Y).
-// A second mode (for the AWQ search) loads an fp16 B operand with TMA instead of dequantising and
-// replaces the store by a per-tile sum of squares.
+// Other modes (for the AWQ search) load an fp16 B operand with TMA instead of dequantising and
+// replace the fp16 store (EPI 0) by a per-tile sum of squares (EPI 1), an fp32 store (EPI 2), or a
+// per-tile sum of D[m, n] * A[m, n] (EPI 3, for N == K: A read back from global memory).
 //
 // Every mbarrier wait is bounded; on timeout the kernel records W4_ERR_DEVICE_TIMEOUT, stops
 // issuing work, drains what it issued and frees TMEM before it exits.
@@ -62,12 +63,14 @@ __device__ __forceinline__ void tc_tile_coords(int t, int m_tiles, int n_tiles, 
     nt = r / gm;
 }
 
-template <bool DEQ, bool SSE, int MT>
+template <bool DEQ, int EPI, int MT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __half* __restrict__ scales, const uint8_t* __restrict__ zeros,
-                   __half* __restrict__ Y, double* __restrict__ sse_part, int M, int N, int K,
-                   int m_tiles, int n_tiles, int* status) {
+                   __half* __restrict__ Y, double* __restrict__ sse_part, float* __restrict__ Cf,
+                   const __half* __restrict__ Adot, int M, int N, int K, int m_tiles, int n_tiles,
+                   int* status) {
+    constexpr bool SSE = EPI == 1 || EPI == 3;  // modes that reduce the tile to one fp64 partial
     using C = TcCfg<DEQ, MT>;
     constexpr int S = C::kStages;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256 + col), v);
                 tmem_wait_ld();
-                if (SSE) {
+                if (EPI == 1) {
                     float a = 0.0f;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -255,6 +258,46 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         a = fmaf(f, f, a);
                     }
                     sq += (double)a;
+                } else if (EPI == 3) {
+                    if (m < M) {  // sum of D[m, n] * A[m, n] over this thread's 32 columns
+                        const int nb = n0 + col;
+                        const __half* arow = Adot + (int64_t)m * K + nb;
+                        float a = 0.0f;
+                        if (nb + 32 <= N) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 8) {
+                                const uint4 h8 = *reinterpret_cast<const uint4*>(arow + i);
+                                const __half2* hp = reinterpret_cast<const __half2*>(&h8);
+#pragma unroll
+                                for (int u = 0; u < 4; ++u) {
+                                    const float2 f = __half22float2(hp[u]);
+                                    a = fmaf(__uint_as_float(v[i + 2 * u]), f.x, a);
+                                    a = fmaf(__uint_as_float(v[i + 2 * u + 1]), f.y, a);
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (nb + i < N) a = fmaf(__uint_as_float(v[i]), __half2float(arow[i]), a);
+                        }
+                        sq += (double)a;
+                    }
+                } else if (EPI == 2) {
+                    if (m < M) {
+                        const int nb = n0 + col;
+                        float* crow = Cf + (int64_t)m * N + nb;
+                        if (nb + 32 <= N) {
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4)
+                                *reinterpret_cast<float4*>(crow + i) =
+                                    make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                                __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (nb + i < N) crow[i] = __uint_as_float(v[i]);
+                        }
+                    }
                 } else if (m < M) {
                     const int nb = n0 + col;
                     __half* yrow = Y + (int64_t)m * N + nb;
@@ -325,7 +368,7 @@ bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
     return r == CUDA_SUCCESS;
 }
 
-template <bool DEQ, bool SSE, int MT>
+template <bool DEQ, int EPI, int MT>
 static cudaError_t set_tc_attrs() {
     static std::once_flag once[64];
     static cudaError_t err[64];
@@ -334,16 +377,16 @@ static cudaError_t set_tc_attrs() {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&]() {
-        err[dev] = cudaFuncSetAttribute(tc_gemm_kernel<DEQ, SSE, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        err[dev] = cudaFuncSetAttribute(tc_gemm_kernel<DEQ, EPI, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)TcCfg<DEQ, MT>::kBytes);
     });
     return err[dev];
 }
 
-template <bool DEQ, bool SSE, int MT>
+template <bool DEQ, int EPI, int MT>
 static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int64_t N, int64_t K,
                              const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, double* sse_part,
-                             int* status, cudaStream_t stream) {
+                             int* status, cudaStream_t stream, float* Cf = nullptr) {
     using C = TcCfg<DEQ, MT>;
     CUtensorMap ta, tb;
     if (!make_tensor_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, TC_BK, C::kBM,
@@ -355,13 +398,13 @@ static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int6
             : make_tensor_map_2d(&tb, Bop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)N, TC_BK, TC_BN,
                           CU_TENSOR_MAP_SWIZZLE_128B);
     if (!okb) return cudaErrorInvalidValue;
-    cudaError_t e = set_tc_attrs<DEQ, SSE, MT>();
+    cudaError_t e = set_tc_attrs<DEQ, EPI, MT>();
     if (e != cudaSuccess) return e;
     const int m_tiles = (int)((M + C::kBM - 1) / C::kBM);
     const int n_tiles = (int)((N + TC_BN - 1) / TC_BN);
-    tc_gemm_kernel<DEQ, SSE, MT><<<m_tiles * n_tiles, TC_THREADS, C::kBytes, stream>>>(
-        ta, tb, reinterpret_cast<const __half*>(scales), zeros, reinterpret_cast<__half*>(Y), sse_part, (int)M,
-        (int)N, (int)K, m_tiles, n_tiles, status);
+    tc_gemm_kernel<DEQ, EPI, MT><<<m_tiles * n_tiles, TC_THREADS, C::kBytes, stream>>>(
+        ta, tb, reinterpret_cast<const __half*>(scales), zeros, reinterpret_cast<__half*>(Y), sse_part, Cf,
+        reinterpret_cast<const __half*>(X), (int)M, (int)N, (int)K, m_tiles, n_tiles, status);
     return cudaGetLastError();
 }
 
@@ -372,15 +415,30 @@ cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, con
                          const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,
                          cudaStream_t stream) {
     if (tc_mt(M) == 2)
-        return launch_tc<true, false, 2>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
-    return launch_tc<true, false, 1>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
+        return launch_tc<true, 0, 2>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
+    return launch_tc<true, 0, 1>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
 }
 
 cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64_t N, int64_t K,
                           double* sse_part, int* status, cudaStream_t stream) {
     if (tc_mt(T) == 2)
-        return launch_tc<false, true, 2>(X, T, E, N, K, nullptr, nullptr, nullptr, sse_part, status, stream);
-    return launch_tc<false, true, 1>(X, T, E, N, K, nullptr, nullptr, nullptr, sse_part, status, stream);
+        return launch_tc<false, 1, 2>(X, T, E, N, K, nullptr, nullptr, nullptr, sse_part, status, stream);
+    return launch_tc<false, 1, 1>(X, T, E, N, K, nullptr, nullptr, nullptr, sse_part, status, stream);
+}
+
+cudaError_t launch_tc_f32(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, float* C,
+                          int* status, cudaStream_t stream) {
+    if (tc_mt(M) == 2)
+        return launch_tc<false, 2, 2>(A, M, B, N, K, nullptr, nullptr, nullptr, nullptr, status, stream, C);
+    return launch_tc<false, 2, 1>(A, M, B, N, K, nullptr, nullptr, nullptr, nullptr, status, stream, C);
+}
+
+cudaError_t launch_tc_dot(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, double* part,
+                          int* status, cudaStream_t stream) {
+    if (N != K) return cudaErrorInvalidValue;  // the epilogue reads A[m, n] with n as a column of A
+    if (tc_mt(M) == 2)
+        return launch_tc<false, 3, 2>(A, M, B, N, K, nullptr, nullptr, nullptr, part, status, stream);
+    return launch_tc<false, 3, 1>(A, M, B, N, K, nullptr, nullptr, nullptr, part, status, stream);
 }
 
 int tc_sse_partials(int64_t T, int64_t N) {

@@ -59,7 +59,13 @@ cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, con
                          cudaStream_t stream);
 cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64_t N, int64_t K,
                           double* sse_part, int* status, cudaStream_t stream);
-int tc_sse_partials(int64_t T, int64_t N);
+int tc_sse_partials(int64_t T, int64_t N);  // tiles of an M = T x N launch (partials of EPI 1 and 3)
+// C [M, N] fp32 = A [M, K] . B [N, K]^T (both fp16, K-major, K % 64 == 0, row strides 16-byte multiples).
+cudaError_t launch_tc_f32(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, float* C,
+                          int* status, cudaStream_t stream);
+// Per-tile sum over (m, n) of (A . B^T)[m, n] * A[m, n] into part[tile] (requires N == K).
+cudaError_t launch_tc_dot(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, double* part,
+                          int* status, cudaStream_t stream);
 // 2-D tensor map (TMA descriptor) over a row-major matrix, through the driver entry point.
 bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, uint32_t elem_bytes,
                         uint64_t inner, uint64_t outer, uint32_t box_inner, uint32_t box_outer,
@@ -74,6 +80,19 @@ AwqLayout awq_layout(int64_t T, int64_t N, int64_t K, int n_alpha);
 cudaError_t launch_awq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int n_alpha,
                        double* mse, int32_t* best_idx, float* best_s, void* ws, int* status,
                        cudaStream_t stream);
+
+// AWQ search, Gram form (awq.cu).  Workspace layout (byte offsets, 256-byte aligned).
+struct AwqGramLayout {
+    size_t colsum, s_all, E, part, XT, G, G64, Gp, d, rd, bytes;
+    int64_t chunk;     // rows of X per Gram chunk (a multiple of 64)
+    int64_t n_chunks;
+    int64_t Tp;        // chunk * n_chunks: calibration rows padded with zeros
+    int n_part;
+};
+AwqGramLayout awq_gram_layout(int64_t T, int64_t N, int64_t K, int n_alpha);
+cudaError_t launch_awq_gram(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int n_alpha,
+                            double* mse, int32_t* best_idx, float* best_s, void* ws, int* status,
+                            cudaStream_t stream);
 
 // AWQ clip search (awq_clip.cu).  Workspace: Gram blocks, then per-split partial Gram blocks.
 struct AwqClipLayout {

@@ -33,6 +33,8 @@ SIGNATURES = {
     "awq_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_scale_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "awq_scale_search_noalloc": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P]),
+    "awq_gram_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
+    "awq_scale_search_gram": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "awq_clip_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_clip_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "w4_check_device_status": (_I32, [_P]),
@@ -215,6 +217,32 @@ def awq_scale_search(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20, group:
                                 ctypes.c_void_p(workspace.data_ptr()),
                                 workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "awq_scale_search")
+    return mse, best, best_s
+
+
+def awq_gram_workspace_size(T: int, N: int, K: int, group: int = 128, n_alpha: int = 20) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().awq_gram_workspace_size(T, N, K, group, n_alpha, ctypes.byref(n)), "awq_gram_workspace_size")
+    return n.value
+
+
+def awq_scale_search_gram(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20, group: int = 128,
+                          workspace: torch.Tensor | None = None, stream=None):
+    """awq_scale_search through the Gram matrix of X.  Returns (mse, best_idx, best_s) on the device."""
+    T, K = X.shape
+    N = W.shape[0]
+    need = awq_gram_workspace_size(T, N, K, group, n_alpha)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
+    mse = torch.empty(n_alpha, dtype=torch.float64, device=X.device)
+    best = torch.empty(1, dtype=torch.int32, device=X.device)
+    best_s = torch.empty(K, dtype=torch.float32, device=X.device)
+    st = lib().awq_scale_search_gram(_dev(X, torch.float16, "X"), T, _dev(W, torch.float16, "W"), N, K,
+                                     group, n_alpha, ctypes.c_void_p(mse.data_ptr()),
+                                     ctypes.c_void_p(best.data_ptr()), ctypes.c_void_p(best_s.data_ptr()),
+                                     ctypes.c_void_p(workspace.data_ptr()),
+                                     workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "awq_scale_search_gram")
     return mse, best, best_s
 
 
