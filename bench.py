@@ -440,17 +440,10 @@ def bench_quantize(world, peaks, l2, reps=10):
     return {"kernel": "quantize_pack_kernel", "bound": "hbm", "layers": res}
 
 
-def bench_awq(world, peaks, reps=2):
-    """awq_scale_search on X_calib [65536, 4096], W [4096, 4096], 20 alphas."""
+def _time_awq_search(world, search, Xd, Wd, ws, reps):
+    """Min over reps of one search call's CUDA-event time (ms), max over ranks."""
     import torch
-    from weight_only_int4_06_b200 import w4a16 as B
-    X, W = synth.awq_case()
-    Xd = torch.from_numpy(X).cuda()
-    Wd = torch.from_numpy(W).cuda()
-    T, K = X.shape
-    N = W.shape[0]
-    ws = torch.empty(B.awq_workspace_size(T, N, K, 128, 20), dtype=torch.uint8, device="cuda")
-    B.awq_scale_search(Xd, Wd, 20, workspace=ws)
+    search(Xd, Wd, 20, workspace=ws)
     torch.cuda.synchronize()
     times = []
     for _ in range(reps):
@@ -459,11 +452,24 @@ def bench_awq(world, peaks, reps=2):
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record()
-        B.awq_scale_search(Xd, Wd, 20, workspace=ws)
+        search(Xd, Wd, 20, workspace=ws)
         e1.record()
         torch.cuda.synchronize()
         times.append(e0.elapsed_time(e1))
-    t = max_over_ranks(min(times), world)
+    return max_over_ranks(min(times), world)
+
+
+def bench_awq(world, peaks, case, reps=2):
+    """awq_scale_search on X_calib [65536, 4096], W [4096, 4096], 20 alphas."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    X, W = case
+    Xd = torch.from_numpy(X).cuda()
+    Wd = torch.from_numpy(W).cuda()
+    T, K = X.shape
+    N = W.shape[0]
+    ws = torch.empty(B.awq_workspace_size(T, N, K, 128, 20), dtype=torch.uint8, device="cuda")
+    t = _time_awq_search(world, B.awq_scale_search, Xd, Wd, ws, reps)
     flops = 20 * 2 * T * K * N
     tf = flops / (t * 1e-3) / 1e12
     del Xd, Wd, ws
@@ -474,15 +480,37 @@ def bench_awq(world, peaks, reps=2):
             "flops": flops}
 
 
+def bench_awq_gram(world, peaks, case, reps=3):
+    """awq_scale_search_gram on the same calibration layer: G = X^T X once, then 20 K x K forms."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    X, W = case
+    Xd = torch.from_numpy(X).cuda()
+    Wd = torch.from_numpy(W).cuda()
+    T, K = X.shape
+    N = W.shape[0]
+    ws = torch.empty(B.awq_gram_workspace_size(T, N, K, 128, 20), dtype=torch.uint8, device="cuda")
+    t = _time_awq_search(world, B.awq_scale_search_gram, Xd, Wd, ws, reps)
+    flops = 2 * T * K * K + 20 * 2 * N * K * K  # Gram + one quadratic-form GEMM per alpha
+    tf = flops / (t * 1e-3) / 1e12
+    del Xd, Wd, ws
+    torch.cuda.empty_cache()
+    return {"kernel": "transpose + 16 x (tc_gemm_kernel<f32 out> + fp64 add) + scale + "
+                      "20 x (fakequant + tc_gemm_kernel<quadratic form>) + finalize",
+            "T": T, "K": K, "N": N, "n_alpha": 20, "ms": round(t, 3), "TFLOPs": round(tf, 1),
+            "bound": "tensor", "tensor_frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 3),
+            "flops": flops}
+
+
 FP32_FMA_PER_CLK_PER_SM = 128     # B200 SM: 4 partitions x 32 fp32 FMA lanes
 B200_SMS, B200_MAX_SM_MHZ = 148, 1965
 
 
-def bench_awq_clip(world, peaks, reps=3, n_ratios=10):
+def bench_awq_clip(world, peaks, case, reps=3, n_ratios=10):
     """awq_clip_search on X_calib [65536, 4096], W [4096, 4096], 10 ratios, with an AWQ scale."""
     import torch
     from weight_only_int4_06_b200 import w4a16 as B
-    X, W = synth.awq_case()
+    X, W = case
     Xd = torch.from_numpy(X).cuda()
     Wd = torch.from_numpy(W).cuda()
     T, K = X.shape
@@ -528,8 +556,11 @@ def other_rows(args, world, peaks, l2):
                        "layers": layer_rows(pre, world, reps, peaks, True)}
     del pre
     torch.cuda.empty_cache()
-    rows["awq"] = bench_awq(world, peaks)
-    rows["awq_clip"] = bench_awq_clip(world, peaks)
+    case = synth.awq_case()
+    rows["awq"] = bench_awq(world, peaks, case)
+    rows["awq_gram"] = bench_awq_gram(world, peaks, case)
+    rows["awq_gram"]["speedup_vs_direct"] = round(rows["awq"]["ms"] / rows["awq_gram"]["ms"], 2)
+    rows["awq_clip"] = bench_awq_clip(world, peaks, case)
     return rows
 
 

@@ -254,9 +254,9 @@ cudaError_t launch_awq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t 
 // Gram form of the same search.  sum_{t,n} (X E_i^T)^2 = sum_n e_n^T G e_n with G = X^T X, so the T
 // calibration rows are read once: G on the tensor cores, then per alpha one GEMM over K x K instead
 // of T x K.  G is formed chunk by chunk: each chunk of at most GRAM_CHUNK rows is one fp32
-// tensor-core product (the same accumulation length as the direct form's K-long dot products; one
-// fp32 accumulator over all 65536 rows showed a systematic 4e-4 relative shortfall), and the chunks
-// are summed in fp64 in chunk order.  G carries the squared activations' dynamic range (beyond
+// tensor-core product (the same accumulation length as the direct form's K-long dot products; with
+// one fp32 accumulator over all 65536 calibration rows the two forms differed by a uniform 4e-4
+// relative), and the chunks are summed in fp64 in chunk order.  G carries the squared activations' dynamic range (beyond
 // fp16), so it is scaled symmetrically: d_k = sqrt(G_kk) (1 for a channel that is zero in every
 // row), G' = D^-1 G D^-1 with entries in [-1, 1] in fp16, and E'_i = E_i D in fp16, so that
 // e^T G e = e'^T G' e'.  The per-alpha GEMM E' G'^T has an epilogue that sums (E' G'^T)[n, k] E'[n, k]
