@@ -35,6 +35,9 @@
  *                          the outputs of that call are unspecified
  *      W4_ERR_DEVICE_TIMEOUT  a bounded wait inside a kernel gave up; that kernel's outputs are
  *                          unspecified and the context stays usable
+ *      W4_ERR_NUMERIC      gptq_quantize: the damped Hessian is not positive definite (a zero
+ *                          damp with fewer calibration rows than K, or non-finite inputs); the
+ *                          outputs of that call are unspecified
  *  - Results are deterministic: the same inputs give bit-identical outputs (no floating-point
  *    atomics; every reduction has a fixed order).
  *  - Thread safety: calls may come from several host threads; the only shared state is the
@@ -66,7 +69,8 @@ typedef enum {
     W4_ERR_WORKSPACE = 5,
     W4_ERR_CUDA = 6,
     W4_ERR_DEVICE_TIMEOUT = 7,
-    W4_ERR_RANGE = 8
+    W4_ERR_RANGE = 8,
+    W4_ERR_NUMERIC = 9
 } w4_status;
 
 /* Kernel families of w4_gemm_ex (w4_gemm picks one per shape). */
@@ -252,6 +256,38 @@ w4_status awq_gram_workspace_size(int64_t T, int64_t N, int64_t K, int group, in
 w4_status awq_scale_search_gram(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N,
                                 int64_t K, int group, int n_alpha, double* mse, int32_t* best_idx,
                                 float* best_s, void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of device workspace gptq_quantize needs for this problem (T does not change it). */
+w4_status gptq_workspace_size(int64_t T, int64_t N, int64_t K, int group, size_t* bytes);
+
+/*
+ * gptq_quantize -- GPTQ: quantise W column by column, paying for each column's rounding error
+ * with the columns not yet quantised, and emit w4_quantize_pack's format (so w4_gemm serves it).
+ *
+ * Follows "GPTQ, AWQ and the rules of post-training quantization", section "GPTQ: pay for the
+ * error with the other weights" (a fixed column order, compensation through the inverse Hessian
+ * of the layer's reconstruction loss via a Cholesky factorisation, lazily batched updates):
+ *     H   = X^T X + lambda I, lambda = damp * mean(diag(X^T X))   (fp64; damp 0.01 is usual)
+ *     U   = the upper triangular factor with H^-1 = U^T U          (fp64)
+ *     for each group of 128 columns, left to right:
+ *         scale s (fp16, rounded up) and zero point z by w4_quantize_pack's rule from the group's
+ *         current weights rounded to fp32;
+ *         for each column k of the group: q_k = clamp(rint(fp32(w_k) / s) + z, 0, 15) (fp32,
+ *         exactly w4_quantize_pack's decision); e = (w_k - (q_k - z) s) / U_kk;
+ *         w_j -= e U_kj for every later column j (fp64; columns beyond the group lazily, one
+ *         product per group).
+ *   X [T, K] fp16 calibration activations; W [N, K] fp16 (not modified).
+ *   packed [N, K/8] uint32, scales [N, K/128] fp16, zeros [N, K/128] uint8 out, as
+ *   w4_quantize_pack's.
+ *   damp >= 0 and finite (else W4_ERR_UNSUPPORTED); K <= 32768 (else W4_ERR_SHAPE).
+ *   ws: device workspace of at least gptq_workspace_size bytes (16 K^2 + 8 N K bytes and a little).
+ * A Hessian that is not positive definite sets W4_ERR_NUMERIC in the device status.  The codes
+ * equal those of the same algorithm in exact arithmetic except where fp64 rounding moves a value
+ * across a rounding boundary of the fp32 quantiser.
+ */
+w4_status gptq_quantize(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K,
+                        int group, double damp, uint32_t* packed, uint16_t* scales, uint8_t* zeros,
+                        void* ws, size_t ws_bytes, void* stream);
 
 /* Bytes of device workspace awq_clip_search needs for this problem. */
 w4_status awq_clip_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_ratios,

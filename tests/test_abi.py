@@ -31,7 +31,7 @@ def test_header_declares_expected_api():
     names = declared_functions()
     for n in ("w4_quantize_pack", "w4_gemm", "w4_gemm_ex", "w4_gemm_host", "w4_gemm_workspace_size",
               "awq_scale_search", "awq_workspace_size", "awq_clip_search", "awq_clip_workspace_size",
-              "awq_scale_search_gram", "awq_gram_workspace_size",
+              "awq_scale_search_gram", "awq_gram_workspace_size", "gptq_quantize", "gptq_workspace_size",
               "w4_check_device_status", "w4_status_string"):
         assert n in names, n
 
@@ -152,3 +152,24 @@ def test_gemm_host_rejects(L):
     assert L.w4_gemm_host(*args(xd=None)) == 1
     assert L.w4_gemm_host(*args(yd=None)) == 1
     assert L.w4_gemm_host(*args(M=0)) == 0  # empty: nothing enqueued
+
+
+def test_gptq_rejects(L):
+    P = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(1 << 12)
+    d = P(ctypes.addressof(buf) + (-ctypes.addressof(buf) % 16))
+    n = ctypes.c_size_t(0)
+    assert L.gptq_workspace_size(100, 64, 512, 128, ctypes.byref(n)) == 0
+    assert n.value >= 512 * 512 * 16 + 64 * 512 * 8  # H and its factors in fp64, W in fp64
+    assert L.gptq_workspace_size(100, 64, 512, 64, ctypes.byref(n)) == 4
+    assert L.gptq_workspace_size(100, 60, 512, 128, ctypes.byref(n)) == 2
+    assert L.gptq_workspace_size(100, 64, 65536, 128, ctypes.byref(n)) == 2  # K above 32768
+    args = lambda **kw: [kw.get("X", d), 100, kw.get("W", d), 64, 512, kw.get("group", 128),
+                         kw.get("damp", 0.01), kw.get("p", d), d, d, kw.get("ws", d), kw.get("ws_bytes", 1 << 40),
+                         None]
+    assert L.gptq_quantize(*args(group=64)) == 4
+    assert L.gptq_quantize(*args(damp=-1.0)) == 4
+    assert L.gptq_quantize(*args(damp=float("nan"))) == 4
+    assert L.gptq_quantize(*args(ws_bytes=16)) == 5
+    assert L.gptq_quantize(*args(X=None)) == 1
+    assert L.gptq_quantize(*args(p=P(d.value + 4))) == 3

@@ -235,6 +235,37 @@ w4_status awq_scale_search_gram(const uint16_t* X, int64_t T, const uint16_t* W,
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
+static w4_status gptq_check(int64_t T, int64_t N, int64_t K, int group) {
+    if (group != 128) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(T, K) || !dims_ok(N, K) || T < 1 || N < 8 || K < 128 || K > 32768 || K % group != 0 ||
+        N % 8 != 0)
+        return W4_ERR_SHAPE;
+    return W4_OK;
+}
+
+w4_status gptq_workspace_size(int64_t T, int64_t N, int64_t K, int group, size_t* bytes) {
+    if (!bytes) return W4_ERR_NULL;
+    w4_status st = gptq_check(T, N, K, group);
+    if (st != W4_OK) return st;
+    *bytes = gptq_layout(N, K).bytes;
+    return W4_OK;
+}
+
+w4_status gptq_quantize(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int group,
+                        double damp, uint32_t* packed, uint16_t* scales, uint8_t* zeros, void* ws,
+                        size_t ws_bytes, void* stream) {
+    w4_status st = gptq_check(T, N, K, group);
+    if (st != W4_OK) return st;
+    if (!(damp >= 0.0) || !(damp < 1.0e300)) return W4_ERR_UNSUPPORTED;  // rejects NaN and inf too
+    if (ws_bytes < gptq_layout(N, K).bytes) return W4_ERR_WORKSPACE;
+    if (!X || !W || !packed || !scales || !zeros || !ws) return W4_ERR_NULL;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(packed) || !aligned16(ws)) return W4_ERR_ALIGN;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_gptq(X, T, W, N, K, damp, packed, scales, zeros, ws, status, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 static w4_status clip_check(int64_t T, int64_t N, int64_t K, int group, int n_ratios) {
     if (group != 128 || n_ratios < 1 || n_ratios > 10) return W4_ERR_UNSUPPORTED;
     if (!dims_ok(T, K) || !dims_ok(N, K) || T < 1 || N < 8 || K < 128 || K % group != 0 || N % 8 != 0)
@@ -288,6 +319,7 @@ const char* w4_status_string(w4_status status) {
         case W4_ERR_CUDA: return "CUDA launch or query failed";
         case W4_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
         case W4_ERR_RANGE: return "fp16 group scale overflow";
+        case W4_ERR_NUMERIC: return "matrix not positive definite (GPTQ Hessian)";
     }
     return "unknown status";
 }

@@ -94,6 +94,15 @@ cudaError_t launch_awq_gram(const uint16_t* X, int64_t T, const uint16_t* W, int
                             double* mse, int32_t* best_idx, float* best_s, void* ws, int* status,
                             cudaStream_t stream);
 
+// GPTQ quantiser (gptq.cu).  Workspace layout (byte offsets, 256-byte aligned).
+struct GptqLayout {
+    size_t H, P, W64, E, lambda, bytes;
+};
+GptqLayout gptq_layout(int64_t N, int64_t K);
+cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, double damp,
+                        uint32_t* packed, uint16_t* scales, uint8_t* zeros, void* ws, int* status,
+                        cudaStream_t stream);
+
 // AWQ clip search (awq_clip.cu).  Workspace: Gram blocks, then per-split partial Gram blocks.
 struct AwqClipLayout {
     size_t gram, part, bytes;

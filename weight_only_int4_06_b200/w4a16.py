@@ -35,6 +35,8 @@ SIGNATURES = {
     "awq_scale_search_noalloc": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P]),
     "awq_gram_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_scale_search_gram": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
+    "gptq_workspace_size": (_I32, [_I64, _I64, _I64, _I32, ctypes.POINTER(_SZ)]),
+    "gptq_quantize": (_I32, [_P, _I64, _P, _I64, _I64, _I32, ctypes.c_double, _P, _P, _P, _P, _SZ, _P]),
     "awq_clip_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_clip_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "w4_check_device_status": (_I32, [_P]),
@@ -244,6 +246,32 @@ def awq_scale_search_gram(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20, g
                                      workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "awq_scale_search_gram")
     return mse, best, best_s
+
+
+def gptq_workspace_size(T: int, N: int, K: int, group: int = 128) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().gptq_workspace_size(T, N, K, group, ctypes.byref(n)), "gptq_workspace_size")
+    return n.value
+
+
+def gptq_quantize(X: torch.Tensor, W: torch.Tensor, damp: float = 0.01, group: int = 128,
+                  workspace: torch.Tensor | None = None, stream=None):
+    """GPTQ on one layer.  Returns (packed [N, K/8] int32 view of uint32, scales [N, K/128] fp16,
+    zeros [N, K/128] uint8) on the device, in w4_quantize_pack's format."""
+    T, K = X.shape
+    N = W.shape[0]
+    need = gptq_workspace_size(T, N, K, group)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
+    packed = torch.empty(N, K // 8, dtype=torch.int32, device=X.device)
+    scales = torch.empty(N, K // group, dtype=torch.float16, device=X.device)
+    zeros = torch.empty(N, K // group, dtype=torch.uint8, device=X.device)
+    st = lib().gptq_quantize(_dev(X, torch.float16, "X"), T, _dev(W, torch.float16, "W"), N, K, group,
+                             float(damp), ctypes.c_void_p(packed.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                             ctypes.c_void_p(zeros.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "gptq_quantize")
+    return packed, scales, zeros
 
 
 def awq_scale_search_noalloc(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20, group: int = 128,
