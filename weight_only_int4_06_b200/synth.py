@@ -18,6 +18,11 @@ on, which are not available here):
   1 % x20 outlier channels, cast to fp16.  T = 65536 mirrors the
   "128 sequences" calibration set of the same page (128 x 512 tokens).
 
+* correlated calibration activations (GPTQ cases): X = Z A * 0.3 + 0.1 E with Z [T, r] and
+  E [T, K] ~ N(0, 1) and a mixing matrix A [r, K] ~ N(0, 1), r = K / 8, cast to fp16.  Real
+  activations have strongly correlated channels, which is what GPTQ's compensation exploits; the
+  independent-channel recipe above leaves it almost nothing to exploit.
+
 Seeds: the single-layer smoke case uses ``seed = 0``; every other case uses the
 sequence seed ``[case_id, M, K, N]`` and draws, in this fixed order, W, X and
 then the outlier channel set.
@@ -97,3 +102,18 @@ def awq_subsample_rows(T: int = AWQ_T, n: int = AWQ_SUBSAMPLE, case_id: int = 5)
     """Seeded row subsample (sorted, without replacement) used to check the search on the CPU."""
     rng = np.random.default_rng([case_id, T, n, 7])
     return np.sort(rng.choice(T, n, replace=False))
+
+
+def correlated_case(T: int, K: int, N: int, case_id: int = 9):
+    """GPTQ calibration layer with correlated channels: X [T, K] (rank K/8 plus noise), W [N, K].
+
+    Returns (X, W) as fp16 numpy arrays.  Draw order: W, Z, A, E.
+    """
+    rng = np.random.default_rng([case_id, T, K, N, 77])
+    W = _to_f16(rng.standard_normal((N, K), dtype=np.float32) * np.float32(W_STD))
+    r = max(1, K // 8)
+    Z = rng.standard_normal((T, r), dtype=np.float32)
+    A = rng.standard_normal((r, K), dtype=np.float32)
+    E = rng.standard_normal((T, K), dtype=np.float32)
+    X = (Z @ A) * np.float32(0.3) + np.float32(0.1) * E
+    return _to_f16(X), W
