@@ -6,8 +6,8 @@ fp32(w); the weights they decide on are fp64 values that differ only by rounding
 factors the Hessian blockwise and applies far-column updates as one product per group).  So the
 codes, scales and zero points must be identical, except in a row whose first difference sits at
 a rounding boundary of the oracle's own decision (margin below 1e-6 of a step): after such a flip
-the row legitimately diverges.  At most one such row per 100 is accepted.  The file sorts after
-the other GPU parity files so that a run stopping at the first failure has already run those."""
+the row legitimately diverges.  At most one such row per 100 is accepted.  The file sorts after every
+other test file so that a run stopping at the first failure has already run all of those."""
 import numpy as np
 import pytest
 import torch
