@@ -257,7 +257,8 @@ w4_status awq_scale_search_gram(const uint16_t* X, int64_t T, const uint16_t* W,
                                 int64_t K, int group, int n_alpha, double* mse, int32_t* best_idx,
                                 float* best_s, void* ws, size_t ws_bytes, void* stream);
 
-/* Bytes of device workspace gptq_quantize needs for this problem (T does not change it). */
+/* Bytes of device workspace gptq_quantize / gptq_quantize_ex need (group 64 or 128; T does not
+ * change it). */
 w4_status gptq_workspace_size(int64_t T, int64_t N, int64_t K, int group, size_t* bytes);
 
 /*
@@ -288,6 +289,71 @@ w4_status gptq_workspace_size(int64_t T, int64_t N, int64_t K, int group, size_t
 w4_status gptq_quantize(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K,
                         int group, double damp, uint32_t* packed, uint16_t* scales, uint8_t* zeros,
                         void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * gptq_quantize_ex -- gptq_quantize at other widths, group sizes and column orders.
+ *
+ * bits in {2, 3, 4, 8} and group in {64, 128} ("AutoGPTQ vs The Stack v2": 2/3/4/8-bit GPTQ with
+ * per-group quantisation; INT3 g128 and INT2 g64 in "GPTQ, AWQ and the rules of post-training
+ * quantization"), else W4_ERR_UNSUPPORTED.  The quantiser is w4_quantize_pack's with L = 2^bits - 1
+ * steps; codes are packed as w4_quantize_pack_bits packs them.
+ * act_order != 0 (desc_act): the columns are processed in decreasing diag(X^T X), ties in index
+ * order; the outputs are stored in PROCESSING order and perm [K] int32 (device, required then)
+ * receives perm[i] = the original column processed i-th.  Serve such weights with
+ * w4_act_prepare(X, perm) followed by the matmul.
+ *   packed [N, K*bits/32] uint32, scales / zeros [N, K/group].  K <= 32768.
+ *   ws: at least gptq_workspace_size(T, N, K, group) bytes.
+ * gptq_quantize(...) is gptq_quantize_ex(bits 4, group 128, act_order 0).
+ */
+w4_status gptq_quantize_ex(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K,
+                           int bits, int group, double damp, int act_order, uint32_t* packed,
+                           uint16_t* scales, uint8_t* zeros, int32_t* perm, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * w4_quantize_pack_bits -- w4_quantize_pack at other widths and group sizes.
+ *
+ * bits in {2, 3, 4, 8}, group in {64, 128} (else W4_ERR_UNSUPPORTED).  The quantiser's rules with
+ * L = 2^bits - 1 steps: lo = min(0, min v), hi = max(0, max v), s32 = (hi - lo) / L, fp16 scale
+ * rounded up (1 for an all-zero group), z = clamp(rint(-lo / s16), 0, L),
+ * q = clamp(rint(v / s16) + z, 0, L).  Codes form one little-endian bit stream per row: code k
+ * occupies bits bits*k .. bits*k + bits - 1, stream bit j is bit j % 32 of word j / 32 (a 3-bit
+ * code may straddle two words; bits 4 gives exactly w4_quantize_pack's layout).
+ *   W [N, K] fp16; act_scale [K] fp32 or NULL; packed [N, K*bits/32] uint32; scales [N, K/group]
+ *   fp16; zeros [N, K/group] uint8.  N % 8 == 0, K % group == 0.
+ */
+w4_status w4_quantize_pack_bits(const uint16_t* W, int64_t N, int64_t K, int bits, int group,
+                                const float* act_scale, uint32_t* packed, uint16_t* scales,
+                                uint8_t* zeros, void* stream);
+
+/* Bytes of device workspace wb_gemm needs: N * K * 2 (the dequantised weights). */
+w4_status wb_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits, int group,
+                                 size_t* bytes);
+
+/*
+ * wb_gemm -- Y = X . dequant(W)^T for w4_quantize_pack_bits' format at any supported width.
+ *
+ * Two passes: every weight is dequantised to fp16 (w = (q - z) s, exact in fp32, rounded once to
+ * fp16) into ws, then the tcgen05 GEMM multiplies with fp32 accumulation and writes fp16 Y.  Not
+ * fused (w4_gemm's fused kernels serve 4-bit, group-128 weights); meant for the other widths.
+ *   X [M, K] fp16, Y [M, N] fp16, ws >= wb_gemm_workspace_size bytes; all 16-byte aligned.
+ */
+w4_status wb_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                  const uint16_t* scales, const uint8_t* zeros, int bits, int group, uint16_t* Y,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * w4_act_prepare -- activations for act-order weights and/or an activation-side scale.
+ *
+ * X_out[m, i] = X[m, src], src = perm[i] (or i when perm is NULL), divided by s[src] when s is
+ * not NULL: fp16(fp32(x) / s) with one IEEE division.  With act-order weights from
+ * gptq_quantize_ex, X_out . dequant(W)^T (w4_gemm or wb_gemm) is the layer's output; with AWQ's
+ * scale s and weights quantised as W * diag(s), it folds the division of the activations into
+ * the same pass.  A perm entry outside [0, K) sets W4_ERR_RANGE and yields 0.
+ *   X, X_out [M, K] fp16 (distinct buffers); perm [K] int32 or NULL; s [K] fp32 or NULL.
+ */
+w4_status w4_act_prepare(const uint16_t* X, int64_t M, int64_t K, const int32_t* perm, const float* s,
+                         uint16_t* X_out, void* stream);
 
 /* Bytes of device workspace awq_clip_search needs for this problem. */
 w4_status awq_clip_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_ratios,

@@ -167,19 +167,7 @@ def dequantize_g_idx(q_orig: np.ndarray, scales: np.ndarray, zeros: np.ndarray, 
 # ----------------------------------------------------------------------------
 # GPTQ at any width, natural or act-order
 # ----------------------------------------------------------------------------
-def gptq_quantize_bits(X: np.ndarray, W: np.ndarray, bits: int = 4, group: int = 128, damp: float = 0.01,
-                       act_order: bool = False):
-    """GPTQ ("GPTQ, AWQ and the rules of post-training quantization", section "GPTQ: pay for the error
-    with the other weights") with b-bit groups, columns in natural or act-order.
-
-    H = X^T X + damp * mean(diag) I in fp64; with act-order, columns, H's rows and columns and W's
-    columns are first permuted by perm.  U = upper Cholesky factor of H^-1.  For each column k in
-    processing order: at a group's first column its scale and zero point come from the group's
-    current weights rounded to fp32; q_k = clamp(rint(fp32(w_k) / s) + z, 0, L);
-    e = (w_k - (q_k - z) s) / U_kk; w_j -= e U_kj for later j.
-    Returns (packed, scales, zeros, perm), outputs in processing order (perm = arange when
-    act_order is False).
-    """
+def _gptq_bits(X, W, bits, group, damp, act_order, stop_after):
     L = levels(bits)
     X64 = np.asarray(X).astype(np.float64)
     Wc = np.asarray(W, dtype=np.float16).astype(np.float64).copy()
@@ -196,7 +184,7 @@ def gptq_quantize_bits(X: np.ndarray, W: np.ndarray, bits: int = 4, group: int =
     s16 = np.zeros((N, G), dtype=np.float16)
     z = np.zeros((N, G), dtype=np.uint8)
     sf = zg = None
-    for k in range(K):
+    for k in range(K if stop_after is None else stop_after):
         if k % group == 0:
             sg, sf, zg = _params(Wc[:, k:k + group].astype(np.float32), L)
             s16[:, k // group] = sg
@@ -207,7 +195,31 @@ def gptq_quantize_bits(X: np.ndarray, W: np.ndarray, bits: int = 4, group: int =
         w_hat = (qk.astype(np.float64) - zg.astype(np.float64)) * sf.astype(np.float64)
         e = (Wc[:, k] - w_hat) / U[k, k]
         Wc[:, k + 1:] -= np.outer(e, U[k, k + 1:])
+    return q, s16, z, Wc, perm
+
+
+def gptq_quantize_bits(X: np.ndarray, W: np.ndarray, bits: int = 4, group: int = 128, damp: float = 0.01,
+                       act_order: bool = False):
+    """GPTQ ("GPTQ, AWQ and the rules of post-training quantization", section "GPTQ: pay for the error
+    with the other weights") with b-bit groups, columns in natural or act-order.
+
+    H = X^T X + damp * mean(diag) I in fp64; with act-order, columns, H's rows and columns and W's
+    columns are first permuted by perm.  U = upper Cholesky factor of H^-1.  For each column k in
+    processing order: at a group's first column its scale and zero point come from the group's
+    current weights rounded to fp32; q_k = clamp(rint(fp32(w_k) / s) + z, 0, L);
+    e = (w_k - (q_k - z) s) / U_kk; w_j -= e U_kj for later j.
+    Returns (packed, scales, zeros, perm), outputs in processing order (perm = arange when
+    act_order is False).
+    """
+    q, s16, z, _, perm = _gptq_bits(X, W, bits, group, damp, act_order, None)
     return pack_bits(q, bits), s16, z, perm
+
+
+def gptq_state_bits(X: np.ndarray, W: np.ndarray, bits: int, group: int, damp: float, act_order: bool,
+                    stop_after: int):
+    """The weights in processing order after the first stop_after columns (for tests), and perm."""
+    _, _, _, Wc, perm = _gptq_bits(X, W, bits, group, damp, act_order, stop_after)
+    return Wc, perm
 
 
 # ----------------------------------------------------------------------------

@@ -32,6 +32,7 @@ def test_header_declares_expected_api():
     for n in ("w4_quantize_pack", "w4_gemm", "w4_gemm_ex", "w4_gemm_host", "w4_gemm_workspace_size",
               "awq_scale_search", "awq_workspace_size", "awq_clip_search", "awq_clip_workspace_size",
               "awq_scale_search_gram", "awq_gram_workspace_size", "gptq_quantize", "gptq_workspace_size",
+              "gptq_quantize_ex", "w4_quantize_pack_bits", "wb_gemm", "wb_gemm_workspace_size", "w4_act_prepare",
               "w4_check_device_status", "w4_status_string"):
         assert n in names, n
 
@@ -161,7 +162,8 @@ def test_gptq_rejects(L):
     n = ctypes.c_size_t(0)
     assert L.gptq_workspace_size(100, 64, 512, 128, ctypes.byref(n)) == 0
     assert n.value >= 512 * 512 * 16 + 64 * 512 * 8  # H and its factors in fp64, W in fp64
-    assert L.gptq_workspace_size(100, 64, 512, 64, ctypes.byref(n)) == 4
+    assert L.gptq_workspace_size(100, 64, 512, 32, ctypes.byref(n)) == 4
+    assert L.gptq_workspace_size(100, 64, 576, 64, ctypes.byref(n)) == 0  # group 64 (quantize_ex)
     assert L.gptq_workspace_size(100, 60, 512, 128, ctypes.byref(n)) == 2
     assert L.gptq_workspace_size(100, 64, 65536, 128, ctypes.byref(n)) == 2  # K above 32768
     args = lambda **kw: [kw.get("X", d), 100, kw.get("W", d), 64, 512, kw.get("group", 128),
@@ -173,3 +175,32 @@ def test_gptq_rejects(L):
     assert L.gptq_quantize(*args(ws_bytes=16)) == 5
     assert L.gptq_quantize(*args(X=None)) == 1
     assert L.gptq_quantize(*args(p=P(d.value + 4))) == 3
+
+
+def test_width_calls_reject(L):
+    P = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(1 << 12)
+    d = P(ctypes.addressof(buf) + (-ctypes.addressof(buf) % 16))
+    q = lambda **kw: [kw.get("W", d), 64, kw.get("K", 512), kw.get("bits", 3), kw.get("group", 128), None, d, d, d,
+                      None]
+    assert L.w4_quantize_pack_bits(*q(bits=5)) == 4
+    assert L.w4_quantize_pack_bits(*q(group=32)) == 4
+    assert L.w4_quantize_pack_bits(*q(K=500)) == 2
+    assert L.w4_quantize_pack_bits(*q(W=None)) == 1
+    assert L.w4_quantize_pack_bits(*q(W=P(d.value + 2))) == 3
+    n = ctypes.c_size_t(0)
+    assert L.wb_gemm_workspace_size(4, 64, 512, 3, 128, ctypes.byref(n)) == 0 and n.value == 64 * 512 * 2
+    assert L.wb_gemm_workspace_size(4, 64, 512, 6, 128, ctypes.byref(n)) == 4
+    g = lambda **kw: [d, 4, 64, 512, d, d, d, kw.get("bits", 2), kw.get("group", 64), kw.get("Y", d), d,
+                      kw.get("ws_bytes", 1 << 30), None]
+    assert L.wb_gemm(*g(bits=1)) == 4
+    assert L.wb_gemm(*g(ws_bytes=100)) == 5
+    assert L.wb_gemm(*g(Y=None)) == 1
+    e = lambda **kw: [d, 100, d, 64, 512, kw.get("bits", 3), kw.get("group", 128), kw.get("damp", 0.01),
+                      kw.get("ao", 0), d, d, d, kw.get("perm", None), d, kw.get("ws_bytes", 1 << 40), None]
+    assert L.gptq_quantize_ex(*e(bits=7)) == 4
+    assert L.gptq_quantize_ex(*e(group=256)) == 4
+    assert L.gptq_quantize_ex(*e(ao=1)) == 1  # act-order needs perm
+    assert L.gptq_quantize_ex(*e(ws_bytes=8)) == 5
+    assert L.w4_act_prepare(None, 2, 128, None, None, d, None) == 1
+    assert L.w4_act_prepare(d, 0, 128, None, None, d, None) == 0

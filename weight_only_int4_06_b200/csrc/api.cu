@@ -235,17 +235,23 @@ w4_status awq_scale_search_gram(const uint16_t* X, int64_t T, const uint16_t* W,
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
-static w4_status gptq_check(int64_t T, int64_t N, int64_t K, int group) {
-    if (group != 128) return W4_ERR_UNSUPPORTED;
-    if (!dims_ok(T, K) || !dims_ok(N, K) || T < 1 || N < 8 || K < 128 || K > 32768 || K % group != 0 ||
+// group 64 or 128 (the Cholesky's 32-wide panels need K % 32 == 0, which K % group == 0 gives)
+static w4_status gptq_shape(int64_t T, int64_t N, int64_t K, int group) {
+    if (!dims_ok(T, K) || !dims_ok(N, K) || T < 1 || N < 8 || K < group || K > 32768 || K % group != 0 ||
         N % 8 != 0)
         return W4_ERR_SHAPE;
     return W4_OK;
 }
 
+static w4_status gptq_check(int64_t T, int64_t N, int64_t K, int group) {
+    if (group != 128) return W4_ERR_UNSUPPORTED;
+    return gptq_shape(T, N, K, group);
+}
+
 w4_status gptq_workspace_size(int64_t T, int64_t N, int64_t K, int group, size_t* bytes) {
     if (!bytes) return W4_ERR_NULL;
-    w4_status st = gptq_check(T, N, K, group);
+    if (group != 64 && group != 128) return W4_ERR_UNSUPPORTED;
+    w4_status st = gptq_shape(T, N, K, group);
     if (st != W4_OK) return st;
     *bytes = gptq_layout(N, K).bytes;
     return W4_OK;
@@ -262,7 +268,80 @@ w4_status gptq_quantize(const uint16_t* X, int64_t T, const uint16_t* W, int64_t
     if (!aligned16(X) || !aligned16(W) || !aligned16(packed) || !aligned16(ws)) return W4_ERR_ALIGN;
     int* status = device_status_ptr();
     if (!status) return W4_ERR_CUDA;
-    cudaError_t e = launch_gptq(X, T, W, N, K, damp, packed, scales, zeros, ws, status, (cudaStream_t)stream);
+    cudaError_t e = launch_gptq(X, T, W, N, K, 4, 128, damp, false, packed, scales, zeros, nullptr, ws, status,
+                                (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+static bool bits_ok(int bits, int group) {
+    return (bits == 2 || bits == 3 || bits == 4 || bits == 8) && (group == 64 || group == 128);
+}
+
+w4_status gptq_quantize_ex(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int bits,
+                           int group, double damp, int act_order, uint32_t* packed, uint16_t* scales,
+                           uint8_t* zeros, int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+    if (!bits_ok(bits, group)) return W4_ERR_UNSUPPORTED;
+    w4_status st = gptq_shape(T, N, K, group);
+    if (st != W4_OK) return st;
+    if (!(damp >= 0.0) || !(damp < 1.0e300)) return W4_ERR_UNSUPPORTED;
+    if (ws_bytes < gptq_layout(N, K).bytes) return W4_ERR_WORKSPACE;
+    if (!X || !W || !packed || !scales || !zeros || !ws || (act_order && !perm)) return W4_ERR_NULL;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(packed) || !aligned16(ws)) return W4_ERR_ALIGN;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_gptq(X, T, W, N, K, bits, group, damp, act_order != 0, packed, scales, zeros,
+                                act_order ? perm : nullptr, ws, status, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status w4_quantize_pack_bits(const uint16_t* W, int64_t N, int64_t K, int bits, int group,
+                                const float* act_scale, uint32_t* packed, uint16_t* scales, uint8_t* zeros,
+                                void* stream) {
+    if (!bits_ok(bits, group)) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(N, K) || K % group != 0 || N % 8 != 0) return W4_ERR_SHAPE;
+    if (N == 0 || K == 0) return W4_OK;
+    if (!W || !packed || !scales || !zeros) return W4_ERR_NULL;
+    if (!aligned16(W) || !aligned16(packed) || (act_scale && !aligned16(act_scale))) return W4_ERR_ALIGN;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_quantize_bits(W, N, K, bits, group, act_scale, packed, scales, zeros, status,
+                                         (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status wb_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits, int group, size_t* bytes) {
+    if (!bytes) return W4_ERR_NULL;
+    if (!bits_ok(bits, group)) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0) return W4_ERR_SHAPE;
+    *bytes = (size_t)N * (size_t)K * 2;
+    return W4_OK;
+}
+
+w4_status wb_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                  const uint16_t* scales, const uint8_t* zeros, int bits, int group, uint16_t* Y, void* ws,
+                  size_t ws_bytes, void* stream) {
+    if (!bits_ok(bits, group)) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0) return W4_ERR_SHAPE;
+    if (M == 0 || N == 0) return W4_OK;
+    if (K == 0) return W4_ERR_SHAPE;
+    if (ws_bytes < (size_t)N * (size_t)K * 2) return W4_ERR_WORKSPACE;
+    if (!X || !packed || !scales || !zeros || !Y || !ws) return W4_ERR_NULL;
+    if (!aligned16(X) || !aligned16(packed) || !aligned16(Y) || !aligned16(ws)) return W4_ERR_ALIGN;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_wb_gemm(X, M, N, K, packed, scales, zeros, bits, group, Y, ws, status,
+                                   (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status w4_act_prepare(const uint16_t* X, int64_t M, int64_t K, const int32_t* perm, const float* s,
+                         uint16_t* X_out, void* stream) {
+    if (!dims_ok(M, K)) return W4_ERR_SHAPE;
+    if (M == 0 || K == 0) return W4_OK;
+    if (!X || !X_out) return W4_ERR_NULL;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_act_prepare(X, M, K, perm, s, X_out, status, (cudaStream_t)stream);
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 

@@ -433,6 +433,13 @@ cudaError_t launch_tc_f32(const uint16_t* A, int64_t M, const uint16_t* B, int64
     return launch_tc<false, 2, 1>(A, M, B, N, K, nullptr, nullptr, nullptr, nullptr, status, stream, C);
 }
 
+cudaError_t launch_tc_f16(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, uint16_t* Y,
+                          int* status, cudaStream_t stream) {
+    if (tc_mt(M) == 2)
+        return launch_tc<false, 0, 2>(A, M, B, N, K, nullptr, nullptr, Y, nullptr, status, stream);
+    return launch_tc<false, 0, 1>(A, M, B, N, K, nullptr, nullptr, Y, nullptr, status, stream);
+}
+
 cudaError_t launch_tc_dot(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, double* part,
                           int* status, cudaStream_t stream) {
     if (N != K) return cudaErrorInvalidValue;  // the epilogue reads A[m, n] with n as a column of A

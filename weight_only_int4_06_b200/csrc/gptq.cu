@@ -5,12 +5,16 @@
 // for by the columns not yet quantised, using the inverse Hessian of the layer's reconstruction
 // loss through its Cholesky factor, and the updates to far columns are applied lazily in blocks.
 //
-// Arithmetic (fp64 except the quantiser's decisions, which are w4_quantize_pack's fp32 rules):
+// Arithmetic (fp64 except the quantiser's decisions, which are w4_quantize_pack's fp32 rules with
+// L = 2^b - 1 steps for b-bit codes):
+//   perm   = the processing order: identity, or with act-order (desc_act, "AutoGPTQ vs The Stack
+//            v2") the columns by decreasing diag(X^T X), ties in index order; H, W and the outputs
+//            are taken in that order (the outputs are stored in processing order with perm)
 //   H      = X^T X + lambda I,  lambda = damp * mean(diag(X^T X))
 //   U      = upper triangular with H^-1 = U^T U.  With J the index reversal, chol(J H J) = L lower
 //            gives H = (J L J)(J L J)^T with J L J upper, hence U = (J L J)^-1 = J L^-1 J: one
 //            Cholesky and one triangular inverse, no explicit H^-1.
-//   sweep  for every block of 128 columns (= one quantisation group):
+//   sweep  for every block of `group` columns (= one quantisation group):
 //            group scale/zero from the block's current weights rounded to fp32 (RTN rule);
 //            for each column k of the block, in order:
 //              q_k = RTN code of fp32(w_k); e_k = (w_k - (q_k - z) s) / U_kk;
@@ -24,12 +28,12 @@
 // trailing update.  Every launch is on the caller's stream; results are deterministic.
 #include "common.cuh"
 #include "internal.h"
-#include "quant_rtn.cuh"
+#include "quant_bits.cuh"
 
 namespace w4 {
 
-constexpr int CH_NB = 32;      // Cholesky / inverse panel width
-constexpr int GQ_BLOCK = 128;  // columns per sweep block (the group size)
+constexpr int CH_NB = 32;  // Cholesky / inverse panel width
+// A sweep block is one quantisation group (64 or 128 columns).
 
 // ------------------------------------------------------------------------------ H = X^T X (fp64)
 // One 64 x 64 tile of H per CTA (lower tiles only; each writes its mirror too).  256 threads, 4 x 4
@@ -102,14 +106,35 @@ __global__ void __launch_bounds__(1024) gptq_damp_kernel(const double* __restric
     if (threadIdx.x == 0) *lambda = damp * (part[0] / (double)K);
 }
 
-// P = J H J + lambda I (P[i][j] = H[K-1-i][K-1-j]).
-__global__ void gptq_reverse_kernel(const double* __restrict__ H, int K, const double* __restrict__ lambda,
-                                    double* __restrict__ P) {
+// Act-order: perm[rank] = i, rank = the number of columns before i in decreasing diag(H) with
+// ties in index order (NaN counts as -inf, so the order is total and perm a permutation).
+__global__ void gptq_perm_kernel(const double* __restrict__ H, int K, int32_t* __restrict__ perm) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= K) return;
+    auto key = [&](int k) {
+        const double d = H[(int64_t)k * K + k];
+        return d != d ? -INFINITY : d;
+    };
+    const double di = key(i);
+    int rank = 0;
+    for (int j = 0; j < K; ++j) {
+        const double dj = key(j);
+        rank += (dj > di || (dj == di && j < i)) ? 1 : 0;
+    }
+    perm[rank] = i;
+}
+
+// P = J H_p J + lambda I with H_p = H[perm][:, perm] (perm null: identity), i.e.
+// P[i][j] = H[perm[K-1-i]][perm[K-1-j]].
+__global__ void gptq_reverse_kernel(const double* __restrict__ H, int K, const int32_t* __restrict__ perm,
+                                    const double* __restrict__ lambda, double* __restrict__ P) {
     const int64_t n = (int64_t)K * K;
     const double lam = *lambda;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
         const int i = (int)(e / K), j = (int)(e - (int64_t)i * K);
-        const double h = H[(int64_t)(K - 1 - i) * K + (K - 1 - j)];
+        const int a = perm ? perm[K - 1 - i] : K - 1 - i;
+        const int b = perm ? perm[K - 1 - j] : K - 1 - j;
+        const double h = H[(int64_t)a * K + b];
         P[e] = i == j ? h + lam : h;
     }
 }
@@ -283,33 +308,42 @@ __global__ void gptq_u_kernel(const double* __restrict__ Li, int K, double* __re
     }
 }
 
-__global__ void gptq_w_init_kernel(const __half* __restrict__ W, int64_t n, double* __restrict__ W64) {
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
-        W64[e] = (double)__half2float(W[e]);
+// W64[n][i] = W[n][perm[i]] in fp64 (perm null: identity).
+__global__ void gptq_w_init_kernel(const __half* __restrict__ W, int64_t N, int K, const int32_t* __restrict__ perm,
+                                   double* __restrict__ W64) {
+    const int64_t total = N * K;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = e / K;
+        const int i = (int)(e - n * K);
+        W64[e] = (double)__half2float(W[n * K + (perm ? perm[i] : i)]);
+    }
 }
 
 // --------------------------------------------------------------------------------- column sweep
-// One warp per weight row over the 128 columns of block b.  Lane l holds columns l, 32 + l, 64 + l
-// and 96 + l of the block; column k's value is broadcast from its lane, every lane takes the same
+// One warp per weight row over the GROUP columns of block b.  Lane l holds columns 32 s + l of the
+// block (s < GROUP / 32); column k's value is broadcast from its lane, every lane takes the same
 // fp32 decision, and each lane updates its own later columns.
 constexpr int SW_WARPS = 8;
+template <int GROUP>
 __global__ void __launch_bounds__(SW_WARPS * 32) gptq_sweep_kernel(double* __restrict__ W64, int N, int K, int b,
-                                                                   const double* __restrict__ U,
+                                                                   int bits, const double* __restrict__ U,
                                                                    uint32_t* __restrict__ packed,
                                                                    __half* __restrict__ scales,
                                                                    uint8_t* __restrict__ zeros,
                                                                    double* __restrict__ E, int* status) {
-    __shared__ uint8_t codes[SW_WARPS][GQ_BLOCK];
+    constexpr int V = GROUP / 32;
+    __shared__ uint8_t codes[SW_WARPS][GROUP];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n = blockIdx.x * SW_WARPS + warp;
     if (n >= N) return;  // whole warps only: nothing below synchronises across warps
+    const int L = (1 << bits) - 1;
     double* wrow = W64 + (int64_t)n * K + b;
-    double w[4];
+    double w[V];
 #pragma unroll
-    for (int s = 0; s < 4; ++s) w[s] = wrow[32 * s + lane];
+    for (int s = 0; s < V; ++s) w[s] = wrow[32 * s + lane];
     float lo = 0.0f, hi = 0.0f;  // zero-inclusive range of the block's fp32 values
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < V; ++s) {
         const float v = __double2float_rn(w[s]);
         lo = fminf(lo, v);
         hi = fmaxf(hi, v);
@@ -319,20 +353,22 @@ __global__ void __launch_bounds__(SW_WARPS * 32) gptq_sweep_kernel(double* __res
         lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
         hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
-    const GroupQuant p = group_params(lo, hi);
+    const GroupQuant p = group_params_steps(lo, hi, L);
     const double sd = (double)p.sf;
-    double ek[4] = {0.0, 0.0, 0.0, 0.0};
-    uint32_t qk[4] = {0, 0, 0, 0};
+    double ek[V];
+    int qk[V];
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < V; ++s) {
+        ek[s] = 0.0;
+        qk[s] = 0;
+    }
+#pragma unroll
+    for (int s = 0; s < V; ++s) {
         for (int kk = 0; kk < 32; ++kk) {
             const int k = 32 * s + kk;  // column within the block
             const double wk = __shfl_sync(0xffffffffu, w[s], kk);
-            // w4_quantize_pack's decision on fp32(w_k); the quotient is clamped first so that the
-            // rounding helper's range holds (values beyond +-64 clamp to code 0 or 15 either way)
-            const float x = fminf(fmaxf(div_rn_from_rcp(__double2float_rn(wk), p.sf, p.rcp), -64.0f), 64.0f);
-            const uint32_t q = (uint32_t)min(max(rint_small(x) + p.z, 0), 15);
-            const double wh = (double)((int)q - p.z) * sd;
+            const int q = quant_code_steps(__double2float_rn(wk), p, L);  // the quantiser's fp32 decision
+            const double wh = (double)(q - p.z) * sd;
             const int64_t kg = (int64_t)b + k;
             const double e = __ddiv_rn(__dsub_rn(wk, wh), U[kg * K + kg]);
             if (lane == kk) {
@@ -341,38 +377,36 @@ __global__ void __launch_bounds__(SW_WARPS * 32) gptq_sweep_kernel(double* __res
             }
             const double* urow = U + kg * K + b;
 #pragma unroll
-            for (int s2 = s; s2 < 4; ++s2) {
+            for (int s2 = s; s2 < V; ++s2) {
                 const int j = 32 * s2 + lane;
                 if (j > k) w[s2] = __dsub_rn(w[s2], __dmul_rn(e, urow[j]));
             }
         }
     }
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < V; ++s) {
         codes[warp][32 * s + lane] = (uint8_t)qk[s];
-        E[(int64_t)n * GQ_BLOCK + 32 * s + lane] = ek[s];
+        E[(int64_t)n * GROUP + 32 * s + lane] = ek[s];
     }
     __syncwarp();
-    const int G = K / GQ_BLOCK;
-    if (lane < GQ_BLOCK / 8) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) word |= (uint32_t)codes[warp][8 * lane + i] << (4 * i);
-        packed[(int64_t)n * (K / 8) + b / 8 + lane] = word;
-    }
+    const int G = K / GROUP;
+    const int nwords = GROUP * bits / 32;
+    if (lane < nwords)
+        packed[(int64_t)n * ((int64_t)K * bits / 32) + (int64_t)(b / GROUP) * nwords + lane] =
+            stream_word(codes[warp], bits, lane);
     if (lane == 0) {
-        scales[(int64_t)n * G + b / GQ_BLOCK] = p.s16;
-        zeros[(int64_t)n * G + b / GQ_BLOCK] = (uint8_t)p.z;
+        scales[(int64_t)n * G + b / GROUP] = p.s16;
+        zeros[(int64_t)n * G + b / GROUP] = (uint8_t)p.z;
         if (p.overflow) record_status(status, W4_ERR_RANGE);
     }
 }
 
-// W64[n][j] -= sum_{c < 128} E[n][c] U[b + c][j] for j >= b + 128: 64 x 64 output tiles, the sum
-// in increasing c.
-__global__ void __launch_bounds__(256) gptq_trailing_kernel(double* __restrict__ W64, int N, int K, int b,
+// W64[n][j] -= sum_{c < group} E[n][c] U[b + c][j] for j >= b + group: 64 x 64 output tiles, the
+// sum in increasing c.
+__global__ void __launch_bounds__(256) gptq_trailing_kernel(double* __restrict__ W64, int N, int K, int b, int group,
                                                             const double* __restrict__ E,
                                                             const double* __restrict__ U) {
-    const int j0 = b + GQ_BLOCK + blockIdx.x * 64;
+    const int j0 = b + group + blockIdx.x * 64;
     const int n0 = blockIdx.y * 64;
     __shared__ double es[64][32 + 1];
     __shared__ double us[32][64 + 1];
@@ -383,10 +417,10 @@ __global__ void __launch_bounds__(256) gptq_trailing_kernel(double* __restrict__
     for (int a = 0; a < 4; ++a)
 #pragma unroll
         for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.0;
-    for (int c0 = 0; c0 < GQ_BLOCK; c0 += 32) {
+    for (int c0 = 0; c0 < group; c0 += 32) {
         for (int e = tid; e < 64 * 32; e += 256) {
             const int rr = e >> 5, cc = e & 31;
-            es[rr][cc] = n0 + rr < N ? E[(int64_t)(n0 + rr) * GQ_BLOCK + c0 + cc] : 0.0;
+            es[rr][cc] = n0 + rr < N ? E[(int64_t)(n0 + rr) * group + c0 + cc] : 0.0;
             const int ur = e >> 6, uc = e & 63;
             us[ur][uc] = j0 + uc < K ? U[(int64_t)(b + c0 + ur) * K + j0 + uc] : 0.0;
         }
@@ -423,21 +457,23 @@ GptqLayout gptq_layout(int64_t N, int64_t K) {
     L.H = off; off = gq_align(off + (size_t)K * K * 8);
     L.P = off; off = gq_align(off + (size_t)K * K * 8);
     L.W64 = off; off = gq_align(off + (size_t)N * K * 8);
-    L.E = off; off = gq_align(off + (size_t)N * GQ_BLOCK * 8);
+    L.E = off; off = gq_align(off + (size_t)N * 128 * 8);
+    L.perm = off; off = gq_align(off + (size_t)K * 4);
     L.lambda = off; off = gq_align(off + 8);
     L.bytes = off;
     return L;
 }
 
-cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, double damp,
-                        uint32_t* packed, uint16_t* scales, uint8_t* zeros, void* ws, int* status,
-                        cudaStream_t stream) {
+cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int bits, int group,
+                        double damp, bool act_order, uint32_t* packed, uint16_t* scales, uint8_t* zeros,
+                        int32_t* perm_out, void* ws, int* status, cudaStream_t stream) {
     const GptqLayout Lo = gptq_layout(N, K);
     unsigned char* base = static_cast<unsigned char*>(ws);
     double* H = reinterpret_cast<double*>(base + Lo.H);   // H, later L^-1
-    double* P = reinterpret_cast<double*>(base + Lo.P);   // J H J + lambda I, then L, then U
+    double* P = reinterpret_cast<double*>(base + Lo.P);   // J H_p J + lambda I, then L, then U
     double* W64 = reinterpret_cast<double*>(base + Lo.W64);
     double* E = reinterpret_cast<double*>(base + Lo.E);
+    int32_t* perm = act_order ? reinterpret_cast<int32_t*>(base + Lo.perm) : nullptr;
     double* lambda = reinterpret_cast<double*>(base + Lo.lambda);
     const int k = (int)K, n = (int)N;
     const unsigned ew = (unsigned)device_sm_count() * 8;
@@ -449,7 +485,14 @@ cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t
     }
     gptq_damp_kernel<<<1, 1024, 0, stream>>>(H, k, damp, lambda);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gptq_reverse_kernel<<<ew, 256, 0, stream>>>(H, k, lambda, P);
+    if (perm) {
+        gptq_perm_kernel<<<(unsigned)((K + 255) / 256), 256, 0, stream>>>(H, k, perm);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (perm_out && (e = cudaMemcpyAsync(perm_out, perm, (size_t)K * 4, cudaMemcpyDeviceToDevice, stream)) !=
+                            cudaSuccess)
+            return e;
+    }
+    gptq_reverse_kernel<<<ew, 256, 0, stream>>>(H, k, perm, lambda, P);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     for (int kb = 0; kb < k; kb += CH_NB) {
         chol_diag_kernel<<<1, CH_NB * CH_NB, 0, stream>>>(P, k, kb, status);
@@ -472,16 +515,22 @@ cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t
     }
     gptq_u_kernel<<<ew, 256, 0, stream>>>(H, k, P);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gptq_w_init_kernel<<<ew, 256, 0, stream>>>(reinterpret_cast<const __half*>(W), N * K, W64);
+    gptq_w_init_kernel<<<ew, 256, 0, stream>>>(reinterpret_cast<const __half*>(W), N, k, perm, W64);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    for (int b = 0; b < k; b += GQ_BLOCK) {
-        gptq_sweep_kernel<<<(unsigned)((N + SW_WARPS - 1) / SW_WARPS), SW_WARPS * 32, 0, stream>>>(
-            W64, n, k, b, P, packed, reinterpret_cast<__half*>(scales), zeros, E, status);
+    __half* sc = reinterpret_cast<__half*>(scales);
+    const unsigned sweep_blocks = (unsigned)((N + SW_WARPS - 1) / SW_WARPS);
+    for (int b = 0; b < k; b += group) {
+        if (group == 64)
+            gptq_sweep_kernel<64><<<sweep_blocks, SW_WARPS * 32, 0, stream>>>(W64, n, k, b, bits, P, packed, sc, zeros,
+                                                                              E, status);
+        else
+            gptq_sweep_kernel<128><<<sweep_blocks, SW_WARPS * 32, 0, stream>>>(W64, n, k, b, bits, P, packed, sc,
+                                                                               zeros, E, status);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        const int rest = k - b - GQ_BLOCK;
+        const int rest = k - b - group;
         if (rest <= 0) break;
         gptq_trailing_kernel<<<dim3((unsigned)((rest + 63) / 64), (unsigned)((N + 63) / 64)), 256, 0, stream>>>(
-            W64, n, k, b, E, P);
+            W64, n, k, b, group, E, P);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -61,6 +61,9 @@ cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64
                           double* sse_part, int* status, cudaStream_t stream);
 int tc_sse_partials(int64_t T, int64_t N);  // tiles of an M = T x N launch (partials of EPI 1 and 3)
 // C [M, N] fp32 = A [M, K] . B [N, K]^T (both fp16, K-major, K % 64 == 0, row strides 16-byte multiples).
+// Y [M, N] fp16 = A B^T with an fp16 B [N, K] (no dequantisation).
+cudaError_t launch_tc_f16(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, uint16_t* Y,
+                          int* status, cudaStream_t stream);
 cudaError_t launch_tc_f32(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, float* C,
                           int* status, cudaStream_t stream);
 // Per-tile sum over (m, n) of (A . B^T)[m, n] * A[m, n] into part[tile] (requires N == K).
@@ -94,14 +97,26 @@ cudaError_t launch_awq_gram(const uint16_t* X, int64_t T, const uint16_t* W, int
                             double* mse, int32_t* best_idx, float* best_s, void* ws, int* status,
                             cudaStream_t stream);
 
+// Other widths and column orders (wbits.cu).
+cudaError_t launch_quantize_bits(const uint16_t* W, int64_t N, int64_t K, int bits, int group, const float* act_scale,
+                                 uint32_t* packed, uint16_t* scales, uint8_t* zeros, int* status,
+                                 cudaStream_t stream);
+cudaError_t launch_wb_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                           const uint16_t* scales, const uint8_t* zeros, int bits, int group, uint16_t* Y,
+                           void* ws, int* status, cudaStream_t stream);
+cudaError_t launch_act_prepare(const uint16_t* X, int64_t M, int64_t K, const int32_t* perm, const float* s,
+                               uint16_t* Xo, int* status, cudaStream_t stream);
+
 // GPTQ quantiser (gptq.cu).  Workspace layout (byte offsets, 256-byte aligned).
 struct GptqLayout {
-    size_t H, P, W64, E, lambda, bytes;
+    size_t H, P, W64, E, perm, lambda, bytes;
 };
 GptqLayout gptq_layout(int64_t N, int64_t K);
-cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, double damp,
-                        uint32_t* packed, uint16_t* scales, uint8_t* zeros, void* ws, int* status,
-                        cudaStream_t stream);
+// bits in {2, 3, 4, 8}, group in {64, 128}; perm_out (K int32) is written when act_order is set
+// and perm_out is not null.
+cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int bits, int group,
+                        double damp, bool act_order, uint32_t* packed, uint16_t* scales, uint8_t* zeros,
+                        int32_t* perm_out, void* ws, int* status, cudaStream_t stream);
 
 // AWQ clip search (awq_clip.cu).  Workspace: Gram blocks, then per-split partial Gram blocks.
 struct AwqClipLayout {

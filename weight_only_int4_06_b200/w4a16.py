@@ -37,6 +37,12 @@ SIGNATURES = {
     "awq_scale_search_gram": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "gptq_workspace_size": (_I32, [_I64, _I64, _I64, _I32, ctypes.POINTER(_SZ)]),
     "gptq_quantize": (_I32, [_P, _I64, _P, _I64, _I64, _I32, ctypes.c_double, _P, _P, _P, _P, _SZ, _P]),
+    "gptq_quantize_ex": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, ctypes.c_double, _I32, _P, _P, _P, _P, _P,
+                                _SZ, _P]),
+    "w4_quantize_pack_bits": (_I32, [_P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P]),
+    "wb_gemm_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
+    "wb_gemm": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P]),
+    "w4_act_prepare": (_I32, [_P, _I64, _I64, _P, _P, _P, _P]),
     "awq_clip_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_clip_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "w4_check_device_status": (_I32, [_P]),
@@ -272,6 +278,76 @@ def gptq_quantize(X: torch.Tensor, W: torch.Tensor, damp: float = 0.01, group: i
                              workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "gptq_quantize")
     return packed, scales, zeros
+
+
+def gptq_quantize_ex(X: torch.Tensor, W: torch.Tensor, bits: int = 4, group: int = 128, damp: float = 0.01,
+                     act_order: bool = False, workspace: torch.Tensor | None = None, stream=None):
+    """GPTQ at `bits` in {2, 3, 4, 8}, group 64 or 128, natural or act-order.  Returns (packed
+    [N, K*bits/32] int32 (uint32 bits), scales, zeros, perm [K] int32 or None), outputs in
+    processing order."""
+    T, K = X.shape
+    N = W.shape[0]
+    need = gptq_workspace_size(T, N, K, group)
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=X.device)
+    packed = torch.empty(N, K * bits // 32, dtype=torch.int32, device=X.device)
+    scales = torch.empty(N, K // group, dtype=torch.float16, device=X.device)
+    zeros = torch.empty(N, K // group, dtype=torch.uint8, device=X.device)
+    perm = torch.empty(K, dtype=torch.int32, device=X.device) if act_order else None
+    st = lib().gptq_quantize_ex(_dev(X, torch.float16, "X"), T, _dev(W, torch.float16, "W"), N, K, bits, group,
+                                float(damp), 1 if act_order else 0, ctypes.c_void_p(packed.data_ptr()),
+                                ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(zeros.data_ptr()),
+                                ctypes.c_void_p(perm.data_ptr()) if perm is not None else None,
+                                ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size(),
+                                _stream(stream))
+    _check(st, "gptq_quantize_ex")
+    return packed, scales, zeros, perm
+
+
+def w4_quantize_pack_bits(W: torch.Tensor, bits: int, group: int = 128, act_scale: torch.Tensor | None = None,
+                          stream=None):
+    """Returns (packed [N, K*bits/32] int32 (uint32 bits), scales [N, K/group] fp16, zeros uint8)."""
+    N, K = W.shape
+    packed = torch.empty((N, K * bits // 32), dtype=torch.int32, device=W.device)
+    scales = torch.empty((N, K // group), dtype=torch.float16, device=W.device)
+    zeros = torch.empty((N, K // group), dtype=torch.uint8, device=W.device)
+    a = _dev(act_scale, torch.float32, "act_scale") if act_scale is not None else None
+    st = lib().w4_quantize_pack_bits(_dev(W, torch.float16, "W"), N, K, bits, group, a,
+                                     ctypes.c_void_p(packed.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                                     ctypes.c_void_p(zeros.data_ptr()), _stream(stream))
+    _check(st, "w4_quantize_pack_bits")
+    return packed, scales, zeros
+
+
+def wb_gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor, bits: int,
+            group: int = 128, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = X dequant(W)^T for b-bit weights (dequantise to fp16, then the tcgen05 GEMM)."""
+    M, K = X.shape
+    N = scales.shape[0]
+    n = ctypes.c_size_t(0)
+    _check(lib().wb_gemm_workspace_size(M, N, K, bits, group, ctypes.byref(n)), "wb_gemm_workspace_size")
+    if workspace is None or workspace.numel() * workspace.element_size() < n.value:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=X.device)
+    Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    st = lib().wb_gemm(_dev(X, torch.float16, "X"), M, N, K, ctypes.c_void_p(packed.data_ptr()),
+                       ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(zeros.data_ptr()), bits, group,
+                       ctypes.c_void_p(Y.data_ptr()), ctypes.c_void_p(workspace.data_ptr()),
+                       workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "wb_gemm")
+    return Y
+
+
+def w4_act_prepare(X: torch.Tensor, perm: torch.Tensor | None = None, s: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """X_out[m, i] = X[m, perm[i]] (optionally / s[perm[i]]) in fp16."""
+    M, K = X.shape
+    out = torch.empty_like(X)
+    p = _dev(perm, torch.int32, "perm") if perm is not None else None
+    sc = _dev(s, torch.float32, "s") if s is not None else None
+    st = lib().w4_act_prepare(_dev(X, torch.float16, "X"), M, K, p, sc, ctypes.c_void_p(out.data_ptr()),
+                              _stream(stream))
+    _check(st, "w4_act_prepare")
+    return out
 
 
 def awq_scale_search_noalloc(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20, group: int = 128,
