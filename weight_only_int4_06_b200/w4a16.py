@@ -192,6 +192,46 @@ def w4_gemm_host(X_host: torch.Tensor, packed: torch.Tensor, scales: torch.Tenso
     return out_host
 
 
+class HostGemmCall:
+    """A w4_gemm_host call whose arguments are checked and marshalled once, for loops that reuse
+    the same buffers (a serving loop refills X_host and reads out_host between runs).
+
+    run() makes the one C call -- copy X_host to x_dev, GEMM into y_dev, copy y_dev to out_host,
+    enqueued on the stream chosen at construction, no synchronisation -- without re-validating or
+    re-converting the arguments.  The tensors are kept alive by this object; they must keep their
+    storage (no resize) for as long as it is used."""
+
+    def __init__(self, X_host: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                 out_host: torch.Tensor, x_dev: torch.Tensor, y_dev: torch.Tensor, group: int = 128,
+                 workspace: torch.Tensor | None = None, variant: int = VARIANT_AUTO, stream=None):
+        M, K = X_host.shape
+        N = packed.shape[0]
+        for t, name, shape in ((X_host, "X_host", (M, K)), (out_host, "out_host", (M, N))):
+            if t.is_cuda or t.dtype != torch.float16 or not t.is_contiguous() or tuple(t.shape) != shape:
+                raise ValueError(f"{name} must be a contiguous float16 host tensor of shape {shape}")
+        if x_dev.numel() < M * K or y_dev.numel() < M * N:
+            raise ValueError("x_dev / y_dev too small")
+        need = _ws_size(M, N, K, group)
+        if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+            raise ValueError("workspace too small: see w4_gemm_workspace_size")
+        ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        self._fn = lib().w4_gemm_host
+        self._args = (ctypes.c_void_p(X_host.data_ptr()), ctypes.c_int64(M), ctypes.c_int64(N), ctypes.c_int64(K),
+                      _dev(packed, torch.int32, "packed"), _dev(scales, torch.float16, "scales"),
+                      _dev(zeros, torch.uint8, "zeros"), ctypes.c_int32(group), ctypes.c_void_p(out_host.data_ptr()),
+                      _dev(x_dev, torch.float16, "x_dev"), _dev(y_dev, torch.float16, "y_dev"), ws_ptr,
+                      ctypes.c_size_t(ws_bytes), ctypes.c_int32(variant), _stream(stream))
+        self._keep = (X_host, packed, scales, zeros, out_host, x_dev, y_dev, workspace)
+        self.out_host = out_host
+
+    def run(self) -> torch.Tensor:
+        st = self._fn(*self._args)
+        if st != W4_OK:
+            raise W4Error(st, "w4_gemm_host")
+        return self.out_host
+
+
 _ws_cache: dict = {}
 
 
