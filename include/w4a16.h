@@ -173,9 +173,9 @@ w4_status awq_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_a
  * awq_scale_search -- the AWQ activation-aware per-channel scale search on one linear layer.
  *
  * Follows "GPTQ, AWQ and the rules of post-training quantization", section "AWQ: find the one
- * percent that matters": the scale of input channel j is the average activation magnitude
- * raised to a power alpha, alpha is chosen by a grid search over [0, 1], and the layer keeps
- * its function when W's channel j is multiplied by s_j and X's channel j divided by s_j.
+ * percent that matters": channel j's scale is its mean |x| over the calibration rows to the
+ * power alpha, alpha is picked from a grid on [0, 1], and multiplying W's channel j by s_j while
+ * dividing X's channel j by s_j leaves the layer's output unchanged.
  *     m_j      = (1/T) sum_t |X[t,j]|                        (exact sum, rounded once to fp64)
  *     alpha_i  = i / n_alpha, i = 0 .. n_alpha-1
  *     s_ij     = max(m_j, 1e-6)^alpha_i / sqrt(max_j(.) * min_j(.))   (fp64, then rounded to fp32)
@@ -266,8 +266,9 @@ w4_status gptq_workspace_size(int64_t T, int64_t N, int64_t K, int group, size_t
  * with the columns not yet quantised, and emit w4_quantize_pack's format (so w4_gemm serves it).
  *
  * Follows "GPTQ, AWQ and the rules of post-training quantization", section "GPTQ: pay for the
- * error with the other weights" (a fixed column order, compensation through the inverse Hessian
- * of the layer's reconstruction loss via a Cholesky factorisation, lazily batched updates):
+ * error with the other weights" (columns in a fixed order; each column's rounding error absorbed
+ * by the later columns through the inverse of H = X^T X, taken via a Cholesky factorisation;
+ * updates of far columns batched):
  *     H   = X^T X + lambda I, lambda = damp * mean(diag(X^T X))   (fp64; damp 0.01 is usual)
  *     U   = the upper triangular factor with H^-1 = U^T U          (fp64)
  *     for each group of 128 columns, left to right:

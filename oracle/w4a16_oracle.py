@@ -10,7 +10,7 @@ Everything here is written for a reader to check by eye against the pages:
 * "GPTQ, AWQ and the rules of post-training quantization" -- section "The problem
   both methods solve" (round-to-nearest rounding of weights to a small integer
   format) and section "AWQ: find the one percent that matters" (INT4 with group
-  size 128; per-channel scale = average activation magnitude raised to alpha;
+  size 128; per-channel scale = the channel's mean |x| to the power alpha;
   alpha on a 20-point grid over [0, 1]; multiply a channel's weights by s and
   divide its activation by s, so the layer computes the same function).
 * "AutoGPTQ vs The Stack v2" -- the GPTQ quantisation blurb (per-group

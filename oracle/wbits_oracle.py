@@ -5,8 +5,8 @@ the matmuls that serve them, and a matmul whose activations are divided by a per
 TEST INFRASTRUCTURE, NOT PRODUCT CODE.  Only the test suite, the smoke check and the benchmark's
 CPU-baseline leg may import this module.  It shares no code with the CUDA library.
 
-Pages: "AutoGPTQ vs The Stack v2" (GPTQ to 2/3/4/8-bit integers with per-group quantisation and
-optional activation description, desc_act); "GPTQ, AWQ and the rules of post-training
+Pages: "AutoGPTQ vs The Stack v2" (GPTQ to 2/3/4/8-bit codes with per-group scales and zero
+points, optional act-order, desc_act); "GPTQ, AWQ and the rules of post-training
 quantization", sections "AWQ: find the one percent that matters" (INT3 with group size 128) and
 "What activation-awareness buys and what it does not" (INT2 with group size 64; AWQ's scaling
 applied before GPTQ).

@@ -1,10 +1,10 @@
 // AWQ activation-aware scale search on one linear layer.
 //
 // "GPTQ, AWQ and the rules of post-training quantization", section "AWQ: find the one percent
-// that matters": the scale of input channel j is the average activation magnitude raised to a
-// power alpha; alpha comes from a grid search over [0, 1]; scaling W's channel j by s_j and
-// dividing X's channel j by s_j keeps the layer's function while the quantisation error of the
-// salient channels shrinks.
+// that matters": channel j's scale is its mean |x| over the calibration rows to the power alpha;
+// alpha is picked from a grid on [0, 1]; multiplying W's channel j by s_j and dividing X's
+// channel j by s_j leaves the output unchanged, while the rounding error of the channels with
+// large activations shrinks.
 //
 // Steps on the device (all on the caller's stream, workspace supplied by the caller):
 //   1. colabs:    c_j = sum_t |X[t, j]| as an exact integer count of 2^-24 units (every fp16 value

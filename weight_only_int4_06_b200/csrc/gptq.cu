@@ -1,9 +1,9 @@
 // GPTQ quantiser emitting the library's packed INT4 format (codes, fp16 scales, 4-bit zero points).
 //
 // "GPTQ, AWQ and the rules of post-training quantization", section "GPTQ: pay for the error with
-// the other weights": columns are quantised in a fixed order; after each one the error is paid
-// for by the columns not yet quantised, using the inverse Hessian of the layer's reconstruction
-// loss through its Cholesky factor, and the updates to far columns are applied lazily in blocks.
+// the other weights": columns are quantised in a fixed order; each column's rounding error is
+// absorbed by the columns still unquantised, weighted by the inverse of H = X^T X through a
+// Cholesky factor, and the updates of far columns are batched per block.
 //
 // Arithmetic (fp64 except the quantiser's decisions, which are w4_quantize_pack's fp32 rules with
 // L = 2^b - 1 steps for b-bit codes):

@@ -1,7 +1,7 @@
 // Other weight widths and column orders.
 //
-// "AutoGPTQ vs The Stack v2": GPTQ to 2/3/4/8-bit integers with per-group quantisation and an
-// optional activation description (desc_act); "GPTQ, AWQ and the rules of post-training
+// "AutoGPTQ vs The Stack v2": GPTQ to 2/3/4/8-bit codes, per-group scales and zero points, and an
+// optional act-order (desc_act); "GPTQ, AWQ and the rules of post-training
 // quantization", sections "AWQ: find the one percent that matters" (INT3, group 128) and "What
 // activation-awareness buys and what it does not" (INT2, group 64).
 //
