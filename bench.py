@@ -552,23 +552,46 @@ def bench_awq_clip(world, peaks, case, reps=3, n_ratios=10):
             "alu_frac": round(tf / peak, 3), "flops": flops}
 
 
-def other_rows(args, world, peaks, l2):
+def _prefill_row(world, peaks, l2):
     import torch
-    rows = {}
-    rows["quantize"] = bench_quantize(world, peaks, l2)
     pre = GemmWorkload(prefill_cases()[0], 4, l2)
-    reps = 10
     pre.run_step(0)
     torch.cuda.synchronize()
-    rows["prefill"] = {"kernel": "tc_gemm_kernel<DEQ>", "bound": "tensor",
-                       "layers": layer_rows(pre, world, reps, peaks, True)}
+    row = {"kernel": "tc_gemm_kernel<DEQ>", "bound": "tensor", "layers": layer_rows(pre, world, 10, peaks, True)}
     del pre
     torch.cuda.empty_cache()
+    return row
+
+
+def other_rows(args, world, peaks, l2):
+    """The rows besides the headline.  On one GPU a row that fails is reported as {"error": ...}
+    and the others still run; with several ranks an error propagates (the ranks' collective steps
+    must stay in step)."""
+    import torch
+    rows = {}
+
+    def row(name, fn):
+        if world > 1:
+            rows[name] = fn()
+            return
+        try:
+            rows[name] = fn()
+        except Exception as e:  # keep the headline line and the other rows
+            rows[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
+            try:
+                torch.cuda.synchronize()
+                torch.cuda.empty_cache()
+            except Exception:
+                pass
+
+    row("quantize", lambda: bench_quantize(world, peaks, l2))
+    row("prefill", lambda: _prefill_row(world, peaks, l2))
     case = synth.awq_case()
-    rows["awq"] = bench_awq(world, peaks, case)
-    rows["awq_gram"] = bench_awq_gram(world, peaks, case)
-    rows["awq_gram"]["speedup_vs_direct"] = round(rows["awq"]["ms"] / rows["awq_gram"]["ms"], 2)
-    rows["awq_clip"] = bench_awq_clip(world, peaks, case)
+    row("awq", lambda: bench_awq(world, peaks, case))
+    row("awq_gram", lambda: bench_awq_gram(world, peaks, case))
+    if "ms" in rows["awq"] and "ms" in rows["awq_gram"]:
+        rows["awq_gram"]["speedup_vs_direct"] = round(rows["awq"]["ms"] / rows["awq_gram"]["ms"], 2)
+    row("awq_clip", lambda: bench_awq_clip(world, peaks, case))
     return rows
 
 
