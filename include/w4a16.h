@@ -222,6 +222,41 @@ w4_status awq_scale_search_noalloc(const uint16_t* X, int64_t T, const uint16_t*
                                    int64_t K, int group, int n_alpha, double* mse,
                                    int32_t* best_idx, float* best_s, void* stream);
 
+/*
+ * The AWQ scale search split by calibration rows, for one part per rank (or any partition of the
+ * rows).  awq_scale_search on all rows equals, up to the association of the fp64 sums:
+ *     1. per part:  awq_colsum(X_part) -> colsum_part
+ *     2. colsum = sum over parts of colsum_part (uint64 integers: exact in any order);
+ *        T_total = sum of the parts' row counts
+ *     3. awq_scales_from_colsum(colsum, T_total) -> s_all [n_alpha, K]  (same on every part)
+ *     4. per part:  awq_sse(X_part, W, s_all) -> sse_part [n_alpha]
+ *     5. awq_select(sse [n_parts, n_alpha], T_total, N, s_all) -> mse, best_idx, best_s
+ * The exchange between ranks is steps 2 and 4 -> 5 (an integer all-reduce of K values and a
+ * gather of n_alpha doubles per rank); no step reads another GPU's memory.
+ *
+ * awq_colsum: colsum [K] uint64 (device, overwritten) = sum_t |X[t, j]| * 2^24, exact (every
+ *   fp16 magnitude is a whole number of 2^-24 units).  T may be 0 (all zeros).
+ * awq_scales_from_colsum: s_all [n_alpha, K] fp32 = awq_scale_search's scales for alpha_i =
+ *   i / n_alpha from the mean m_j = colsum_j * 2^-24 / T_total.
+ * awq_sse: sse [n_alpha] fp64 = sum over this part's rows t and all n of (X E_i^T)[t, n]^2 with
+ *   awq_scale_search's E_i (fp32 tensor-core accumulation, fixed-order fp64 sums).  ws: at least
+ *   awq_sse_workspace_size bytes.
+ * awq_select: sse [n_parts, n_alpha] fp64 (part-major); MSE_i = (sum over parts in part order) /
+ *   (T_total N); best = lowest index among the minima; best_s = s_all[best].
+ * All arrays are device memory; errors as for awq_scale_search.
+ */
+w4_status awq_colsum(const uint16_t* X, int64_t T, int64_t K, uint64_t* colsum, void* stream);
+w4_status awq_scales_from_colsum(const uint64_t* colsum, int64_t T_total, int64_t K, int n_alpha,
+                                 float* s_all, void* stream);
+w4_status awq_sse_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha,
+                                 size_t* bytes);
+w4_status awq_sse(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int group,
+                  int n_alpha, const float* s_all, double* sse, void* ws, size_t ws_bytes,
+                  void* stream);
+w4_status awq_select(const double* sse, int n_parts, int n_alpha, int64_t T_total, int64_t N,
+                     const float* s_all, int64_t K, double* mse, int32_t* best_idx, float* best_s,
+                     void* stream);
+
 /* Bytes of device workspace awq_scale_search_gram needs for this problem. */
 w4_status awq_gram_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha,
                                   size_t* bytes);

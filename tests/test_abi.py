@@ -33,6 +33,7 @@ def test_header_declares_expected_api():
               "awq_scale_search", "awq_workspace_size", "awq_clip_search", "awq_clip_workspace_size",
               "awq_scale_search_gram", "awq_gram_workspace_size", "gptq_quantize", "gptq_workspace_size",
               "gptq_quantize_ex", "w4_quantize_pack_bits", "wb_gemm", "wb_gemm_workspace_size", "w4_act_prepare",
+              "awq_colsum", "awq_scales_from_colsum", "awq_sse", "awq_sse_workspace_size", "awq_select",
               "w4_check_device_status", "w4_status_string"):
         assert n in names, n
 
@@ -204,3 +205,20 @@ def test_width_calls_reject(L):
     assert L.gptq_quantize_ex(*e(ws_bytes=8)) == 5
     assert L.w4_act_prepare(None, 2, 128, None, None, d, None) == 1
     assert L.w4_act_prepare(d, 0, 128, None, None, d, None) == 0
+
+
+def test_row_split_calls_reject(L):
+    P = ctypes.c_void_p
+    buf = ctypes.create_string_buffer(1 << 12)
+    d = P(ctypes.addressof(buf) + (-ctypes.addressof(buf) % 16))
+    assert L.awq_colsum(d, 10, 500, d, None) == 2
+    assert L.awq_colsum(None, 10, 512, d, None) == 1
+    assert L.awq_colsum(P(d.value + 2), 10, 512, d, None) == 3
+    assert L.awq_scales_from_colsum(d, 0, 512, 20, d, None) == 2
+    assert L.awq_scales_from_colsum(d, 10, 512, 65, d, None) == 4
+    n = ctypes.c_size_t(0)
+    assert L.awq_sse_workspace_size(100, 64, 512, 128, 20, ctypes.byref(n)) == 0 and n.value > 64 * 512 * 2
+    assert L.awq_sse(d, 100, d, 64, 512, 128, 20, d, d, d, 16, None) == 5
+    assert L.awq_sse(d, 100, d, 64, 512, 128, 20, None, d, d, 1 << 30, None) == 1
+    assert L.awq_select(d, 0, 20, 100, 64, d, 512, d, d, d, None) == 2
+    assert L.awq_select(d, 2, 0, 100, 64, d, 512, d, d, d, None) == 4

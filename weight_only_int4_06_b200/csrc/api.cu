@@ -212,6 +212,54 @@ w4_status awq_scale_search(const uint16_t* X, int64_t T, const uint16_t* W, int6
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
+w4_status awq_colsum(const uint16_t* X, int64_t T, int64_t K, uint64_t* colsum, void* stream) {
+    if (!dims_ok(T, K) || T < 0 || K < 128 || K % 128 != 0) return W4_ERR_SHAPE;
+    if ((T > 0 && !X) || !colsum) return W4_ERR_NULL;
+    if ((T > 0 && !aligned16(X)) || !aligned16(colsum)) return W4_ERR_ALIGN;
+    cudaError_t e = launch_awq_colsum(X, T, K, colsum, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status awq_scales_from_colsum(const uint64_t* colsum, int64_t T_total, int64_t K, int n_alpha, float* s_all,
+                                 void* stream) {
+    if (n_alpha < 1 || n_alpha > 64) return W4_ERR_UNSUPPORTED;
+    if (T_total < 1 || K < 128 || K % 128 != 0 || K >= ((int64_t)1 << 31)) return W4_ERR_SHAPE;
+    if (!colsum || !s_all) return W4_ERR_NULL;
+    cudaError_t e = launch_awq_scales_from_colsum(colsum, T_total, K, n_alpha, s_all, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status awq_sse_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha, size_t* bytes) {
+    if (!bytes) return W4_ERR_NULL;
+    w4_status st = awq_check(T, N, K, group, n_alpha);
+    if (st != W4_OK) return st;
+    *bytes = awq_sse_layout(T, N, K, n_alpha).bytes;
+    return W4_OK;
+}
+
+w4_status awq_sse(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int group, int n_alpha,
+                  const float* s_all, double* sse, void* ws, size_t ws_bytes, void* stream) {
+    w4_status st = awq_check(T, N, K, group, n_alpha);
+    if (st != W4_OK) return st;
+    if (ws_bytes < awq_sse_layout(T, N, K, n_alpha).bytes) return W4_ERR_WORKSPACE;
+    if (!X || !W || !s_all || !sse || !ws) return W4_ERR_NULL;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(s_all) || !aligned16(ws)) return W4_ERR_ALIGN;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_awq_sse(X, T, W, N, K, n_alpha, s_all, sse, ws, status, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
+w4_status awq_select(const double* sse, int n_parts, int n_alpha, int64_t T_total, int64_t N, const float* s_all,
+                     int64_t K, double* mse, int32_t* best_idx, float* best_s, void* stream) {
+    if (n_alpha < 1 || n_alpha > 64) return W4_ERR_UNSUPPORTED;
+    if (n_parts < 1 || T_total < 1 || N < 1 || K < 1 || K >= ((int64_t)1 << 31)) return W4_ERR_SHAPE;
+    if (!sse || !s_all || !mse || !best_idx || !best_s) return W4_ERR_NULL;
+    cudaError_t e = launch_awq_select(sse, n_parts, n_alpha, T_total, N, s_all, K, mse, best_idx, best_s,
+                                      (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 w4_status awq_gram_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha, size_t* bytes) {
     if (!bytes) return W4_ERR_NULL;
     w4_status st = awq_check(T, N, K, group, n_alpha);

@@ -251,6 +251,113 @@ cudaError_t launch_awq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t 
 }
 
 // ==================================================================================================
+// The search split by calibration rows (one part per rank, or any row partition): every part
+// computes its exact column sums and, once the scales are known, its per-alpha sums of squares;
+// the parts' column sums add exactly (integers), the parts' sums of squares add in part order.
+
+// sse[i] = the fixed-order sum of alpha i's tile partials (the reduction of awq_finalize_kernel).
+__global__ void __launch_bounds__(256) awq_sum_parts_kernel(const double* __restrict__ part, int n_part,
+                                                            double* __restrict__ sse) {
+    __shared__ double red[256];
+    const int i = blockIdx.x;
+    double acc = 0.0;
+    for (int p = threadIdx.x; p < n_part; p += blockDim.x) acc += part[(int64_t)i * n_part + p];
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = 128; w; w >>= 1) {
+        if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) sse[i] = red[0];
+}
+
+// MSE_i = (sum over parts p, in order, of sse[p][i]) / denom; best = lowest index among the
+// minima; best_s = s_all[best].
+__global__ void __launch_bounds__(256) awq_select_kernel(const double* __restrict__ sse, int n_parts, int n_alpha,
+                                                         double denom, const float* __restrict__ s_all, int K,
+                                                         double* __restrict__ mse, int32_t* __restrict__ best_idx,
+                                                         float* __restrict__ best_s) {
+    __shared__ double vals[64];
+    __shared__ int best_sh;
+    if (threadIdx.x < n_alpha) {
+        double acc = 0.0;
+        for (int p = 0; p < n_parts; ++p) acc += sse[(int64_t)p * n_alpha + threadIdx.x];
+        vals[threadIdx.x] = acc / denom;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int b = 0;
+        for (int i = 0; i < n_alpha; ++i) {
+            mse[i] = vals[i];
+            if (vals[i] < vals[b]) b = i;
+        }
+        *best_idx = b;
+        best_sh = b;
+    }
+    __syncthreads();
+    const int b = best_sh;
+    for (int j = threadIdx.x; j < K; j += blockDim.x) best_s[j] = s_all[(int64_t)b * K + j];
+}
+
+cudaError_t launch_awq_colsum(const uint16_t* X, int64_t T, int64_t K, uint64_t* colsum, cudaStream_t stream) {
+    cudaError_t e = cudaMemsetAsync(colsum, 0, (size_t)K * 8, stream);
+    if (e != cudaSuccess || T == 0) return e;
+    const int chunks = (int)(K / 8);
+    dim3 grid((chunks + 255) / 256, (unsigned)((T + CA_ROWS - 1) / CA_ROWS));
+    colabs_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(X), T, (int)K,
+                                            reinterpret_cast<unsigned long long*>(colsum));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_awq_scales_from_colsum(const uint64_t* colsum, int64_t T_total, int64_t K, int n_alpha,
+                                          float* s_all, cudaStream_t stream) {
+    awq_scales_kernel<<<n_alpha, 1024, 0, stream>>>(reinterpret_cast<const unsigned long long*>(colsum), T_total,
+                                                    (int)K, n_alpha, s_all);
+    return cudaGetLastError();
+}
+
+AwqSseLayout awq_sse_layout(int64_t T, int64_t N, int64_t K, int n_alpha) {
+    AwqSseLayout L;
+    L.n_part = tc_sse_partials(T, N);
+    size_t off = 0;
+    L.E = off; off = align256(off + (size_t)N * K * 2);
+    L.part = off; off = align256(off + (size_t)n_alpha * L.n_part * 8);
+    L.bytes = off;
+    return L;
+}
+
+cudaError_t launch_awq_sse(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int n_alpha,
+                           const float* s_all, double* sse, void* ws, int* status, cudaStream_t stream) {
+    const AwqSseLayout L = awq_sse_layout(T, N, K, n_alpha);
+    unsigned char* base = static_cast<unsigned char*>(ws);
+    uint16_t* E = reinterpret_cast<uint16_t*>(base + L.E);
+    double* part = reinterpret_cast<double*>(base + L.part);
+    cudaError_t e;
+    const int64_t G = K / 128;
+    const int64_t n_groups = N * G;
+    const int64_t want = ((n_groups + 1) / 2 + 7) / 8;
+    const int64_t cap = (int64_t)device_sm_count() * 8;
+    const int fq_blocks = (int)(want < cap ? want : cap);
+    for (int i = 0; i < n_alpha; ++i) {
+        awq_fakequant_kernel<<<fq_blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(W), s_all + (int64_t)i * K,
+                                                             n_groups, (int)G, reinterpret_cast<uint4*>(E), status);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        e = launch_tc_sse(X, T, E, N, K, part + (int64_t)i * L.n_part, status, stream);
+        if (e != cudaSuccess) return e;
+    }
+    awq_sum_parts_kernel<<<n_alpha, 256, 0, stream>>>(part, L.n_part, sse);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_awq_select(const double* sse, int n_parts, int n_alpha, int64_t T_total, int64_t N,
+                              const float* s_all, int64_t K, double* mse, int32_t* best_idx, float* best_s,
+                              cudaStream_t stream) {
+    awq_select_kernel<<<1, 256, 0, stream>>>(sse, n_parts, n_alpha, (double)T_total * (double)N, s_all, (int)K, mse,
+                                             best_idx, best_s);
+    return cudaGetLastError();
+}
+
+// ==================================================================================================
 // Gram form of the same search.  sum_{t,n} (X E_i^T)^2 = sum_n e_n^T G e_n with G = X^T X, so the T
 // calibration rows are read once: G on the tensor cores, then per alpha one GEMM over K x K instead
 // of T x K.  G is formed chunk by chunk: each chunk of at most GRAM_CHUNK rows is one fp32

@@ -84,6 +84,21 @@ cudaError_t launch_awq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t 
                        double* mse, int32_t* best_idx, float* best_s, void* ws, int* status,
                        cudaStream_t stream);
 
+// AWQ search split by calibration rows (awq.cu).
+struct AwqSseLayout {
+    size_t E, part, bytes;
+    int n_part;
+};
+AwqSseLayout awq_sse_layout(int64_t T, int64_t N, int64_t K, int n_alpha);
+cudaError_t launch_awq_colsum(const uint16_t* X, int64_t T, int64_t K, uint64_t* colsum, cudaStream_t stream);
+cudaError_t launch_awq_scales_from_colsum(const uint64_t* colsum, int64_t T_total, int64_t K, int n_alpha,
+                                          float* s_all, cudaStream_t stream);
+cudaError_t launch_awq_sse(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int n_alpha,
+                           const float* s_all, double* sse, void* ws, int* status, cudaStream_t stream);
+cudaError_t launch_awq_select(const double* sse, int n_parts, int n_alpha, int64_t T_total, int64_t N,
+                              const float* s_all, int64_t K, double* mse, int32_t* best_idx, float* best_s,
+                              cudaStream_t stream);
+
 // AWQ search, Gram form (awq.cu).  Workspace layout (byte offsets, 256-byte aligned).
 struct AwqGramLayout {
     size_t colsum, s_all, E, part, XT, G, G64, Gp, d, rd, bytes;

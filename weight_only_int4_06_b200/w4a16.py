@@ -43,6 +43,11 @@ SIGNATURES = {
     "wb_gemm_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "wb_gemm": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P]),
     "w4_act_prepare": (_I32, [_P, _I64, _I64, _P, _P, _P, _P]),
+    "awq_colsum": (_I32, [_P, _I64, _I64, _P, _P]),
+    "awq_scales_from_colsum": (_I32, [_P, _I64, _I64, _I32, _P, _P]),
+    "awq_sse_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
+    "awq_sse": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _SZ, _P]),
+    "awq_select": (_I32, [_P, _I32, _I32, _I64, _I64, _P, _I64, _P, _P, _P, _P]),
     "awq_clip_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_clip_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "w4_check_device_status": (_I32, [_P]),
@@ -388,6 +393,56 @@ def w4_act_prepare(X: torch.Tensor, perm: torch.Tensor | None = None, s: torch.T
                               _stream(stream))
     _check(st, "w4_act_prepare")
     return out
+
+
+def awq_colsum(X: torch.Tensor, stream=None) -> torch.Tensor:
+    """[K] int64 (uint64 bits) exact column sums of |X| in units of 2^-24."""
+    T, K = X.shape
+    out = torch.empty(K, dtype=torch.int64, device=X.device)
+    _check(lib().awq_colsum(_dev(X, torch.float16, "X"), T, K, ctypes.c_void_p(out.data_ptr()), _stream(stream)),
+           "awq_colsum")
+    return out
+
+
+def awq_scales_from_colsum(colsum: torch.Tensor, T_total: int, n_alpha: int = 20, stream=None) -> torch.Tensor:
+    """[n_alpha, K] fp32 scales from the (all-part) column sums and total row count."""
+    K = colsum.shape[0]
+    s_all = torch.empty(n_alpha, K, dtype=torch.float32, device=colsum.device)
+    _check(lib().awq_scales_from_colsum(_dev(colsum, torch.int64, "colsum"), T_total, K, n_alpha,
+                                        ctypes.c_void_p(s_all.data_ptr()), _stream(stream)), "awq_scales_from_colsum")
+    return s_all
+
+
+def awq_sse(X: torch.Tensor, W: torch.Tensor, s_all: torch.Tensor, group: int = 128,
+            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """[n_alpha] fp64 sums of squared output errors over this part's rows."""
+    T, K = X.shape
+    N = W.shape[0]
+    n_alpha = s_all.shape[0]
+    n = ctypes.c_size_t(0)
+    _check(lib().awq_sse_workspace_size(T, N, K, group, n_alpha, ctypes.byref(n)), "awq_sse_workspace_size")
+    if workspace is None or workspace.numel() * workspace.element_size() < n.value:
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8, device=X.device)
+    sse = torch.empty(n_alpha, dtype=torch.float64, device=X.device)
+    _check(lib().awq_sse(_dev(X, torch.float16, "X"), T, _dev(W, torch.float16, "W"), N, K, group, n_alpha,
+                         _dev(s_all, torch.float32, "s_all"), ctypes.c_void_p(sse.data_ptr()),
+                         ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size(),
+                         _stream(stream)), "awq_sse")
+    return sse
+
+
+def awq_select(sse_by_part: torch.Tensor, T_total: int, N: int, s_all: torch.Tensor, stream=None):
+    """sse_by_part [n_parts, n_alpha] fp64 -> (mse [n_alpha] fp64, best [1] int32, best_s [K] fp32)."""
+    n_parts, n_alpha = sse_by_part.shape
+    K = s_all.shape[1]
+    mse = torch.empty(n_alpha, dtype=torch.float64, device=s_all.device)
+    best = torch.empty(1, dtype=torch.int32, device=s_all.device)
+    best_s = torch.empty(K, dtype=torch.float32, device=s_all.device)
+    _check(lib().awq_select(_dev(sse_by_part, torch.float64, "sse_by_part"), n_parts, n_alpha, T_total, N,
+                            _dev(s_all, torch.float32, "s_all"), K, ctypes.c_void_p(mse.data_ptr()),
+                            ctypes.c_void_p(best.data_ptr()), ctypes.c_void_p(best_s.data_ptr()), _stream(stream)),
+           "awq_select")
+    return mse, best, best_s
 
 
 def awq_scale_search_noalloc(X: torch.Tensor, W: torch.Tensor, n_alpha: int = 20, group: int = 128,
