@@ -191,6 +191,18 @@ def test_special_groups():
     assert z[1, 0] == 15 and q[1, 100] == 0 and np.all(np.delete(q[1], 100) == 15)
 
 
+def test_strictly_negative_group_uses_zero_as_its_top():
+    """v_k = -1 - k/128 (all below zero): the range is [min v, 0], so the scale is the smallest fp16
+    at or above (1 + 127/128) / 15, the zero point is 15 and v = -1 lands on the nearest level."""
+    v = (-1.0 - np.arange(128) / 128.0).astype(np.float16)[None, :]
+    q, s, z = O.quantize_rtn(v)
+    s_exact = exact_fp16_ru(float(np.float32(1.0 + 127.0 / 128.0) / np.float32(15)))
+    assert float(s[0, 0]) == s_exact and z[0, 0] == 15
+    levels = [Fraction(c - 15) * Fraction(s_exact) for c in range(16)]
+    dist = [abs(Fraction(-1) - L) for L in levels]
+    assert q[0, 0] == dist.index(min(dist))
+
+
 def test_ramp_group_closed_form():
     """W[k] = (k - 64) / 64: lo = -1, hi = 63/64, d = 127/64.
 
@@ -313,6 +325,24 @@ def test_awq_scales_alpha0_and_normalisation():
         order = np.argsort(np.maximum(m, 1e-6), kind="stable")
         assert np.all(np.diff(s[order]) >= 0)
     assert np.allclose(O.awq_alpha_grid(20), np.arange(20) / 20)
+
+
+def test_awq_scales_floor_closed_form():
+    """Means 0, 1e-4, 1, 4 at alpha = 1/2: floored to 1e-6, their roots are 1e-3, 1e-2, 1, 2 and the
+    normaliser is sqrt(2 * 1e-3), so s = sqrt(5e-4) * (1, 10, 1000, 2000)."""
+    s = O.awq_scales(np.array([0.0, 1e-4, 1.0, 4.0]), 0.5)
+    r = 0.022360679774997897  # sqrt(5e-4)
+    assert np.allclose(s, [r, 10 * r, 1000 * r, 2000 * r], rtol=1e-13, atol=0)
+
+
+def test_awq_exact_ties_pick_the_lowest_alpha():
+    """Every |x| = 1: all channel means are equal, so every alpha gives s = 1 and the very same MSE;
+    the lowest index is chosen."""
+    rng = np.random.default_rng(19)
+    X = np.where(rng.random((64, 256)) < 0.5, -1.0, 1.0).astype(np.float16)
+    W = rng_w(20, 16, 256)
+    mse, best, s_best, s_all = O.awq_scale_search(X, W, n_alpha=8)
+    assert np.all(s_all == 1.0) and np.all(mse == mse[0]) and best == 0
 
 
 def _awq_small():
