@@ -157,3 +157,53 @@ def test_scaled_activations():
     s = np.float32(2.0) ** np.random.default_rng(4).integers(-3, 4, 256).astype(np.float32)
     want = (X.astype(np.float64) / s.astype(np.float64)).astype(np.float16)  # exact: powers of two
     assert np.array_equal(B.scale_activations(X, s).view(np.uint16), want.view(np.uint16))
+
+
+def test_all_zero_group_any_width():
+    for bits, group in ((2, 64), (3, 128), (8, 64)):
+        q, s, z = B.quantize_rtn_bits(np.zeros((1, 2 * group), np.float16), bits, group)
+        assert np.all(s == 1.0) and not z.any() and not q.any()
+
+
+def test_act_order_ties_keep_index_order():
+    """Channels in pairs of equal energy (exact copies): ties are broken by the lower index."""
+    rng = np.random.default_rng(9)
+    base = rng.standard_normal((40, 8)).astype(np.float16)
+    X = np.ascontiguousarray(base[:, np.arange(256) % 8])  # column k copies column k % 8
+    perm = B.act_order_perm(X)
+    d = np.einsum("tk,tk->k", X.astype(np.float64), X.astype(np.float64))
+    for i in range(255):
+        a, b = perm[i], perm[i + 1]
+        assert d[a] > d[b] or (d[a] == d[b] and a < b)
+
+
+def _fp32_rn(f):
+    """The fp32 value nearest to the rational f (ties to even), by exact comparison."""
+    from fractions import Fraction
+    c = np.float32(float(f))
+    cands = [c, np.nextafter(c, np.float32(np.inf)), np.nextafter(c, np.float32(-np.inf))]
+    best = min(cands, key=lambda v: (abs(Fraction(float(v)) - f), int(np.float32(v).view(np.uint32)) & 1))
+    return np.float32(best)
+
+
+def test_scaled_activations_are_one_division_then_fp16():
+    """fp16(RN32(x / s)) with the quotient rounded once, checked with exact rationals on a random
+    block and on elements chosen where multiplying by a rounded reciprocal would give another
+    fp16 value (so a two-rounding implementation cannot pass)."""
+    from fractions import Fraction
+    rng = np.random.default_rng(12)
+    X = (rng.standard_normal((40, 512)) * 3).astype(np.float16)
+    s = rng.uniform(0.3, 7.0, 512).astype(np.float32)
+    cases = [(X[m, k], s[k]) for m in range(0, 40, 4) for k in range(0, 512, 4)]
+    xs = (rng.standard_normal(400000) * 3).astype(np.float16)
+    ss = rng.uniform(0.3, 7.0, 400000).astype(np.float32)
+    x32 = xs.astype(np.float32)
+    hard = np.nonzero((x32 / ss).astype(np.float16) != (x32 * (np.float32(1) / ss)).astype(np.float16))[0][:64]
+    assert len(hard) >= 8
+    cases += [(xs[i], ss[i]) for i in hard]
+    xa = np.array([c[0] for c in cases], np.float16)[None, :]
+    sa = np.array([c[1] for c in cases], np.float32)
+    got = B.scale_activations(xa, sa)[0]
+    for i, (x, sv) in enumerate(cases):
+        want = np.float16(_fp32_rn(Fraction(float(x)) / Fraction(float(sv))))
+        assert got[i].view(np.uint16) == want.view(np.uint16), (float(x), float(sv))
