@@ -522,6 +522,62 @@ def bench_awq_gram(world, peaks, case, reps=3):
             "flops": flops}
 
 
+def bench_gptq(world, peaks, reps=2):
+    """gptq_quantize on the calibration layer's 4096-row subsample, K = N = 4096 (fp64 CUDA cores)."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    X, W = synth.awq_case()
+    Xs = torch.from_numpy(np.ascontiguousarray(X[synth.awq_subsample_rows()])).cuda()
+    Wd = torch.from_numpy(W).cuda()
+    T, K = Xs.shape
+    N = Wd.shape[0]
+    ws = torch.empty(B.gptq_workspace_size(T, N, K), dtype=torch.uint8, device="cuda")
+    B.gptq_quantize(Xs, Wd, workspace=ws)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        B.gptq_quantize(Xs, Wd, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    t = max_over_ranks(min(times), world)
+    flops = 2 * T * K * K + 2 * K ** 3 // 3 + N * K * K  # H, Cholesky + inverse, sweep updates (fp64)
+    del Xs, Wd, ws
+    torch.cuda.empty_cache()
+    return {"kernel": "gptq_gram + blocked Cholesky/inverse + 32 x (sweep + trailing), fp64", "T": T, "K": K,
+            "N": N, "ms": round(t, 3), "TFLOPs_fp64": round(flops / (t * 1e-3) / 1e12, 2), "flops": flops,
+            "bound": "fp64 FMA"}
+
+
+def bench_wb_gemm(world, peaks, reps=20):
+    """wb_gemm (dequantise to fp16 + tcgen05 GEMM) for 3-bit g128 and 2-bit g64 at M = 1 and 2048."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    K = N = 4096
+    _, W = synth.layer_case(6, 1, K, N)
+    Wd = torch.from_numpy(W).cuda()
+    ws = torch.empty(N * K * 2, dtype=torch.uint8, device="cuda")
+    res = []
+    for bits, group in ((3, 128), (2, 64)):
+        p, s, z = B.w4_quantize_pack_bits(Wd, bits, group)
+        for M in (1, 2048):
+            X, _ = synth.layer_case(6, M, K, 8)
+            Xd = torch.from_numpy(X).cuda()
+            B.wb_gemm(Xd, p, s, z, bits, group, ws)
+            g = capture(lambda i: B.wb_gemm(Xd, p, s, z, bits, group, ws), reps, 0)
+            g.replay()
+            t = max_over_ranks(time_graph(g, world) / reps, world)
+            res.append({"bits": bits, "group": group, "M": M, "K": K, "N": N, "us": round(t * 1e3, 2)})
+            del g
+    del Wd, ws
+    torch.cuda.empty_cache()
+    return {"kernel": "dequant_bits_kernel + tc_gemm_kernel<fp16 B>", "layers": res}
+
+
 FP32_FMA_PER_CLK_PER_SM = 128     # B200 SM: 4 partitions x 32 fp32 FMA lanes
 B200_SMS, B200_MAX_SM_MHZ = 148, 1965
 
@@ -604,6 +660,9 @@ def other_rows(args, world, peaks, l2):
     if "ms" in rows["awq"] and "ms" in rows["awq_gram"]:
         rows["awq_gram"]["speedup_vs_direct"] = round(rows["awq"]["ms"] / rows["awq_gram"]["ms"], 2)
     row("awq_clip", lambda: bench_awq_clip(world, peaks, case))
+    if getattr(args, "extra_rows", False):  # rows whose kernels await their first parity run
+        row("gptq", lambda: bench_gptq(world, peaks))
+        row("wb_gemm", lambda: bench_wb_gemm(world, peaks))
     return rows
 
 
@@ -644,6 +703,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the secondary rows (quantize, prefill, awq) in the JSON line")
+    ap.add_argument("--extra-rows", action="store_true",
+                    help="also time GPTQ and the other-width matmul (not part of the default line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
