@@ -1,0 +1,53 @@
+"""More GPU parity cases for validated calls at shapes the other files do not reach, and the
+prepared host call.  The file sorts after the validated GPU parity files so that a run stopping at
+the first failure has already run those.
+
+Pages: "GPTQ, AWQ and the rules of post-training quantization", section "AWQ: find the one percent
+that matters" (the scale search); "AutoAWQ vs The Stack v2" (the W4A16 matmul)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from weight_only_int4_06_b200 import synth
+from weight_only_int4_06_b200 import w4a16 as B
+
+pytestmark = pytest.mark.gpu
+
+
+def test_gram_form_search_at_the_down_projection_width():
+    """K = 11008 (86 groups; the Gram GEMMs' N = K is not a multiple of the 256-wide tile)."""
+    X, W = synth.awq_case(T=2048, K=11008, N=264, case_id=44)
+    mse, best, s = B.awq_scale_search_gram(torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda(), 5)
+    assert B.w4_check_device_status() == 0
+    mse_o, best_o, _, s_all = oracle.awq_scale_search(X, W, 5)
+    mse = mse.cpu().numpy()
+    assert np.all(np.abs(mse - mse_o) <= 1e-3 * mse_o)
+    b = int(best.item())
+    order = np.argsort(mse_o, kind="stable")
+    if (mse_o[order[1]] - mse_o[order[0]]) <= 2e-3 * mse_o[order[0]]:
+        assert b in (int(order[0]), int(order[1]))
+    else:
+        assert b == best_o
+    assert np.array_equal(s.cpu().numpy(), s_all[b])
+
+
+def test_prepared_host_call_matches_w4_gemm():
+    X, W = synth.layer_case(45, 1, 4096, 11008)
+    p, s, z = B.w4_quantize_pack(torch.from_numpy(W).cuda())
+    Xh = torch.from_numpy(X).pin_memory()
+    out = torch.empty((1, 11008), dtype=torch.float16).pin_memory()
+    xd = torch.empty((1, 4096), dtype=torch.float16, device="cuda")
+    yd = torch.empty((1, 11008), dtype=torch.float16, device="cuda")
+    call = B.HostGemmCall(Xh, p, s, z, out, xd, yd)
+    for _ in range(3):
+        call.run()
+    torch.cuda.current_stream().synchronize()
+    ref = B.w4_gemm(torch.from_numpy(X).cuda(), p, s, z).cpu()
+    assert torch.equal(out, ref)  # same kernel, same inputs: same bits
+    Xh.copy_(torch.from_numpy(X[:, ::-1].copy()))  # new contents in the same buffer
+    call.run()
+    torch.cuda.current_stream().synchronize()
+    ref2 = B.w4_gemm(torch.from_numpy(X[:, ::-1].copy()).cuda(), p, s, z).cpu()
+    assert torch.equal(out, ref2)
+    assert B.w4_check_device_status() == 0
