@@ -24,7 +24,8 @@
  *      W4_ERR_NULL         a required pointer is NULL
  *      W4_ERR_SHAPE        a size is negative, K % group != 0, N % 8 != 0, or a size exceeds the
  *                          library's limits (every dimension < 2^31, every matrix < 2^40 elements)
- *      W4_ERR_UNSUPPORTED  group != 128, or n_alpha outside 1..64
+ *      W4_ERR_UNSUPPORTED  group != 128 (64 or 128 where a call says so), bits outside
+ *                          {2, 3, 4, 8}, n_alpha outside 1..64, or a negative / non-finite damp
  *      W4_ERR_ALIGN        X, W, packed, Y or act_scale is not 16-byte aligned
  *      W4_ERR_WORKSPACE    ws_bytes is smaller than the size the matching query returns
  *      W4_ERR_CUDA         a CUDA launch or query failed (the CUDA error is left for the caller
