@@ -425,6 +425,15 @@ w4_status awq_clip_search(const uint16_t* X, int64_t T, const uint16_t* W, int64
                           void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * w4_selftest_bounded_wait -- self-test of the library's bounded waits (no counterpart on the
+ * pages).  Launches one kernel that waits on a barrier nothing ever arrives at; after limit_ns
+ * (1 us .. 5 s, else W4_ERR_UNSUPPORTED) the wait gives up, W4_ERR_DEVICE_TIMEOUT is recorded in
+ * the device status word and the kernel returns.  The call itself returns W4_OK once the launch is
+ * enqueued; w4_check_device_status then reports the timeout, and the context stays usable.
+ */
+w4_status w4_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
+/*
  * w4_check_device_status -- synchronise `stream`, then read and clear the current device's
  * status word.  Returns W4_OK, W4_ERR_RANGE, W4_ERR_DEVICE_TIMEOUT, or W4_ERR_CUDA if the
  * synchronisation itself failed.

@@ -35,6 +35,7 @@ int main(void) {
     CHECK(w4_quantize_pack_bits(NULL, 64, 512, 5, 128, NULL, NULL, NULL, NULL, NULL) == W4_ERR_UNSUPPORTED,
           "5-bit codes rejected");
     CHECK(w4_gemm(NULL, 1, 64, 512, NULL, NULL, NULL, 128, NULL, NULL, 0, NULL) == W4_ERR_NULL, "NULL GEMM operands");
+    CHECK(w4_selftest_bounded_wait(10000000000ull, NULL) == W4_ERR_UNSUPPORTED, "self-test limit above 5 s");
     CHECK(strcmp(w4_status_string(W4_OK), "ok") == 0, "status string ok");
     CHECK(strlen(w4_status_string(W4_ERR_NUMERIC)) > 0, "status string for a non-positive-definite Hessian");
     printf("%d failed\n", fails);

@@ -8,7 +8,7 @@ from weight_only_int4_06_b200 import w4a16 as B
 
 HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "w4a16.h")
 
-SCALARS = {"int64_t": ctypes.c_int64, "int": ctypes.c_int, "size_t": ctypes.c_size_t, "double": ctypes.c_double,
+SCALARS = {"int64_t": ctypes.c_int64, "uint64_t": ctypes.c_uint64, "int": ctypes.c_int, "size_t": ctypes.c_size_t, "double": ctypes.c_double,
            "w4_status": ctypes.c_int}
 
 

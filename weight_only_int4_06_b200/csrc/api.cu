@@ -435,6 +435,14 @@ w4_status w4_check_device_status(void* stream) {
     return (w4_status)v;
 }
 
+w4_status w4_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+    if (limit_ns < 1000u || limit_ns > 5000000000ull) return W4_ERR_UNSUPPORTED;
+    int* status = device_status_ptr();
+    if (!status) return W4_ERR_CUDA;
+    cudaError_t e = launch_selftest_wait(limit_ns, status, (cudaStream_t)stream);
+    return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
+}
+
 const char* w4_status_string(w4_status status) {
     switch (status) {
         case W4_OK: return "ok";

@@ -122,6 +122,9 @@ cudaError_t launch_wb_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, c
 cudaError_t launch_act_prepare(const uint16_t* X, int64_t M, int64_t K, const int32_t* perm, const float* s,
                                uint16_t* Xo, int* status, cudaStream_t stream);
 
+// Self-test of the bounded waits (selftest.cu).
+cudaError_t launch_selftest_wait(uint64_t limit_ns, int* status, cudaStream_t stream);
+
 // GPTQ quantiser (gptq.cu).  Workspace layout (byte offsets, 256-byte aligned).
 struct GptqLayout {
     size_t H, P, W64, E, perm, lambda, bytes;

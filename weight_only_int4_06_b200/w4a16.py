@@ -48,6 +48,7 @@ SIGNATURES = {
     "awq_sse_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_sse": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _SZ, _P]),
     "awq_select": (_I32, [_P, _I32, _I32, _I64, _I64, _P, _I64, _P, _P, _P, _P]),
+    "w4_selftest_bounded_wait": (_I32, [ctypes.c_uint64, _P]),
     "awq_clip_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_clip_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
     "w4_check_device_status": (_I32, [_P]),
@@ -498,6 +499,11 @@ def awq_clip_search(X: torch.Tensor, W: torch.Tensor, act_scale: torch.Tensor | 
 
 def w4_check_device_status(stream=None) -> int:
     return lib().w4_check_device_status(_stream(stream))
+
+
+def w4_selftest_bounded_wait(limit_ns: int = 200_000_000, stream=None) -> None:
+    """Launch the bounded-wait self-test (a wait that must time out after limit_ns)."""
+    _check(lib().w4_selftest_bounded_wait(limit_ns, _stream(stream)), "w4_selftest_bounded_wait")
 
 
 def w4_status_string(status: int) -> str:
