@@ -20,8 +20,7 @@ Everything here is written for a reader to check by eye against the pages:
 * "AutoAWQ vs The Stack v2" -- the WQLinear blurb (INT4 storage, FP16 compute,
   weights dequantised on the fly inside the matmul).
 
-Readings adopted where the pages are silent (each one is also listed in the
-design notes of the repository):
+Readings adopted where the pages are silent:
 
 * the group range includes zero: lo = min(0, min v), hi = max(0, max v);
 * scale: s32 = (hi - lo) / 15 in fp32 (IEEE round to nearest), then the fp16 scale
@@ -57,7 +56,8 @@ class QuantRangeError(ValueError):
 # fp16 rounding toward +infinity
 # ----------------------------------------------------------------------------
 def fp16_round_up(x32: np.ndarray) -> np.ndarray:
-    """Round fp32 values to fp16 toward +infinity.
+    """Round fp32 values to fp16 toward +infinity (the scale's rounding: the pages fix an fp16
+    scale but not how it is rounded; rounding up keeps the 16 levels over the group's range).
 
     numpy's float32 -> float16 cast rounds to nearest (ties to even); where that
     result lies below the fp32 value, step one fp16 ulp up.
@@ -77,6 +77,10 @@ def fp16_round_up(x32: np.ndarray) -> np.ndarray:
 def quantize_rtn(W: np.ndarray, act_scale: np.ndarray | None = None, group: int = GROUP,
                  clip_ratio: np.ndarray | None = None):
     """Group-wise asymmetric INT4 round-to-nearest quantisation of W (or of W * diag(act_scale)).
+
+    "GPTQ, AWQ and the rules of post-training quantization", section "The problem both methods solve" (round to the nearest
+    level of a small integer format); "AutoGPTQ vs The Stack v2" (a scale and a zero point per group,
+    group size 128); the steps the pages leave open follow the readings in this module's header.
 
     W: [N, K] fp16.  act_scale: [K] (cast to fp32) or None.
     clip_ratio: [N, K/group] fp32 or None.  When given, both ends of each group's zero-inclusive
@@ -117,6 +121,8 @@ def quantize_rtn(W: np.ndarray, act_scale: np.ndarray | None = None, group: int 
 # Packing: 8 nibbles per uint32, lowest k in the lowest nibble
 # ----------------------------------------------------------------------------
 def pack_nibbles(q: np.ndarray) -> np.ndarray:
+    """8 codes per uint32, the lowest k in the lowest nibble ("AutoAWQ vs The Stack v2": INT4
+    storage; the pages do not fix the nibble order)."""
     q = np.asarray(q, dtype=np.uint32)
     N, K = q.shape
     assert K % 8 == 0
@@ -128,6 +134,7 @@ def pack_nibbles(q: np.ndarray) -> np.ndarray:
 
 
 def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
+    """Inverse of pack_nibbles."""
     packed = np.asarray(packed, dtype=np.uint32)
     N, W8 = packed.shape
     q = np.zeros((N, W8, 8), dtype=np.uint8)
@@ -146,7 +153,8 @@ def quantize_pack(W: np.ndarray, act_scale: np.ndarray | None = None, group: int
 # Dequantisation and the fp64 matmul
 # ----------------------------------------------------------------------------
 def dequantize(packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray, group: int = GROUP) -> np.ndarray:
-    """w[n, k] = (q[n, k] - z[n, k // group]) * s16[n, k // group], exact in fp64."""
+    """w[n, k] = (q[n, k] - z[n, k // group]) * s16[n, k // group], exact in fp64 ("AutoAWQ vs The
+    Stack v2": the weights are dequantised for FP16 compute)."""
     q = unpack_nibbles(packed).astype(np.float64)
     N, K = q.shape
     s = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), group, axis=1)
@@ -157,7 +165,8 @@ def dequantize(packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray, group:
 
 def gemm(X: np.ndarray, packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray,
          group: int = GROUP) -> np.ndarray:
-    """Y = X . dequant(W)^T in fp64.  X: [M, K] fp16.  Returns [M, N] float64."""
+    """Y = X . dequant(W)^T in fp64 (the W4A16 matmul of "AutoAWQ vs The Stack v2": activations stay
+    fp16, weights are INT4).  X: [M, K] fp16.  Returns [M, N] float64."""
     Wd = dequantize(packed, scales, zeros, group)
     return np.asarray(X).astype(np.float64) @ Wd.T
 
@@ -180,7 +189,8 @@ def gemm_entries(X: np.ndarray, packed: np.ndarray, scales: np.ndarray, zeros: n
 # AWQ activation-aware scale search
 # ----------------------------------------------------------------------------
 def channel_mean_abs(X: np.ndarray) -> np.ndarray:
-    """m_j = (1/T) sum_t |X[t, j]|, with the sum taken exactly.
+    """m_j = (1/T) sum_t |X[t, j]|, with the sum taken exactly ("GPTQ, AWQ and the rules of post-training quantization",
+    section "AWQ: find the one percent that matters": a channel's mean activation magnitude).
 
     Every fp16 value is an integer multiple of 2**-24 below 2**16, so |X| * 2**24 is an
     exact int64 and the column sums (at most 2**16 * 2**40 < 2**63) are exact; the one
@@ -194,18 +204,23 @@ def channel_mean_abs(X: np.ndarray) -> np.ndarray:
 
 
 def awq_alpha_grid(n_alpha: int = 20) -> np.ndarray:
+    """alpha_i = i / n_alpha, i < n_alpha (the 20-point grid on [0, 1] of "GPTQ, AWQ and the rules of post-training quantization",
+    section "AWQ: find the one percent that matters"; 1.0 itself is not a grid point)."""
     return np.array([i / n_alpha for i in range(n_alpha)], dtype=np.float64)
 
 
 def awq_scales(m: np.ndarray, alpha: float) -> np.ndarray:
-    """s_j = max(m_j, 1e-6) ** alpha, normalised by sqrt(max(s) * min(s)) (fp64)."""
+    """s_j = max(m_j, 1e-6) ** alpha, normalised by sqrt(max(s) * min(s)) (fp64; "GPTQ, AWQ and the rules of post-training quantization",
+    section "AWQ: find the one percent that matters"; the floor and the normaliser are readings)."""
     s = np.maximum(np.asarray(m, dtype=np.float64), 1e-6) ** alpha
     return s / np.sqrt(s.max() * s.min())
 
 
 def awq_scale_search(X: np.ndarray, W: np.ndarray, n_alpha: int = 20, group: int = GROUP,
                      quantizer=None):
-    """Grid search of the AWQ per-channel scale exponent alpha.
+    """Grid search of the AWQ per-channel scale exponent alpha ("GPTQ, AWQ and the rules of post-training quantization",
+    section "AWQ: find the one percent that matters": scale W's channels by s, divide X's by s, and
+    keep the alpha whose quantised layer output is closest to the original).
 
     X: [T, K] fp16 calibration activations; W: [N, K] fp16 weights.
     quantizer(W16, s32) -> fake-quantised W * diag(s32) as fp64 [N, K]; the default is
@@ -241,13 +256,16 @@ def awq_scale_search(X: np.ndarray, W: np.ndarray, n_alpha: int = 20, group: int
 # AWQ clip search: per-group shrinking of the quantisation range
 # ----------------------------------------------------------------------------
 def clip_ratio_grid(n_ratios: int = 10) -> np.ndarray:
-    """Shrink ratios r_j = 1 - j/20, j = 0 .. n_ratios-1 (fp32; 1.0 first)."""
+    """Shrink ratios r_j = 1 - j/20, j = 0 .. n_ratios-1 (fp32; 1.0 first).  The pages name the
+    clipping ("AutoAWQ vs The Stack v2") without a grid; this grid is a reading."""
     return np.array([1.0 - j / 20.0 for j in range(n_ratios)], dtype=np.float64).astype(np.float32)
 
 
 def awq_clip_search(X: np.ndarray, W: np.ndarray, act_scale: np.ndarray | None = None,
                     n_ratios: int = 10, group: int = GROUP):
-    """Choose, for every (row n, group g), the range shrink ratio with the least output error.
+    """Choose, for every (row n, group g), the range shrink ratio with the least output error
+    (activation-guided clipping, "AutoAWQ vs The Stack v2"; the objective is a reading: each
+    group's own contribution to the output error).
 
     The layer sees activations X diag(1/a) and quantises W diag(a) (a = act_scale, or 1).  For
     ratio r_j the group is quantised with its range shrunk by r_j (quantize_rtn's clip_ratio) and
@@ -287,7 +305,8 @@ def awq_clip_search(X: np.ndarray, W: np.ndarray, act_scale: np.ndarray | None =
 # GPTQ: quantise one column at a time and let the later columns absorb the error
 # ----------------------------------------------------------------------------
 def _group_params_rtn(v32: np.ndarray):
-    """Scale and zero point of quantize_rtn for one group per row: v32 [N, group] fp32."""
+    """Scale and zero point of quantize_rtn for one group per row: v32 [N, group] fp32 (the same
+    steps as quantize_rtn)."""
     lo = np.minimum(v32.min(axis=1), np.float32(0))
     hi = np.maximum(v32.max(axis=1), np.float32(0))
     d = hi - lo

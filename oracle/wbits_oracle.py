@@ -11,7 +11,7 @@ quantization", sections "AWQ: find the one percent that matters" (INT3 with grou
 "What activation-awareness buys and what it does not" (INT2 with group size 64; AWQ's scaling
 applied before GPTQ).
 
-Readings adopted where the pages are silent (also listed in the design notes):
+Readings adopted where the pages are silent:
 * a b-bit group has L = 2^b - 1 steps: the rules of the INT4 quantiser with 15 replaced by L
   (zero-inclusive range, s32 = (hi - lo) / L in fp32, fp16 scale rounded up, z = clamp(rint(-lo /
   s16), 0, L), q = clamp(rint(v / s16) + z, 0, L), half to even, one rounding per fp32 step);
@@ -40,6 +40,7 @@ BITS = (2, 3, 4, 8)
 
 
 def levels(bits: int) -> int:
+    """L = 2^bits - 1 quantisation steps ("AutoGPTQ vs The Stack v2": 2/3/4/8-bit codes)."""
     assert bits in BITS, bits
     return (1 << bits) - 1
 
@@ -48,7 +49,8 @@ def levels(bits: int) -> int:
 # Round-to-nearest groups of any width
 # ----------------------------------------------------------------------------
 def _params(v32: np.ndarray, L: int):
-    """Scale and zero point of groups of fp32 values v32 [..., group] (last axis is the group)."""
+    """Scale and zero point of groups of fp32 values v32 [..., group] (last axis is the group): the
+    INT4 quantiser's rules with L steps (the first reading in this module's header)."""
     lo = np.minimum(v32.min(axis=-1), np.float32(0))
     hi = np.maximum(v32.max(axis=-1), np.float32(0))
     d = hi - lo
@@ -62,7 +64,9 @@ def _params(v32: np.ndarray, L: int):
 
 
 def quantize_rtn_bits(W: np.ndarray, bits: int, group: int, act_scale: np.ndarray | None = None):
-    """Returns (q [N, K] uint8 codes 0..L, scales [N, K/group] fp16, zeros [N, K/group] uint8)."""
+    """Round-to-nearest b-bit groups ("GPTQ, AWQ and the rules of post-training quantization", section
+    "The problem both methods solve"; INT3 g128 and INT2 g64 in its AWQ sections).
+    Returns (q [N, K] uint8 codes 0..L, scales [N, K/group] fp16, zeros [N, K/group] uint8)."""
     L = levels(bits)
     W = np.asarray(W, dtype=np.float16)
     N, K = W.shape
@@ -81,7 +85,8 @@ def quantize_rtn_bits(W: np.ndarray, bits: int, group: int, act_scale: np.ndarra
 # Bit streams
 # ----------------------------------------------------------------------------
 def pack_bits(q: np.ndarray, bits: int) -> np.ndarray:
-    """[N, K] codes -> [N, K * bits / 32] uint32 (little-endian bit stream per row)."""
+    """[N, K] codes -> [N, K * bits / 32] uint32 (little-endian bit stream per row; the pages fix no
+    layout, this is the packing reading in this module's header)."""
     q = np.asarray(q, dtype=np.uint64)
     N, K = q.shape
     assert (K * bits) % 32 == 0
@@ -98,6 +103,7 @@ def pack_bits(q: np.ndarray, bits: int) -> np.ndarray:
 
 
 def unpack_bits(packed: np.ndarray, bits: int, K: int) -> np.ndarray:
+    """Inverse of pack_bits."""
     p = np.asarray(packed, dtype=np.uint64)
     N = p.shape[0]
     assert p.shape[1] * 32 == K * bits
@@ -114,13 +120,15 @@ def unpack_bits(packed: np.ndarray, bits: int, K: int) -> np.ndarray:
 
 
 def quantize_pack_bits(W: np.ndarray, bits: int, group: int, act_scale: np.ndarray | None = None):
+    """quantize_rtn_bits followed by pack_bits."""
     q, s16, z = quantize_rtn_bits(W, bits, group, act_scale)
     return pack_bits(q, bits), s16, z
 
 
 def dequantize_bits(packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray, bits: int, group: int,
                     K: int) -> np.ndarray:
-    """w[n, k] = (q - z[n, k // group]) * s16[n, k // group], exact in fp64."""
+    """w[n, k] = (q - z[n, k // group]) * s16[n, k // group], exact in fp64 (dequantisation for fp16
+    compute, "AutoAWQ vs The Stack v2")."""
     q = unpack_bits(packed, bits, K).astype(np.float64)
     s = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), group, axis=1)
     z = np.repeat(np.asarray(zeros).astype(np.float64), group, axis=1)
@@ -129,6 +137,7 @@ def dequantize_bits(packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray, b
 
 def gemm_bits(X: np.ndarray, packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray, bits: int,
               group: int) -> np.ndarray:
+    """Y = X . dequant(W)^T in fp64."""
     X64 = np.asarray(X).astype(np.float64)
     return X64 @ dequantize_bits(packed, scales, zeros, bits, group, X64.shape[1]).T
 
@@ -137,7 +146,8 @@ def gemm_bits(X: np.ndarray, packed: np.ndarray, scales: np.ndarray, zeros: np.n
 # Act-order layout
 # ----------------------------------------------------------------------------
 def act_order_perm(X: np.ndarray) -> np.ndarray:
-    """perm[i] = original column processed i-th: decreasing diag(X^T X), stable."""
+    """perm[i] = original column processed i-th: decreasing diag(X^T X), stable (desc_act,
+    "AutoGPTQ vs The Stack v2"; the order criterion is the act-order reading in this header)."""
     X64 = np.asarray(X).astype(np.float64)
     d = np.einsum("tk,tk->k", X64, X64)
     return np.argsort(-d, kind="stable")
