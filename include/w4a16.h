@@ -338,14 +338,19 @@ w4_status gptq_quantize(const uint16_t* X, int64_t T, const uint16_t* W, int64_t
  * order; the outputs are stored in PROCESSING order and perm [K] int32 (device, required then)
  * receives perm[i] = the original column processed i-th.  Serve such weights with
  * w4_act_prepare(X, perm) followed by the matmul.
+ * act_scale [K] fp32 (device) or NULL: AWQ's per-channel scale s applied first ("GPTQ, AWQ and
+ * the rules of post-training quantization", section "What activation-awareness buys and what it
+ * does not": the scaling is independent of GPTQ's update and goes before it).  GPTQ then runs on
+ * X / s and W * s (both formed in fp64; s must be positive and finite) and the layer's output is
+ * (X / s) . dequant(W)^T, e.g. w4_act_prepare(X, perm, s) followed by the matmul.
  *   packed [N, K*bits/32] uint32, scales / zeros [N, K/group].  K <= 32768.
  *   ws: at least gptq_workspace_size(T, N, K, group) bytes.
  * gptq_quantize(...) is gptq_quantize_ex(bits 4, group 128, act_order 0).
  */
 w4_status gptq_quantize_ex(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K,
-                           int bits, int group, double damp, int act_order, uint32_t* packed,
-                           uint16_t* scales, uint8_t* zeros, int32_t* perm, void* ws,
-                           size_t ws_bytes, void* stream);
+                           int bits, int group, double damp, int act_order, const float* act_scale,
+                           uint32_t* packed, uint16_t* scales, uint8_t* zeros, int32_t* perm,
+                           void* ws, size_t ws_bytes, void* stream);
 
 /*
  * w4_quantize_pack_bits -- w4_quantize_pack at other widths and group sizes.

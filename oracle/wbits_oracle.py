@@ -177,13 +177,21 @@ def dequantize_g_idx(q_orig: np.ndarray, scales: np.ndarray, zeros: np.ndarray, 
 # ----------------------------------------------------------------------------
 # GPTQ at any width, natural or act-order
 # ----------------------------------------------------------------------------
-def _gptq_bits(X, W, bits, group, damp, act_order, stop_after):
+def _gptq_bits(X, W, bits, group, damp, act_order, stop_after, act_scale=None):
     L = levels(bits)
     X64 = np.asarray(X).astype(np.float64)
     Wc = np.asarray(W, dtype=np.float16).astype(np.float64).copy()
     N, K = Wc.shape
     assert K % group == 0
-    perm = act_order_perm(X) if act_order else np.arange(K)
+    if act_scale is not None:  # AWQ's scaling first: X / s and W * s (both in fp64)
+        s64 = np.asarray(act_scale, dtype=np.float32).astype(np.float64)
+        X64 = X64 / s64[None, :]
+        Wc = Wc * s64[None, :]
+    if act_order:
+        d = np.einsum("tk,tk->k", X64, X64)
+        perm = np.argsort(-d, kind="stable")
+    else:
+        perm = np.arange(K)
     X64 = X64[:, perm]
     Wc = Wc[:, perm]
     H = X64.T @ X64
@@ -209,7 +217,7 @@ def _gptq_bits(X, W, bits, group, damp, act_order, stop_after):
 
 
 def gptq_quantize_bits(X: np.ndarray, W: np.ndarray, bits: int = 4, group: int = 128, damp: float = 0.01,
-                       act_order: bool = False):
+                       act_order: bool = False, act_scale: np.ndarray | None = None):
     """GPTQ ("GPTQ, AWQ and the rules of post-training quantization", section "GPTQ: pay for the error
     with the other weights") with b-bit groups, columns in natural or act-order.
 
@@ -218,17 +226,21 @@ def gptq_quantize_bits(X: np.ndarray, W: np.ndarray, bits: int = 4, group: int =
     processing order: at a group's first column its scale and zero point come from the group's
     current weights rounded to fp32; q_k = clamp(rint(fp32(w_k) / s) + z, 0, L);
     e = (w_k - (q_k - z) s) / U_kk; w_j -= e U_kj for later j.
+    act_scale [K] (fp32): AWQ's per-channel scale applied first ("GPTQ, AWQ and the rules of
+    post-training quantization", section "What activation-awareness buys and what it does not":
+    the scaling is independent of the second-order update and goes before it): GPTQ then runs on
+    X / s and W * s, both formed in fp64, and the layer computes (X / s) dequant(W)^T.
     Returns (packed, scales, zeros, perm), outputs in processing order (perm = arange when
     act_order is False).
     """
-    q, s16, z, _, perm = _gptq_bits(X, W, bits, group, damp, act_order, None)
+    q, s16, z, _, perm = _gptq_bits(X, W, bits, group, damp, act_order, None, act_scale)
     return pack_bits(q, bits), s16, z, perm
 
 
 def gptq_state_bits(X: np.ndarray, W: np.ndarray, bits: int, group: int, damp: float, act_order: bool,
-                    stop_after: int):
+                    stop_after: int, act_scale: np.ndarray | None = None):
     """The weights in processing order after the first stop_after columns (for tests), and perm."""
-    _, _, _, Wc, perm = _gptq_bits(X, W, bits, group, damp, act_order, stop_after)
+    _, _, _, Wc, perm = _gptq_bits(X, W, bits, group, damp, act_order, stop_after, act_scale)
     return Wc, perm
 
 

@@ -198,7 +198,7 @@ def test_width_calls_reject(L):
     assert L.wb_gemm(*g(ws_bytes=100)) == 5
     assert L.wb_gemm(*g(Y=None)) == 1
     e = lambda **kw: [d, 100, d, 64, 512, kw.get("bits", 3), kw.get("group", 128), kw.get("damp", 0.01),
-                      kw.get("ao", 0), d, d, d, kw.get("perm", None), d, kw.get("ws_bytes", 1 << 40), None]
+                      kw.get("ao", 0), None, d, d, d, kw.get("perm", None), d, kw.get("ws_bytes", 1 << 40), None]
     assert L.gptq_quantize_ex(*e(bits=7)) == 4
     assert L.gptq_quantize_ex(*e(group=256)) == 4
     assert L.gptq_quantize_ex(*e(ao=1)) == 1  # act-order needs perm

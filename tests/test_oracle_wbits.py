@@ -207,3 +207,21 @@ def test_scaled_activations_are_one_division_then_fp16():
     for i, (x, sv) in enumerate(cases):
         want = np.float16(_fp32_rn(Fraction(float(x)) / Fraction(float(sv))))
         assert got[i].view(np.uint16) == want.view(np.uint16), (float(x), float(sv))
+
+
+def test_gptq_act_scale_of_ones_changes_nothing():
+    X, W = synth.correlated_case(T=300, K=256, N=16, case_id=66)
+    a = B.gptq_quantize_bits(X, W, 3, 128, act_order=True)
+    b = B.gptq_quantize_bits(X, W, 3, 128, act_order=True, act_scale=np.ones(256, np.float32))
+    for u, v in zip(a, b):
+        assert np.array_equal(np.asarray(u).view(np.uint8), np.asarray(v).view(np.uint8))
+
+
+def test_gptq_uniform_power_of_two_act_scale_scales_only_the_scales():
+    """s = 4 everywhere: X / 4 and W * 4 are exact, every later step scales exactly by a power of two,
+    so the codes, zero points and order are unchanged and each fp16 scale is exactly 4 times larger."""
+    X, W = synth.correlated_case(T=300, K=256, N=16, case_id=67)
+    p, s, z, perm = B.gptq_quantize_bits(X, W, 2, 64, act_order=True)
+    p4, s4, z4, perm4 = B.gptq_quantize_bits(X, W, 2, 64, act_order=True, act_scale=np.full(256, 4.0, np.float32))
+    assert np.array_equal(p, p4) and np.array_equal(z, z4) and np.array_equal(perm, perm4)
+    assert np.array_equal(s4.astype(np.float64), 4.0 * s.astype(np.float64))

@@ -90,29 +90,30 @@ def test_act_prepare_rejects_a_perm_entry_out_of_range():
     assert np.all(g[:, 17] == 0) and np.array_equal(g[:, :17], X[:, :17])
 
 
-def _margin(X, W_row, bits, group, damp, act_order, k_first):
+def _margin(X, W_row, bits, group, damp, act_order, k_first, act_scale=None):
     """Distance of the oracle's decision at processing column k_first (or at its group's scale and
     zero point) from a rounding boundary, in units of a step."""
     L = (1 << bits) - 1
     g0 = (k_first // group) * group
-    Wc, _ = OB.gptq_state_bits(X, W_row, bits, group, damp, act_order, g0)
+    Wc, _ = OB.gptq_state_bits(X, W_row, bits, group, damp, act_order, g0, act_scale)
     v = Wc[0, g0:g0 + group].astype(np.float32)
     lo, hi = min(np.float32(0), v.min()), max(np.float32(0), v.max())
     s32 = (hi - lo) / np.float32(L)
     s16 = O.fp16_round_up(np.array([s32], np.float32))[0]
     below = np.nextafter(np.float16(s16), np.float16(0))
     m = [abs(float(s32) - float(below)) / float(s16), abs(abs(float(-lo / np.float32(s16)) % 1.0) - 0.5)]
-    Wc, _ = OB.gptq_state_bits(X, W_row, bits, group, damp, act_order, k_first)
+    Wc, _ = OB.gptq_state_bits(X, W_row, bits, group, damp, act_order, k_first, act_scale)
     x = np.float32(Wc[0, k_first]) / np.float32(s16)
     m.append(abs(abs(float(x) % 1.0) - 0.5))
     return min(m)
 
 
-def _check_gptq(X, W, bits, group, act_order, damp=0.01):
+def _check_gptq(X, W, bits, group, act_order, damp=0.01, act_scale=None):
+    sd = torch.from_numpy(act_scale).cuda() if act_scale is not None else None
     p, s, z, perm = B.gptq_quantize_ex(torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda(), bits, group, damp,
-                                       act_order)
+                                       act_order, act_scale=sd)
     assert B.w4_check_device_status() == 0
-    po, so, zo, permo = OB.gptq_quantize_bits(X, W, bits, group, damp, act_order)
+    po, so, zo, permo = OB.gptq_quantize_bits(X, W, bits, group, damp, act_order, act_scale)
     K = W.shape[1]
     if act_order:
         assert np.array_equal(perm.cpu().numpy(), permo.astype(np.int32))
@@ -126,7 +127,7 @@ def _check_gptq(X, W, bits, group, act_order, damp=0.01):
         grp = np.nonzero((s_[n].view(np.uint16) != so[n].view(np.uint16)) | (z_[n] != zo[n]))[0]
         firsts = ([int(cols[0])] if len(cols) else []) + ([int(grp[0]) * group] if len(grp) else [])
         k_first = min(firsts)
-        mg = _margin(X, W[n:n + 1], bits, group, damp, act_order, k_first)
+        mg = _margin(X, W[n:n + 1], bits, group, damp, act_order, k_first, act_scale)
         assert mg < 1e-6, f"row {n} differs at processing column {k_first}, margin {mg:.3g}"
     return p, s, z, perm
 
@@ -165,3 +166,17 @@ def test_int3_gptq_served_by_wb_gemm():
     p, s, z, _ = _check_gptq(X, W, 3, 128, False)
     Y = B.wb_gemm(torch.from_numpy(X[:16]).cuda(), p, s, z, 3, 128).cpu().numpy()
     _check_gemm(Y, OB.gemm_bits(X[:16], _u32(p), s.cpu().numpy(), z.cpu().numpy(), 3, 128))
+
+
+@pytest.mark.parametrize("bits,group,act_order", [(2, 64, False), (4, 128, True)])
+def test_gptq_after_awq_scaling_matches_oracle(bits, group, act_order):
+    """AWQ's per-channel scale first, then GPTQ on X / s and W * s; served as (X / s) dequant(W)^T."""
+    X, W = synth.correlated_case(T=600, K=384, N=40, case_id=80)
+    a = np.random.default_rng(80).uniform(0.5, 2.0, 384).astype(np.float32)
+    p, s, z, perm = _check_gptq(X, W, bits, group, act_order, act_scale=a)
+    if bits == 4 and group == 128:
+        Xp = B.w4_act_prepare(torch.from_numpy(X[:8]).cuda(), perm, torch.from_numpy(a).cuda())
+        Y = B.w4_gemm(Xp, p, s, z).cpu().numpy()
+        Xs = OB.scale_activations(X[:8], a)
+        Yref = OB.gemm_act_order(Xs, _u32(p), s.cpu().numpy(), z.cpu().numpy(), perm.cpu().numpy(), 4, 128)
+        _check_gemm(Y, Yref)

@@ -316,8 +316,8 @@ w4_status gptq_quantize(const uint16_t* X, int64_t T, const uint16_t* W, int64_t
     if (!aligned16(X) || !aligned16(W) || !aligned16(packed) || !aligned16(ws)) return W4_ERR_ALIGN;
     int* status = device_status_ptr();
     if (!status) return W4_ERR_CUDA;
-    cudaError_t e = launch_gptq(X, T, W, N, K, 4, 128, damp, false, packed, scales, zeros, nullptr, ws, status,
-                                (cudaStream_t)stream);
+    cudaError_t e = launch_gptq(X, T, W, N, K, 4, 128, damp, false, nullptr, packed, scales, zeros, nullptr, ws,
+                                status, (cudaStream_t)stream);
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }
 
@@ -326,8 +326,9 @@ static bool bits_ok(int bits, int group) {
 }
 
 w4_status gptq_quantize_ex(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int bits,
-                           int group, double damp, int act_order, uint32_t* packed, uint16_t* scales,
-                           uint8_t* zeros, int32_t* perm, void* ws, size_t ws_bytes, void* stream) {
+                           int group, double damp, int act_order, const float* act_scale, uint32_t* packed,
+                           uint16_t* scales, uint8_t* zeros, int32_t* perm, void* ws, size_t ws_bytes,
+                           void* stream) {
     if (!bits_ok(bits, group)) return W4_ERR_UNSUPPORTED;
     w4_status st = gptq_shape(T, N, K, group);
     if (st != W4_OK) return st;
@@ -337,7 +338,7 @@ w4_status gptq_quantize_ex(const uint16_t* X, int64_t T, const uint16_t* W, int6
     if (!aligned16(X) || !aligned16(W) || !aligned16(packed) || !aligned16(ws)) return W4_ERR_ALIGN;
     int* status = device_status_ptr();
     if (!status) return W4_ERR_CUDA;
-    cudaError_t e = launch_gptq(X, T, W, N, K, bits, group, damp, act_order != 0, packed, scales, zeros,
+    cudaError_t e = launch_gptq(X, T, W, N, K, bits, group, damp, act_order != 0, act_scale, packed, scales, zeros,
                                 act_order ? perm : nullptr, ws, status, (cudaStream_t)stream);
     return e == cudaSuccess ? W4_OK : W4_ERR_CUDA;
 }

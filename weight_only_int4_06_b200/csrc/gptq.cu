@@ -7,6 +7,9 @@
 //
 // Arithmetic (fp64 except the quantiser's decisions, which are w4_quantize_pack's fp32 rules with
 // L = 2^b - 1 steps for b-bit codes):
+//   scale  = optionally AWQ's per-channel scale s first: X / s and W * s in fp64 replace X and W
+//            ("GPTQ, AWQ and the rules of post-training quantization", section "What
+//            activation-awareness buys and what it does not": the scaling goes before GPTQ)
 //   perm   = the processing order: identity, or with act-order (desc_act, "AutoGPTQ vs The Stack
 //            v2") the columns by decreasing diag(X^T X), ties in index order; H, W and the outputs
 //            are taken in that order (the outputs are stored in processing order with perm)
@@ -37,11 +40,12 @@ constexpr int CH_NB = 32;  // Cholesky / inverse panel width
 
 // ------------------------------------------------------------------------------ H = X^T X (fp64)
 // One 64 x 64 tile of H per CTA (lower tiles only; each writes its mirror too).  256 threads, 4 x 4
-// outputs each; X rows staged 16 at a time as fp64.  Products of fp16 values are exact in fp64 and
-// every sum runs over t in increasing order, so H[i][j] and H[j][i] are the same bits.
+// outputs each; X rows staged 16 at a time as fp64 (divided by the activation scale s in fp64 when
+// one is given).  Every sum runs over t in increasing order, so H[i][j] and H[j][i] are the same
+// bits.
 constexpr int GM_T = 16;
 __global__ void __launch_bounds__(256) gptq_gram_kernel(const __half* __restrict__ X, int64_t T, int K,
-                                                        double* __restrict__ H) {
+                                                        const float* __restrict__ s, double* __restrict__ H) {
     const int ti = blockIdx.y, tj = blockIdx.x;
     if (tj > ti) return;
     __shared__ double xi[GM_T][64 + 1];
@@ -61,8 +65,14 @@ __global__ void __launch_bounds__(256) gptq_gram_kernel(const __half* __restrict
             const int row = e >> 6, col = e & 63;
             const int64_t t = t0 + row;
             const bool ok = t < T;
-            xi[row][col] = ok && i0 + col < K ? (double)__half2float(X[t * K + i0 + col]) : 0.0;
-            xj[row][col] = ok && j0 + col < K ? (double)__half2float(X[t * K + j0 + col]) : 0.0;
+            double vi = ok && i0 + col < K ? (double)__half2float(X[t * K + i0 + col]) : 0.0;
+            double vj = ok && j0 + col < K ? (double)__half2float(X[t * K + j0 + col]) : 0.0;
+            if (s) {
+                if (i0 + col < K) vi = __ddiv_rn(vi, (double)s[i0 + col]);
+                if (j0 + col < K) vj = __ddiv_rn(vj, (double)s[j0 + col]);
+            }
+            xi[row][col] = vi;
+            xj[row][col] = vj;
         }
         __syncthreads();
 #pragma unroll 4
@@ -308,14 +318,17 @@ __global__ void gptq_u_kernel(const double* __restrict__ Li, int K, double* __re
     }
 }
 
-// W64[n][i] = W[n][perm[i]] in fp64 (perm null: identity).
+// W64[n][i] = W[n][c] * s[c] in fp64 with c = perm[i] (perm null: identity; s null: 1).  The
+// product of an fp16 and an fp32 value is exact in fp64.
 __global__ void gptq_w_init_kernel(const __half* __restrict__ W, int64_t N, int K, const int32_t* __restrict__ perm,
-                                   double* __restrict__ W64) {
+                                   const float* __restrict__ s, double* __restrict__ W64) {
     const int64_t total = N * K;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
         const int64_t n = e / K;
         const int i = (int)(e - n * K);
-        W64[e] = (double)__half2float(W[n * K + (perm ? perm[i] : i)]);
+        const int c = perm ? perm[i] : i;
+        const double w = (double)__half2float(W[n * K + c]);
+        W64[e] = s ? w * (double)s[c] : w;
     }
 }
 
@@ -465,8 +478,8 @@ GptqLayout gptq_layout(int64_t N, int64_t K) {
 }
 
 cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int bits, int group,
-                        double damp, bool act_order, uint32_t* packed, uint16_t* scales, uint8_t* zeros,
-                        int32_t* perm_out, void* ws, int* status, cudaStream_t stream) {
+                        double damp, bool act_order, const float* act_scale, uint32_t* packed, uint16_t* scales,
+                        uint8_t* zeros, int32_t* perm_out, void* ws, int* status, cudaStream_t stream) {
     const GptqLayout Lo = gptq_layout(N, K);
     unsigned char* base = static_cast<unsigned char*>(ws);
     double* H = reinterpret_cast<double*>(base + Lo.H);   // H, later L^-1
@@ -480,7 +493,8 @@ cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t
     cudaError_t e;
     {
         const unsigned tiles = (unsigned)((K + 63) / 64);
-        gptq_gram_kernel<<<dim3(tiles, tiles), 256, 0, stream>>>(reinterpret_cast<const __half*>(X), T, k, H);
+        gptq_gram_kernel<<<dim3(tiles, tiles), 256, 0, stream>>>(reinterpret_cast<const __half*>(X), T, k, act_scale,
+                                                                 H);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     gptq_damp_kernel<<<1, 1024, 0, stream>>>(H, k, damp, lambda);
@@ -515,7 +529,7 @@ cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t
     }
     gptq_u_kernel<<<ew, 256, 0, stream>>>(H, k, P);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gptq_w_init_kernel<<<ew, 256, 0, stream>>>(reinterpret_cast<const __half*>(W), N, k, perm, W64);
+    gptq_w_init_kernel<<<ew, 256, 0, stream>>>(reinterpret_cast<const __half*>(W), N, k, perm, act_scale, W64);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     __half* sc = reinterpret_cast<__half*>(scales);
     const unsigned sweep_blocks = (unsigned)((N + SW_WARPS - 1) / SW_WARPS);

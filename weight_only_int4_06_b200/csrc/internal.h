@@ -133,8 +133,8 @@ GptqLayout gptq_layout(int64_t N, int64_t K);
 // bits in {2, 3, 4, 8}, group in {64, 128}; perm_out (K int32) is written when act_order is set
 // and perm_out is not null.
 cudaError_t launch_gptq(const uint16_t* X, int64_t T, const uint16_t* W, int64_t N, int64_t K, int bits, int group,
-                        double damp, bool act_order, uint32_t* packed, uint16_t* scales, uint8_t* zeros,
-                        int32_t* perm_out, void* ws, int* status, cudaStream_t stream);
+                        double damp, bool act_order, const float* act_scale, uint32_t* packed, uint16_t* scales,
+                        uint8_t* zeros, int32_t* perm_out, void* ws, int* status, cudaStream_t stream);
 
 // AWQ clip search (awq_clip.cu).  Workspace: Gram blocks, then per-split partial Gram blocks.
 struct AwqClipLayout {

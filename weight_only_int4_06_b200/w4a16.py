@@ -38,7 +38,7 @@ SIGNATURES = {
     "gptq_workspace_size": (_I32, [_I64, _I64, _I64, _I32, ctypes.POINTER(_SZ)]),
     "gptq_quantize": (_I32, [_P, _I64, _P, _I64, _I64, _I32, ctypes.c_double, _P, _P, _P, _P, _SZ, _P]),
     "gptq_quantize_ex": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, ctypes.c_double, _I32, _P, _P, _P, _P, _P,
-                                _SZ, _P]),
+                                _P, _SZ, _P]),
     "w4_quantize_pack_bits": (_I32, [_P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _P]),
     "wb_gemm_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "wb_gemm": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _I32, _P, _P, _SZ, _P]),
@@ -327,7 +327,8 @@ def gptq_quantize(X: torch.Tensor, W: torch.Tensor, damp: float = 0.01, group: i
 
 
 def gptq_quantize_ex(X: torch.Tensor, W: torch.Tensor, bits: int = 4, group: int = 128, damp: float = 0.01,
-                     act_order: bool = False, workspace: torch.Tensor | None = None, stream=None):
+                     act_order: bool = False, act_scale: torch.Tensor | None = None,
+                     workspace: torch.Tensor | None = None, stream=None):
     """GPTQ at `bits` in {2, 3, 4, 8}, group 64 or 128, natural or act-order.  Returns (packed
     [N, K*bits/32] int32 (uint32 bits), scales, zeros, perm [K] int32 or None), outputs in
     processing order."""
@@ -341,7 +342,9 @@ def gptq_quantize_ex(X: torch.Tensor, W: torch.Tensor, bits: int = 4, group: int
     zeros = torch.empty(N, K // group, dtype=torch.uint8, device=X.device)
     perm = torch.empty(K, dtype=torch.int32, device=X.device) if act_order else None
     st = lib().gptq_quantize_ex(_dev(X, torch.float16, "X"), T, _dev(W, torch.float16, "W"), N, K, bits, group,
-                                float(damp), 1 if act_order else 0, ctypes.c_void_p(packed.data_ptr()),
+                                float(damp), 1 if act_order else 0,
+                                _dev(act_scale, torch.float32, "act_scale") if act_scale is not None else None,
+                                ctypes.c_void_p(packed.data_ptr()),
                                 ctypes.c_void_p(scales.data_ptr()), ctypes.c_void_p(zeros.data_ptr()),
                                 ctypes.c_void_p(perm.data_ptr()) if perm is not None else None,
                                 ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size(),
