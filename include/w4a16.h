@@ -108,7 +108,8 @@ typedef enum {
  *
  *   W          [N, K] fp16, device, 16-byte aligned.
  *   act_scale  [K] fp32, device, 16-byte aligned, or NULL.  AWQ use: quantise W*diag(s) here and
- *              feed X*diag(1/s) to w4_gemm (or fold 1/s into the producer of X).
+ *              feed X*diag(1/s) to w4_gemm (w4_act_prepare(X, NULL, s) forms it in one pass, or
+ *              fold 1/s into the producer of X).
  *   packed     [N, K/8] uint32 out, 16-byte aligned.  scales [N, K/group] fp16 out.
  *   zeros      [N, K/group] uint8 out.   group must be 128.
  * N == 0 is a no-op.  Errors: see the conventions above; W4_ERR_RANGE is reported through the
