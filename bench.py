@@ -380,7 +380,8 @@ def run_gemm_bench(args, rank, world, local, kind, with_extras=True):
                 "traffic": load_traffic("decode") if kind == "decode" else None}
         kern = ("gemv_stream_kernel<MT> (persistent TMA ring, mma.sync, metadata by bulk copy)"
                 if kind == "decode" else
-                "gemv_stream_kernel<MT> for M <= 8, skinny_kernel (cluster split-K) above")
+                "gemv_stream_kernel<MT> in launches of <= 8 rows where 8 staged rows fit, else "
+                "skinny_kernel (cluster split-K)")
     roof["traffic_unit"] = "DRAM bytes per step (ncu, see profiles/)"
     roof["peak_source"] = peaks["source"]
     roof["kernel"] = kern

@@ -79,9 +79,9 @@ typedef enum {
     W4_VARIANT_AUTO = 0,
     W4_VARIANT_SKINNY = 1, /* warp-level tensor-core GEMV / skinny GEMM, split-K over a cluster */
     W4_VARIANT_TC = 2,     /* tcgen05/TMEM tensor-core GEMM with dequantisation in the smem path */
-    W4_VARIANT_GEMV = 3,   /* persistent TMA-fed mma.sync GEMV, up to 8 activation rows per launch;
-                            * needs 16-byte aligned scales and zeros (else W4_ERR_ALIGN; w4_gemm
-                            * then uses the skinny family) */
+    W4_VARIANT_GEMV = 3,   /* persistent TMA-fed mma.sync GEMV, up to 8 activation rows per launch
+                            * (more rows: several launches); needs 16-byte aligned scales and zeros
+                            * (else W4_ERR_ALIGN; w4_gemm then uses the skinny family) */
     W4_VARIANT_GEMV_TC = 4, /* tcgen05 GEMV, weights as a TMEM operand, up to 8 rows per launch */
     /* Flag, OR-ed into the variant: packed/scales/zeros are not written by any work still in
      * flight on the stream (static weights).  The call may then use programmatic dependent launch
@@ -133,8 +133,9 @@ w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, siz
  *   X [M, K] fp16, packed/scales/zeros as produced by w4_quantize_pack, Y [M, N] fp16 out.
  *   ws / ws_bytes: device workspace of at least w4_gemm_workspace_size bytes (may be NULL when
  *   that size is 0).  M == 0 or N == 0 is a no-op; K == 0 writes Y = 0.
- * Families (w4_gemm picks by M: GEMV for M <= 8 when its staged activations fit shared memory
- * and scales/zeros are 16-byte aligned, skinny for M <= 32, TC above):
+ * Families (w4_gemm picks by M: GEMV, in launches of up to 8 activation rows, for M <= 32 when
+ * 8 staged activation rows fit shared memory and scales/zeros are 16-byte aligned; skinny for
+ * the other M <= 32; TC above):
  *   - GEMV: tensor-core sums of x with the raw operands 1024+q / 1024+16q, offsets and z removed
  *     per group with fp32 activation sums (fixed order), times s16 in fp32;
  *   - skinny: sum_k x_k (q_k - z) exactly per group on tensor cores in fp32, times s16 in fp32;

@@ -134,7 +134,12 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     const bool meta_aligned = aligned16(scales) && aligned16(zeros);  // the GEMV bulk-copies metadata
     if (family == W4_VARIANT_GEMV && !gemv_fits) return W4_ERR_SHAPE;
     if (family == W4_VARIANT_GEMV && !meta_aligned) return W4_ERR_ALIGN;
-    if (family == W4_VARIANT_GEMV || (family == W4_VARIANT_AUTO && M <= 8 && gemv_fits && meta_aligned)) {
+    // AUTO takes the GEMV up to 32 rows, as ceil(M / 8) launches of at most 8 rows each: measured
+    // at K = 8192, two M = 8 launches (2 x 16.7 us at N = 8192, 2 x 40.6 us at N = 28672) beat
+    // one skinny launch at M = 16 (44.9 / 126.6 us) and four tie with it at M = 32 (66.6 vs 67.0,
+    // 162.6 vs 168.8 us), before any L2 reuse of the weights between the launches.  The skinny
+    // kernel keeps the shapes whose 8 activation rows do not fit the GEMV's shared memory.
+    if (family == W4_VARIANT_GEMV || (family == W4_VARIANT_AUTO && M <= 32 && gemv_fits && meta_aligned)) {
         // up to 8 activation rows per launch (token-by-token decode has M == 1)
         for (int64_t m0 = 0; m0 < M; m0 += 8) {
             const int64_t mc = (M - m0) < 8 ? (M - m0) : 8;
