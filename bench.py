@@ -157,6 +157,18 @@ def prefill_cases():
             "prefill, compute-bound")
 
 
+def gemm_launches(M, K):
+    """Kernel launches of one w4_gemm call at the bench's shapes (decode M = 1; small batch M <= 32 at
+    K = 8192 or 28672; prefill M >= 512): for 8 < M <= 32 the GEMV takes up to 8 rows per launch
+    where 8 staged activation rows fit shared memory (K = 8192; not K = 28672, which keeps one
+    skinny launch); every other case is one launch."""
+    if M <= 8:
+        return 1
+    if M <= 32 and K <= 8192:
+        return (M + 7) // 8
+    return 1
+
+
 class GemmWorkload:
     """Device-resident inputs for a list of (M, K, N) layers, with rotating weight copies."""
 
@@ -188,7 +200,7 @@ class GemmWorkload:
         torch.cuda.synchronize()
         self.bytes_per_step = sum(gemm_bytes(M, K, N) for (M, K, N) in cases)
         self.flops_per_step = sum(2 * M * K * N for (M, K, N) in cases)
-        self.launches_per_step = len(cases)
+        self.launches_per_step = sum(gemm_launches(M, K) for (M, K, N) in cases)
         self.host_calls = None  # prepared w4_gemm_host calls, built on first use
         self.host_path_note = None
 
