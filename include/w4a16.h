@@ -212,9 +212,12 @@ w4_status awq_scale_search(const uint16_t* X, int64_t T, const uint16_t* W, int6
  *   - Limit: problems whose awq_workspace_size exceeds W4_NOALLOC_SCRATCH_BYTES are rejected
  *     with W4_ERR_WORKSPACE before anything is enqueued (e.g. T = 4096, K = N = 2048 fits;
  *     K = N = 4096 does not).
+ *   - The stream must belong to the current device (else W4_ERR_CUDA, nothing enqueued); the
+ *     scratch used is that device's copy of the array.
  *   - The first call on each device looks up that device's copy of the scratch array
  *     (cudaGetSymbolAddress, with the device current); make that first call before any stream
- *     capture on the device.
+ *     capture on the device.  A lookup that fails returns W4_ERR_CUDA and is tried again by the
+ *     next call.
  *   - Every call shares the one array and leaves its contents behind; the call clears what must
  *     start at zero itself.  Calls whose work overlaps on the GPU (for example on two streams)
  *     race on the array and give wrong results: serialise them.

@@ -2,8 +2,7 @@
 awq_sse, awq_select) against awq_scale_search on all rows, with the parts emulated in one process
 on one GPU (no kernel waits on another).  Column sums add exactly; the scales are bit-identical;
 the MSEs differ only by the grouping of rows into fp32 tensor-core tiles (parts do not start on
-tile boundaries), well inside 1e-5 relative.  The file sorts after the validated GPU parity files
-so that a run stopping at the first failure has already run those."""
+tile boundaries), well inside 1e-5 relative."""
 import numpy as np
 import pytest
 import torch

@@ -6,8 +6,7 @@ fp32(w); the weights they decide on are fp64 values that differ only by rounding
 factors the Hessian blockwise and applies far-column updates as one product per group).  So the
 codes, scales and zero points must be identical, except in a row whose first difference sits at
 a rounding boundary of the oracle's own decision (margin below 1e-6 of a step): after such a flip
-the row legitimately diverges.  At most one such row per 100 is accepted.  The file sorts after every
-other test file so that a run stopping at the first failure has already run all of those."""
+the row legitimately diverges.  At most one such row per 100 is accepted."""
 import numpy as np
 import pytest
 import torch
@@ -88,14 +87,20 @@ def test_gptq_diagonal_hessian_is_rtn():
 
 
 def test_gptq_output_error_below_rtn_and_served_by_gemm():
+    """The layer's output error of the GPU's GPTQ codes equals the oracle's GPTQ output error on the
+    same input (how far below RTN it lies is a property of the input, not of the kernel: on these
+    independent channels the oracle itself reaches 0.94 of RTN), and lies below RTN's."""
     X, W = synth.awq_case(T=1024, K=512, N=64, case_id=96)
     p, s, z = B.gptq_quantize(torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda())
     Wq_g = O.dequantize(p.cpu().numpy().view(np.uint32), s.cpu().numpy(), z.cpu().numpy())
+    po, so, zo, _ = O.gptq_quantize(X, W)
     pr, sr, zr = O.quantize_pack(W)
     X64, W64 = X.astype(np.float64), W.astype(np.float64)
     e_g = np.sum((X64 @ (Wq_g - W64).T) ** 2)
+    e_o = np.sum((X64 @ (O.dequantize(po, so, zo) - W64).T) ** 2)
     e_r = np.sum((X64 @ (O.dequantize(pr, sr, zr) - W64).T) ** 2)
-    assert e_g < 0.9 * e_r
+    assert abs(e_g - e_o) <= 1e-3 * e_o
+    assert e_g < e_r
     # the GEMM serves GPTQ's output unchanged
     Y = B.w4_gemm(torch.from_numpy(X[:64]).cuda(), p, s, z).cpu().numpy().astype(np.float64)
     Yref = X64[:64] @ Wq_g.T

@@ -1,6 +1,5 @@
 """More GPU parity cases for validated calls at shapes the other files do not reach, and the
-prepared host call.  The file sorts after the validated GPU parity files so that a run stopping at
-the first failure has already run those.
+prepared host call.
 
 Pages: "GPTQ, AWQ and the rules of post-training quantization", section "AWQ: find the one percent
 that matters" (the scale search); "AutoAWQ vs The Stack v2" (the W4A16 matmul)."""

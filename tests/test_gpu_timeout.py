@@ -1,6 +1,6 @@
 """The bounded waits on a GPU: a wait that nothing can satisfy gives up after its limit, the
 device status reports W4_ERR_DEVICE_TIMEOUT, and the context stays usable (a quantise + GEMM right
-after still matches the oracle).  The file sorts after the validated GPU parity files."""
+after still matches the oracle)."""
 import time
 
 import numpy as np

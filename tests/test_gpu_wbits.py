@@ -5,8 +5,7 @@ act-order with the same near-tie rule as the INT4 GPTQ parity tests, and act-ord
 end to end.
 
 Pages: "AutoGPTQ vs The Stack v2" (2/3/4/8-bit GPTQ, per-group quantisation, desc_act); "GPTQ, AWQ
-and the rules of post-training quantization" (INT3 g128, INT2 g64).  The file sorts after every
-other test file so that a run stopping at the first failure has already run all of those."""
+and the rules of post-training quantization" (INT3 g128, INT2 g64)."""
 import numpy as np
 import pytest
 import torch

@@ -10,7 +10,8 @@
 // The scratch is a file-scope __device__ array of W4_NOALLOC_SCRATCH_BYTES.  Every GPU that loads
 // the library holds it until the process exits.  In host code the array's name is only a host-side
 // stand-in, so its device address is looked up with cudaGetSymbolAddress once per device (with
-// that device current) on the first call, and that address is what the kernels receive.
+// that device current) on the first call that succeeds there, and that address is what the
+// kernels receive.
 #include <mutex>
 
 #include "common.cuh"
@@ -22,9 +23,23 @@ static __device__ __align__(256) unsigned char g_awq_scratch[W4_NOALLOC_SCRATCH_
 
 namespace {
 constexpr int kMaxDev = 64;
-std::once_flag g_scratch_once[kMaxDev];
-void* g_scratch_ptr[kMaxDev];
-cudaError_t g_scratch_err[kMaxDev];
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDev];  // set once the lookup has succeeded on that device
+
+// Device address of `dev`'s copy of the scratch array; `dev` must be the current device.  A failed
+// lookup is not remembered: the next call tries again.
+void* scratch_on(int dev) {
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_awq_scratch) == cudaSuccess) {
+            g_scratch_ptr[dev] = p;
+        } else {
+            (void)cudaGetLastError();  // leave no error behind for the caller's next check
+        }
+    }
+    return g_scratch_ptr[dev];
+}
 }  // namespace
 
 }  // namespace w4
@@ -38,13 +53,20 @@ extern "C" w4_status awq_scale_search_noalloc(const uint16_t* X, int64_t T, cons
     const w4_status st = awq_workspace_size(T, N, K, group, n_alpha, &need);
     if (st != W4_OK) return st;
     if (need > (size_t)W4_NOALLOC_SCRATCH_BYTES) return W4_ERR_WORKSPACE;  // problem too large for the scratch
+    // The scratch used is the copy on the stream's device, which must be the current device (the
+    // kernels are launched there, and only there can the symbol's address be looked up).
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return W4_ERR_CUDA;
-    std::call_once(g_scratch_once[dev], [dev]() {
-        // with `dev` current: the device address of this device's copy of the array
-        g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_ptr[dev], g_awq_scratch);
-    });
-    if (g_scratch_err[dev] != cudaSuccess || !g_scratch_ptr[dev]) return W4_ERR_CUDA;
-    return awq_scale_search(X, T, W, N, K, group, n_alpha, mse, best_idx, best_s, g_scratch_ptr[dev],
+    if (stream) {
+        int sdev = -1;
+        if (cudaStreamGetDevice((cudaStream_t)stream, &sdev) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return W4_ERR_CUDA;
+        }
+        if (sdev != dev) return W4_ERR_CUDA;  // a stream of another device: nothing enqueued
+    }
+    void* scratch = scratch_on(dev);
+    if (!scratch) return W4_ERR_CUDA;
+    return awq_scale_search(X, T, W, N, K, group, n_alpha, mse, best_idx, best_s, scratch,
                             (size_t)W4_NOALLOC_SCRATCH_BYTES, stream);
 }
