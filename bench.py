@@ -21,8 +21,10 @@ reported time is the maximum over ranks.  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -34,7 +36,6 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from weight_only_int4_06_b200 import synth  # noqa: E402
-from weight_only_int4_06_b200.ncu_traffic import load_traffic  # noqa: E402
 
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
@@ -51,6 +52,51 @@ def load_peaks():
     except Exception:
         return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
                 "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------- DRAM-traffic records
+# An ncu capture (dram__bytes_read.sum, dram__bytes_write.sum per launch) of one step of a workload
+# is summed into profiles/traffic_<workload>.json together with a digest of the kernel's sources;
+# the roofline line reports that traffic only while the digest still matches, so a kernel edited
+# after the capture reports none.
+KERNEL_SOURCES = {
+    "decode": ["weight_only_int4_06_b200/csrc/decode_stream.cu", "weight_only_int4_06_b200/csrc/sm100.cuh",
+               "weight_only_int4_06_b200/csrc/common.cuh"],
+    "prefill": ["weight_only_int4_06_b200/csrc/gemm_tc.cu", "weight_only_int4_06_b200/csrc/sm100.cuh",
+                "weight_only_int4_06_b200/csrc/common.cuh"],
+}
+
+_COMMENT = re.compile(r"/\*.*?\*/|//[^\n]*", re.S)
+
+
+def code_only(text: str) -> str:
+    """C/C++ source without comments and with whitespace collapsed: what the compiler sees."""
+    return " ".join(_COMMENT.sub(" ", text).split())
+
+
+def source_digest(workload: str) -> str:
+    """Digest of the kernel sources' code (comments and layout excluded)."""
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES[workload]:
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + code_only(fh.read()).encode())
+    return h.hexdigest()
+
+
+def traffic_record_path(workload: str) -> str:
+    return os.path.join(ROOT, "profiles", f"traffic_{workload}.json")
+
+
+def load_traffic(workload: str):
+    """DRAM bytes per step, or None (no record, or the kernel sources changed since)."""
+    try:
+        with open(traffic_record_path(workload)) as f:
+            rec = json.load(f)
+        if rec.get("source_sha256") != source_digest(workload):
+            return None
+        return int(rec["dram_bytes_per_step"])
+    except (OSError, KeyError, ValueError):
+        return None
 
 
 def gemm_bytes(M, K, N):
@@ -269,6 +315,29 @@ def time_graph(g, world, stream=None):
     return e0.elapsed_time(e1)  # ms
 
 
+class L2Flush:
+    """Writes a buffer of twice the L2 size, evicting whatever the previous replay left there."""
+
+    def __init__(self, l2_bytes):
+        import torch
+        self.buf = torch.empty(max(1, int(2 * l2_bytes) // 4), dtype=torch.int32, device="cuda")
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def time_graph_median(g, world, replays, flush=None):
+    """Median over `replays` replays of the graph's CUDA-event time (ms), each replay bracketed by a
+    barrier and device synchronisations (time_graph), the L2 flushed before each replay outside
+    the timed region; then the maximum of the ranks' medians."""
+    times = []
+    for _ in range(replays):
+        if flush is not None:
+            flush()
+        times.append(time_graph(g, world))
+    return max_over_ranks(statistics.median(times), world), times
+
+
 def oracle_cpu_baseline(cases, case_id, budget_s=20.0):
     """The CPU oracle as it stands, on a bounded sample of the same step."""
     import oracle
@@ -295,13 +364,14 @@ def oracle_cpu_baseline(cases, case_id, budget_s=20.0):
                        + "; oracle = numpy dequantise + fp64 matmul (OpenBLAS threads)")}
 
 
-def layer_rows(wl, world, reps, peaks, compute_bound):
-    """Per-layer device time, one layer at a time, same graph protocol."""
+def layer_rows(wl, world, reps, peaks, compute_bound, flush=None, replays=5):
+    """Per-layer device time, one layer at a time: a graph of `reps` calls of that layer (rotating
+    weight sets), median of `replays` replays."""
     rows = []
     for i, L in enumerate(wl.layers):
         gi = capture(lambda s, i=i: wl.run_step(s, only=i), reps, 0)
         gi.replay()
-        t = max_over_ranks(time_graph(gi, world) / reps, world)
+        t = time_graph_median(gi, world, replays, flush)[0] / reps
         b = gemm_bytes(L["M"], L["K"], L["N"])
         fl = 2 * L["M"] * L["K"] * L["N"]
         r = {"M": L["M"], "K": L["K"], "N": L["N"], "us": round(t * 1e3, 3),
@@ -345,9 +415,9 @@ def run_gemm_bench(args, rank, world, local, kind, with_extras=True):
         while time.time() < t_end:   # keep the GPU busy while the sampler settles
             g_warm.replay()
         torch.cuda.synchronize()
-    ms = time_graph(g_timed, world)
+    flush = L2Flush(l2)
+    ms, replay_ms = time_graph_median(g_timed, world, args.replays, flush)
     clocks = sampler.stop() if sampler else None
-    ms = max_over_ranks(ms, world)
     ms_per_step = ms / K_steps
     del g_timed, g_warm
 
@@ -355,11 +425,11 @@ def run_gemm_bench(args, rank, world, local, kind, with_extras=True):
     wl.variant = 0
     g_plain = capture(wl.run_step, K_steps, 0)
     g_plain.replay()
-    ms_plain = max_over_ranks(time_graph(g_plain, world), world) / K_steps
+    ms_plain = time_graph_median(g_plain, world, max(3, args.replays // 4), flush)[0] / K_steps
     del g_plain
     wl.variant = variant
 
-    per_layer = layer_rows(wl, world, max(W_steps, 20), peaks, compute_bound)
+    per_layer = layer_rows(wl, world, max(W_steps, 20), peaks, compute_bound, flush)
 
     # end to end through the public API with host buffers (pinned X in, Y out, every step)
     h2d, d2h = wl.h2d_d2h_bytes()
@@ -390,9 +460,9 @@ def run_gemm_bench(args, rank, world, local, kind, with_extras=True):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
                 "traffic": load_traffic("decode") if kind == "decode" else None}
-        kern = ("gemv_stream_kernel<MT> (persistent TMA ring, mma.sync, metadata by bulk copy)"
+        kern = ("decode_stream_kernel<MT> (one half-SM CTA per SM, TMA ring of 8 KB stages, mma.sync, metadata by bulk copy)"
                 if kind == "decode" else
-                "gemv_stream_kernel<MT> in launches of <= 8 rows where 8 staged rows fit, else "
+                "decode_stream_kernel<MT> in launches of <= 8 rows where 8 staged rows fit, else "
                 "skinny_kernel (cluster split-K)")
     roof["traffic_unit"] = "DRAM bytes per step (ncu, see profiles/)"
     roof["peak_source"] = peaks["source"]
@@ -420,6 +490,10 @@ def run_gemm_bench(args, rank, world, local, kind, with_extras=True):
         "roofline": roof,
         "plain_launch_us_per_step": round(ms_plain * 1e3, 3),
         "layers": per_layer,
+        "timing": {"replays": len(replay_ms), "statistic": "median of replays, each exactly K steps",
+                   "replay_us_per_step_min_max": [round(min(replay_ms) / K_steps * 1e3, 3),
+                                                  round(max(replay_ms) / K_steps * 1e3, 3)],
+                   "l2": "flushed (2x L2 write) before every replay, outside the timed region"},
         "e2e": {"value": round(e2e_ms * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "path": wl.host_path_note or ("one w4_gemm_host C call per layer (pinned X in, GEMM, Y out), "
@@ -713,6 +787,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode", choices=["decode", "small_batch", "prefill"])
+    ap.add_argument("--replays", type=int, default=20,
+                    help="graph replays of the K timed steps; the median is reported (>= 20 by default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the secondary rows (quantize, prefill, awq) in the JSON line")

@@ -130,7 +130,8 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
         return W4_OK;
     }
     const int64_t gemv_rows = M < 8 ? M : 8;
-    const bool gemv_fits = gemv_stream_smem(gemv_rows, K) <= 227 * 1024;
+    DecodePlan dplan;
+    const bool gemv_fits = plan_decode_stream(gemv_rows, N, K, &dplan);
     const bool meta_aligned = aligned16(scales) && aligned16(zeros);  // the GEMV bulk-copies metadata
     if (family == W4_VARIANT_GEMV && !gemv_fits) return W4_ERR_SHAPE;
     if (family == W4_VARIANT_GEMV && !meta_aligned) return W4_ERR_ALIGN;
@@ -143,7 +144,7 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
         // up to 8 activation rows per launch (token-by-token decode has M == 1)
         for (int64_t m0 = 0; m0 < M; m0 += 8) {
             const int64_t mc = (M - m0) < 8 ? (M - m0) : 8;
-            cudaError_t e = launch_gemv_stream(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N,
+            cudaError_t e = launch_decode_stream(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N,
                                                weights_static, status, s);
             if (e != cudaSuccess) return W4_ERR_CUDA;
         }

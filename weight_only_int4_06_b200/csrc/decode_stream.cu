@@ -1,0 +1,531 @@
+// Decode GEMV / skinny GEMM for M <= 8: Y = X dequant(W)^T, streamed at HBM rate.
+//
+// "AutoAWQ vs The Stack v2" (WQLinear blurb): the GEMV kernel serves token-by-token generation,
+// where the layer is bound by memory traffic and weight reuse is minimal.  The traffic is the
+// packed weights (0.5 B/weight) plus 3 B of scale and zero point per group of 128.
+//
+// Design (sm_100a):
+//  * One CTA per SM (or per tile when there are fewer tiles than SMs).  CTA c owns a contiguous,
+//    balanced range of 16-row tiles over the whole K (CTA sizes differ by at most one tile), so
+//    every output is finished inside one CTA: no split-K workspace, no cluster barrier.
+//  * A producer warp streams each tile through a shared-memory ring of 32 KB stages with TMA: one
+//    stage is 16 rows x 32 groups (4096 k, 2 KB of each row).  A tile's scales and zero points are
+//    one contiguous block of each array and ride on the tile's first stage as two bulk copies.
+//    The ring is as deep as the SM's shared memory allows (6 stages at K = 4096).  With static
+//    weights the kernel is launched early (programmatic dependent launch) and the producer fills
+//    the ring before the preceding kernel has finished; everything that reads the activations or
+//    writes Y waits for it.
+//  * Sixteen consumer warps; warp w takes the two consecutive groups 2w, 2w + 1 of every stage
+//    and runs mma.sync m16n8k16 with the 16 weight rows as the A operand and the (up to 8)
+//    activation rows as B.  Dequantisation is one LOP3 per two weights: the operands are the raw
+//    fp16 values 1024+q (low nibble of a byte) and 1024+16q (high nibble); activations that meet
+//    high nibbles are staged pre-multiplied by 1/16, and the constant offsets and the zero point
+//    are removed per group in fp32 with the activation sums
+//        sum_k x_k (q_k - z) = raw - 1024 (Sl + Sh') - z (Sl + 16 Sh'),
+//    Sl = sum of x over low-nibble slots, Sh' = sum of the staged x/16 over high-nibble slots,
+//    both summed in fp32 in a fixed tree order (deterministic; their rounding is of the same order
+//    as the MMA's own fp32 accumulation of the offset operands).  The group's fp16 scale then
+//    multiplies that sum in fp32.
+//  * Each consumer warp stages only the activations of its own groups, each 8-k chunk as
+//    [x0, x4, x1/16, x5/16, x2, x6, x3/16, x7/16] so that one 16-byte shared load yields the B
+//    fragments of the two MMAs that consume one packed word; no CTA-wide barrier stands between
+//    the preceding kernel's end and the first MMA.  Lanes whose B column is not an activation row
+//    skip the loads and feed zeros.
+//  * Shared memory is read through 32-bit shared addresses with immediate offsets; a stage's
+//    scales and zero points are read as vectors when the group count allows.
+//  * At the end of a tile every consumer warp parks its partial sums in a shared slot and moves
+//    on; a reducer warp adds the warps' partials in warp order (deterministic) and writes Y, so
+//    the ring never waits for a reduction.
+//  * The kernel is instantiated per activation-row bound MT (1, 2, 4, 8): columns >= MT of the
+//    MMA fragments are never folded or parked.
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace w4 {
+
+// A stage is 16 rows x SG groups (SG = 16 or 32: 16 or 32 KB); consumer warp w takes the SG / 8
+// consecutive groups w * SG / 8 ... of every stage.
+__host__ __device__ constexpr uint32_t ds_stage_bytes(int SG) { return 16u * 64u * (uint32_t)SG; }
+constexpr int DS_CW = 16;                           // consumer warps (then a producer and a reducer warp)
+constexpr int DS_PWARP = DS_CW;                     // producer warp
+constexpr int DS_RWARP = DS_CW + 1;                 // reducer warp
+constexpr int DS_THREADS = 32 * (DS_CW + 2);
+constexpr int DS_MAXM = 8;
+constexpr int DS_MAXNS = 24;                        // ring stages at most
+constexpr int DS_MINNS = 2;                         // ring stages at least
+constexpr int DS_MAXMS = 4;                         // metadata slots at most
+constexpr int DS_RSLOTS = 2;                        // partial-sum slots of the reducer
+// Dynamic shared memory per CTA (alignment slack included): one CTA per SM.
+constexpr uint32_t DS_FULL_SMEM = 227 * 1024;
+
+struct DsLayout {
+    uint32_t ring, meta, mslot, xs, corr, red, bars, total;
+};
+
+// Byte offsets of the shared-memory regions for `ns` ring stages and `nms` metadata slots.
+__host__ __device__ inline DsLayout ds_layout(int SG, int MT, int M, int K, int ns, int nms) {
+    DsLayout L;
+    const uint32_t G = (uint32_t)(K / 128);
+    L.ring = 0;
+    L.meta = (uint32_t)ns * ds_stage_bytes(SG);
+    L.mslot = 48u * G;                                                  // 16 rows x G x (2 + 1) bytes
+    L.xs = L.meta + (uint32_t)nms * L.mslot;
+    L.corr = L.xs + (uint32_t)M * (uint32_t)(K + 8) * 2;                // float2 [G][MT] (+ 8 spare)
+    L.red = L.corr + (G * (uint32_t)MT + 8) * 8;                        // [slot][warp][16][MT] fp32
+    L.bars = L.red + (uint32_t)DS_RSLOTS * DS_CW * 16 * (uint32_t)MT * 4;
+    // full, empty [DS_MAXNS]; meta_empty [DS_MAXMS]; tile_full, red_empty [DS_RSLOTS]; abort flag
+    L.total = L.bars + (2 * DS_MAXNS + DS_MAXMS + 2 * DS_RSLOTS) * 8 + 8;
+    return L;
+}
+
+// 16-byte chunk swizzle of a staged activation row (row stride padded to 16 mod 128 bytes):
+// makes the B-fragment loads of a warp bank-conflict free for up to 8 activation rows.
+__device__ __forceinline__ int ds_swz(int ch) { return ch ^ ((ch >> 2) & 2); }
+
+// Sum of the two fp16 halves of a packed pair, in fp32.
+__device__ __forceinline__ float half2_sum(uint32_t h) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    return f.x + f.y;
+}
+
+constexpr int DS_XILP = 4;  // activation chunks each consumer thread loads before using any
+
+// Shared-memory loads through 32-bit shared addresses (volatile: they stay behind the mbarrier waits).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
+    return r;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 r;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a));
+    return r;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t r;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(a));
+    return r;
+}
+__device__ __forceinline__ unsigned short lds_u16(uint32_t a) {
+    unsigned short r;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(a));
+    return r;
+}
+__device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
+    uint32_t r;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(r) : "r"(a));
+    return r;
+}
+
+// Half h (0: low, 1: high) of a packed fp16 pair, as fp32.
+__device__ __forceinline__ float ds_half(uint32_t v, int h) {
+    return __half2float(__ushort_as_half((unsigned short)(h ? (v >> 16) : (v & 0xFFFFu))));
+}
+
+// One group (16 rows x 128 k) for this thread: raw tensor-core sums, then the offsets and the zero
+// point removed with the group's activation sums and the scale applied, into acc.
+template <int MT>
+__device__ __forceinline__ void ds_group(uint32_t a_addr, uint32_t b_addr, uint32_t xg, const uint32_t (&xofs)[4],
+                                         bool xlane, uint32_t corr_addr, float fsa, float fsb, float fza, float fzb,
+                                         float (&acc)[4]) {
+    const uint4 A = lds128(a_addr);
+    const uint4 B = lds128(b_addr);
+    float c0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, c1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const uint32_t wA[4] = {A.x, A.y, A.z, A.w};
+    const uint32_t wB[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t a = wA[j], b = wB[j], a8 = a >> 8, b8 = b >> 8;
+        const uint4 xf = xlane ? lds128(xg + xofs[j]) : make_uint4(0u, 0u, 0u, 0u);
+        float(&cc)[4] = (j & 1) ? c1 : c0;  // two independent accumulation chains
+        mma_16816(cc, lop3_and_or(a, 0x000F000Fu, 0x64006400u), lop3_and_or(b, 0x000F000Fu, 0x64006400u),
+                  lop3_and_or(a, 0x00F000F0u, 0x64006400u), lop3_and_or(b, 0x00F000F0u, 0x64006400u), xf.x, xf.y);
+        mma_16816(cc, lop3_and_or(a8, 0x000F000Fu, 0x64006400u), lop3_and_or(b8, 0x000F000Fu, 0x64006400u),
+                  lop3_and_or(a8, 0x00F000F0u, 0x64006400u), lop3_and_or(b8, 0x00F000F0u, 0x64006400u), xf.z, xf.w);
+    }
+    // rows g8 + 8 of a half tile (N % 16 == 8) hold stale metadata; never stored
+    if (MT == 1) {
+        const uint2 cv = lds64(corr_addr);
+        const float C = __uint_as_float(cv.x), S = __uint_as_float(cv.y);
+        acc[0] = fmaf(fsa, (c0[0] + c1[0]) - fmaf(fza, S, C), acc[0]);  // row g8,   col 0
+        acc[2] = fmaf(fsb, (c0[2] + c1[2]) - fmaf(fzb, S, C), acc[2]);  // row g8+8, col 0
+    } else {
+        const uint4 cv = lds128(corr_addr);
+        const float C0 = __uint_as_float(cv.x), S0 = __uint_as_float(cv.y);
+        const float C1 = __uint_as_float(cv.z), S1 = __uint_as_float(cv.w);
+        acc[0] = fmaf(fsa, (c0[0] + c1[0]) - fmaf(fza, S0, C0), acc[0]);  // row g8,   col 2c
+        acc[1] = fmaf(fsa, (c0[1] + c1[1]) - fmaf(fza, S1, C1), acc[1]);  // row g8,   col 2c+1
+        acc[2] = fmaf(fsb, (c0[2] + c1[2]) - fmaf(fzb, S0, C0), acc[2]);  // row g8+8, col 2c
+        acc[3] = fmaf(fsb, (c0[3] + c1[3]) - fmaf(fzb, S1, C1), acc[3]);  // row g8+8, col 2c+1
+    }
+}
+
+template <int MT, int SG>
+__global__ void __launch_bounds__(DS_THREADS, 1)
+    decode_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __half* __restrict__ X,
+                         const unsigned short* __restrict__ scales, const uint8_t* __restrict__ zeros,
+                         __half* __restrict__ Y, int M, int N, int K, int n_tiles, int ns, int nms,
+                         int weights_early, int* status) {
+    constexpr int ROWB = SG * 64;                    // bytes of one row in a stage
+    constexpr uint32_t STAGE_BYTES = 16u * ROWB;
+    constexpr int GPW = SG / DS_CW;                  // groups per consumer warp per stage
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // TMA destinations need an aligned base: round up (the launch reserves 1 KB of slack)
+    unsigned char* smem = smem_align1024(smem_raw);
+    const DsLayout L = ds_layout(SG, MT, M, K, ns, nms);
+    const uint32_t sbase = smem_u32(smem);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = K >> 7;
+    const int NC = (G + SG - 1) / SG;  // stages per tile
+    // balanced contiguous tile ranges: CTA sizes differ by at most one tile
+    const int t0 = (int)(((int64_t)blockIdx.x * n_tiles) / gridDim.x);
+    const int t1 = (int)(((int64_t)(blockIdx.x + 1) * n_tiles) / gridDim.x);
+    const int n_units = (t1 - t0) * NC;
+    const uint32_t bar0 = sbase + L.bars;
+    auto full_bar = [&](int s) { return bar0 + 8 * s; };
+    auto empty_bar = [&](int s) { return bar0 + 8 * (DS_MAXNS + s); };
+    auto meta_empty = [&](int i) { return bar0 + 8 * (2 * DS_MAXNS + i); };
+    auto tile_full = [&](int i) { return bar0 + 8 * (2 * DS_MAXNS + DS_MAXMS + i); };
+    auto red_empty = [&](int i) { return bar0 + 8 * (2 * DS_MAXNS + DS_MAXMS + DS_RSLOTS + i); };
+    volatile int* abort_flag =
+        reinterpret_cast<volatile int*>(smem + L.bars + 8 * (2 * DS_MAXNS + DS_MAXMS + 2 * DS_RSLOTS));
+    float* red = reinterpret_cast<float*>(smem + L.red);
+
+    if (tid == 0) {
+        for (int s = 0; s < ns; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), DS_CW);
+        }
+        for (int i = 0; i < nms; ++i) mbar_init(meta_empty(i), DS_CW);
+        for (int i = 0; i < DS_RSLOTS; ++i) {
+            mbar_init(tile_full(i), 32 * DS_CW);  // every consumer lane arrives after parking
+            mbar_init(red_empty(i), 1);
+        }
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    pdl_launch_dependents();  // the next kernel may claim the other half of the SM and start streaming
+
+    if (warp == DS_PWARP) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmW);
+            if (!weights_early) pdl_wait();
+            int issued = 0, t = t0, kc = 0, s = 0, ms = 0;
+            uint32_t ph = 0, mph = 0;
+            for (int u = 0; u < n_units; ++u) {
+                // The ring is full: from here on progress depends on the consumers, who first
+                // wait for the preceding kernel; start the bounded waits only after that point.
+                if (u == ns && weights_early) pdl_wait();
+                if ((kc == 0 && !mbar_wait_bounded(meta_empty(ms), mph ^ 1, abort_flag)) ||
+                    !mbar_wait_bounded(empty_bar(s), ph ^ 1, abort_flag)) {
+                    *abort_flag = 1;
+                    record_status(status, W4_ERR_DEVICE_TIMEOUT);
+                    break;
+                }
+                uint32_t sb = 0, zb = 0;
+                const int64_t mofs = (int64_t)t * 16 * G;  // first metadata entry of the tile
+                const uint32_t mdst = L.meta + ms * L.mslot;
+                if (kc == 0) {  // the tile's metadata rides on its first stage
+                    const int rows = N - t * 16 < 16 ? N - t * 16 : 16;  // 8 or 16 (N % 8 == 0)
+                    sb = (uint32_t)(rows * 2 * G);
+                    zb = (uint32_t)(rows * G) & ~15u;
+                    if (zb != (uint32_t)(rows * G))  // 8 trailing zero points (8 rows, odd G): plain copy
+                        *reinterpret_cast<uint2*>(smem + mdst + 32 * G + zb) =
+                            *reinterpret_cast<const uint2*>(zeros + mofs + zb);
+                }
+                mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES + sb + zb);
+                tma_load_2d(sbase + L.ring + s * STAGE_BYTES, &tmW, kc * (ROWB / 8), t * 16, full_bar(s));
+                if (sb) bulk_load_1d(sbase + mdst, scales + mofs, sb, full_bar(s));
+                if (zb) bulk_load_1d(sbase + mdst + 32 * G, zeros + mofs, zb, full_bar(s));
+                ++issued;
+                if (++kc == NC) {
+                    kc = 0;
+                    ++t;
+                    if (++ms == nms) { ms = 0; mph ^= 1; }
+                }
+                if (++s == ns) { s = 0; ph ^= 1; }
+            }
+            for (int u = issued - ns; u < issued; ++u)  // no loads in flight at exit
+                if (u >= 0) mbar_wait_bounded(full_bar(u % ns), (u / ns) & 1, nullptr, 200000000ull);
+        }
+        return;
+    }
+
+    if (warp == DS_RWARP) {
+        // ------------------------------------------------------------ reducer: Y, in warp order
+        pdl_wait();  // Y may be read by the preceding kernel
+        int rs = 0;
+        uint32_t rph = 0;
+        for (int t = t0; t < t1; ++t) {
+            if (!mbar_wait_bounded(tile_full(rs), rph, abort_flag)) {
+                *abort_flag = 1;
+                record_status(status, W4_ERR_DEVICE_TIMEOUT);
+                break;
+            }
+            const float* rsl = red + (size_t)rs * (DS_CW * 16 * MT);
+#pragma unroll
+            for (int o0 = 0; o0 < 16 * MT; o0 += 32) {
+                const int o = o0 + lane, row = o / MT, m = o - row * MT;
+                const int n = t * 16 + row;
+                if (o < 16 * MT && m < M && n < N) {
+                    float sum = 0.0f;
+#pragma unroll
+                    for (int w = 0; w < DS_CW; ++w) sum += rsl[w * (16 * MT) + o];
+                    Y[(int64_t)m * N + n] = __float2half_rn(sum);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(red_empty(rs));
+            if (++rs == DS_RSLOTS) { rs = 0; rph ^= 1; }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    // Consumer warp w owns the GPW consecutive groups w*GPW .. w*GPW+GPW-1 of every stage: in stage
+    // kc of a tile, groups kc*SG + w*GPW + e.  It stages exactly the activations of those groups,
+    // with their offset sums, so no other warp waits for them (one memory round trip after the
+    // preceding kernel has finished).  The 16 chunks of one group sit in 16 consecutive lanes,
+    // which reduce the sums with shuffles in a fixed order.
+    pdl_wait();  // the activations may be produced by the preceding kernel
+    const uint32_t xs_u = sbase + L.xs;
+    const uint32_t corr_u = sbase + L.corr;
+    __half* xs = reinterpret_cast<__half*>(smem + L.xs);
+    float2* corr = reinterpret_cast<float2*>(smem + L.corr);
+    const int RS = K + 8;  // staged row stride in halves (16 bytes of padding)
+    {
+        const __half2 sixteenth = __float2half2_rn(0.0625f);
+        const unsigned half_mask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;
+        const int per_warp = M * NC * GPW * 16;  // chunks of 8 k this warp stages (a multiple of 16)
+        for (int base = 0; base < per_warp; base += 32 * DS_XILP) {
+            uint4 raw[DS_XILP];
+#pragma unroll
+            for (int v = 0; v < DS_XILP; ++v) {
+                const int i = base + v * 32 + lane;
+                const int q = i >> 4, e = q % GPW, r = q / GPW, kc = r % NC, m = r / NC;
+                const int g = kc * SG + warp * GPW + e;
+                if (i < per_warp && g < G) raw[v] = ldg_cached(X + (int64_t)m * K + g * 128 + (i & 15) * 8);
+            }
+#pragma unroll
+            for (int v = 0; v < DS_XILP; ++v) {
+                const int i = base + v * 32 + lane;
+                const int q = i >> 4, e = q % GPW, r = q / GPW, kc = r % NC, m = r / NC;
+                const int g = kc * SG + warp * GPW + e;
+                if (i >= per_warp || g >= G) continue;  // uniform per 16-lane half (one group)
+                const int ch = g * 16 + (i & 15);       // chunk index within the row
+                const uint4 w = raw[v];
+                uint4 p;
+                p.x = __byte_perm(w.x, w.z, 0x5410);         // x0, x4
+                uint32_t h = __byte_perm(w.x, w.z, 0x7632);  // x1, x5
+                __half2 hh = __hmul2(*reinterpret_cast<__half2*>(&h), sixteenth);
+                p.y = *reinterpret_cast<uint32_t*>(&hh);
+                p.z = __byte_perm(w.y, w.w, 0x5410);  // x2, x6
+                h = __byte_perm(w.y, w.w, 0x7632);    // x3, x7
+                hh = __hmul2(*reinterpret_cast<__half2*>(&h), sixteenth);
+                p.w = *reinterpret_cast<uint32_t*>(&hh);
+                *reinterpret_cast<uint4*>(xs + (int64_t)m * RS + ds_swz(ch) * 8) = p;
+                float lo = half2_sum(p.x) + half2_sum(p.z);  // staged low-nibble partners
+                float hi = half2_sum(p.y) + half2_sum(p.w);  // staged high-nibble partners (x/16)
+#pragma unroll
+                for (int o = 8; o; o >>= 1) {
+                    lo += __shfl_xor_sync(half_mask, lo, o);
+                    hi += __shfl_xor_sync(half_mask, hi, o);
+                }
+                if ((i & 15) == 0)  // C = 1024 (Sl + Sh'), S = Sl + 16 Sh'
+                    corr[g * MT + m] = make_float2(1024.0f * (lo + hi), fmaf(16.0f, hi, lo));
+            }
+        }
+    }
+    // corr entries of activation rows >= M stay unset: they only feed columns that are never stored
+    __syncwarp();
+
+    const int g8 = lane >> 2, c = lane & 3;
+    const bool xlane = g8 < M;  // B column g8 holds activation row g8; other lanes use zeros
+    const uint32_t xrow = xs_u + (uint32_t)(xlane ? g8 : 0) * (uint32_t)RS * 2u;
+    uint32_t xofs[4];  // swizzled byte offset of word j's chunk within a group, for this lane
+#pragma unroll
+    for (int j = 0; j < 4; ++j) xofs[j] = (uint32_t)ds_swz(c * 4 + j) * 16u;
+    const int ccol = 2 * c < MT ? 2 * c : 0;  // first activation column of this thread's C pair
+    const bool mvec = (G % GPW) == 0;         // metadata of the warp's groups is vector-aligned
+    // this thread's W bytes inside a stage: rows g8 and g8 + 8 of the warp's groups, 16 bytes at 16 c
+    const uint32_t wlane = (uint32_t)(g8 * ROWB + warp * GPW * 64 + c * 16);
+    int s = 0, kc = 0, ms = 0, rs = 0;
+    uint32_t ph = 0, rph = 0;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // rows (g8, g8+8) x cols (2c, 2c+1)
+    bool dead = false;
+    for (int u = 0; u < n_units; ++u) {
+        // After a timeout every wait is skipped; the loop still runs to the end.
+        if (!dead && !mbar_wait_bounded(full_bar(s), ph, abort_flag)) {
+            *abort_flag = 1;
+            record_status(status, W4_ERR_DEVICE_TIMEOUT);
+            dead = true;
+        }
+        const int g0 = kc * SG + warp * GPW;
+        const int ng = g0 >= G ? 0 : min(GPW, G - g0);
+        if (!dead && ng > 0) {
+            const uint32_t st = sbase + L.ring + (uint32_t)s * STAGE_BYTES + wlane;
+            const uint32_t xg = xrow + (uint32_t)g0 * 256u;
+            const uint32_t msa = sbase + L.meta + (uint32_t)ms * L.mslot;  // scales [16][G] fp16
+            const uint32_t mza = msa + 32u * (uint32_t)G;                   // zeros [16][G] u8
+            const uint32_t ia = (uint32_t)(g8 * G + g0), ib = ia + 8u * (uint32_t)G;
+            if (ng == GPW && mvec) {
+                // the scales and zero points of the warp's groups, packed: GPW fp16 and GPW bytes per row
+                uint32_t sa[GPW / 2], sb[GPW / 2], za, zb;
+                if constexpr (GPW == 4) {
+                    const uint2 va = lds64(msa + 2u * ia), vb = lds64(msa + 2u * ib);
+                    sa[0] = va.x; sa[1] = va.y; sb[0] = vb.x; sb[1] = vb.y;
+                    za = lds32(mza + ia);
+                    zb = lds32(mza + ib);
+                } else {
+                    sa[0] = lds32(msa + 2u * ia);
+                    sb[0] = lds32(msa + 2u * ib);
+                    za = lds_u16(mza + ia);
+                    zb = lds_u16(mza + ib);
+                }
+#pragma unroll
+                for (int e = 0; e < GPW; ++e) {
+                    const float fsa = ds_half(sa[e >> 1], e & 1), fsb = ds_half(sb[e >> 1], e & 1);
+                    const float fza = (float)((za >> (8 * e)) & 0xFFu), fzb = (float)((zb >> (8 * e)) & 0xFFu);
+                    ds_group<MT>(st + e * 64, st + e * 64 + 8 * ROWB, xg + e * 256, xofs, xlane,
+                                 corr_u + (uint32_t)((g0 + e) * MT + ccol) * 8u, fsa, fsb, fza, fzb, acc);
+                }
+            } else {
+                for (int e = 0; e < ng; ++e) {
+                    const float fsa = __half2float(__ushort_as_half(lds_u16(msa + 2u * (ia + e))));
+                    const float fsb = __half2float(__ushort_as_half(lds_u16(msa + 2u * (ib + e))));
+                    const float fza = (float)lds_u8(mza + ia + e);
+                    const float fzb = (float)lds_u8(mza + ib + e);
+                    ds_group<MT>(st + e * 64, st + e * 64 + 8 * ROWB, xg + e * 256, xofs, xlane,
+                                 corr_u + (uint32_t)((g0 + e) * MT + ccol) * 8u, fsa, fsb, fza, fzb, acc);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));
+        if (++s == ns) { s = 0; ph ^= 1; }
+        if (++kc == NC) {
+            // tile done: release its metadata, park this warp's partials for the reducer
+            if (lane == 0) mbar_arrive(meta_empty(ms));
+            if (++ms == nms) ms = 0;
+            if (!dead && !mbar_wait_bounded(red_empty(rs), rph ^ 1, abort_flag)) {
+                *abort_flag = 1;
+                record_status(status, W4_ERR_DEVICE_TIMEOUT);
+                dead = true;
+            }
+            float* mine = red + (size_t)rs * (DS_CW * 16 * MT) + warp * (16 * MT);
+            if (2 * c < MT) { mine[g8 * MT + 2 * c] = acc[0]; mine[(g8 + 8) * MT + 2 * c] = acc[2]; }
+            if (2 * c + 1 < MT) { mine[g8 * MT + 2 * c + 1] = acc[1]; mine[(g8 + 8) * MT + 2 * c + 1] = acc[3]; }
+            mbar_arrive(tile_full(rs));  // every lane: its own stores are released with it
+            if (++rs == DS_RSLOTS) { rs = 0; rph ^= 1; }
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+            kc = 0;
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------ host side
+static int ds_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+
+// Launch plan: stage size (32 groups: every consumer warp takes two groups of a stage), ring
+// depth and metadata slots within one SM's shared memory; one CTA per SM (or per tile when there
+// are fewer tiles than SMs).
+bool plan_decode_stream(int64_t M, int64_t N, int64_t K, DecodePlan* p) {
+    if (M < 1 || M > DS_MAXM || N < 8 || K < 128 || K % 128 != 0 || K > 65536 || N % 8 != 0) return false;
+    const int mt = ds_mt(M);
+    const int G = (int)(K / 128);
+    const int64_t T = (N + 15) / 16;
+    const int sms = device_sm_count();
+    const int grid = (int)std::min<int64_t>(T, sms);
+    const int64_t tpc = (T + grid - 1) / grid;  // tiles of the largest CTA
+    {
+        const uint32_t budget = DS_FULL_SMEM;
+        bool found = false;
+        int64_t best_bytes = -1;
+        for (int sg : {32}) {
+            const int NC = (G + sg - 1) / sg;
+            const int64_t units = tpc * NC;
+            const int nms = (int)std::min<int64_t>(DS_MAXMS, std::min<int64_t>(tpc, 2 + (int64_t)DS_MAXNS / NC));
+            const uint32_t fixed = ds_layout(sg, mt, (int)M, (int)K, 0, nms).total + 1024;  // alignment slack
+            const uint32_t sb = ds_stage_bytes(sg);
+            const int64_t want = std::min<int64_t>(DS_MINNS, units);
+            if (fixed + want * sb > budget) continue;
+            const int64_t ns = std::min<int64_t>(std::min<int64_t>((budget - fixed) / sb, DS_MAXNS), units);
+            const int64_t bytes = ns * sb;
+            if (bytes > best_bytes) {
+                best_bytes = bytes;
+                p->sg = sg;
+                p->mt = mt;
+                p->ns = (int)ns;
+                p->nms = nms;
+                p->n_tiles = (int)T;
+                p->grid = grid;
+                p->smem = ds_layout(sg, mt, (int)M, (int)K, (int)ns, nms).total + 1024;
+                found = true;
+            }
+        }
+        if (found) return true;
+    }
+    return false;
+}
+
+template <int MT, int SG>
+static cudaError_t ds_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                             const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, const DecodePlan& p,
+                             bool weights_static, int* status, cudaStream_t stream) {
+    static std::once_flag once[64];
+    static cudaError_t attr_err[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [&]() {
+        attr_err[dev] = cudaFuncSetAttribute(decode_stream_kernel<MT, SG>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DS_FULL_SMEM);
+    });
+    if (attr_err[dev] != cudaSuccess) return attr_err[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.grid, 1, 1);
+    cfg.blockDim = dim3(DS_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = weights_static ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<MT, SG>, tm, reinterpret_cast<const __half*>(X),
+                              reinterpret_cast<const unsigned short*>(scales), zeros, reinterpret_cast<__half*>(Y),
+                              (int)M, (int)N, (int)K, p.n_tiles, p.ns, p.nms, weights_static ? 1 : 0, status);
+}
+
+template <int SG>
+static cudaError_t ds_launch_mt(const CUtensorMap& tm, const uint16_t* X, int64_t M, int64_t N, int64_t K,
+                                const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, const DecodePlan& p,
+                                bool weights_static, int* status, cudaStream_t stream) {
+    switch (p.mt) {
+        case 1: return ds_launch<1, SG>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
+        case 2: return ds_launch<2, SG>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
+        case 4: return ds_launch<4, SG>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
+        default: return ds_launch<8, SG>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
+    }
+}
+
+cudaError_t launch_decode_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                                 const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, bool weights_static,
+                                 int* status, cudaStream_t stream) {
+    DecodePlan p;
+    if (!plan_decode_stream(M, N, K, &p)) return cudaErrorInvalidValue;
+    CUtensorMap tm;  // packed rows as 8-byte elements: a box of 8 SG elements is one stage's share of a row
+    if (!make_tensor_map_2d(&tm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)(K / 16), (uint64_t)N,
+                            (uint32_t)(8 * p.sg), 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    return ds_launch_mt<32>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
+}
+
+}  // namespace w4

@@ -35,11 +35,20 @@ cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           uint16_t* Y, const SkinnyPlan& plan, bool weights_static,
                           cudaStream_t stream);
 
-// Decode GEMV for M <= 8, persistent TMA-fed (gemv_stream.cu).
-cudaError_t launch_gemv_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                               const uint16_t* scales, const uint8_t* zeros, uint16_t* Y,
-                               bool weights_static, int* status, cudaStream_t stream);
-size_t gemv_stream_smem(int64_t M, int64_t K);  // SIZE_MAX when the shape cannot use the kernel
+// Decode GEMV for M <= 8, one TMA-fed CTA per SM (decode_stream.cu).
+struct DecodePlan {
+    int sg;             // groups of 128 k per 16-row stage (32: 32 KB)
+    int mt;             // activation-row bound of the instantiation: 1, 2, 4 or 8
+    int ns;             // ring stages
+    int nms;            // metadata slots
+    int n_tiles;        // 16-row tiles in all (balanced over the CTAs)
+    int grid;           // CTAs
+    uint32_t smem;      // dynamic shared memory per CTA
+};
+bool plan_decode_stream(int64_t M, int64_t N, int64_t K, DecodePlan* plan);  // false: shape not served
+cudaError_t launch_decode_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                                 const uint16_t* scales, const uint8_t* zeros, uint16_t* Y,
+                                 bool weights_static, int* status, cudaStream_t stream);
 
 // Decode GEMV for M <= 8 on tcgen05 with the weights as a TMEM operand (gemv_tc.cu).
 struct GemvTcPlan {
