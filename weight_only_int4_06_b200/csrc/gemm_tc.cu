@@ -33,24 +33,26 @@
 
 namespace w4 {
 
-constexpr int TC_BN = 256;
+constexpr int TC_BN = 256;  // W rows per tile (the AWQ modes; w4_gemm also has 128-row W tiles)
 constexpr int TC_BK = 64;
 constexpr int TC_THREADS = 384;
 constexpr int TC_DEQ_THREADS = 256;
 constexpr uint32_t TC_A1_BYTES = 128 * TC_BK * 2;   // 16 KB per 128-row X tile
-constexpr uint32_t TC_B_BYTES = TC_BN * TC_BK * 2;  // 32 KB
-constexpr uint32_t TC_P_BYTES = TC_BN * TC_BK / 2;  // 8 KB of packed codes
 constexpr int TC_GROUP_M = 8;  // raster: CTAs in flight share X and W tiles through L2
 
-template <bool DEQ, int MT>
+// Tile of (128 MT) rows of X by BN rows of W; as many ring stages as fit (at most 6).
+template <bool DEQ, int MT, int BN>
 struct TcCfg {
     static constexpr int kBM = 128 * MT;
     static constexpr uint32_t kA = TC_A1_BYTES * MT;
-    static constexpr uint32_t kStage = kA + TC_B_BYTES + (DEQ ? TC_P_BYTES : 0);
-    static constexpr int kStages = (MT == 1) ? 4 : 3;
+    static constexpr uint32_t kB = BN * TC_BK * 2;  // fp16 W tile (dequantised or loaded)
+    static constexpr uint32_t kP = BN * TC_BK / 2;  // packed codes of the W tile
+    static constexpr uint32_t kStage = kA + kB + (DEQ ? kP : 0);
+    static constexpr int kFit = (int)((227u * 1024u - 1280u) / kStage);
+    static constexpr int kStages = kFit < 6 ? kFit : 6;
     static constexpr uint32_t kBarOff = kStage * kStages;
     static constexpr uint32_t kBytes = kBarOff + 256 + 1024;  // barriers + slack for 1 KB alignment
-    static constexpr uint32_t kTmemCols = 256 * MT;
+    static constexpr uint32_t kTmemCols = BN * MT;
 };
 
 __device__ __forceinline__ void tc_tile_coords(int t, int m_tiles, int n_tiles, int& mt, int& nt) {
@@ -63,7 +65,7 @@ __device__ __forceinline__ void tc_tile_coords(int t, int m_tiles, int n_tiles, 
     nt = r / gm;
 }
 
-template <bool DEQ, int EPI, int MT>
+template <bool DEQ, int EPI, int MT, int BN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __half* __restrict__ scales, const uint8_t* __restrict__ zeros,
@@ -71,14 +73,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                    const __half* __restrict__ Adot, int M, int N, int K, int m_tiles, int n_tiles,
                    int* status) {
     constexpr bool SSE = EPI == 1 || EPI == 3;  // modes that reduce the tile to one fp64 partial
-    using C = TcCfg<DEQ, MT>;
+    using C = TcCfg<DEQ, MT, BN>;
     constexpr int S = C::kStages;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = smem_align1024(smem_raw);
     const uint32_t sbase = smem_u32(smem);
     auto a_addr = [&](int s) { return sbase + s * C::kStage; };
     auto b_addr = [&](int s) { return sbase + s * C::kStage + C::kA; };
-    auto p_addr = [&](int s) { return sbase + s * C::kStage + C::kA + TC_B_BYTES; };
+    auto p_addr = [&](int s) { return sbase + s * C::kStage + C::kA + C::kB; };
     const uint32_t bar0 = sbase + C::kBarOff;
     auto full_bar = [&](int s) { return bar0 + 8 * s; };
     auto deq_bar = [&](int s) { return bar0 + 8 * (S + s); };
@@ -91,7 +93,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int mt, nt;
     tc_tile_coords(blockIdx.x, m_tiles, n_tiles, mt, nt);
-    const int m0 = mt * C::kBM, n0 = nt * TC_BN;
+    const int m0 = mt * C::kBM, n0 = nt * BN;
     const int nk = K / TC_BK;
     const int G = K >> 7;
 
@@ -124,7 +126,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const uint32_t tx = C::kA + (DEQ ? TC_P_BYTES : TC_B_BYTES);
+            const uint32_t tx = C::kA + (DEQ ? C::kP : C::kB);
             int issued = 0;
             for (int kb = 0; kb < nk; ++kb) {
                 const int s = kb % S;
@@ -145,7 +147,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16_f32(128, TC_BN);
+            constexpr uint32_t idesc = idesc_f16_f32(128, BN);
             bool ok = true;
             for (int kb = 0; kb < nk && ok; ++kb) {
                 const int s = kb % S;
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     for (int t = 0; t < MT; ++t) {
                         const uint64_t ad = sw128_kmajor_desc(a_addr(s) + t * TC_A1_BYTES);
                         // +32 bytes along K per MMA inside the 128-byte swizzled row
-                        mma_f16_ss(tmem_d + t * 256, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+                        mma_f16_ss(tmem_d + t * BN, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
                     }
                 }
                 tc_commit(empty_bar(s));
@@ -171,7 +173,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int d = tid - 128;  // 0..255
         if (DEQ) {
             // -------------------------------------------------------- dequantisation
-            const int r = d;  // tile row (row of W)
+            // W tile rows are shared by 256 / BN threads, each dequantising WPT of the row's 8 words
+            constexpr int WPT = 8 * BN / TC_DEQ_THREADS;
+            const int r = d % BN;  // tile row (row of W)
+            const int part = d / BN;
             const int n = n0 + r;
             const bool nvalid = n < N;
             uint32_t s2 = 0, zl = 0, zh = 0;
@@ -199,14 +204,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     zh = (0xD400u | (z << 4)) * 0x10001u;
                 }
                 if (!mbar_wait_bounded(full_bar(s), ph, abort_flag)) { fail(); break; }
-                const unsigned char* prow = smem + (p_addr(s) - sbase) + r * 32;
-                const uint4 w0 = *reinterpret_cast<const uint4*>(prow);
-                const uint4 w1 = *reinterpret_cast<const uint4*>(prow + 16);
-                const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                const unsigned char* prow = smem + (p_addr(s) - sbase) + r * 32 + part * (WPT * 4);
+                uint32_t words[WPT];
+#pragma unroll
+                for (int i = 0; i < WPT; i += 4) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(prow + 4 * i);
+                    words[i] = w4.x; words[i + 1] = w4.y; words[i + 2] = w4.z; words[i + 3] = w4.w;
+                }
                 unsigned char* brow = smem + (b_addr(s) - sbase) + b_row;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint32_t w = words[c];
+                for (int cw = 0; cw < WPT; ++cw) {
+                    const int c = part * WPT + cw;  // word (8 k) within the row's 64 k
+                    const uint32_t w = words[cw];
                     uint32_t lo0 = hsub2_u32(lop3_and_or(w, 0x000F000Fu, 0x64006400u), zl);            // n0,n4
                     uint32_t hi0 = hfma2_u32(lop3_and_or(w, 0x00F000F0u, 0x64006400u), 0x2C002C00u, zh);  // n1,n5
                     const uint32_t w8 = w >> 8;
@@ -230,13 +239,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         // ------------------------------------------------------------ epilogue
         // warp (4 + 4*slot + q) reads TMEM lanes [32q, 32q + 32) (the quarter it may access):
-        // MT == 1: columns [128*slot, 128*slot + 128) of the single accumulator;
-        // MT == 2: all 256 columns of accumulator `slot`.
+        // MT == 1: columns [BN/2 * slot, BN/2 * slot + BN/2) of the single accumulator;
+        // MT == 2: all BN columns of accumulator `slot`.
         const int q = warp & 3;
         const int slot = (warp - 4) >> 2;
         const int acc = MT == 1 ? 0 : slot;
-        const int c_begin = MT == 1 ? slot * 128 : 0;
-        const int c_count = MT == 1 ? 128 : 256;
+        const int c_begin = MT == 1 ? slot * (BN / 2) : 0;
+        const int c_count = MT == 1 ? BN / 2 : BN;
         // not cut short by the abort flag: TMEM is freed only after every issued MMA completed
         const bool ok = mbar_wait_bounded(accum_bar, 0, nullptr, 4000000000ull);
         if (!ok) fail();
@@ -248,7 +257,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int cc = 0; cc < c_count; cc += 32) {
                 const int col = c_begin + cc;
                 uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * 256 + col), v);
+                tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + col), v);
                 tmem_wait_ld();
                 if (EPI == 1) {
                     float a = 0.0f;
@@ -341,6 +350,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 }
 
 // ------------------------------------------------------------------------------------ host side
+// Relative time of one tile of each w4_gemm tile shape (MT x 128 rows of X, BN rows of W), in
+// units of a (1 x 128) x 128 tile at the same K.  Measured on B200 at M = 4096, K = N = 4096 (many
+// waves of every shape, rotating weights): 113.0, 172.9, 150.7 and 205.1 us for 256, 512, 512
+// and 1024 tiles, i.e. per-tile times 2.20 : 1.69 : 1.47 : 1.00.  Larger tiles cost more per tile
+// but much less per flop (each dequantised weight feeds MT MMAs, each X tile BN rows of W).
+#ifndef TC_TT_2_256
+#define TC_TT_2_256 2.20
+#define TC_TT_1_256 1.69
+#define TC_TT_2_128 1.47
+#define TC_TT_1_128 1.00
+#endif
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -368,7 +388,7 @@ bool make_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType 
     return r == CUDA_SUCCESS;
 }
 
-template <bool DEQ, int EPI, int MT>
+template <bool DEQ, int EPI, int MT, int BN>
 static cudaError_t set_tc_attrs() {
     static std::once_flag once[64];
     static cudaError_t err[64];
@@ -377,32 +397,32 @@ static cudaError_t set_tc_attrs() {
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&]() {
-        err[dev] = cudaFuncSetAttribute(tc_gemm_kernel<DEQ, EPI, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)TcCfg<DEQ, MT>::kBytes);
+        err[dev] = cudaFuncSetAttribute(tc_gemm_kernel<DEQ, EPI, MT, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)TcCfg<DEQ, MT, BN>::kBytes);
     });
     return err[dev];
 }
 
-template <bool DEQ, int EPI, int MT>
+template <bool DEQ, int EPI, int MT, int BN = TC_BN>
 static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int64_t N, int64_t K,
                              const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, double* sse_part,
                              int* status, cudaStream_t stream, float* Cf = nullptr) {
-    using C = TcCfg<DEQ, MT>;
+    using C = TcCfg<DEQ, MT, BN>;
     CUtensorMap ta, tb;
     if (!make_tensor_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, TC_BK, C::kBM,
                      CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const bool okb =
         DEQ ? make_tensor_map_2d(&tb, Bop, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)(K / 8), (uint64_t)N, TC_BK / 8,
-                          TC_BN, CU_TENSOR_MAP_SWIZZLE_NONE)
-            : make_tensor_map_2d(&tb, Bop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)N, TC_BK, TC_BN,
+                          BN, CU_TENSOR_MAP_SWIZZLE_NONE)
+            : make_tensor_map_2d(&tb, Bop, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)N, TC_BK, BN,
                           CU_TENSOR_MAP_SWIZZLE_128B);
     if (!okb) return cudaErrorInvalidValue;
-    cudaError_t e = set_tc_attrs<DEQ, EPI, MT>();
+    cudaError_t e = set_tc_attrs<DEQ, EPI, MT, BN>();
     if (e != cudaSuccess) return e;
     const int m_tiles = (int)((M + C::kBM - 1) / C::kBM);
-    const int n_tiles = (int)((N + TC_BN - 1) / TC_BN);
-    tc_gemm_kernel<DEQ, EPI, MT><<<m_tiles * n_tiles, TC_THREADS, C::kBytes, stream>>>(
+    const int n_tiles = (int)((N + BN - 1) / BN);
+    tc_gemm_kernel<DEQ, EPI, MT, BN><<<m_tiles * n_tiles, TC_THREADS, C::kBytes, stream>>>(
         ta, tb, reinterpret_cast<const __half*>(scales), zeros, reinterpret_cast<__half*>(Y), sse_part, Cf,
         reinterpret_cast<const __half*>(X), (int)M, (int)N, (int)K, m_tiles, n_tiles, status);
     return cudaGetLastError();
@@ -411,12 +431,42 @@ static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int6
 // 256-row tiles once M is large enough to fill them; 128-row tiles otherwise.
 static int tc_mt(int64_t M) { return M > 128 ? 2 : 1; }
 
+// Tile shape of w4_gemm's tensor-core path: the fewest waves of one-CTA-per-SM tiles, weighed by
+// each shape's per-tile time (larger tiles share every dequantised weight between more rows of X
+// and every X tile between more rows of W, so they run closer to the tensor peak).
+void tc_w4_pick(int64_t M, int64_t N, int* mt_out, int* bn_out) {
+    const int64_t sms = device_sm_count();
+    const int shapes[4][2] = {{2, 256}, {1, 256}, {2, 128}, {1, 128}};
+    // relative time of one tile, from the measured per-tile rates of each shape
+    const double tile_time[4] = {TC_TT_2_256, TC_TT_1_256, TC_TT_2_128, TC_TT_1_128};
+    double best = -1.0;
+    *mt_out = 2;
+    *bn_out = 256;
+    for (int i = 0; i < 4; ++i) {
+        const int mt = shapes[i][0], bn = shapes[i][1];
+        if (mt == 2 && M <= 128) continue;
+        const int64_t tiles = ((M + 128 * mt - 1) / (128 * mt)) * ((N + bn - 1) / bn);
+        const double t = (double)((tiles + sms - 1) / sms) * tile_time[i];
+        if (best < 0.0 || t < best) {
+            best = t;
+            *mt_out = mt;
+            *bn_out = bn;
+        }
+    }
+}
+
 cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                          const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,
                          cudaStream_t stream) {
-    if (tc_mt(M) == 2)
-        return launch_tc<true, 0, 2>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
-    return launch_tc<true, 0, 1>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
+    int mt = 2, bn = 256;
+    tc_w4_pick(M, N, &mt, &bn);
+    if (mt == 2 && bn == 256)
+        return launch_tc<true, 0, 2, 256>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
+    if (mt == 1 && bn == 256)
+        return launch_tc<true, 0, 1, 256>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
+    if (mt == 2)
+        return launch_tc<true, 0, 2, 128>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
+    return launch_tc<true, 0, 1, 128>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream);
 }
 
 cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64_t N, int64_t K,
