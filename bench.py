@@ -203,16 +203,10 @@ def prefill_cases():
             "prefill, compute-bound")
 
 
-def gemm_launches(M, K):
-    """Kernel launches of one w4_gemm call at the bench's shapes (decode M = 1; small batch M <= 32 at
-    K = 8192 or 28672; prefill M >= 512): for 8 < M <= 32 the GEMV takes up to 8 rows per launch
-    where 8 staged activation rows fit shared memory (K = 8192; not K = 28672, which keeps one
-    skinny launch); every other case is one launch."""
-    if M <= 8:
-        return 1
-    if M <= 32 and K <= 8192:
-        return (M + 7) // 8
-    return 1
+def gemm_launches(M, K, N, variant=0, scales=None, zeros=None):
+    """Kernel launches of one w4_gemm call, as the library's own dispatch decides them."""
+    from weight_only_int4_06_b200 import w4a16 as B
+    return B.w4_gemm_plan(M, N, K, 128, variant, scales, zeros)[1]
 
 
 class GemmWorkload:
@@ -224,6 +218,9 @@ class GemmWorkload:
         self.B = B
         self.variant = variant
         self.cases = cases
+        # Weight copies per layer: the step rotates through n_sets copies of every layer (more than
+        # 3x L2 between two uses of a copy); a layer timed alone rotates through its own copies,
+        # at least 3x L2 of that layer's weights.
         step_w = sum(N * K // 2 + N * (K // 128) * 3 for (M, K, N) in cases)
         self.n_sets = max(1, min(16, int(np.ceil(3 * l2_bytes / max(step_w, 1))) + 1))
         self.layers = []
@@ -233,7 +230,9 @@ class GemmWorkload:
             Wd = torch.from_numpy(W).cuda()
             packed, scales, zeros = B.w4_quantize_pack(Wd)
             copies = [(packed, scales, zeros)]
-            for c in range(1, self.n_sets):
+            layer_w = N * K // 2 + N * (K // 128) * 3
+            n_layer = max(self.n_sets, min(64, int(np.ceil(3 * l2_bytes / layer_w)) + 1))
+            for c in range(1, n_layer):
                 copies.append((packed.clone(), scales.clone(), zeros.clone()))
             del Wd
             Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
@@ -246,40 +245,48 @@ class GemmWorkload:
         torch.cuda.synchronize()
         self.bytes_per_step = sum(gemm_bytes(M, K, N) for (M, K, N) in cases)
         self.flops_per_step = sum(2 * M * K * N for (M, K, N) in cases)
-        self.launches_per_step = sum(gemm_launches(M, K) for (M, K, N) in cases)
+        self.launches_per_step = sum(gemm_launches(M, K, N, variant, L["copies"][0][1], L["copies"][0][2])
+                                     for (M, K, N), L in zip(cases, self.layers))
         self.host_calls = None  # prepared w4_gemm_host calls, built on first use
         self.host_path_note = None
 
     def run_step(self, step, only=None):
-        s = step % self.n_sets
         for i, L in enumerate(self.layers):
             if only is not None and i != only:
                 continue
-            p, sc, z = L["copies"][s]
+            copies = L["copies"] if only is not None else L["copies"][:self.n_sets]
+            p, sc, z = copies[step % len(copies)]
             self.B.w4_gemm(L["X"], p, sc, z, out=L["Y"], workspace=L["ws"], variant=self.variant)
 
     def run_step_host(self, step):
-        """The same step through the public API with host (pinned) activations and results:
-        every layer is one w4_gemm_host call (copy X in, GEMM, copy Y out on the stream), prepared
-        once per layer and weight copy as a serving loop over fixed buffers would; the step ends
-        when the stream has drained (the results are then readable on the host)."""
+        """The same step through the public API with host (pinned) activations and results: one
+        w4_gemm_host_batch C call per step (every layer's X in one host-to-device copy, the layers'
+        GEMMs, every Y in one device-to-host copy), prepared once per weight set as a serving loop
+        over fixed buffers would; the step ends when the stream has drained (the results are then
+        readable on the host)."""
         import torch
         if self.host_calls is None:
             try:
-                self.host_calls = [[self.B.HostGemmCall(L["Xh"], *L["copies"][c], L["Yh"], L["xs"], L["Y"],
-                                                        workspace=L["ws"]) for L in self.layers]
-                                   for c in range(self.n_sets)]
-            except Exception as e:  # the same C call, marshalled on every call instead
                 self.host_calls = []
-                self.host_path_note = f"prepared calls unavailable ({type(e).__name__}: {e}); per-call w4_gemm_host"
+                for c in range(self.n_sets):
+                    b = self.B.HostGemmBatch([L["copies"][c] for L in self.layers],
+                                             [(L["M"], L["K"], L["N"]) for L in self.layers],
+                                             workspace=self.layers[0]["ws"], variant=self.variant)
+                    for i, L in enumerate(self.layers):
+                        b.x(i).copy_(L["Xh"])
+                    self.host_calls.append(b)
+            except Exception as e:  # the per-layer C call instead
+                self.host_calls = []
+                self.host_path_note = f"batched call unavailable ({type(e).__name__}: {e}); per-layer w4_gemm_host"
         if self.host_calls:
-            for call in self.host_calls[step % self.n_sets]:
-                call.run()
-        else:
-            s = step % self.n_sets
-            for L in self.layers:
-                p, sc, z = L["copies"][s]
-                self.B.w4_gemm_host(L["Xh"], p, sc, z, L["Yh"], L["xs"], L["Y"], workspace=L["ws"])
+            b = self.host_calls[step % self.n_sets]
+            b.run()
+            torch.cuda.current_stream().synchronize()
+            return [b.y(i) for i in range(len(self.layers))]
+        s = step % self.n_sets
+        for L in self.layers:
+            p, sc, z = L["copies"][s]
+            self.B.w4_gemm_host(L["Xh"], p, sc, z, L["Yh"], L["xs"], L["Y"], workspace=L["ws"])
         torch.cuda.current_stream().synchronize()
         return [L["Yh"] for L in self.layers]
 
@@ -369,9 +376,11 @@ def layer_rows(wl, world, reps, peaks, compute_bound, flush=None, replays=5):
     weight sets), median of `replays` replays."""
     rows = []
     for i, L in enumerate(wl.layers):
-        gi = capture(lambda s, i=i: wl.run_step(s, only=i), reps, 0)
+        # every call of the graph uses a different copy of the layer's weights (cold L2)
+        n = max(reps, len(L["copies"]))
+        gi = capture(lambda s, i=i: wl.run_step(s, only=i), n, 0)
         gi.replay()
-        t = time_graph_median(gi, world, replays, flush)[0] / reps
+        t = time_graph_median(gi, world, replays, flush)[0] / n
         b = gemm_bytes(L["M"], L["K"], L["N"])
         fl = 2 * L["M"] * L["K"] * L["N"]
         r = {"M": L["M"], "K": L["K"], "N": L["N"], "us": round(t * 1e3, 3),
@@ -496,9 +505,10 @@ def run_gemm_bench(args, rank, world, local, kind, with_extras=True):
                    "l2": "flushed (2x L2 write) before every replay, outside the timed region"},
         "e2e": {"value": round(e2e_ms * 1e3, 3), "unit": "us/step", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "path": wl.host_path_note or ("one w4_gemm_host C call per layer (pinned X in, GEMM, Y out), "
-                                              "prepared once per buffer set (HostGemmCall); one stream "
-                                              "synchronisation per step")},
+                "path": wl.host_path_note or ("one w4_gemm_host_batch C call per step (all layers' X in one "
+                                              "pinned host-to-device copy, the GEMMs, all Y in one "
+                                              "device-to-host copy), prepared once per weight set "
+                                              "(HostGemmBatch); one stream synchronisation per step")},
         "gpu_launches": wl.launches_per_step * K_steps,
         "clocks": clocks,
     }
@@ -707,6 +717,26 @@ def bench_awq_clip(world, peaks, case, reps=3, n_ratios=10):
             "alu_frac": round(tf / peak, 3), "flops": flops}
 
 
+def _small_batch_row(world, peaks, l2):
+    """Config-3 shapes one at a time: M in {4, 8, 16, 32} x the 70B-class (K, N)."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    cases = small_batch_cases()[0]
+    wl = GemmWorkload(cases, 3, l2, variant=B.FLAG_WEIGHTS_STATIC)
+    wl.run_step(0)
+    torch.cuda.synchronize()
+    flush = L2Flush(l2)
+    layers = layer_rows(wl, world, 10, peaks, False, flush)
+    for r, (M, K, N), L in zip(layers, cases, wl.layers):
+        fam, n = B.w4_gemm_plan(M, N, K, 128, 0, L["copies"][0][1], L["copies"][0][2])
+        r["family"] = {B.VARIANT_GEMV: "gemv", B.VARIANT_SKINNY: "skinny", B.VARIANT_TC: "tc"}.get(fam, str(fam))
+        r["launches"] = n
+    del wl, flush
+    torch.cuda.empty_cache()
+    return {"kernel": "w4_gemm (per-shape family: decode_stream_kernel in launches of <= 8 rows, "
+                      "skinny_kernel where 8 staged rows do not fit)", "bound": "hbm", "layers": layers}
+
+
 def _prefill_row(world, peaks, l2):
     import torch
     pre = GemmWorkload(prefill_cases()[0], 4, l2)
@@ -739,6 +769,7 @@ def other_rows(args, world, peaks, l2):
             except Exception:
                 pass
 
+    row("small_batch", lambda: _small_batch_row(world, peaks, l2))
     row("quantize", lambda: bench_quantize(world, peaks, l2))
     row("prefill", lambda: _prefill_row(world, peaks, l2))
     case = synth.awq_case()
@@ -751,6 +782,54 @@ def other_rows(args, world, peaks, l2):
         row("gptq", lambda: bench_gptq(world, peaks))
         row("wb_gemm", lambda: bench_wb_gemm(world, peaks))
     return rows
+
+
+def run_dispatch(args):
+    """Every kernel family that can serve each decode and small-batch shape, timed alone (cold L2,
+    median of replays), next to the family w4_gemm picks: the measurement behind the dispatch."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    l2 = getattr(torch.cuda.get_device_properties(torch.cuda.current_device()), "L2_cache_size", 126 * 2 ** 20)
+    flush = L2Flush(l2)
+    peaks = load_peaks()
+    names = {B.VARIANT_GEMV: "gemv", B.VARIANT_SKINNY: "skinny", B.VARIANT_TC: "tc"}
+    shapes = decode_cases()[0] + small_batch_cases()[0]
+    table = []
+    for (M, K, N) in shapes:
+        X, W = synth.layer_case(3, M, K, N)
+        Xd = torch.from_numpy(X).cuda()
+        p, sc, z = B.w4_quantize_pack(torch.from_numpy(W).cuda())
+        layer_w = N * K // 2 + N * (K // 128) * 3
+        n = max(8, min(64, int(np.ceil(3 * l2 / layer_w)) + 1))
+        copies = [(p, sc, z)] + [(p.clone(), sc.clone(), z.clone()) for _ in range(n - 1)]
+        Y = torch.empty((M, N), dtype=torch.float16, device="cuda")
+        row = {"M": M, "K": K, "N": N, "auto": names.get(B.w4_gemm_plan(M, N, K, 128, 0, sc, z)[0])}
+        for fam in (B.VARIANT_GEMV, B.VARIANT_SKINNY, B.VARIANT_TC):
+            try:
+                B.w4_gemm_plan(M, N, K, 128, fam, sc, z)
+            except B.W4Error:
+                row[names[fam]] = None
+                continue
+            var = fam | B.FLAG_WEIGHTS_STATIC
+
+            def step(i, var=var):
+                pp, ss, zz = copies[i % n]
+                B.w4_gemm(Xd, pp, ss, zz, out=Y, variant=var)
+            step(0)
+            torch.cuda.synchronize()
+            g = capture(step, n, 0)
+            g.replay()
+            t = time_graph_median(g, 1, 3, flush)[0] / n
+            row[names[fam]] = {"us": round(t * 1e3, 3),
+                               "hbm_frac": round(gemm_bytes(M, K, N) / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+            del g
+        timed = {k: v["us"] for k, v in row.items() if isinstance(v, dict)}
+        row["fastest"] = min(timed, key=timed.get) if timed else None
+        table.append(row)
+        del copies, Xd, Y
+        torch.cuda.empty_cache()
+    return {"workload": "dispatch table: decode and small-batch shapes x kernel family", "table": table,
+            "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]}
 
 
 def run_reference(args, rank, world):
@@ -786,7 +865,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "small_batch", "prefill"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "small_batch", "prefill", "dispatch"])
     ap.add_argument("--replays", type=int, default=20,
                     help="graph replays of the K timed steps; the median is reported (>= 20 by default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -800,6 +879,8 @@ def main():
     rank, world, local = dist_setup(args)
     if args.impl == "reference":
         out = run_reference(args, rank, world)
+    elif args.workload == "dispatch":
+        out = run_dispatch(args) if rank == 0 else None
     else:
         out = run_gemm_bench(args, rank, world, local, args.workload)
     if rank == 0 and out is not None:

@@ -153,6 +153,22 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
                      void* ws, size_t ws_bytes, int variant, void* stream);
 
 /*
+ * w4_gemm_plan -- which kernel family a w4_gemm_ex call with these arguments runs, and how many
+ * kernel launches it makes.  Nothing is enqueued and no device is touched beyond the cached
+ * per-device attributes; the decision is the one w4_gemm_ex takes (the same code).
+ *   variant: as for w4_gemm_ex.  scales / zeros: the metadata pointers the call will receive (the
+ *   GEMV family needs both 16-byte aligned), or NULL to assume aligned ones.
+ *   family_out: W4_VARIANT_GEMV, W4_VARIANT_SKINNY, W4_VARIANT_TC or W4_VARIANT_GEMV_TC (host int);
+ *   W4_VARIANT_AUTO with launches_out = 0 when the call launches no kernel (M, N or K zero).
+ *   launches_out: kernel launches of the call (host int).
+ * Errors: those w4_gemm_ex would return for the shape and variant (W4_ERR_SHAPE when an explicit
+ * family cannot serve the shape, W4_ERR_ALIGN for misaligned metadata with the explicit GEMV).
+ * The pages have no counterpart to this query; it lets a caller account for the launches.
+ */
+w4_status w4_gemm_plan(int64_t M, int64_t N, int64_t K, int group, int variant, const void* scales,
+                       const void* zeros, int* family_out, int* launches_out);
+
+/*
  * w4_gemm_host -- w4_gemm with X and Y in host memory.
  *
  * Enqueues on `stream`: one copy of X_host [M, K] into the caller's device buffer x_dev, the
@@ -167,6 +183,39 @@ w4_status w4_gemm_host(const uint16_t* X_host, int64_t M, int64_t N, int64_t K, 
                        const uint16_t* scales, const uint8_t* zeros, int group, uint16_t* Y_host,
                        uint16_t* x_dev, uint16_t* y_dev, void* ws, size_t ws_bytes, int variant,
                        void* stream);
+
+/*
+ * w4_gemm_host_batch -- several w4_gemm layers with their activations and results in host memory,
+ * moved with one copy each way.
+ *
+ * Enqueues on `stream`: one copy of x_bytes from x_host into the caller's device buffer x_dev,
+ * then for every layer i in order the GEMM of w4_gemm_ex (same `variant`) reading X_i at x_dev +
+ * layers[i].x_offset and writing Y_i at y_dev + layers[i].y_offset, then one copy of y_bytes from
+ * y_dev into y_host.  Returns once enqueued; y_host holds every layer's result when the stream has
+ * drained.
+ *   layers[i].M, N, K: the layer's shape; packed/scales/zeros: its device weights (as for w4_gemm).
+ *   x_offset / y_offset: byte offsets, multiples of 16; X_i [M, K] fp16 must lie inside [0, x_bytes)
+ *   and Y_i [M, N] fp16 inside [0, y_bytes).
+ *   x_host, y_host: host buffers (pinned for asynchronous copies); x_dev, y_dev: 16-byte aligned
+ *   device buffers the caller owns.  x_bytes may be 0 (no input copy).
+ *   ws: device workspace of at least the largest w4_gemm_workspace_size of the layers.
+ * Every layer is validated before anything is enqueued; errors as w4_gemm_ex (W4_ERR_SHAPE also for
+ * a region outside its buffer or n_layers < 1, W4_ERR_ALIGN for an offset that is not a multiple
+ * of 16), plus W4_ERR_CUDA if a copy cannot be enqueued.
+ * The pages have no counterpart to this call; it exists so that a decode step pays for two copies
+ * instead of two per layer.
+ */
+typedef struct {
+    int64_t M, N, K;
+    const uint32_t* packed;
+    const uint16_t* scales;
+    const uint8_t* zeros;
+    int64_t x_offset;
+    int64_t y_offset;
+} w4_gemm_layer;
+w4_status w4_gemm_host_batch(const w4_gemm_layer* layers, int n_layers, int group, const void* x_host,
+                             void* x_dev, size_t x_bytes, void* y_host, void* y_dev, size_t y_bytes, void* ws,
+                             size_t ws_bytes, int variant, void* stream);
 
 /* Bytes of device workspace awq_scale_search needs for this problem. */
 w4_status awq_workspace_size(int64_t T, int64_t N, int64_t K, int group, int n_alpha,

@@ -222,3 +222,50 @@ def test_row_split_calls_reject(L):
     assert L.awq_sse(d, 100, d, 64, 512, 128, 20, None, d, d, 1 << 30, None) == 1
     assert L.awq_select(d, 0, 20, 100, 64, d, 512, d, d, d, None) == 2
     assert L.awq_select(d, 2, 0, 100, 64, d, 512, d, d, d, None) == 4
+
+
+def _layers(specs):
+    arr = (B.GemmLayer * max(1, len(specs)))()
+    for i, (M, N, K, xo, yo) in enumerate(specs):
+        arr[i] = B.GemmLayer(M, N, K, GOOD.value, GOOD.value, GOOD.value, xo, yo)
+    return ctypes.cast(arr, P), arr
+
+
+def test_host_batch_rejects_before_enqueuing(L):
+    """w4_gemm_host_batch validates every layer first (CPU only: the pointers are never used)."""
+    f = L.w4_gemm_host_batch
+    ok = [(1, 4096, 4096, 0, 0), (1, 12288, 4096, 8192, 8192)]
+    xb, yb = 8192 * 2, 8192 + 2 * 12288
+
+    def call(specs, n=None, x_bytes=xb, y_bytes=yb, xdev=GOOD, ydev=GOOD, group=128, variant=0):
+        p, keep = _layers(specs)
+        return f(p, len(specs) if n is None else n, group, GOOD, xdev, x_bytes, GOOD, ydev, y_bytes, None, 0,
+                 variant, None)
+
+    assert call(ok, n=0) == 2                                        # no layer: W4_ERR_SHAPE
+    assert call(ok, group=64) == 4                                   # W4_ERR_UNSUPPORTED
+    assert call(ok, variant=77) == 4
+    assert call([(1, 4096, 4096, 8, 0)]) == 3                        # x_offset not a multiple of 16
+    assert call([(1, 4096, 4096, 0, 0), (1, 12288, 4096, 8208, 8192)]) == 2  # second X beyond x_bytes
+    assert call(ok, x_bytes=xb - 16) == 2                            # X region outside the buffer
+    assert call(ok, y_bytes=yb - 16) == 2                            # Y region outside the buffer
+    assert call([(1, 4100, 4096, 0, 0)]) == 2                        # N % 8 != 0
+    assert call(ok, xdev=BAD_ALIGN) == 3
+    assert call(ok, ydev=P(0)) == 1                                  # W4_ERR_NULL
+    assert f(None, 1, 128, GOOD, GOOD, xb, GOOD, GOOD, yb, None, 0, 0, None) == 1
+
+
+def test_gemm_plan_query(L):
+    """The dispatch query (CPU: no device work) agrees with the documented rule."""
+    assert B.w4_gemm_plan(1, 4096, 4096) == (B.VARIANT_GEMV, 1)
+    assert B.w4_gemm_plan(16, 8192, 8192) == (B.VARIANT_GEMV, 2)
+    assert B.w4_gemm_plan(32, 8192, 8192) == (B.VARIANT_GEMV, 4)
+    assert B.w4_gemm_plan(4, 8192, 28672) == (B.VARIANT_SKINNY, 1)  # 4 staged rows of K = 28672 do not fit
+    assert B.w4_gemm_plan(33, 4096, 4096) == (B.VARIANT_TC, 1)
+    assert B.w4_gemm_plan(0, 4096, 4096) == (B.VARIANT_AUTO, 0)
+    assert B.w4_gemm_plan(64, 4096, 4096, variant=B.VARIANT_SKINNY) == (B.VARIANT_SKINNY, 2)
+    fam, n = ctypes.c_int(0), ctypes.c_int(0)
+    assert L.w4_gemm_plan(1, 4096, 4096, 128, B.VARIANT_GEMV, BAD_ALIGN, GOOD, ctypes.byref(fam),
+                          ctypes.byref(n)) == 3  # explicit GEMV with misaligned scales: W4_ERR_ALIGN
+    assert L.w4_gemm_plan(1, 4096, 4096, 128, 0, BAD_ALIGN, GOOD, ctypes.byref(fam), ctypes.byref(n)) == 0
+    assert (fam.value, n.value) == (B.VARIANT_SKINNY, 1)  # AUTO falls back to the skinny kernel

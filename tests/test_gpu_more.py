@@ -50,3 +50,25 @@ def test_prepared_host_call_matches_w4_gemm():
     ref2 = B.w4_gemm(torch.from_numpy(X[:, ::-1].copy()).cuda(), p, s, z).cpu()
     assert torch.equal(out, ref2)
     assert B.w4_check_device_status() == 0
+
+
+def test_host_batch_matches_per_layer_gemm():
+    """w4_gemm_host_batch (one copy in, the layers' GEMMs, one copy out) gives every layer the bits
+    w4_gemm gives it, twice in a row with new inputs in the same buffers."""
+    shapes = [(1, 4096, 4096), (1, 4096, 12288), (5, 1152, 520), (1, 11008, 4096), (40, 512, 264)]
+    weights, Xs = [], []
+    for i, (M, K, N) in enumerate(shapes):
+        X, W = synth.layer_case(46 + i, M, K, N)
+        weights.append(B.w4_quantize_pack(torch.from_numpy(W).cuda()))
+        Xs.append(X)
+    batch = B.HostGemmBatch(weights, shapes)
+    for rep in range(2):
+        for i, X in enumerate(Xs):
+            batch.x(i).copy_(torch.from_numpy(X if rep == 0 else X[:, ::-1].copy()))
+        batch.run()
+        torch.cuda.current_stream().synchronize()
+        for i, X in enumerate(Xs):
+            Xi = X if rep == 0 else X[:, ::-1].copy()
+            ref = B.w4_gemm(torch.from_numpy(Xi).cuda(), *weights[i]).cpu()
+            assert torch.equal(batch.y(i), ref), (rep, shapes[i])
+    assert B.w4_check_device_status() == 0

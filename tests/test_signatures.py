@@ -33,6 +33,8 @@ def _expected(param):
         return SCALARS[base]
     if base == "size_t":
         return ctypes.POINTER(ctypes.c_size_t)
+    if base == "int":  # host int outputs of the queries
+        return ctypes.POINTER(ctypes.c_int)
     return ctypes.c_void_p
 
 

@@ -57,6 +57,47 @@ int* device_status_ptr() {
     return g_status_ptr[dev];
 }
 
+// The kernel family and number of launches of one w4_gemm_ex call (shape already validated).
+// AUTO: the tensor-core GEMM above 32 activation rows; up to 32 rows the TMA-fed GEMV in
+// launches of up to 8 rows where 8 staged activation rows fit its shared memory and the metadata
+// is 16-byte aligned (it bulk-copies scales and zero points), else the skinny kernel in launches
+// of up to 32 rows; from 17 rows on, the tensor-core GEMM instead when its 128-row W tiles alone
+// fill the SMs.  Measured per shape on B200 (bench.py --workload dispatch, cold L2): decode M = 1
+// GEMV 4.6 / 9.5 / 8.6 / 8.7 us vs skinny 6.2 / 19.6 / 18.9 / 14.3; at K = 8192 two and four
+// 8-row GEMV launches beat one skinny launch at M = 16 and 32 (32.6 vs 46.9, 63.4 vs 69.0 us at
+// N = 8192); at M = 32, N = 28672 the tensor-core GEMM (89.4 us) beats four GEMV launches (156.1)
+// and at M = 16 it does not (88.8 vs 79.0); at K = 28672 (8 rows of X do not fit the GEMV) the
+// skinny kernel beats or ties the tensor-core GEMM at every M.
+w4_status gemm_plan(int64_t M, int64_t N, int64_t K, int family, bool meta_aligned, int* chosen, int* launches) {
+    const bool tc_fills = (N + 127) / 128 >= device_sm_count();
+    if (family == W4_VARIANT_TC || (family == W4_VARIANT_AUTO && (M > 32 || (M > 16 && K <= 8192 && tc_fills)))) {
+        *chosen = W4_VARIANT_TC;
+        *launches = 1;
+        return W4_OK;
+    }
+    if (family == W4_VARIANT_GEMV_TC) {
+        GemvTcPlan gtp;
+        if (!plan_gemv_tc(M < 8 ? M : 8, N, K, &gtp)) return W4_ERR_SHAPE;
+        *chosen = W4_VARIANT_GEMV_TC;
+        *launches = (int)((M + 7) / 8);
+        return W4_OK;
+    }
+    DecodePlan dplan;
+    const bool gemv_fits = plan_decode_stream(M < 8 ? M : 8, N, K, &dplan);
+    if (family == W4_VARIANT_GEMV && !gemv_fits) return W4_ERR_SHAPE;
+    if (family == W4_VARIANT_GEMV && !meta_aligned) return W4_ERR_ALIGN;
+    if (family == W4_VARIANT_GEMV || (family == W4_VARIANT_AUTO && M <= 32 && gemv_fits && meta_aligned)) {
+        *chosen = W4_VARIANT_GEMV;
+        *launches = (int)((M + 7) / 8);
+        return W4_OK;
+    }
+    SkinnyPlan plan;
+    if (!plan_skinny(M < 32 ? M : 32, N, K, &plan)) return W4_ERR_SHAPE;
+    *chosen = W4_VARIANT_SKINNY;
+    *launches = (int)((M + 31) / 32);
+    return W4_OK;
+}
+
 }  // namespace w4
 
 using namespace w4;
@@ -113,14 +154,16 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     int* status = device_status_ptr();
     if (!status) return W4_ERR_CUDA;
 
-    const bool use_tc = family == W4_VARIANT_TC || (family == W4_VARIANT_AUTO && M > 32);
-    if (use_tc) {
+    int chosen = 0, launches = 0;
+    st = gemm_plan(M, N, K, family, aligned16(scales) && aligned16(zeros), &chosen, &launches);
+    if (st != W4_OK) return st;
+    if (chosen == W4_VARIANT_TC) {
         return launch_tc_w4(X, M, N, K, packed, scales, zeros, Y, status, s) == cudaSuccess ? W4_OK
                                                                                             : W4_ERR_CUDA;
     }
-    GemvTcPlan gtp;
-    if (family == W4_VARIANT_GEMV_TC && !plan_gemv_tc(M < 8 ? M : 8, N, K, &gtp)) return W4_ERR_SHAPE;
-    if (family == W4_VARIANT_GEMV_TC) {  // chosen explicitly only: slower than the mma.sync GEMV so far
+    if (chosen == W4_VARIANT_GEMV_TC) {  // chosen explicitly only: slower than the mma.sync GEMV so far
+        GemvTcPlan gtp;
+        if (!plan_gemv_tc(M < 8 ? M : 8, N, K, &gtp)) return W4_ERR_SHAPE;
         for (int64_t m0 = 0; m0 < M; m0 += 8) {  // up to 8 activation rows per launch
             const int64_t mc = (M - m0) < 8 ? (M - m0) : 8;
             cudaError_t e = launch_gemv_tc(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N, gtp,
@@ -129,23 +172,12 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
         }
         return W4_OK;
     }
-    const int64_t gemv_rows = M < 8 ? M : 8;
-    DecodePlan dplan;
-    const bool gemv_fits = plan_decode_stream(gemv_rows, N, K, &dplan);
-    const bool meta_aligned = aligned16(scales) && aligned16(zeros);  // the GEMV bulk-copies metadata
-    if (family == W4_VARIANT_GEMV && !gemv_fits) return W4_ERR_SHAPE;
-    if (family == W4_VARIANT_GEMV && !meta_aligned) return W4_ERR_ALIGN;
-    // AUTO takes the GEMV up to 32 rows, as ceil(M / 8) launches of at most 8 rows each: measured
-    // at K = 8192, two M = 8 launches (2 x 16.7 us at N = 8192, 2 x 40.6 us at N = 28672) beat
-    // one skinny launch at M = 16 (44.9 / 126.6 us) and four tie with it at M = 32 (66.6 vs 67.0,
-    // 162.6 vs 168.8 us), before any L2 reuse of the weights between the launches.  The skinny
-    // kernel keeps the shapes whose 8 activation rows do not fit the GEMV's shared memory.
-    if (family == W4_VARIANT_GEMV || (family == W4_VARIANT_AUTO && M <= 32 && gemv_fits && meta_aligned)) {
+    if (chosen == W4_VARIANT_GEMV) {
         // up to 8 activation rows per launch (token-by-token decode has M == 1)
         for (int64_t m0 = 0; m0 < M; m0 += 8) {
             const int64_t mc = (M - m0) < 8 ? (M - m0) : 8;
             cudaError_t e = launch_decode_stream(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N,
-                                               weights_static, status, s);
+                                                 weights_static, status, s);
             if (e != cudaSuccess) return W4_ERR_CUDA;
         }
         return W4_OK;
@@ -160,6 +192,23 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
         if (e != cudaSuccess) return W4_ERR_CUDA;
     }
     return W4_OK;
+}
+
+w4_status w4_gemm_plan(int64_t M, int64_t N, int64_t K, int group, int variant, const void* scales,
+                       const void* zeros, int* family_out, int* launches_out) {
+    if (!family_out || !launches_out) return W4_ERR_NULL;
+    if (group != 128) return W4_ERR_UNSUPPORTED;
+    const int family = variant & ~W4_FLAG_WEIGHTS_STATIC;
+    if (family < W4_VARIANT_AUTO || family > W4_VARIANT_GEMV_TC) return W4_ERR_UNSUPPORTED;
+    if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0)
+        return W4_ERR_SHAPE;
+    if (M == 0 || N == 0 || K == 0) {  // no kernel (K == 0: one memset of Y)
+        *family_out = W4_VARIANT_AUTO;
+        *launches_out = 0;
+        return W4_OK;
+    }
+    const bool meta_aligned = (!scales || aligned16(scales)) && (!zeros || aligned16(zeros));
+    return gemm_plan(M, N, K, family, meta_aligned, family_out, launches_out);
 }
 
 w4_status w4_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
@@ -183,6 +232,54 @@ w4_status w4_gemm_host(const uint16_t* X_host, int64_t M, int64_t N, int64_t K, 
     const w4_status st = w4_gemm_ex(x_dev, M, N, K, packed, scales, zeros, group, y_dev, ws, ws_bytes, variant, stream);
     if (st != W4_OK) return st;
     if (cudaMemcpyAsync(Y_host, y_dev, (size_t)M * (size_t)N * 2, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return W4_ERR_CUDA;
+    return W4_OK;
+}
+
+w4_status w4_gemm_host_batch(const w4_gemm_layer* layers, int n_layers, int group, const void* x_host, void* x_dev,
+                             size_t x_bytes, void* y_host, void* y_dev, size_t y_bytes, void* ws, size_t ws_bytes,
+                             int variant, void* stream) {
+    if (group != 128) return W4_ERR_UNSUPPORTED;
+    const int family = variant & ~W4_FLAG_WEIGHTS_STATIC;
+    if (family < W4_VARIANT_AUTO || family > W4_VARIANT_GEMV_TC) return W4_ERR_UNSUPPORTED;
+    if (!layers || n_layers < 1) return n_layers < 1 ? W4_ERR_SHAPE : W4_ERR_NULL;
+    if ((x_bytes > 0 && (!x_host || !x_dev)) || !y_host || !y_dev) return W4_ERR_NULL;
+    if ((x_dev && !aligned16(x_dev)) || !aligned16(y_dev)) return W4_ERR_ALIGN;
+    // validate every layer before anything is enqueued
+    for (int i = 0; i < n_layers; ++i) {
+        const w4_gemm_layer& L = layers[i];
+        const int64_t M = L.M, N = L.N, K = L.K;
+        if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0)
+            return W4_ERR_SHAPE;
+        if (L.x_offset < 0 || L.y_offset < 0) return W4_ERR_SHAPE;
+        if ((L.x_offset & 15) || (L.y_offset & 15)) return W4_ERR_ALIGN;
+        if ((uint64_t)L.y_offset + (uint64_t)(M * N * 2) > (uint64_t)y_bytes) return W4_ERR_SHAPE;
+        if (M == 0 || N == 0 || K == 0) continue;
+        if ((uint64_t)L.x_offset + (uint64_t)(M * K * 2) > (uint64_t)x_bytes || !x_dev) return W4_ERR_SHAPE;
+        if (!L.packed || !L.scales || !L.zeros) return W4_ERR_NULL;
+        if (!aligned16(L.packed)) return W4_ERR_ALIGN;
+        size_t need = 0;
+        w4_status st = w4_gemm_workspace_size(M, N, K, group, &need);
+        if (st != W4_OK) return st;
+        if (ws_bytes < need) return W4_ERR_WORKSPACE;
+        if (need > 0 && !ws) return W4_ERR_NULL;
+        int chosen = 0, launches = 0;
+        st = gemm_plan(M, N, K, family, aligned16(L.scales) && aligned16(L.zeros), &chosen, &launches);
+        if (st != W4_OK) return st;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    if (x_bytes > 0 && cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return W4_ERR_CUDA;
+    for (int i = 0; i < n_layers; ++i) {
+        const w4_gemm_layer& L = layers[i];
+        const w4_status st =
+            w4_gemm_ex(reinterpret_cast<const uint16_t*>(static_cast<const char*>(x_dev) + L.x_offset), L.M, L.N,
+                       L.K, L.packed, L.scales, L.zeros, group,
+                       reinterpret_cast<uint16_t*>(static_cast<char*>(y_dev) + L.y_offset), ws, ws_bytes, variant,
+                       stream);
+        if (st != W4_OK) return st;
+    }
+    if (y_bytes > 0 && cudaMemcpyAsync(y_host, y_dev, y_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return W4_ERR_CUDA;
     return W4_OK;
 }

@@ -30,6 +30,9 @@ SIGNATURES = {
     "w4_gemm": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ, _P]),
     "w4_gemm_ex": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P, _P, _SZ, _I32, _P]),
     "w4_gemm_host": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P, _I32, _P, _P, _P, _P, _SZ, _I32, _P]),
+    "w4_gemm_host_batch": (_I32, [_P, _I32, _I32, _P, _P, _SZ, _P, _P, _SZ, _P, _SZ, _I32, _P]),
+    "w4_gemm_plan": (_I32, [_I64, _I64, _I64, _I32, _I32, _P, _P, ctypes.POINTER(ctypes.c_int),
+                            ctypes.POINTER(ctypes.c_int)]),
     "awq_workspace_size": (_I32, [_I64, _I64, _I64, _I32, _I32, ctypes.POINTER(_SZ)]),
     "awq_scale_search": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P, _SZ, _P]),
     "awq_scale_search_noalloc": (_I32, [_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P, _P]),
@@ -123,6 +126,17 @@ def w4_gemm_workspace_size(M: int, N: int, K: int, group: int = 128) -> int:
     n = ctypes.c_size_t(0)
     _check(lib().w4_gemm_workspace_size(M, N, K, group, ctypes.byref(n)), "w4_gemm_workspace_size")
     return n.value
+
+
+def w4_gemm_plan(M: int, N: int, K: int, group: int = 128, variant: int = VARIANT_AUTO, scales=None,
+                 zeros=None) -> tuple[int, int]:
+    """(kernel family, kernel launches) of a w4_gemm call with these arguments (no device work).
+    scales / zeros: the metadata tensors the call will use (their alignment matters), or None."""
+    fam, n = ctypes.c_int(0), ctypes.c_int(0)
+    sp = ctypes.c_void_p(scales.data_ptr()) if scales is not None else None
+    zp = ctypes.c_void_p(zeros.data_ptr()) if zeros is not None else None
+    _check(lib().w4_gemm_plan(M, N, K, group, variant, sp, zp, ctypes.byref(fam), ctypes.byref(n)), "w4_gemm_plan")
+    return fam.value, n.value
 
 
 def w4_gemm(X: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
@@ -236,6 +250,75 @@ class HostGemmCall:
         if st != W4_OK:
             raise W4Error(st, "w4_gemm_host")
         return self.out_host
+
+
+class GemmLayer(ctypes.Structure):
+    """One layer of w4_gemm_host_batch (the C struct w4_gemm_layer)."""
+    _fields_ = [("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("packed", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("zeros", ctypes.c_void_p),
+                ("x_offset", ctypes.c_int64), ("y_offset", ctypes.c_int64)]
+
+
+def _align16(n: int) -> int:
+    return (n + 15) // 16 * 16
+
+
+class HostGemmBatch:
+    """w4_gemm_host_batch over fixed buffers: every layer's X is packed into one pinned host buffer
+    (x_host, 16-byte aligned regions in layer order) and every Y into another (y_host); run() makes
+    the one C call: one host-to-device copy, the layers' GEMMs, one device-to-host copy, enqueued
+    on the stream chosen at construction, no synchronisation.
+
+    weights: [(packed, scales, zeros)] device tensors per layer; shapes: [(M, K, N)] per layer.
+    x(i) / y(i) are views of layer i's input and result inside the host buffers."""
+
+    def __init__(self, weights, shapes, group: int = 128, workspace: torch.Tensor | None = None,
+                 variant: int = VARIANT_AUTO, stream=None):
+        if len(weights) != len(shapes) or not shapes:
+            raise ValueError("one (packed, scales, zeros) per layer shape")
+        self.shapes = [tuple(int(v) for v in sh) for sh in shapes]
+        self.x_off, self.y_off, xo, yo = [], [], 0, 0
+        for (M, K, N) in self.shapes:
+            self.x_off.append(xo)
+            self.y_off.append(yo)
+            xo += _align16(2 * M * K)
+            yo += _align16(2 * M * N)
+        self.x_bytes, self.y_bytes = xo, yo
+        self.x_host = torch.empty(max(xo, 16), dtype=torch.uint8).pin_memory()
+        self.y_host = torch.empty(max(yo, 16), dtype=torch.uint8).pin_memory()
+        self.x_dev = torch.empty(max(xo, 16), dtype=torch.uint8, device="cuda")
+        self.y_dev = torch.empty(max(yo, 16), dtype=torch.uint8, device="cuda")
+        arr = (GemmLayer * len(self.shapes))()
+        for i, ((p, sc, z), (M, K, N)) in enumerate(zip(weights, self.shapes)):
+            if tuple(p.shape) != (N, K // 8) or tuple(sc.shape) != (N, K // group):
+                raise ValueError(f"layer {i}: weights do not match shape (M={M}, K={K}, N={N})")
+            arr[i] = GemmLayer(M, N, K, _dev(p, torch.int32, "packed").value, _dev(sc, torch.float16, "scales").value,
+                               _dev(z, torch.uint8, "zeros").value, self.x_off[i], self.y_off[i])
+        need = max(_ws_size(M, N, K, group) for (M, K, N) in self.shapes)
+        if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+            raise ValueError("workspace too small: see w4_gemm_workspace_size")
+        ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
+        ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+        self._fn = lib().w4_gemm_host_batch
+        self._args = (ctypes.cast(arr, ctypes.c_void_p), ctypes.c_int32(len(self.shapes)), ctypes.c_int32(group),
+                      ctypes.c_void_p(self.x_host.data_ptr()), ctypes.c_void_p(self.x_dev.data_ptr()),
+                      ctypes.c_size_t(self.x_bytes), ctypes.c_void_p(self.y_host.data_ptr()),
+                      ctypes.c_void_p(self.y_dev.data_ptr()), ctypes.c_size_t(self.y_bytes), ws_ptr,
+                      ctypes.c_size_t(ws_bytes), ctypes.c_int32(variant), _stream(stream))
+        self._keep = (arr, weights, workspace)
+
+    def x(self, i: int) -> torch.Tensor:
+        M, K, _ = self.shapes[i]
+        return self.x_host[self.x_off[i]:self.x_off[i] + 2 * M * K].view(torch.float16).view(M, K)
+
+    def y(self, i: int) -> torch.Tensor:
+        M, _, N = self.shapes[i]
+        return self.y_host[self.y_off[i]:self.y_off[i] + 2 * M * N].view(torch.float16).view(M, N)
+
+    def run(self):
+        st = self._fn(*self._args)
+        if st != W4_OK:
+            raise W4Error(st, "w4_gemm_host_batch")
 
 
 _ws_cache: dict = {}
