@@ -832,6 +832,46 @@ def run_dispatch(args):
             "peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": peaks["source"]}
 
 
+def run_profile_case(args):
+    """A short, self-checking run for ncu captures (no timing): the workload's layers with one
+    weight copy each (ncu flushes the caches between its passes), `args.profile_only` steps, then
+    the device status.  Workloads: decode, small_batch, prefill (w4_gemm per layer), awq / awq_gram
+    (the scale search on the calibration layer's 16384-row subsample), quantize (w4_quantize_pack of
+    the decode layers' weights), awq_clip (the clip search, 10 ratios, on the same subsample)."""
+    import torch
+    from weight_only_int4_06_b200 import w4a16 as B
+    steps = max(1, args.profile_only)
+    kind = args.workload
+    if kind in ("awq", "awq_gram", "awq_clip"):
+        X, W = synth.awq_case()
+        Xd = torch.from_numpy(X[:16384].copy()).cuda()
+        Wd = torch.from_numpy(W).cuda()
+        for _ in range(steps):
+            if kind == "awq_clip":
+                B.awq_clip_search(Xd, Wd, None, 10)
+            else:
+                (B.awq_scale_search if kind == "awq" else B.awq_scale_search_gram)(Xd, Wd, 20)
+    elif kind == "quantize":
+        Ws = [torch.from_numpy(synth.layer_case(2, 1, K, N)[1]).cuda() for (K, N) in synth.DECODE_7B_SHAPES]
+        for _ in range(steps):
+            for Wd in Ws:
+                B.w4_quantize_pack(Wd)
+    else:
+        cases, case_id, _ = {"decode": decode_cases, "small_batch": small_batch_cases,
+                             "prefill": prefill_cases}[kind]()
+        layers = []
+        for (M, K, N) in cases:
+            X, W = synth.layer_case(case_id, M, K, N)
+            layers.append((torch.from_numpy(X).cuda(), *B.w4_quantize_pack(torch.from_numpy(W).cuda())))
+        for _ in range(steps):
+            for (Xd, p, sc, z) in layers:
+                B.w4_gemm(Xd, p, sc, z, variant=B.FLAG_WEIGHTS_STATIC)
+    torch.cuda.synchronize()
+    st = B.w4_check_device_status()
+    assert st == 0, B.STATUS_NAMES.get(st, st)
+    return {"profile_case": kind, "steps": steps, "status": "ok"}
+
+
 def run_reference(args, rank, world):
     """The reference arm: the CPU oracle timed on a bounded sample of the same workload."""
     if rank != 0:
@@ -865,7 +905,11 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "small_batch", "prefill", "dispatch"])
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "small_batch", "prefill", "dispatch", "awq", "awq_gram", "awq_clip",
+                             "quantize"])
+    ap.add_argument("--profile-only", type=int, default=0, metavar="S",
+                    help="run S untimed steps of the workload for an ncu capture, check the status, exit")
     ap.add_argument("--replays", type=int, default=20,
                     help="graph replays of the K timed steps; the median is reported (>= 20 by default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -879,8 +923,12 @@ def main():
     rank, world, local = dist_setup(args)
     if args.impl == "reference":
         out = run_reference(args, rank, world)
+    elif args.profile_only:
+        out = run_profile_case(args) if rank == 0 else None
     elif args.workload == "dispatch":
         out = run_dispatch(args) if rank == 0 else None
+    elif args.workload in ("awq", "awq_gram", "awq_clip", "quantize"):
+        raise SystemExit(f"--workload {args.workload} is a profiling case only: add --profile-only S")
     else:
         out = run_gemm_bench(args, rank, world, local, args.workload)
     if rank == 0 and out is not None:
