@@ -247,7 +247,7 @@ class GemmWorkload:
         self.flops_per_step = sum(2 * M * K * N for (M, K, N) in cases)
         self.launches_per_step = sum(gemm_launches(M, K, N, variant, L["copies"][0][1], L["copies"][0][2])
                                      for (M, K, N), L in zip(cases, self.layers))
-        self.host_calls = None  # prepared w4_gemm_host calls, built on first use
+        self.host_calls = None  # prepared w4_gemm_host_batch calls, built on first use
         self.host_path_note = None
 
     def run_step(self, step, only=None):
@@ -279,7 +279,8 @@ class GemmWorkload:
                 self.host_calls = []
                 self.host_path_note = f"batched call unavailable ({type(e).__name__}: {e}); per-layer w4_gemm_host"
         if self.host_calls:
-            b = self.host_calls[step % self.n_sets]
+            c = step % self.n_sets
+            b = self.host_calls[c]
             b.run()
             torch.cuda.current_stream().synchronize()
             return [b.y(i) for i in range(len(self.layers))]
@@ -610,13 +611,18 @@ def bench_awq_gram(world, peaks, case, reps=3):
     t = _time_awq_search(world, B.awq_scale_search_gram, Xd, Wd, ws, reps)
     flops = 2 * T * K * K + 20 * 2 * N * K * K  # Gram + one quadratic-form GEMM per alpha
     tf = flops / (t * 1e-3) / 1e12
+    # executed: G is formed as its 256 x 256 tiles on and below the diagonal
+    nt = (K + 255) // 256
+    executed = 2 * T * K * K * (nt * (nt + 1) // 2) / (nt * nt) + 20 * 2 * N * K * K
+    tf_exec = executed / (t * 1e-3) / 1e12
     del Xd, Wd, ws
     torch.cuda.empty_cache()
-    return {"kernel": "transpose + 16 x (tc_gemm_kernel<f32 out> + fp64 add) + scale + "
+    return {"kernel": "transpose + 16 x (tc_gemm_kernel<f32 out, lower-triangle tiles> + fp64 add) + scale + "
                       "20 x (fakequant + tc_gemm_kernel<quadratic form>) + finalize",
             "T": T, "K": K, "N": N, "n_alpha": 20, "ms": round(t, 3), "TFLOPs": round(tf, 1),
             "bound": "tensor", "tensor_frac_sustained": round(tf / peaks["bf16_tflops_sustained"], 3),
-            "flops": flops}
+            "flops": flops, "flops_executed": int(executed),
+            "tensor_frac_sustained_executed": round(tf_exec / peaks["bf16_tflops_sustained"], 3)}
 
 
 def bench_gptq(world, peaks, reps=2):

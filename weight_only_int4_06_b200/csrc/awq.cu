@@ -397,10 +397,16 @@ __global__ void __launch_bounds__(256) transpose_pad_kernel(const unsigned short
         if (t < Tp) XT[(c * K + k0 + r) * L + tt] = tile[threadIdx.x][r];
 }
 
-// G64 = Gc (first chunk) or G64 += Gc, elementwise in fp64.
-__global__ void gram_accumulate_kernel(const float* __restrict__ Gc, int64_t n, bool first, double* __restrict__ G64) {
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
-        G64[e] = first ? (double)Gc[e] : G64[e] + (double)Gc[e];
+// G64 = Gc (first chunk) or G64 += Gc in fp64, on and below the diagonal (row i, columns j <= i;
+// lower = 0: every entry).  One block row of the grid per row of G.
+__global__ void gram_accumulate_kernel(const float* __restrict__ Gc, int K, bool first, int lower,
+                                       double* __restrict__ G64) {
+    for (int i = blockIdx.x; i < K; i += gridDim.x) {
+        const int jn = lower ? i + 1 : K;
+        const int64_t r = (int64_t)i * K;
+        for (int j = threadIdx.x; j < jn; j += blockDim.x)
+            G64[r + j] = first ? (double)Gc[r + j] : G64[r + j] + (double)Gc[r + j];
+    }
 }
 
 // d_k = sqrt(G_kk) (1 when G_kk is 0) and rd = 1 / d, from the fp64 G rounded once to fp32.
@@ -413,13 +419,15 @@ __global__ void gram_diag_kernel(const double* __restrict__ G64, int K, float* _
     rd[k] = __frcp_rn(dk);
 }
 
-// G' = D^-1 G D^-1 in fp16.
-__global__ void gram_scale_kernel(const double* __restrict__ G64, const float* __restrict__ rd, int K,
+// G' = D^-1 G D^-1 in fp16, every entry; with `lower` only G's lower triangle holds values and
+// entry (i, j) above the diagonal is read as its mirror (j, i), which makes G' exactly symmetric.
+__global__ void gram_scale_kernel(const double* __restrict__ G64, const float* __restrict__ rd, int K, int lower,
                                   __half* __restrict__ Gp) {
     const int64_t n = (int64_t)K * K;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x) {
         const int i = (int)(e / K), j = (int)(e - (int64_t)i * K);
-        Gp[e] = __double2half(G64[e] * (double)rd[i] * (double)rd[j]);
+        const double g = (lower && j > i) ? G64[(int64_t)j * K + i] : G64[e];
+        Gp[e] = __double2half(g * (double)rd[i] * (double)rd[j]);
     }
 }
 
@@ -533,16 +541,20 @@ cudaError_t launch_awq_gram(const uint16_t* X, int64_t T, const uint16_t* W, int
         reinterpret_cast<const unsigned short*>(X), T, (int)K, L.chunk, L.Tp, reinterpret_cast<unsigned short*>(XT));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const unsigned ew_blocks = (unsigned)device_sm_count() * 8;
+    // G is symmetric: for K > 128 only the 256 x 256 tiles on and below the diagonal are formed
+    // (half the tensor-core work, one wave at K = 4096), accumulated and read back mirrored.
+    const int lower = K > 128 ? 1 : 0;
     for (int64_t c = 0; c < L.n_chunks; ++c) {  // G = sum over chunks of X_c^T X_c
         const uint16_t* XTc = XT + c * K * L.chunk;
-        e = launch_tc_f32(XTc, K, XTc, K, L.chunk, Gc, status, stream);
+        e = lower ? launch_tc_f32_lower(XTc, K, L.chunk, Gc, status, stream)
+                  : launch_tc_f32(XTc, K, XTc, K, L.chunk, Gc, status, stream);
         if (e != cudaSuccess) return e;
-        gram_accumulate_kernel<<<ew_blocks, 256, 0, stream>>>(Gc, K * K, c == 0, G64);
+        gram_accumulate_kernel<<<(unsigned)(K < 4096 ? K : 4096), 256, 0, stream>>>(Gc, (int)K, c == 0, lower, G64);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     gram_diag_kernel<<<(unsigned)((K + 255) / 256), 256, 0, stream>>>(G64, (int)K, d, rd);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    gram_scale_kernel<<<ew_blocks, 256, 0, stream>>>(G64, rd, (int)K, Gp);
+    gram_scale_kernel<<<ew_blocks, 256, 0, stream>>>(G64, rd, (int)K, lower, Gp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int64_t G = K / 128;
     const int64_t n_groups = N * G;

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                    const __half* __restrict__ scales, const uint8_t* __restrict__ zeros,
                    __half* __restrict__ Y, double* __restrict__ sse_part, float* __restrict__ Cf,
                    const __half* __restrict__ Adot, int M, int N, int K, int m_tiles, int n_tiles,
-                   int* status) {
+                   int lower, int* status) {
     constexpr bool SSE = EPI == 1 || EPI == 3;  // modes that reduce the tile to one fp64 partial
     using C = TcCfg<DEQ, MT, BN>;
     constexpr int S = C::kStages;
@@ -92,7 +92,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int mt, nt;
-    tc_tile_coords(blockIdx.x, m_tiles, n_tiles, mt, nt);
+    if (lower) {  // only the tiles on or below the diagonal of a square product (one per CTA)
+        const int t = blockIdx.x;
+        mt = (int)((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
+        while ((mt + 1) * (mt + 2) / 2 <= t) ++mt;
+        while (mt * (mt + 1) / 2 > t) --mt;
+        nt = t - mt * (mt + 1) / 2;
+    } else {
+        tc_tile_coords(blockIdx.x, m_tiles, n_tiles, mt, nt);
+    }
     const int m0 = mt * C::kBM, n0 = nt * BN;
     const int nk = K / TC_BK;
     const int G = K >> 7;
@@ -406,7 +414,7 @@ static cudaError_t set_tc_attrs() {
 template <bool DEQ, int EPI, int MT, int BN = TC_BN>
 static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int64_t N, int64_t K,
                              const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, double* sse_part,
-                             int* status, cudaStream_t stream, float* Cf = nullptr) {
+                             int* status, cudaStream_t stream, float* Cf = nullptr, bool lower = false) {
     using C = TcCfg<DEQ, MT, BN>;
     CUtensorMap ta, tb;
     if (!make_tensor_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, TC_BK, C::kBM,
@@ -422,9 +430,11 @@ static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int6
     if (e != cudaSuccess) return e;
     const int m_tiles = (int)((M + C::kBM - 1) / C::kBM);
     const int n_tiles = (int)((N + BN - 1) / BN);
-    tc_gemm_kernel<DEQ, EPI, MT, BN><<<m_tiles * n_tiles, TC_THREADS, C::kBytes, stream>>>(
+    if (lower && (M != N || C::kBM != BN)) return cudaErrorInvalidValue;  // square tiles of a square product
+    const int grid = lower ? m_tiles * (m_tiles + 1) / 2 : m_tiles * n_tiles;
+    tc_gemm_kernel<DEQ, EPI, MT, BN><<<grid, TC_THREADS, C::kBytes, stream>>>(
         ta, tb, reinterpret_cast<const __half*>(scales), zeros, reinterpret_cast<__half*>(Y), sse_part, Cf,
-        reinterpret_cast<const __half*>(X), (int)M, (int)N, (int)K, m_tiles, n_tiles, status);
+        reinterpret_cast<const __half*>(X), (int)M, (int)N, (int)K, m_tiles, n_tiles, lower ? 1 : 0, status);
     return cudaGetLastError();
 }
 
@@ -481,6 +491,11 @@ cudaError_t launch_tc_f32(const uint16_t* A, int64_t M, const uint16_t* B, int64
     if (tc_mt(M) == 2)
         return launch_tc<false, 2, 2>(A, M, B, N, K, nullptr, nullptr, nullptr, nullptr, status, stream, C);
     return launch_tc<false, 2, 1>(A, M, B, N, K, nullptr, nullptr, nullptr, nullptr, status, stream, C);
+}
+
+cudaError_t launch_tc_f32_lower(const uint16_t* A, int64_t M, int64_t K, float* C, int* status, cudaStream_t stream) {
+    if (tc_mt(M) != 2) return cudaErrorInvalidValue;
+    return launch_tc<false, 2, 2>(A, M, A, M, K, nullptr, nullptr, nullptr, nullptr, status, stream, C, true);
 }
 
 cudaError_t launch_tc_f16(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, uint16_t* Y,

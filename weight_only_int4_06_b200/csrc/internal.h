@@ -75,6 +75,9 @@ cudaError_t launch_tc_f16(const uint16_t* A, int64_t M, const uint16_t* B, int64
                           int* status, cudaStream_t stream);
 cudaError_t launch_tc_f32(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, float* C,
                           int* status, cudaStream_t stream);
+// C [M, M] fp32 = A A^T on and below the diagonal only (256 x 256 tiles; M > 128): entries above the
+// diagonal are not written.
+cudaError_t launch_tc_f32_lower(const uint16_t* A, int64_t M, int64_t K, float* C, int* status, cudaStream_t stream);
 // Per-tile sum over (m, n) of (A . B^T)[m, n] * A[m, n] into part[tile] (requires N == K).
 cudaError_t launch_tc_dot(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, double* part,
                           int* status, cudaStream_t stream);

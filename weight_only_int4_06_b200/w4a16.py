@@ -320,6 +320,24 @@ class HostGemmBatch:
         if st != W4_OK:
             raise W4Error(st, "w4_gemm_host_batch")
 
+    def capture(self) -> "torch.cuda.CUDAGraph":
+        """The batch call (both copies and every GEMM) captured once into a CUDA graph; replay() on
+        the current stream then enqueues all of it with one launch.  The graph reads x_host and
+        writes y_host in place, so refill x(i) and read y(i) around each replay as with run().
+        Capture the graph on the stream the batch was built for (the default: the current one)."""
+        self.run()  # one direct call first: kernel set-up happens outside the capture
+        torch.cuda.current_stream().synchronize()
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                st = lib().w4_gemm_host_batch(*self._args[:-1], ctypes.c_void_p(side.cuda_stream))
+        torch.cuda.current_stream().wait_stream(side)
+        if st != W4_OK:
+            raise W4Error(st, "w4_gemm_host_batch (capture)")
+        return g
+
 
 _ws_cache: dict = {}
 
