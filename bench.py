@@ -674,11 +674,17 @@ def bench_wb_gemm(world, peaks, reps=20):
             g = capture(lambda i: B.wb_gemm(Xd, p, s, z, bits, group, ws), reps, 0)
             g.replay()
             t = max_over_ranks(time_graph(g, world) / reps, world)
-            res.append({"bits": bits, "group": group, "M": M, "K": K, "N": N, "us": round(t * 1e3, 2)})
+            byts = N * K * bits // 8 + 3 * N * (K // group) + 2 * M * K + 2 * M * N  # algorithmic (b/8 B/weight)
+            r = {"bits": bits, "group": group, "M": M, "K": K, "N": N, "us": round(t * 1e3, 2),
+                 "hbm_frac_of_algorithmic": round(byts / (t * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+            if M > 1:
+                r["tensor_frac"] = round(2 * M * N * K / (t * 1e-3) / 1e12 / peaks["bf16_tflops"], 3)
+            res.append(r)
             del g
     del Wd, ws
     torch.cuda.empty_cache()
-    return {"kernel": "dequant_bits_kernel + tc_gemm_kernel<fp16 B>", "layers": res}
+    return {"kernel": "dequant_bits_kernel + tc_gemm_kernel<fp16 B> (two passes through an fp16 workspace; "
+                      "not fused)", "layers": res}
 
 
 FP32_FMA_PER_CLK_PER_SM = 128     # B200 SM: 4 partitions x 32 fp32 FMA lanes
@@ -784,9 +790,8 @@ def other_rows(args, world, peaks, l2):
     if "ms" in rows["awq"] and "ms" in rows["awq_gram"]:
         rows["awq_gram"]["speedup_vs_direct"] = round(rows["awq"]["ms"] / rows["awq_gram"]["ms"], 2)
     row("awq_clip", lambda: bench_awq_clip(world, peaks, case))
-    if getattr(args, "extra_rows", False):  # rows whose kernels await their first parity run
-        row("gptq", lambda: bench_gptq(world, peaks))
-        row("wb_gemm", lambda: bench_wb_gemm(world, peaks))
+    row("gptq", lambda: bench_gptq(world, peaks))
+    row("wb_gemm", lambda: bench_wb_gemm(world, peaks))
     return rows
 
 
@@ -922,7 +927,7 @@ def main():
     ap.add_argument("--no-rows", action="store_true",
                     help="skip the secondary rows (quantize, prefill, awq) in the JSON line")
     ap.add_argument("--extra-rows", action="store_true",
-                    help="also time GPTQ and the other-width matmul (not part of the default line)")
+                    help="accepted for compatibility: GPTQ and the other-width matmul are in the default line")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
