@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                    const __half* __restrict__ scales, const uint8_t* __restrict__ zeros,
                    __half* __restrict__ Y, double* __restrict__ sse_part, float* __restrict__ Cf,
                    const __half* __restrict__ Adot, int M, int N, int K, int m_tiles, int n_tiles,
-                   int lower, int* status) {
+                   int lower, int ksplit, int* status) {
     constexpr bool SSE = EPI == 1 || EPI == 3;  // modes that reduce the tile to one fp64 partial
     using C = TcCfg<DEQ, MT, BN>;
     constexpr int S = C::kStages;
@@ -92,18 +92,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int mt, nt;
+    // ksplit > 1: CTA b computes K slice b % ksplit of tile b / ksplit (whole groups of 128 k) and
+    // stores its fp32 partial tile into slice (b % ksplit) of Cf
+    const int slice = ksplit > 1 ? (int)(blockIdx.x % ksplit) : 0;
+    const int tile_id = ksplit > 1 ? (int)(blockIdx.x / ksplit) : (int)blockIdx.x;
     if (lower) {  // only the tiles on or below the diagonal of a square product (one per CTA)
-        const int t = blockIdx.x;
+        const int t = tile_id;
         mt = (int)((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
         while ((mt + 1) * (mt + 2) / 2 <= t) ++mt;
         while (mt * (mt + 1) / 2 > t) --mt;
         nt = t - mt * (mt + 1) / 2;
     } else {
-        tc_tile_coords(blockIdx.x, m_tiles, n_tiles, mt, nt);
+        tc_tile_coords(tile_id, m_tiles, n_tiles, mt, nt);
     }
     const int m0 = mt * C::kBM, n0 = nt * BN;
-    const int nk = K / TC_BK;
     const int G = K >> 7;
+    // this CTA's k-blocks [kb0, kb0 + nk): two per group of 128, a slice starts on a group
+    const int kb0 = 2 * (int)(((int64_t)slice * G) / (ksplit > 1 ? ksplit : 1));
+    const int nk = 2 * (int)(((int64_t)(slice + 1) * G) / (ksplit > 1 ? ksplit : 1)) - kb0;
+    if (ksplit > 1 && EPI == 2) Cf += (int64_t)slice * M * N;
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -136,9 +143,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (lane == 0) {
             const uint32_t tx = C::kA + (DEQ ? C::kP : C::kB);
             int issued = 0;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (kb / S) & 1;
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % S, kb = kb0 + i;
+                const uint32_t ph = (i / S) & 1;
                 if (!mbar_wait_bounded(empty_bar(s), ph ^ 1, abort_flag)) { fail(); break; }
                 mbar_arrive_expect_tx(full_bar(s), tx);
                 tma_load_2d(a_addr(s), &tmA, kb * TC_BK, m0, full_bar(s));
@@ -157,9 +164,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_f16_f32(128, BN);
             bool ok = true;
-            for (int kb = 0; kb < nk && ok; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (kb / S) & 1;
+            for (int i = 0; i < nk && ok; ++i) {
+                const int s = i % S;
+                const uint32_t ph = (i / S) & 1;
                 if (!mbar_wait_bounded(full_bar(s), ph, abort_flag)) { fail(); ok = false; break; }
                 if (DEQ && !mbar_wait_bounded(deq_bar(s), ph, abort_flag)) { fail(); ok = false; break; }
                 tc_fence_after();
@@ -170,7 +177,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                     for (int t = 0; t < MT; ++t) {
                         const uint64_t ad = sw128_kmajor_desc(a_addr(s) + t * TC_A1_BYTES);
                         // +32 bytes along K per MMA inside the 128-byte swizzled row
-                        mma_f16_ss(tmem_d + t * BN, ad + 2 * j, bd + 2 * j, idesc, (kb | j) != 0);
+                        mma_f16_ss(tmem_d + t * BN, ad + 2 * j, bd + 2 * j, idesc, (i | j) != 0);
                     }
                 }
                 tc_commit(empty_bar(s));
@@ -194,12 +201,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             // scale/zero of the next group are fetched one group (two stages) ahead
             uint32_t sc_next = 0, z_next = 0;
             if (nvalid) {
-                sc_next = __ldg(srow);
-                z_next = __ldg(zrow);
+                sc_next = __ldg(srow + kb0 / 2);
+                z_next = __ldg(zrow + kb0 / 2);
             }
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % S;
-                const uint32_t ph = (kb / S) & 1;
+            for (int i = 0; i < nk; ++i) {
+                const int s = i % S, kb = kb0 + i;
+                const uint32_t ph = (i / S) & 1;
                 if ((kb & 1) == 0) {  // a new group of 128 every second stage
                     const int g = kb >> 1;
                     const uint32_t sb = sc_next, z = z_next;
@@ -414,7 +421,8 @@ static cudaError_t set_tc_attrs() {
 template <bool DEQ, int EPI, int MT, int BN = TC_BN>
 static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int64_t N, int64_t K,
                              const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, double* sse_part,
-                             int* status, cudaStream_t stream, float* Cf = nullptr, bool lower = false) {
+                             int* status, cudaStream_t stream, float* Cf = nullptr, bool lower = false,
+                             int ksplit = 1) {
     using C = TcCfg<DEQ, MT, BN>;
     CUtensorMap ta, tb;
     if (!make_tensor_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, TC_BK, C::kBM,
@@ -431,10 +439,10 @@ static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int6
     const int m_tiles = (int)((M + C::kBM - 1) / C::kBM);
     const int n_tiles = (int)((N + BN - 1) / BN);
     if (lower && (M != N || C::kBM != BN)) return cudaErrorInvalidValue;  // square tiles of a square product
-    const int grid = lower ? m_tiles * (m_tiles + 1) / 2 : m_tiles * n_tiles;
+    const int grid = (lower ? m_tiles * (m_tiles + 1) / 2 : m_tiles * n_tiles) * ksplit;
     tc_gemm_kernel<DEQ, EPI, MT, BN><<<grid, TC_THREADS, C::kBytes, stream>>>(
         ta, tb, reinterpret_cast<const __half*>(scales), zeros, reinterpret_cast<__half*>(Y), sse_part, Cf,
-        reinterpret_cast<const __half*>(X), (int)M, (int)N, (int)K, m_tiles, n_tiles, lower ? 1 : 0, status);
+        reinterpret_cast<const __half*>(X), (int)M, (int)N, (int)K, m_tiles, n_tiles, lower ? 1 : 0, ksplit, status);
     return cudaGetLastError();
 }
 
@@ -465,9 +473,59 @@ void tc_w4_pick(int64_t M, int64_t N, int* mt_out, int* bn_out) {
     }
 }
 
+// K slices of w4_gemm's tensor-core path: 256 x 256 tiles that fill fewer than half the SMs (M >
+// 128) are split along K into up to 8 slices of whole groups, at least 8 k-blocks of 64 each,
+// so that tiles x slices fill the SMs; 1 = no split.
+int tc_w4_split(int64_t M, int64_t N, int64_t K) {
+    if (M <= 128) return 1;
+    const int64_t sms = device_sm_count();
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    if (2 * tiles >= sms) return 1;
+    int64_t s = sms / tiles;
+    const int64_t max_by_k = (K / TC_BK) / 8;
+    if (s > max_by_k) s = max_by_k;
+    if (s > 8) s = 8;
+    return s >= 2 ? (int)s : 1;
+}
+
+size_t tc_w4_workspace(int64_t M, int64_t N, int64_t K) {
+    const int s = tc_w4_split(M, N, K);
+    return s > 1 ? (size_t)s * (size_t)M * (size_t)N * 4 : 0;
+}
+
+// Y = fp16(sum over the slices of the fp32 partials, in slice order): deterministic.
+__global__ void splitk_reduce_kernel(const float* __restrict__ P, int slices, int64_t mn, __half* __restrict__ Y) {
+    const int64_t n4 = mn / 4;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
+        float4 a = reinterpret_cast<const float4*>(P)[e];
+        for (int s = 1; s < slices; ++s) {
+            const float4 b = reinterpret_cast<const float4*>(P + (int64_t)s * mn)[e];
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        uint2 o;
+        o.x = pack_half2(a.x, a.y);
+        o.y = pack_half2(a.z, a.w);
+        reinterpret_cast<uint2*>(Y)[e] = o;
+    }
+}
+
 cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                         const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,
+                         const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, void* ws, int* status,
                          cudaStream_t stream) {
+    const int ks = tc_w4_split(M, N, K);
+    if (ks > 1) {  // M * N is a multiple of 8 (N % 8 == 0): whole float4s
+        if (!ws) return cudaErrorInvalidValue;
+        float* P = static_cast<float*>(ws);
+        cudaError_t e = launch_tc<true, 2, 2, 256>(X, M, packed, N, K, scales, zeros, nullptr, nullptr, status,
+                                                    stream, P, false, ks);
+        if (e != cudaSuccess) return e;
+        const int64_t mn = M * N;
+        const int64_t want = (mn / 4 + 255) / 256;
+        const int64_t cap = (int64_t)device_sm_count() * 8;
+        splitk_reduce_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, stream>>>(
+            P, ks, mn, reinterpret_cast<__half*>(Y));
+        return cudaGetLastError();
+    }
     int mt = 2, bn = 256;
     tc_w4_pick(M, N, &mt, &bn);
     if (mt == 2 && bn == 256)

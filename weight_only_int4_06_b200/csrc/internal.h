@@ -63,9 +63,12 @@ cudaError_t launch_gemv_tc(const uint16_t* X, int64_t M, int64_t N, int64_t K, c
                            bool weights_static, int* status, cudaStream_t stream);
 
 // tcgen05 GEMM (gemm_tc.cu).
+// ws: tc_w4_workspace(M, N, K) bytes (fp32 partial tiles of the K slices), may be null when 0.
 cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                         const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, int* status,
+                         const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, void* ws, int* status,
                          cudaStream_t stream);
+int tc_w4_split(int64_t M, int64_t N, int64_t K);         // K slices of the tensor-core path (1: none)
+size_t tc_w4_workspace(int64_t M, int64_t N, int64_t K);  // bytes of fp32 partials when split
 cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64_t N, int64_t K,
                           double* sse_part, int* status, cudaStream_t stream);
 int tc_sse_partials(int64_t T, int64_t N);  // tiles of an M = T x N launch (partials of EPI 1 and 3)

@@ -295,7 +295,9 @@ class HostGemmBatch:
             arr[i] = GemmLayer(M, N, K, _dev(p, torch.int32, "packed").value, _dev(sc, torch.float16, "scales").value,
                                _dev(z, torch.uint8, "zeros").value, self.x_off[i], self.y_off[i])
         need = max(_ws_size(M, N, K, group) for (M, K, N) in self.shapes)
-        if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        if need and workspace is None:  # the largest layer's partial tiles (held by this object)
+            workspace = torch.empty(need, dtype=torch.uint8, device="cuda")
+        if need and workspace.numel() * workspace.element_size() < need:
             raise ValueError("workspace too small: see w4_gemm_workspace_size")
         ws_ptr = ctypes.c_void_p(workspace.data_ptr()) if workspace is not None else None
         ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
