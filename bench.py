@@ -683,8 +683,9 @@ def bench_wb_gemm(world, peaks, reps=20):
             del g
     del Wd, ws
     torch.cuda.empty_cache()
-    return {"kernel": "dequant_bits_kernel + tc_gemm_kernel<fp16 B> (two passes through an fp16 workspace; "
-                      "not fused)", "layers": res}
+    return {"kernel": "M <= 8: wb_gemv_kernel (fused: bit stream read once, codes dequantised in registers, "
+                      "fp32 CUDA-core sums); larger M: dequant_bits_kernel + tc_gemm_kernel<fp16 B> (two passes "
+                      "through an fp16 workspace)", "layers": res}
 
 
 FP32_FMA_PER_CLK_PER_SM = 128     # B200 SM: 4 partitions x 32 fp32 FMA lanes

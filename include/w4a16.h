@@ -429,9 +429,11 @@ w4_status wb_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int bits, int 
 /*
  * wb_gemm -- Y = X . dequant(W)^T for w4_quantize_pack_bits' format at any supported width.
  *
- * Two passes: every weight is dequantised to fp16 (w = (q - z) s, exact in fp32, rounded once to
- * fp16) into ws, then the tcgen05 GEMM multiplies with fp32 accumulation and writes fp16 Y.  Not
- * fused (w4_gemm's fused kernels serve 4-bit, group-128 weights); meant for the other widths.
+ * M <= 8: one fused pass: the bit stream is read once and every weight (q - z) s is formed exactly
+ * in fp32 in registers, sum_k x_k (q_k - z) s accumulated in fp32 (ws unused).  Larger M: two
+ * passes: every weight is dequantised to fp16 (w = (q - z) s, exact in fp32, rounded once to fp16)
+ * into ws, then the tcgen05 GEMM multiplies with fp32 accumulation.  Y is rounded once to fp16;
+ * results are deterministic.  Meant for the other widths (w4_gemm serves 4-bit, group-128 weights).
  *   X [M, K] fp16, Y [M, N] fp16, ws >= wb_gemm_workspace_size bytes; all 16-byte aligned.
  */
 w4_status wb_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,

@@ -179,3 +179,16 @@ def test_gptq_after_awq_scaling_matches_oracle(bits, group, act_order):
         Xs = OB.scale_activations(X[:8], a)
         Yref = OB.gemm_act_order(Xs, _u32(p), s.cpu().numpy(), z.cpu().numpy(), perm.cpu().numpy(), 4, 128)
         _check_gemm(Y, Yref)
+
+
+@pytest.mark.parametrize("bits,group", WIDTHS)
+@pytest.mark.parametrize("M,K,N", [(1, 4096, 1032), (3, 11008, 264), (8, 1024, 136)])
+def test_wb_gemm_decode_sizes_match_oracle(bits, group, M, K, N):
+    """Decode-sized M takes the fused b-bit GEMV (bit stream read once, codes dequantised in
+    registers, fp32 sums); same tolerance as every GEMM."""
+    X, W = synth.layer_case(81, M, K, N)
+    p, s, z = OB.quantize_pack_bits(W, bits, group)
+    Y = B.wb_gemm(torch.from_numpy(X).cuda(), torch.from_numpy(p.view(np.int32)).cuda(), torch.from_numpy(s).cuda(),
+                  torch.from_numpy(z).cuda(), bits, group)
+    assert B.w4_check_device_status() == 0
+    _check_gemm(Y.cpu().numpy(), OB.gemm_bits(X, p, s, z, bits, group))
