@@ -470,10 +470,12 @@ def run_gemm_bench(args, rank, world, local, kind, with_extras=True):
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4),
                 "traffic": load_traffic("decode") if kind == "decode" else None}
-        kern = ("decode_stream_kernel<MT> (one half-SM CTA per SM, TMA ring of 8 KB stages, mma.sync, metadata by bulk copy)"
+        kern = ("decode_stream_kernel<MT> (one full-SM CTA per SM, TMA ring of 32 KB stages, mma.sync, "
+                "metadata by bulk copy)"
                 if kind == "decode" else
-                "decode_stream_kernel<MT> in launches of <= 8 rows where 8 staged rows fit, else "
-                "skinny_kernel (cluster split-K)")
+                "w4_gemm per shape: decode_stream_kernel in launches of <= 8 rows (K cut into slices of "
+                "4096 + splitk_reduce where the rows would leave a shallow ring), the tcgen05 GEMM at "
+                "M = 32 on wide layers")
     roof["traffic_unit"] = "DRAM bytes per step (ncu, see profiles/)"
     roof["peak_source"] = peaks["source"]
     roof["kernel"] = kern
@@ -746,8 +748,9 @@ def _small_batch_row(world, peaks, l2):
         r["launches"] = n
     del wl, flush
     torch.cuda.empty_cache()
-    return {"kernel": "w4_gemm (per-shape family: decode_stream_kernel in launches of <= 8 rows, "
-                      "skinny_kernel where 8 staged rows do not fit)", "bound": "hbm", "layers": layers}
+    return {"kernel": "w4_gemm (per-shape family: decode_stream_kernel in launches of <= 8 rows, K cut "
+                      "into slices of 4096 + splitk_reduce where the rows would leave a shallow ring; the "
+                      "tcgen05 GEMM where its tiles fill the SMs)", "bound": "hbm", "layers": layers}
 
 
 def _prefill_row(world, peaks, l2):

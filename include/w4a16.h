@@ -119,7 +119,10 @@ w4_status w4_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int group,
                            const float* act_scale, uint32_t* packed, uint16_t* scales,
                            uint8_t* zeros, void* stream);
 
-/* Bytes of device workspace w4_gemm / w4_gemm_ex need for this shape (may be 0). */
+/* Bytes of device workspace w4_gemm / w4_gemm_ex need for this shape (may be 0): fp32 partial
+ * sums when the tensor-core GEMM (M > 128 with few output tiles) or the GEMV (activation rows too
+ * long to stage whole next to a deep enough ring, K/128 a multiple of 16) cut K into slices.  A
+ * function of M, N, K and group only; no device is touched. */
 w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, size_t* bytes);
 
 /*
@@ -131,11 +134,14 @@ w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, siz
  * w = (q - z) * s16 as above.
  *
  *   X [M, K] fp16, packed/scales/zeros as produced by w4_quantize_pack, Y [M, N] fp16 out.
- *   ws / ws_bytes: device workspace of at least w4_gemm_workspace_size bytes (may be NULL when
- *   that size is 0).  M == 0 or N == 0 is a no-op; K == 0 writes Y = 0.
+ *   ws / ws_bytes: device workspace of at least w4_gemm_workspace_size bytes, 16-byte aligned
+ *   (may be NULL when that size is 0; misaligned: W4_ERR_ALIGN).  M == 0 or N == 0 is a no-op;
+ *   K == 0 writes Y = 0.
  * Families (w4_gemm picks by M: GEMV, in launches of up to 8 activation rows, for M <= 32 when
- * 8 staged activation rows fit shared memory and scales/zeros are 16-byte aligned; skinny for
- * the other M <= 32; TC above):
+ * scales/zeros are 16-byte aligned and 8 staged activation rows fit shared memory or K/128 is a
+ * multiple of 16 (then K is cut into slices of 4096, their fp32 partials summed in slice order by
+ * a second launch); skinny for the other M <= 32; TC above, or from M = 17 when its 128-row
+ * weight tiles alone fill the SMs at K <= 8192):
  *   - GEMV: tensor-core sums of x with the raw operands 1024+q / 1024+16q, offsets and z removed
  *     per group with fp32 activation sums (fixed order), times s16 in fp32;
  *   - skinny: sum_k x_k (q_k - z) exactly per group on tensor cores in fp32, times s16 in fp32;

@@ -87,6 +87,12 @@ def test_gemm_rejects(L):
     assert g(*args(Y=BAD_ALIGN)) == 3
     assert g(*args(M=0)) == 0
     assert g(*args(N=0)) == 0
+    # a shape whose GEMV cuts K: no workspace, a short one, a misaligned one
+    need = 7 * 8 * 8192 * 4
+    big = [GOOD, 8, 8192, 28672, GOOD, GOOD, GOOD, 128, GOOD]
+    assert g(*big, None, 0, 0, None) == 5
+    assert g(*big, GOOD, need - 1, 0, None) == 5
+    assert g(*big, BAD_ALIGN, need, 0, None) == 3
 
 
 def test_workspace_queries(L):
@@ -95,6 +101,13 @@ def test_workspace_queries(L):
     assert L.w4_gemm_workspace_size(1, 4096, 4000, 128, ctypes.byref(n)) == 2
     assert L.w4_gemm_workspace_size(1, 4096, 4096, 64, ctypes.byref(n)) == 4
     assert L.w4_gemm_workspace_size(1, 4096, 4096, 128, None) == 1
+    # decode shapes need none; the GEMV's K slices (K = 28672: 7 slices of 4096) need fp32 partials
+    assert L.w4_gemm_workspace_size(1, 4096, 11008, 128, ctypes.byref(n)) == 0 and n.value == 0
+    assert L.w4_gemm_workspace_size(4, 8192, 8192, 128, ctypes.byref(n)) == 0 and n.value == 0
+    assert L.w4_gemm_workspace_size(8, 8192, 28672, 128, ctypes.byref(n)) == 0
+    assert n.value == 7 * 8 * 8192 * 4
+    assert L.w4_gemm_workspace_size(32, 8192, 28672, 128, ctypes.byref(n)) == 0
+    assert n.value == 7 * 8 * 8192 * 4  # launches of 8 rows reuse one workspace in turn
     assert L.awq_workspace_size(256, 64, 512, 128, 0, ctypes.byref(n)) == 4
     assert L.awq_workspace_size(256, 64, 500, 128, 20, ctypes.byref(n)) == 2
     assert L.awq_clip_workspace_size(256, 64, 512, 128, 10, ctypes.byref(n)) == 0 and n.value > 0
@@ -258,9 +271,14 @@ def test_host_batch_rejects_before_enqueuing(L):
 def test_gemm_plan_query(L):
     """The dispatch query (CPU: no device work) agrees with the documented rule."""
     assert B.w4_gemm_plan(1, 4096, 4096) == (B.VARIANT_GEMV, 1)
-    assert B.w4_gemm_plan(16, 8192, 8192) == (B.VARIANT_GEMV, 2)
-    assert B.w4_gemm_plan(32, 8192, 8192) == (B.VARIANT_GEMV, 4)
-    assert B.w4_gemm_plan(4, 8192, 28672) == (B.VARIANT_SKINNY, 1)  # 4 staged rows of K = 28672 do not fit
+    # 8 rows of K = 8192 leave 2 ring stages whole: K is cut in two, + 1 reducing launch each
+    assert B.w4_gemm_plan(4, 8192, 8192) == (B.VARIANT_GEMV, 1)
+    assert B.w4_gemm_plan(16, 8192, 8192) == (B.VARIANT_GEMV, 4)
+    assert B.w4_gemm_plan(32, 8192, 8192) == (B.VARIANT_GEMV, 8)
+    # K = 28672 is cut into slices (4 rows of it do not fit whole): the GEMV, then the slice sum
+    assert B.w4_gemm_plan(4, 8192, 28672) == (B.VARIANT_GEMV, 2)
+    assert B.w4_gemm_plan(32, 8192, 28672) == (B.VARIANT_GEMV, 8)
+    assert B.w4_gemm_plan(4, 8192, 28800) == (B.VARIANT_SKINNY, 1)  # K/128 = 225: no slices, no fit
     assert B.w4_gemm_plan(33, 4096, 4096) == (B.VARIANT_TC, 1)
     assert B.w4_gemm_plan(0, 4096, 4096) == (B.VARIANT_AUTO, 0)
     assert B.w4_gemm_plan(64, 4096, 4096, variant=B.VARIANT_SKINNY) == (B.VARIANT_SKINNY, 2)

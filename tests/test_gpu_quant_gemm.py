@@ -286,7 +286,11 @@ def test_gemm_tc_ragged(M, K, N):
                                    (1, 11008, 40), (1, 28672, 264), (3, 2048, 520), (1, 8192, 28672),
                                    # full-SM shapes with 3 and 2 ring stages (larger staged activations)
                                    (4, 8192, 264), (8, 4096, 1032), (3, 16384, 136), (5, 8192, 520),
-                                   (2, 28672, 72), (8, 8192, 264), (7, 8192, 136)])
+                                   (2, 28672, 72), (8, 8192, 264), (7, 8192, 136),
+                                   # K cut into slices: one stage each (the last one partial), two
+                                   # stages each, seven; half tiles (N % 16 == 8)
+                                   (8, 6144, 264), (8, 10240, 1032), (3, 16384, 136), (6, 28672, 520),
+                                   (1, 28672, 4104)])
 def test_gemm_gemv_ragged(M, K, N):
     X, p, s, z = oracle_case(28, M, K, N)
     assert_close(gpu_gemm(X, p, s, z, B.VARIANT_GEMV), oracle.gemm(X, p, s, z), f"gemv {M}x{K}x{N}")

@@ -64,6 +64,13 @@ def test_wb_gemm_matches_oracle(bits, group, M, K, N):
     _check_gemm(Y.cpu().numpy(), OB.gemm_bits(X, p, s, z, bits, group))
 
 
+@pytest.mark.parametrize("bits", [2, 4])
+@pytest.mark.parametrize("M,K,N", [(130, 192, 136), (40, 320, 264)])
+def test_wb_gemm_odd_multiple_of_64(bits, M, K, N):
+    """Group 64 with K an odd multiple of 64: the tensor-core GEMM's last k-block is a half group."""
+    test_wb_gemm_matches_oracle(bits, 64, M, K, N)
+
+
 def test_act_prepare_bit_exact():
     X, _ = synth.layer_case(74, 5, 384, 8)
     rng = np.random.default_rng(74)

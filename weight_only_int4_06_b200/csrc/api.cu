@@ -59,15 +59,17 @@ int* device_status_ptr() {
 
 // The kernel family and number of launches of one w4_gemm_ex call (shape already validated).
 // AUTO: the tensor-core GEMM above 32 activation rows; up to 32 rows the TMA-fed GEMV in
-// launches of up to 8 rows where 8 staged activation rows fit its shared memory and the metadata
-// is 16-byte aligned (it bulk-copies scales and zero points), else the skinny kernel in launches
-// of up to 32 rows; from 17 rows on, the tensor-core GEMM instead when its 128-row W tiles alone
-// fill the SMs.  Measured per shape on B200 (bench.py --workload dispatch, cold L2): decode M = 1
-// GEMV 4.6 / 9.5 / 8.6 / 8.7 us vs skinny 6.2 / 19.6 / 18.9 / 14.3; at K = 8192 two and four
-// 8-row GEMV launches beat one skinny launch at M = 16 and 32 (32.6 vs 46.9, 63.4 vs 69.0 us at
-// N = 8192); at M = 32, N = 28672 the tensor-core GEMM (89.4 us) beats four GEMV launches (156.1)
-// and at M = 16 it does not (88.8 vs 79.0); at K = 28672 (8 rows of X do not fit the GEMV) the
-// skinny kernel beats or ties the tensor-core GEMM at every M.
+// launches of up to 8 rows where its metadata is 16-byte aligned (it bulk-copies scales and zero
+// points) and either 8 staged activation rows fit its shared memory or K/128 is a multiple of 16
+// (K then cut into slices of 4096, + 1 reducing launch), else the skinny kernel in launches of up
+// to 32 rows; from 17 rows on, the tensor-core GEMM instead when its 128-row W tiles alone fill
+// the SMs.  Measured per shape on B200 (bench.py --workload dispatch, cold L2, us): decode M = 1
+// GEMV 4.7 / 9.5 / 8.6 / 8.8 vs skinny 6.2 / 19.5 / 18.8 / 14.2; at K = 8192 the GEMV beats the
+// skinny kernel at M = 4 .. 32 (12.9 / 15.4 / 28.0 / 54.3 vs 29.7 / 29.8 / 46.7 / 68.7 at
+// N = 8192, cutting K in two at M = 8: 15.4 vs 17.4 whole); at M = 32, N = 28672 the tensor-core
+// GEMM (90.8) beats four GEMV launches (146.3), at M = 16 it does not (89.7 vs 74.0); at
+// K = 28672 the sliced GEMV beats the skinny kernel at every M (31.9 / 37.6 / 73.2 / 145.2 vs
+// 90.7 / 91.6 / 144.0 / 220.5) and the tensor-core GEMM (224).
 w4_status gemm_plan(int64_t M, int64_t N, int64_t K, int family, bool meta_aligned, int* chosen, int* launches) {
     const bool tc_fills = (N + 127) / 128 >= device_sm_count();
     if (family == W4_VARIANT_TC || (family == W4_VARIANT_AUTO && (M > 32 || (M > 16 && K <= 8192 && tc_fills)))) {
@@ -88,7 +90,9 @@ w4_status gemm_plan(int64_t M, int64_t N, int64_t K, int family, bool meta_align
     if (family == W4_VARIANT_GEMV && !meta_aligned) return W4_ERR_ALIGN;
     if (family == W4_VARIANT_GEMV || (family == W4_VARIANT_AUTO && M <= 32 && gemv_fits && meta_aligned)) {
         *chosen = W4_VARIANT_GEMV;
-        *launches = (int)((M + 7) / 8);
+        *launches = 0;
+        for (int64_t m0 = 0; m0 < M; m0 += 8)  // launches of up to 8 rows, each + 1 when K is cut
+            *launches += decode_stream_slices(M - m0 < 8 ? M - m0 : 8, K) > 1 ? 2 : 1;
         return W4_OK;
     }
     SkinnyPlan plan;
@@ -124,8 +128,11 @@ w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, siz
     if (group != 128) return W4_ERR_UNSUPPORTED;
     if (!dims_ok(M, K) || !dims_ok(N, K) || !dims_ok(M, N) || K % group != 0 || N % 8 != 0)
         return W4_ERR_SHAPE;
-    // fp32 partial tiles when AUTO's tensor-core path splits K (prefill shapes with few tiles)
-    *bytes = M > 32 && K > 0 && N > 0 ? tc_w4_workspace(M, N, K) : 0;
+    // fp32 partials when the tensor-core path splits K (prefill shapes with few tiles) or the
+    // GEMV cuts K into slices (activation rows too long to stage whole next to a deep ring)
+    const size_t tc = M > 32 && K > 0 && N > 0 ? tc_w4_workspace(M, N, K) : 0;
+    const size_t gv = K > 0 && N > 0 ? decode_stream_workspace(M, N, K) : 0;
+    *bytes = tc > gv ? tc : gv;
     return W4_OK;
 }
 
@@ -143,6 +150,7 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     if (st != W4_OK) return st;
     if (ws_bytes < need) return W4_ERR_WORKSPACE;
     if (need > 0 && !ws) return W4_ERR_NULL;
+    if (need > 0 && !aligned16(ws)) return W4_ERR_ALIGN;
     if (M == 0 || N == 0) return W4_OK;
     if (!Y) return W4_ERR_NULL;
     if (!aligned16(Y)) return W4_ERR_ALIGN;
@@ -178,7 +186,7 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
         // up to 8 activation rows per launch (token-by-token decode has M == 1)
         for (int64_t m0 = 0; m0 < M; m0 += 8) {
             const int64_t mc = (M - m0) < 8 ? (M - m0) : 8;
-            cudaError_t e = launch_decode_stream(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N,
+            cudaError_t e = launch_decode_stream(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N, ws,
                                                  weights_static, status, s);
             if (e != cudaSuccess) return W4_ERR_CUDA;
         }

@@ -66,13 +66,18 @@ struct DsLayout {
     uint32_t ring, meta, mslot, xs, corr, red, bars, total;
 };
 
-// Byte offsets of the shared-memory regions for `ns` ring stages and `nms` metadata slots.
-__host__ __device__ inline DsLayout ds_layout(int SG, int MT, int M, int K, int ns, int nms) {
+// Metadata of one stage in split mode: scales [16][SG] fp16, then zero points [16][SG] u8.
+__host__ __device__ constexpr uint32_t ds_stage_meta_bytes(int SG) { return 48u * (uint32_t)SG; }
+
+// Byte offsets of the shared-memory regions for `ns` ring stages and `nms` metadata slots; K is
+// the staged length of k (the whole K, or one K slice in split mode, where every ring stage has a
+// metadata slot of its own: nms == ns).
+__host__ __device__ inline DsLayout ds_layout(int SG, int MT, int M, int K, int ns, int nms, bool ks) {
     DsLayout L;
     const uint32_t G = (uint32_t)(K / 128);
     L.ring = 0;
     L.meta = (uint32_t)ns * ds_stage_bytes(SG);
-    L.mslot = 48u * G;                                                  // 16 rows x G x (2 + 1) bytes
+    L.mslot = ks ? ds_stage_meta_bytes(SG) : 48u * G;                   // 16 rows x groups x (2 + 1) bytes
     L.xs = L.meta + (uint32_t)nms * L.mslot;
     L.corr = L.xs + (uint32_t)M * (uint32_t)(K + 8) * 2;                // float2 [G][MT] (+ 8 spare)
     L.red = L.corr + (G * (uint32_t)MT + 8) * 8;                        // [slot][warp][16][MT] fp32
@@ -164,27 +169,35 @@ __device__ __forceinline__ void ds_group(uint32_t a_addr, uint32_t b_addr, uint3
     }
 }
 
-template <int MT, int SG>
+// KS (split mode): blockIdx.y is a K slice of `ncs` whole stages; the CTA stages the activations of
+// its slice only, every stage brings its own scales and zero points (two 2-D TMA boxes of 16 rows x
+// SG groups), and the reducer writes fp32 partial sums to P [slice][M][N] instead of Y.
+template <int MT, int SG, bool KS>
 __global__ void __launch_bounds__(DS_THREADS, 1)
-    decode_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __half* __restrict__ X,
+    decode_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
+                         const __grid_constant__ CUtensorMap tmZ, const __half* __restrict__ X,
                          const unsigned short* __restrict__ scales, const uint8_t* __restrict__ zeros,
-                         __half* __restrict__ Y, int M, int N, int K, int n_tiles, int ns, int nms,
-                         int weights_early, int* status) {
+                         __half* __restrict__ Y, float* __restrict__ P, int M, int N, int K, int n_tiles, int ns,
+                         int nms, int ncs, int weights_early, int* status) {
     constexpr int ROWB = SG * 64;                    // bytes of one row in a stage
     constexpr uint32_t STAGE_BYTES = 16u * ROWB;
     constexpr int GPW = SG / DS_CW;                  // groups per consumer warp per stage
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // TMA destinations need an aligned base: round up (the launch reserves 1 KB of slack)
     unsigned char* smem = smem_align1024(smem_raw);
-    const DsLayout L = ds_layout(SG, MT, M, K, ns, nms);
-    const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = K >> 7;
-    const int NC = (G + SG - 1) / SG;  // stages per tile
+    const int NC = (G + SG - 1) / SG;  // stages of the whole K
+    // this CTA's stages of every tile: [kc0, kc0 + NCl)
+    const int kc0 = KS ? (int)blockIdx.y * ncs : 0;
+    const int NCl = KS ? min(ncs, NC - kc0) : NC;
+    const int KL = KS ? ncs * SG * 128 : K;  // staged k per activation row
+    const DsLayout L = ds_layout(SG, MT, M, KL, ns, nms, KS);
+    const uint32_t sbase = smem_u32(smem);
     // balanced contiguous tile ranges: CTA sizes differ by at most one tile
     const int t0 = (int)(((int64_t)blockIdx.x * n_tiles) / gridDim.x);
     const int t1 = (int)(((int64_t)(blockIdx.x + 1) * n_tiles) / gridDim.x);
-    const int n_units = (t1 - t0) * NC;
+    const int n_units = (t1 - t0) * NCl;
     const uint32_t bar0 = sbase + L.bars;
     auto full_bar = [&](int s) { return bar0 + 8 * s; };
     auto empty_bar = [&](int s) { return bar0 + 8 * (DS_MAXNS + s); };
@@ -200,7 +213,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), DS_CW);
         }
-        for (int i = 0; i < nms; ++i) mbar_init(meta_empty(i), DS_CW);
+        if (!KS)
+            for (int i = 0; i < nms; ++i) mbar_init(meta_empty(i), DS_CW);
         for (int i = 0; i < DS_RSLOTS; ++i) {
             mbar_init(tile_full(i), 32 * DS_CW);  // every consumer lane arrives after parking
             mbar_init(red_empty(i), 1);
@@ -215,6 +229,10 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&tmW);
+            if (KS) {
+                prefetch_tmap(&tmS);
+                prefetch_tmap(&tmZ);
+            }
             if (!weights_early) pdl_wait();
             int issued = 0, t = t0, kc = 0, s = 0, ms = 0;
             uint32_t ph = 0, mph = 0;
@@ -222,29 +240,40 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
                 // The ring is full: from here on progress depends on the consumers, who first
                 // wait for the preceding kernel; start the bounded waits only after that point.
                 if (u == ns && weights_early) pdl_wait();
-                if ((kc == 0 && !mbar_wait_bounded(meta_empty(ms), mph ^ 1, abort_flag)) ||
+                if ((!KS && kc == 0 && !mbar_wait_bounded(meta_empty(ms), mph ^ 1, abort_flag)) ||
                     !mbar_wait_bounded(empty_bar(s), ph ^ 1, abort_flag)) {
                     *abort_flag = 1;
                     record_status(status, W4_ERR_DEVICE_TIMEOUT);
                     break;
                 }
-                uint32_t sb = 0, zb = 0;
-                const int64_t mofs = (int64_t)t * 16 * G;  // first metadata entry of the tile
-                const uint32_t mdst = L.meta + ms * L.mslot;
-                if (kc == 0) {  // the tile's metadata rides on its first stage
-                    const int rows = N - t * 16 < 16 ? N - t * 16 : 16;  // 8 or 16 (N % 8 == 0)
-                    sb = (uint32_t)(rows * 2 * G);
-                    zb = (uint32_t)(rows * G) & ~15u;
-                    if (zb != (uint32_t)(rows * G))  // 8 trailing zero points (8 rows, odd G): plain copy
-                        *reinterpret_cast<uint2*>(smem + mdst + 32 * G + zb) =
-                            *reinterpret_cast<const uint2*>(zeros + mofs + zb);
+                if constexpr (KS) {
+                    // weights, scales and zero points of stage kc0 + kc of tile t (the boxes' rows past
+                    // N and groups past K/128 are zero-filled and counted in full)
+                    const int kg = kc0 + kc;
+                    const uint32_t mdst = sbase + L.meta + (uint32_t)s * L.mslot;
+                    mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES + ds_stage_meta_bytes(SG));
+                    tma_load_2d(sbase + L.ring + s * STAGE_BYTES, &tmW, kg * (ROWB / 8), t * 16, full_bar(s));
+                    tma_load_2d(mdst, &tmS, kg * SG, t * 16, full_bar(s));
+                    tma_load_2d(mdst + 32u * SG, &tmZ, kg * SG, t * 16, full_bar(s));
+                } else {
+                    uint32_t sb = 0, zb = 0;
+                    const int64_t mofs = (int64_t)t * 16 * G;  // first metadata entry of the tile
+                    const uint32_t mdst = L.meta + ms * L.mslot;
+                    if (kc == 0) {  // the tile's metadata rides on its first stage
+                        const int rows = N - t * 16 < 16 ? N - t * 16 : 16;  // 8 or 16 (N % 8 == 0)
+                        sb = (uint32_t)(rows * 2 * G);
+                        zb = (uint32_t)(rows * G) & ~15u;
+                        if (zb != (uint32_t)(rows * G))  // 8 trailing zero points (8 rows, odd G): plain copy
+                            *reinterpret_cast<uint2*>(smem + mdst + 32 * G + zb) =
+                                *reinterpret_cast<const uint2*>(zeros + mofs + zb);
+                    }
+                    mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES + sb + zb);
+                    tma_load_2d(sbase + L.ring + s * STAGE_BYTES, &tmW, kc * (ROWB / 8), t * 16, full_bar(s));
+                    if (sb) bulk_load_1d(sbase + mdst, scales + mofs, sb, full_bar(s));
+                    if (zb) bulk_load_1d(sbase + mdst + 32 * G, zeros + mofs, zb, full_bar(s));
                 }
-                mbar_arrive_expect_tx(full_bar(s), STAGE_BYTES + sb + zb);
-                tma_load_2d(sbase + L.ring + s * STAGE_BYTES, &tmW, kc * (ROWB / 8), t * 16, full_bar(s));
-                if (sb) bulk_load_1d(sbase + mdst, scales + mofs, sb, full_bar(s));
-                if (zb) bulk_load_1d(sbase + mdst + 32 * G, zeros + mofs, zb, full_bar(s));
                 ++issued;
-                if (++kc == NC) {
+                if (++kc == NCl) {
                     kc = 0;
                     ++t;
                     if (++ms == nms) { ms = 0; mph ^= 1; }
@@ -262,6 +291,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
         pdl_wait();  // Y may be read by the preceding kernel
         int rs = 0;
         uint32_t rph = 0;
+        float* Pl = KS ? P + (int64_t)blockIdx.y * M * N : nullptr;  // this slice's partials
         for (int t = t0; t < t1; ++t) {
             if (!mbar_wait_bounded(tile_full(rs), rph, abort_flag)) {
                 *abort_flag = 1;
@@ -277,7 +307,10 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
                     float sum = 0.0f;
 #pragma unroll
                     for (int w = 0; w < DS_CW; ++w) sum += rsl[w * (16 * MT) + o];
-                    Y[(int64_t)m * N + n] = __float2half_rn(sum);
+                    if (KS)
+                        Pl[(int64_t)m * N + n] = sum;
+                    else
+                        Y[(int64_t)m * N + n] = __float2half_rn(sum);
                 }
             }
             __syncwarp();
@@ -289,36 +322,38 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
 
     // ---------------------------------------------------------------- consumers
     // Consumer warp w owns the GPW consecutive groups w*GPW .. w*GPW+GPW-1 of every stage: in stage
-    // kc of a tile, groups kc*SG + w*GPW + e.  It stages exactly the activations of those groups,
-    // with their offset sums, so no other warp waits for them (one memory round trip after the
-    // preceding kernel has finished).  The 16 chunks of one group sit in 16 consecutive lanes,
-    // which reduce the sums with shuffles in a fixed order.
+    // kc0 + kc of a tile, groups (kc0 + kc)*SG + w*GPW + e, staged at local group kc*SG + w*GPW + e.
+    // It stages exactly the activations of those groups, with their offset sums, so no other warp
+    // waits for them (one memory round trip after the preceding kernel has finished).  The 16
+    // chunks of one group sit in 16 consecutive lanes, which reduce the sums with shuffles in a
+    // fixed order.
     pdl_wait();  // the activations may be produced by the preceding kernel
     const uint32_t xs_u = sbase + L.xs;
     const uint32_t corr_u = sbase + L.corr;
     __half* xs = reinterpret_cast<__half*>(smem + L.xs);
     float2* corr = reinterpret_cast<float2*>(smem + L.corr);
-    const int RS = K + 8;  // staged row stride in halves (16 bytes of padding)
+    const int RS = KL + 8;  // staged row stride in halves (16 bytes of padding)
     {
         const __half2 sixteenth = __float2half2_rn(0.0625f);
         const unsigned half_mask = (lane & 16) ? 0xFFFF0000u : 0x0000FFFFu;
-        const int per_warp = M * NC * GPW * 16;  // chunks of 8 k this warp stages (a multiple of 16)
+        const int per_warp = M * NCl * GPW * 16;  // chunks of 8 k this warp stages (a multiple of 16)
         for (int base = 0; base < per_warp; base += 32 * DS_XILP) {
             uint4 raw[DS_XILP];
 #pragma unroll
             for (int v = 0; v < DS_XILP; ++v) {
                 const int i = base + v * 32 + lane;
-                const int q = i >> 4, e = q % GPW, r = q / GPW, kc = r % NC, m = r / NC;
-                const int g = kc * SG + warp * GPW + e;
+                const int q = i >> 4, e = q % GPW, r = q / GPW, kc = r % NCl, m = r / NCl;
+                const int g = (kc0 + kc) * SG + warp * GPW + e;
                 if (i < per_warp && g < G) raw[v] = ldg_cached(X + (int64_t)m * K + g * 128 + (i & 15) * 8);
             }
 #pragma unroll
             for (int v = 0; v < DS_XILP; ++v) {
                 const int i = base + v * 32 + lane;
-                const int q = i >> 4, e = q % GPW, r = q / GPW, kc = r % NC, m = r / NC;
-                const int g = kc * SG + warp * GPW + e;
+                const int q = i >> 4, e = q % GPW, r = q / GPW, kc = r % NCl, m = r / NCl;
+                const int g = (kc0 + kc) * SG + warp * GPW + e;
                 if (i >= per_warp || g >= G) continue;  // uniform per 16-lane half (one group)
-                const int ch = g * 16 + (i & 15);       // chunk index within the row
+                const int gl = kc * SG + warp * GPW + e;  // staged (local) group
+                const int ch = gl * 16 + (i & 15);        // chunk index within the staged row
                 const uint4 w = raw[v];
                 uint4 p;
                 p.x = __byte_perm(w.x, w.z, 0x5410);         // x0, x4
@@ -338,7 +373,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
                     hi += __shfl_xor_sync(half_mask, hi, o);
                 }
                 if ((i & 15) == 0)  // C = 1024 (Sl + Sh'), S = Sl + 16 Sh'
-                    corr[g * MT + m] = make_float2(1024.0f * (lo + hi), fmaf(16.0f, hi, lo));
+                    corr[gl * MT + m] = make_float2(1024.0f * (lo + hi), fmaf(16.0f, hi, lo));
             }
         }
     }
@@ -352,7 +387,8 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
 #pragma unroll
     for (int j = 0; j < 4; ++j) xofs[j] = (uint32_t)ds_swz(c * 4 + j) * 16u;
     const int ccol = 2 * c < MT ? 2 * c : 0;  // first activation column of this thread's C pair
-    const bool mvec = (G % GPW) == 0;         // metadata of the warp's groups is vector-aligned
+    // metadata of the warp's groups is vector-aligned (always in split mode: rows of SG groups)
+    const bool mvec = KS || (G % GPW) == 0;
     // this thread's W bytes inside a stage: rows g8 and g8 + 8 of the warp's groups, 16 bytes at 16 c
     const uint32_t wlane = (uint32_t)(g8 * ROWB + warp * GPW * 64 + c * 16);
     int s = 0, kc = 0, ms = 0, rs = 0;
@@ -366,14 +402,17 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
             record_status(status, W4_ERR_DEVICE_TIMEOUT);
             dead = true;
         }
-        const int g0 = kc * SG + warp * GPW;
+        const int g0 = (kc0 + kc) * SG + warp * GPW;  // first group of the warp in this stage
+        const int gl0 = kc * SG + warp * GPW;         // its staged (local) index
         const int ng = g0 >= G ? 0 : min(GPW, G - g0);
         if (!dead && ng > 0) {
             const uint32_t st = sbase + L.ring + (uint32_t)s * STAGE_BYTES + wlane;
-            const uint32_t xg = xrow + (uint32_t)g0 * 256u;
-            const uint32_t msa = sbase + L.meta + (uint32_t)ms * L.mslot;  // scales [16][G] fp16
-            const uint32_t mza = msa + 32u * (uint32_t)G;                   // zeros [16][G] u8
-            const uint32_t ia = (uint32_t)(g8 * G + g0), ib = ia + 8u * (uint32_t)G;
+            const uint32_t xg = xrow + (uint32_t)gl0 * 256u;
+            // scales [16][mG] fp16, then zeros [16][mG] u8: the tile's (mG = K/128) or the stage's (mG = SG)
+            const uint32_t mG = KS ? (uint32_t)SG : (uint32_t)G;
+            const uint32_t msa = sbase + L.meta + (uint32_t)(KS ? s : ms) * L.mslot;
+            const uint32_t mza = msa + 32u * mG;
+            const uint32_t ia = g8 * mG + (uint32_t)(KS ? warp * GPW : g0), ib = ia + 8u * mG;
             if (ng == GPW && mvec) {
                 // the scales and zero points of the warp's groups, packed: GPW fp16 and GPW bytes per row
                 uint32_t sa[GPW / 2], sb[GPW / 2], za, zb;
@@ -393,7 +432,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
                     const float fsa = ds_half(sa[e >> 1], e & 1), fsb = ds_half(sb[e >> 1], e & 1);
                     const float fza = (float)((za >> (8 * e)) & 0xFFu), fzb = (float)((zb >> (8 * e)) & 0xFFu);
                     ds_group<MT>(st + e * 64, st + e * 64 + 8 * ROWB, xg + e * 256, xofs, xlane,
-                                 corr_u + (uint32_t)((g0 + e) * MT + ccol) * 8u, fsa, fsb, fza, fzb, acc);
+                                 corr_u + (uint32_t)((gl0 + e) * MT + ccol) * 8u, fsa, fsb, fza, fzb, acc);
                 }
             } else {
                 for (int e = 0; e < ng; ++e) {
@@ -402,16 +441,16 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
                     const float fza = (float)lds_u8(mza + ia + e);
                     const float fzb = (float)lds_u8(mza + ib + e);
                     ds_group<MT>(st + e * 64, st + e * 64 + 8 * ROWB, xg + e * 256, xofs, xlane,
-                                 corr_u + (uint32_t)((g0 + e) * MT + ccol) * 8u, fsa, fsb, fza, fzb, acc);
+                                 corr_u + (uint32_t)((gl0 + e) * MT + ccol) * 8u, fsa, fsb, fza, fzb, acc);
                 }
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar(s));
         if (++s == ns) { s = 0; ph ^= 1; }
-        if (++kc == NC) {
+        if (++kc == NCl) {
             // tile done: release its metadata, park this warp's partials for the reducer
-            if (lane == 0) mbar_arrive(meta_empty(ms));
+            if (!KS && lane == 0) mbar_arrive(meta_empty(ms));
             if (++ms == nms) ms = 0;
             if (!dead && !mbar_wait_bounded(red_empty(rs), rph ^ 1, abort_flag)) {
                 *abort_flag = 1;
@@ -432,52 +471,92 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
 // ------------------------------------------------------------------------------------ host side
 static int ds_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
-// Launch plan: stage size (32 groups: every consumer warp takes two groups of a stage), ring
-// depth and metadata slots within one SM's shared memory; one CTA per SM (or per tile when there
-// are fewer tiles than SMs).
-bool plan_decode_stream(int64_t M, int64_t N, int64_t K, DecodePlan* p) {
-    if (M < 1 || M > DS_MAXM || N < 8 || K < 128 || K % 128 != 0 || K > 65536 || N % 8 != 0) return false;
-    const int mt = ds_mt(M);
-    const int G = (int)(K / 128);
-    const int64_t T = (N + 15) / 16;
-    const int sms = device_sm_count();
-    const int grid = (int)std::min<int64_t>(T, sms);
-    const int64_t tpc = (T + grid - 1) / grid;  // tiles of the largest CTA
-    {
-        const uint32_t budget = DS_FULL_SMEM;
-        bool found = false;
-        int64_t best_bytes = -1;
-        for (int sg : {32}) {
-            const int NC = (G + sg - 1) / sg;
-            const int64_t units = tpc * NC;
-            const int nms = (int)std::min<int64_t>(DS_MAXMS, std::min<int64_t>(tpc, 2 + (int64_t)DS_MAXNS / NC));
-            const uint32_t fixed = ds_layout(sg, mt, (int)M, (int)K, 0, nms).total + 1024;  // alignment slack
-            const uint32_t sb = ds_stage_bytes(sg);
-            const int64_t want = std::min<int64_t>(DS_MINNS, units);
-            if (fixed + want * sb > budget) continue;
-            const int64_t ns = std::min<int64_t>(std::min<int64_t>((budget - fixed) / sb, DS_MAXNS), units);
-            const int64_t bytes = ns * sb;
-            if (bytes > best_bytes) {
-                best_bytes = bytes;
-                p->sg = sg;
-                p->mt = mt;
-                p->ns = (int)ns;
-                p->nms = nms;
-                p->n_tiles = (int)T;
-                p->grid = grid;
-                p->smem = ds_layout(sg, mt, (int)M, (int)K, (int)ns, nms).total + 1024;
-                found = true;
-            }
-        }
-        if (found) return true;
-    }
-    return false;
+constexpr int DS_SG = 32;       // groups per stage (32 KB stages: every consumer warp takes two groups)
+constexpr int DS_GOOD_NS = 4;   // ring depth below which the plan cuts K into slices (when it may)
+
+// Metadata slots of the unsplit kernel: enough to run two tiles ahead of the consumers.
+static int ds_nms(int64_t tpc, int NC) {
+    return (int)std::min<int64_t>(DS_MAXMS, std::min<int64_t>(tpc, 2 + (int64_t)DS_MAXNS / NC));
 }
 
-template <int MT, int SG>
-static cudaError_t ds_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M, int64_t N, int64_t K,
-                             const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, const DecodePlan& p,
-                             bool weights_static, int* status, cudaStream_t stream) {
+// Ring stages that fit in one SM's shared memory with `ncs` stages of k staged per activation row
+// (split mode) or the whole K (ncs == 0, with nms metadata slots); 0 when not even DS_MINNS fit.
+static int ds_fit(int64_t M, int64_t K, int ncs, int nms) {
+    const int mt = ds_mt(M);
+    const bool ks = ncs > 0;
+    const int KL = ks ? ncs * DS_SG * 128 : (int)K;
+    const uint32_t fixed = ds_layout(DS_SG, mt, (int)M, KL, 0, 0, ks).total + (ks ? 0u : (uint32_t)nms * 48u * (uint32_t)(K / 128)) +
+                           1024;  // alignment slack
+    const uint32_t per = ds_stage_bytes(DS_SG) + (ks ? ds_stage_meta_bytes(DS_SG) : 0u);
+    if (fixed + (uint32_t)DS_MINNS * per > DS_FULL_SMEM) return 0;
+    return (int)std::min<uint32_t>((DS_FULL_SMEM - fixed) / per, DS_MAXNS);
+}
+
+// Stages per K slice (0: K is not cut).  A function of M and K alone, so the workspace query needs
+// no device.  K is cut when the whole K leaves fewer than DS_GOOD_NS ring stages (or does not fit
+// at all) and the metadata rows allow 2-D TMA boxes (K/128 a multiple of 16: 16-byte row strides
+// of the zero points); the slices are equal (their count divides the stages of K), the longest
+// that leave DS_GOOD_NS stages, else one stage each.
+static int ds_split_stages(int64_t M, int64_t K) {
+    const int G = (int)(K / 128);
+    const int NC = (G + DS_SG - 1) / DS_SG;
+    if (ds_fit(M, K, 0, ds_nms(DS_MAXMS, NC)) >= DS_GOOD_NS || G % 16 != 0 || NC < 2) return 0;
+    for (int ncs = NC - 1; ncs >= 1; --ncs)
+        if (NC % ncs == 0 && ds_fit(M, K, ncs, 0) >= DS_GOOD_NS) return ncs;
+    return ds_fit(M, K, 1, 0) > ds_fit(M, K, 0, ds_nms(DS_MAXMS, NC)) ? 1 : 0;
+}
+
+int decode_stream_slices(int64_t M, int64_t K) {
+    const int ncs = ds_split_stages(M, K);
+    const int NC = (int)((K / 128 + DS_SG - 1) / DS_SG);
+    return ncs ? (NC + ncs - 1) / ncs : 1;
+}
+
+// Launch plan: ring depth and metadata slots within one SM's shared memory; one CTA per SM (or
+// per tile when there are fewer tiles than SMs), the SMs shared out over the K slices.
+bool plan_decode_stream(int64_t M, int64_t N, int64_t K, DecodePlan* p) {
+    if (M < 1 || M > DS_MAXM || N < 8 || K < 128 || K % 128 != 0 || K > 65536 || N % 8 != 0) return false;
+    const int G = (int)(K / 128);
+    const int NC = (G + DS_SG - 1) / DS_SG;
+    const int64_t T = (N + 15) / 16;
+    const int sms = device_sm_count();
+    const int ncs = ds_split_stages(M, K);
+    const int ks = ncs ? (NC + ncs - 1) / ncs : 1;
+    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(T, sms / ks));
+    const int64_t tpc = (T + grid - 1) / grid;  // tiles of the largest CTA
+    const int units = (int)std::min<int64_t>(tpc * (ncs ? ncs : NC), DS_MAXNS);
+    const int nms = ncs ? 0 : ds_nms(tpc, NC);
+    const int ns = std::min(ds_fit(M, K, ncs, nms), units);
+    if (ns < std::min(DS_MINNS, units) || ns < 1) return false;
+    p->sg = DS_SG;
+    p->mt = ds_mt(M);
+    p->ns = ns;
+    p->nms = ncs ? ns : nms;
+    p->ks = ks;
+    p->ncs = ncs;
+    p->n_tiles = (int)T;
+    p->grid = grid;
+    const int KL = ncs ? ncs * DS_SG * 128 : (int)K;
+    p->smem = ds_layout(DS_SG, p->mt, (int)M, KL, ns, p->nms, ncs > 0).total + 1024;
+    return true;
+}
+
+size_t decode_stream_workspace(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || N < 1 || K < 128 || K % 128 != 0) return 0;
+    // launches of up to 8 rows; each takes its slices' fp32 partials from the start of the workspace
+    size_t need = 0;
+    for (int64_t mc : {std::min<int64_t>(M, DS_MAXM), M % DS_MAXM}) {
+        if (mc < 1) continue;
+        const int ks = decode_stream_slices(mc, K);
+        if (ks > 1) need = std::max(need, (size_t)ks * (size_t)mc * (size_t)N * 4);
+    }
+    return need;
+}
+
+template <int MT, bool KS>
+static cudaError_t ds_launch(const CUtensorMap& tm, const CUtensorMap& tmS, const CUtensorMap& tmZ, const uint16_t* X,
+                             int64_t M, int64_t N, int64_t K, const uint16_t* scales, const uint8_t* zeros, uint16_t* Y,
+                             float* P, const DecodePlan& p, bool weights_static, int* status, cudaStream_t stream) {
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
     int dev = 0;
@@ -485,12 +564,12 @@ static cudaError_t ds_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&]() {
-        attr_err[dev] = cudaFuncSetAttribute(decode_stream_kernel<MT, SG>,
+        attr_err[dev] = cudaFuncSetAttribute(decode_stream_kernel<MT, DS_SG, KS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DS_FULL_SMEM);
     });
     if (attr_err[dev] != cudaSuccess) return attr_err[dev];
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.grid, 1, 1);
+    cfg.gridDim = dim3((unsigned)p.grid, (unsigned)p.ks, 1);
     cfg.blockDim = dim3(DS_THREADS, 1, 1);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = stream;
@@ -499,33 +578,49 @@ static cudaError_t ds_launch(const CUtensorMap& tm, const uint16_t* X, int64_t M
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = weights_static ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<MT, SG>, tm, reinterpret_cast<const __half*>(X),
-                              reinterpret_cast<const unsigned short*>(scales), zeros, reinterpret_cast<__half*>(Y),
-                              (int)M, (int)N, (int)K, p.n_tiles, p.ns, p.nms, weights_static ? 1 : 0, status);
+    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<MT, DS_SG, KS>, tm, tmS, tmZ,
+                              reinterpret_cast<const __half*>(X), reinterpret_cast<const unsigned short*>(scales),
+                              zeros, reinterpret_cast<__half*>(Y), P, (int)M, (int)N, (int)K, p.n_tiles, p.ns, p.nms,
+                              p.ncs, weights_static ? 1 : 0, status);
 }
 
-template <int SG>
-static cudaError_t ds_launch_mt(const CUtensorMap& tm, const uint16_t* X, int64_t M, int64_t N, int64_t K,
-                                const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, const DecodePlan& p,
-                                bool weights_static, int* status, cudaStream_t stream) {
+template <bool KS>
+static cudaError_t ds_launch_mt(const CUtensorMap& tm, const CUtensorMap& tmS, const CUtensorMap& tmZ,
+                                const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint16_t* scales,
+                                const uint8_t* zeros, uint16_t* Y, float* P, const DecodePlan& p, bool weights_static,
+                                int* status, cudaStream_t stream) {
     switch (p.mt) {
-        case 1: return ds_launch<1, SG>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
-        case 2: return ds_launch<2, SG>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
-        case 4: return ds_launch<4, SG>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
-        default: return ds_launch<8, SG>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
+        case 1: return ds_launch<1, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
+        case 2: return ds_launch<2, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
+        case 4: return ds_launch<4, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
+        default: return ds_launch<8, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
     }
 }
 
 cudaError_t launch_decode_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                                 const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, bool weights_static,
-                                 int* status, cudaStream_t stream) {
+                                 const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, void* ws,
+                                 bool weights_static, int* status, cudaStream_t stream) {
     DecodePlan p;
     if (!plan_decode_stream(M, N, K, &p)) return cudaErrorInvalidValue;
     CUtensorMap tm;  // packed rows as 8-byte elements: a box of 8 SG elements is one stage's share of a row
     if (!make_tensor_map_2d(&tm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)(K / 16), (uint64_t)N,
                             (uint32_t)(8 * p.sg), 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    return ds_launch_mt<32>(tm, X, M, N, K, scales, zeros, Y, p, weights_static, status, stream);
+    if (p.ks == 1) return ds_launch_mt<false>(tm, tm, tm, X, M, N, K, scales, zeros, Y, nullptr, p, weights_static,
+                                              status, stream);
+    // split mode: [16][SG] boxes of the scales and zero points, fp32 partials in ws, then their sum
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15)) return cudaErrorInvalidValue;
+    CUtensorMap tmS, tmZ;
+    const uint64_t G = (uint64_t)(K / 128);
+    if (!make_tensor_map_2d(&tmS, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, G, (uint64_t)N, (uint32_t)p.sg, 16,
+                            CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tensor_map_2d(&tmZ, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, G, (uint64_t)N, (uint32_t)p.sg, 16,
+                            CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    float* P = static_cast<float*>(ws);
+    cudaError_t e = ds_launch_mt<true>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
+    if (e != cudaSuccess) return e;
+    return launch_splitk_reduce(P, p.ks, M * N, Y, stream);
 }
 
 }  // namespace w4

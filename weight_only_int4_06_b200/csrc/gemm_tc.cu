@@ -107,9 +107,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     const int m0 = mt * C::kBM, n0 = nt * BN;
     const int G = K >> 7;
-    // this CTA's k-blocks [kb0, kb0 + nk): two per group of 128, a slice starts on a group
-    const int kb0 = 2 * (int)(((int64_t)slice * G) / (ksplit > 1 ? ksplit : 1));
-    const int nk = 2 * (int)(((int64_t)(slice + 1) * G) / (ksplit > 1 ? ksplit : 1)) - kb0;
+    // this CTA's k-blocks [kb0, kb0 + nk): all K / 64 of them, or with ksplit > 1 (K a multiple of
+    // 128) two per group of 128, a slice starting on a group
+    const int kb0 = ksplit > 1 ? 2 * (int)(((int64_t)slice * G) / ksplit) : 0;
+    const int nk = ksplit > 1 ? 2 * (int)(((int64_t)(slice + 1) * G) / ksplit) - kb0 : K / TC_BK;
     if (ksplit > 1 && EPI == 2) Cf += (int64_t)slice * M * N;
 
     if (tid == 0) {
@@ -493,8 +494,12 @@ size_t tc_w4_workspace(int64_t M, int64_t N, int64_t K) {
     return s > 1 ? (size_t)s * (size_t)M * (size_t)N * 4 : 0;
 }
 
-// Y = fp16(sum over the slices of the fp32 partials, in slice order): deterministic.
+// Y = fp16(sum over the slices of the fp32 partials, in slice order): deterministic.  Launched as a
+// programmatic dependent of the kernel that writes the partials: it waits for that kernel's end
+// before reading them, and lets its own dependent start streaming weights meanwhile.
 __global__ void splitk_reduce_kernel(const float* __restrict__ P, int slices, int64_t mn, __half* __restrict__ Y) {
+    pdl_launch_dependents();
+    pdl_wait();
     const int64_t n4 = mn / 4;
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
         float4 a = reinterpret_cast<const float4*>(P)[e];
@@ -509,6 +514,23 @@ __global__ void splitk_reduce_kernel(const float* __restrict__ P, int slices, in
     }
 }
 
+cudaError_t launch_splitk_reduce(const float* P, int slices, int64_t mn, uint16_t* Y, cudaStream_t stream) {
+    if (mn % 4 != 0 || (reinterpret_cast<uintptr_t>(P) & 15) || (reinterpret_cast<uintptr_t>(Y) & 7))
+        return cudaErrorInvalidValue;
+    const int64_t want = (mn / 4 + 255) / 256;
+    const int64_t cap = (int64_t)device_sm_count() * 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(want < cap ? want : cap), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, splitk_reduce_kernel, P, slices, mn, reinterpret_cast<__half*>(Y));
+}
+
 cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                          const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, void* ws, int* status,
                          cudaStream_t stream) {
@@ -519,12 +541,7 @@ cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, con
         cudaError_t e = launch_tc<true, 2, 2, 256>(X, M, packed, N, K, scales, zeros, nullptr, nullptr, status,
                                                     stream, P, false, ks);
         if (e != cudaSuccess) return e;
-        const int64_t mn = M * N;
-        const int64_t want = (mn / 4 + 255) / 256;
-        const int64_t cap = (int64_t)device_sm_count() * 8;
-        splitk_reduce_kernel<<<(unsigned)(want < cap ? want : cap), 256, 0, stream>>>(
-            P, ks, mn, reinterpret_cast<__half*>(Y));
-        return cudaGetLastError();
+        return launch_splitk_reduce(P, ks, M * N, Y, stream);
     }
     int mt = 2, bn = 256;
     tc_w4_pick(M, N, &mt, &bn);

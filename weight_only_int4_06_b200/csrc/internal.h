@@ -40,15 +40,25 @@ struct DecodePlan {
     int sg;             // groups of 128 k per 16-row stage (32: 32 KB)
     int mt;             // activation-row bound of the instantiation: 1, 2, 4 or 8
     int ns;             // ring stages
-    int nms;            // metadata slots
-    int n_tiles;        // 16-row tiles in all (balanced over the CTAs)
-    int grid;           // CTAs
+    int nms;            // metadata slots (split mode: one per ring stage)
+    int ks;             // K slices (1: K is not cut)
+    int ncs;            // stages per K slice (0 when K is not cut)
+    int n_tiles;        // 16-row tiles in all (balanced over the CTAs of each slice)
+    int grid;           // CTAs per K slice
     uint32_t smem;      // dynamic shared memory per CTA
 };
 bool plan_decode_stream(int64_t M, int64_t N, int64_t K, DecodePlan* plan);  // false: shape not served
+// K slices of one launch of M <= 8 rows (1: K is not cut; then a second, reducing launch follows).
+int decode_stream_slices(int64_t M, int64_t K);
+// Bytes of fp32 partials a w4_gemm call of M rows on this path needs (0 when K is never cut); the
+// function of M, N and K alone.
+size_t decode_stream_workspace(int64_t M, int64_t N, int64_t K);
+// ws: decode_stream_workspace(M, N, K) bytes, 16-byte aligned (may be null when that is 0).
 cudaError_t launch_decode_stream(const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                                 const uint16_t* scales, const uint8_t* zeros, uint16_t* Y,
+                                 const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, void* ws,
                                  bool weights_static, int* status, cudaStream_t stream);
+// Y [mn] fp16 = sum over `slices` fp32 partial arrays P [slices][mn], in slice order (mn % 4 == 0).
+cudaError_t launch_splitk_reduce(const float* P, int slices, int64_t mn, uint16_t* Y, cudaStream_t stream);
 
 // Decode GEMV for M <= 8 on tcgen05 with the weights as a TMEM operand (gemv_tc.cu).
 struct GemvTcPlan {
