@@ -74,18 +74,20 @@ __device__ __forceinline__ uint32_t quant_code(float v, const GroupQuant& p) {
 // Eight codes of an unclipped group packed into one word (lowest k in the lowest nibble).
 // Same codes as quant_code: on the zero-inclusive range rint(v / s16) + z is never below 0
 // (RN and rint are odd-symmetric and monotone, and z = rint(-lo / s16) is never clamped since
-// -lo / s16 <= 15 (1 + 2^-23)), so only the upper clamp remains; z joins the bias of rint_small
-// in one integer add, and nibbles are placed by adds (fields never overlap).  A group whose
-// scale overflowed has unspecified codes (its status is reported); adds keep them inside the
-// group's own words.
+// -lo / s16 <= 15 (1 + 2^-23)), so only the upper clamp remains.  It is taken on the biased sum
+// t = RN(v / s16) + 1.5 * 2^23 (see rint_small) against the float whose bit pattern is that of
+// 1.5 * 2^23 + 15 - z: both are positive floats of one binade, so the float minimum is the integer
+// minimum of the patterns.  The word is then sum_i (bits(t_i) - bits(1.5 * 2^23) + z) 16^i, formed
+// modulo 2^32 as (z - bits(1.5 * 2^23)) * 0x11111111 + sum_i bits(t_i) 16^i: every field lies in
+// [0, 15], so the modular sum has the fields of the exact one.  A group whose scale overflowed
+// has unspecified codes (its status is reported); the arithmetic keeps them inside the word.
 __device__ __forceinline__ uint32_t quant_pack8_rtn(const float (&v)[8], const GroupQuant& p) {
-    const int zoff = p.z - 0x4B400000;  // bit pattern of 1.5 * 2^23, see rint_small
-    uint32_t word = 0;
+    const float top = __int_as_float(0x4B400000 + 15 - p.z);
+    uint32_t word = (uint32_t)(p.z - 0x4B400000) * 0x11111111u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float t = __fadd_rn(div_rn_from_rcp(v[i], p.sf, p.rcp), 12582912.0f);
-        const int q = min(__float_as_int(t) + zoff, 15);
-        word += (uint32_t)q << (4 * i);
+        const float t = fminf(__fadd_rn(div_rn_from_rcp(v[i], p.sf, p.rcp), 12582912.0f), top);
+        word += __float_as_uint(t) * (1u << (4 * i));
     }
     return word;
 }
