@@ -94,3 +94,42 @@ def test_host_batch_graph_replay_matches():
             ref = B.w4_gemm(torch.from_numpy(X if rep == 0 else -X).cuda(), *weights[i]).cpu()
             assert torch.equal(batch.y(i), ref), (rep, shapes[i])
     assert B.w4_check_device_status() == 0
+
+
+@pytest.mark.parametrize("pinned", [False, True])
+def test_host_batch_pageable_and_ragged_buffers(pinned):
+    """Host buffers the SMs cannot address (pageable), or whose sizes are not 16-byte multiples,
+    go through the copy engines; pinned 16-byte multiples through the SM copies: same bits."""
+    import ctypes
+    shapes = [(1, 1152, 520), (3, 512, 136)]  # 2304 + 3072 bytes of X: y_bytes 1040 + 816 = 1856
+    weights, Xs = [], []
+    for i, (M, K, N) in enumerate(shapes):
+        X, W = synth.layer_case(58 + i, M, K, N)
+        weights.append(B.w4_quantize_pack(torch.from_numpy(W).cuda()))
+        Xs.append(X)
+    x_off = [0, 2304]
+    y_off = [0, 1040]
+    x_bytes, y_bytes = 2304 + 3072, 1040 + 816 + 8  # y_bytes not a multiple of 16
+    xh = torch.zeros(x_bytes, dtype=torch.uint8)
+    yh = torch.zeros(y_bytes, dtype=torch.uint8)
+    if pinned:
+        xh, yh = xh.pin_memory(), yh.pin_memory()
+    for i, X in enumerate(Xs):
+        xh[x_off[i]:x_off[i] + X.nbytes].copy_(torch.from_numpy(X.view(np.uint8).reshape(-1)))
+    xd = torch.empty(x_bytes, dtype=torch.uint8, device="cuda")
+    yd = torch.empty(y_bytes, dtype=torch.uint8, device="cuda")
+    arr = (B.GemmLayer * 2)()
+    for i, ((p, s, z), (M, K, N)) in enumerate(zip(weights, shapes)):
+        arr[i] = B.GemmLayer(M, N, K, p.data_ptr(), s.data_ptr(), z.data_ptr(), x_off[i], y_off[i])
+    st = B.lib().w4_gemm_host_batch(ctypes.cast(arr, ctypes.c_void_p), 2, 128, ctypes.c_void_p(xh.data_ptr()),
+                                    ctypes.c_void_p(xd.data_ptr()), ctypes.c_size_t(x_bytes),
+                                    ctypes.c_void_p(yh.data_ptr()), ctypes.c_void_p(yd.data_ptr()),
+                                    ctypes.c_size_t(y_bytes), None, ctypes.c_size_t(0), 0,
+                                    ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    torch.cuda.current_stream().synchronize()
+    for i, (M, K, N) in enumerate(shapes):
+        got = yh[y_off[i]:y_off[i] + 2 * M * N].view(torch.float16).view(M, N)
+        ref = B.w4_gemm(torch.from_numpy(Xs[i]).cuda(), *weights[i]).cpu()
+        assert torch.equal(got, ref), shapes[i]
+    assert B.w4_check_device_status() == 0

@@ -290,7 +290,11 @@ def test_gemm_tc_ragged(M, K, N):
                                    # K cut into slices: one stage each (the last one partial), two
                                    # stages each, seven; half tiles (N % 16 == 8)
                                    (8, 6144, 264), (8, 10240, 1032), (3, 16384, 136), (6, 28672, 520),
-                                   (1, 28672, 4104)])
+                                   (1, 28672, 4104),
+                                   # 16-row launches: one slice (Y written directly), slices of 2048,
+                                   # 3 slices with a ragged N, 14 slices; 16 + 8 and 16 + 16 rows
+                                   (16, 2048, 520), (9, 4096, 264), (13, 6144, 1032), (16, 28672, 136),
+                                   (24, 8192, 264), (32, 4096, 136), (12, 1536, 136)])
 def test_gemm_gemv_ragged(M, K, N):
     X, p, s, z = oracle_case(28, M, K, N)
     assert_close(gpu_gemm(X, p, s, z, B.VARIANT_GEMV), oracle.gemm(X, p, s, z), f"gemv {M}x{K}x{N}")

@@ -85,14 +85,15 @@ w4_status gemm_plan(int64_t M, int64_t N, int64_t K, int family, bool meta_align
         return W4_OK;
     }
     DecodePlan dplan;
-    const bool gemv_fits = plan_decode_stream(M < 8 ? M : 8, N, K, &dplan);
+    const int64_t rows = decode_stream_rows(M, K);  // activation rows per GEMV launch
+    const bool gemv_fits = plan_decode_stream(M < rows ? M : rows, N, K, &dplan);
     if (family == W4_VARIANT_GEMV && !gemv_fits) return W4_ERR_SHAPE;
     if (family == W4_VARIANT_GEMV && !meta_aligned) return W4_ERR_ALIGN;
     if (family == W4_VARIANT_GEMV || (family == W4_VARIANT_AUTO && M <= 32 && gemv_fits && meta_aligned)) {
         *chosen = W4_VARIANT_GEMV;
         *launches = 0;
-        for (int64_t m0 = 0; m0 < M; m0 += 8)  // launches of up to 8 rows, each + 1 when K is cut
-            *launches += decode_stream_slices(M - m0 < 8 ? M - m0 : 8, K) > 1 ? 2 : 1;
+        for (int64_t m0 = 0; m0 < M; m0 += rows)  // launches of up to `rows` rows, each + 1 when K is cut
+            *launches += decode_stream_slices(M - m0 < rows ? M - m0 : rows, K) > 1 ? 2 : 1;
         return W4_OK;
     }
     SkinnyPlan plan;
@@ -183,9 +184,11 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
         return W4_OK;
     }
     if (chosen == W4_VARIANT_GEMV) {
-        // up to 8 activation rows per launch (token-by-token decode has M == 1)
-        for (int64_t m0 = 0; m0 < M; m0 += 8) {
-            const int64_t mc = (M - m0) < 8 ? (M - m0) : 8;
+        // up to 16 activation rows per launch (8 where the 16-row instantiation cannot serve K;
+        // token-by-token decode has M == 1)
+        const int64_t rows = decode_stream_rows(M, K);
+        for (int64_t m0 = 0; m0 < M; m0 += rows) {
+            const int64_t mc = (M - m0) < rows ? (M - m0) : rows;
             cudaError_t e = launch_decode_stream(X + m0 * K, mc, N, K, packed, scales, zeros, Y + m0 * N, ws,
                                                  weights_static, status, s);
             if (e != cudaSuccess) return W4_ERR_CUDA;
@@ -278,8 +281,16 @@ w4_status w4_gemm_host_batch(const w4_gemm_layer* layers, int n_layers, int grou
         if (st != W4_OK) return st;
     }
     cudaStream_t s = (cudaStream_t)stream;
-    if (x_bytes > 0 && cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return W4_ERR_CUDA;
+    // Pinned, mapped host buffers (16-byte multiples) are copied by the SMs: one PCIe round trip
+    // each way, chained to the GEMMs by programmatic dependent launch; other host memory through
+    // the copy engines.
+    const void* xh = x_bytes % 16 == 0 ? mapped_host_address(x_host) : nullptr;
+    void* yh = y_bytes % 16 == 0 ? mapped_host_address(y_host) : nullptr;
+    if (x_bytes > 0) {
+        const cudaError_t e = xh && aligned16(xh) ? launch_host_copy(xh, x_dev, x_bytes, false, s)
+                                                  : cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return W4_ERR_CUDA;
+    }
     for (int i = 0; i < n_layers; ++i) {
         const w4_gemm_layer& L = layers[i];
         const w4_status st =
@@ -289,8 +300,11 @@ w4_status w4_gemm_host_batch(const w4_gemm_layer* layers, int n_layers, int grou
                        stream);
         if (st != W4_OK) return st;
     }
-    if (y_bytes > 0 && cudaMemcpyAsync(y_host, y_dev, y_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        return W4_ERR_CUDA;
+    if (y_bytes > 0) {
+        const cudaError_t e = yh && aligned16(yh) ? launch_host_copy(y_dev, yh, y_bytes, true, s)
+                                                  : cudaMemcpyAsync(y_host, y_dev, y_bytes, cudaMemcpyDeviceToHost, s);
+        if (e != cudaSuccess) return W4_ERR_CUDA;
+    }
     return W4_OK;
 }
 

@@ -54,7 +54,7 @@ constexpr int DS_CW = 16;                           // consumer warps (then a pr
 constexpr int DS_PWARP = DS_CW;                     // producer warp
 constexpr int DS_RWARP = DS_CW + 1;                 // reducer warp
 constexpr int DS_THREADS = 32 * (DS_CW + 2);
-constexpr int DS_MAXM = 8;
+constexpr int DS_MAXM = 16;
 constexpr int DS_MAXNS = 24;                        // ring stages at most
 constexpr int DS_MINNS = 2;                         // ring stages at least
 constexpr int DS_MAXMS = 4;                         // metadata slots at most
@@ -171,7 +171,47 @@ __device__ __forceinline__ void ds_group(uint32_t a_addr, uint32_t b_addr, uint3
 
 // KS (split mode): blockIdx.y is a K slice of `ncs` whole stages; the CTA stages the activations of
 // its slice only, every stage brings its own scales and zero points (two 2-D TMA boxes of 16 rows x
-// SG groups), and the reducer writes fp32 partial sums to P [slice][M][N] instead of Y.
+// SG groups), and with several slices the reducer writes fp32 partial sums to P [slice][M][N]
+// instead of Y (P null: one slice, Y directly).
+// MT == 16: the same for two column blocks (activation rows 0-7 and 8-15) that share every
+// dequantised A fragment; one accumulation chain per block.  acc: rows (g8, g8+8) x cols
+// (2c, 2c+1) of block 0, then of block 1.
+__device__ __forceinline__ void ds_group16(uint32_t a_addr, uint32_t b_addr, uint32_t xg0, uint32_t xg1,
+                                           const uint32_t (&xofs)[4], bool x0, bool x1, uint32_t corr0,
+                                           uint32_t corr1, float fsa, float fsb, float fza, float fzb,
+                                           float (&acc)[8]) {
+    const uint4 A = lds128(a_addr);
+    const uint4 B = lds128(b_addr);
+    float c0[4] = {0.0f, 0.0f, 0.0f, 0.0f}, c1[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const uint32_t wA[4] = {A.x, A.y, A.z, A.w};
+    const uint32_t wB[4] = {B.x, B.y, B.z, B.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t a = wA[j], b = wB[j], a8 = a >> 8, b8 = b >> 8;
+        const uint4 xf0 = x0 ? lds128(xg0 + xofs[j]) : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 xf1 = x1 ? lds128(xg1 + xofs[j]) : make_uint4(0u, 0u, 0u, 0u);
+        uint32_t f0 = lop3_and_or(a, 0x000F000Fu, 0x64006400u), f1 = lop3_and_or(b, 0x000F000Fu, 0x64006400u);
+        uint32_t f2 = lop3_and_or(a, 0x00F000F0u, 0x64006400u), f3 = lop3_and_or(b, 0x00F000F0u, 0x64006400u);
+        mma_16816(c0, f0, f1, f2, f3, xf0.x, xf0.y);
+        mma_16816(c1, f0, f1, f2, f3, xf1.x, xf1.y);
+        f0 = lop3_and_or(a8, 0x000F000Fu, 0x64006400u);
+        f1 = lop3_and_or(b8, 0x000F000Fu, 0x64006400u);
+        f2 = lop3_and_or(a8, 0x00F000F0u, 0x64006400u);
+        f3 = lop3_and_or(b8, 0x00F000F0u, 0x64006400u);
+        mma_16816(c0, f0, f1, f2, f3, xf0.z, xf0.w);
+        mma_16816(c1, f0, f1, f2, f3, xf1.z, xf1.w);
+    }
+    const uint4 u = lds128(corr0), v = lds128(corr1);
+    acc[0] = fmaf(fsa, c0[0] - fmaf(fza, __uint_as_float(u.y), __uint_as_float(u.x)), acc[0]);
+    acc[1] = fmaf(fsa, c0[1] - fmaf(fza, __uint_as_float(u.w), __uint_as_float(u.z)), acc[1]);
+    acc[2] = fmaf(fsb, c0[2] - fmaf(fzb, __uint_as_float(u.y), __uint_as_float(u.x)), acc[2]);
+    acc[3] = fmaf(fsb, c0[3] - fmaf(fzb, __uint_as_float(u.w), __uint_as_float(u.z)), acc[3]);
+    acc[4] = fmaf(fsa, c1[0] - fmaf(fza, __uint_as_float(v.y), __uint_as_float(v.x)), acc[4]);
+    acc[5] = fmaf(fsa, c1[1] - fmaf(fza, __uint_as_float(v.w), __uint_as_float(v.z)), acc[5]);
+    acc[6] = fmaf(fsb, c1[2] - fmaf(fzb, __uint_as_float(v.y), __uint_as_float(v.x)), acc[6]);
+    acc[7] = fmaf(fsb, c1[3] - fmaf(fzb, __uint_as_float(v.w), __uint_as_float(v.z)), acc[7]);
+}
+
 template <int MT, int SG, bool KS>
 __global__ void __launch_bounds__(DS_THREADS, 1)
     decode_stream_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmS,
@@ -291,7 +331,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
         pdl_wait();  // Y may be read by the preceding kernel
         int rs = 0;
         uint32_t rph = 0;
-        float* Pl = KS ? P + (int64_t)blockIdx.y * M * N : nullptr;  // this slice's partials
+        float* Pl = KS && P ? P + (int64_t)blockIdx.y * M * N : nullptr;  // this slice's partials
         for (int t = t0; t < t1; ++t) {
             if (!mbar_wait_bounded(tile_full(rs), rph, abort_flag)) {
                 *abort_flag = 1;
@@ -307,7 +347,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
                     float sum = 0.0f;
 #pragma unroll
                     for (int w = 0; w < DS_CW; ++w) sum += rsl[w * (16 * MT) + o];
-                    if (KS)
+                    if (KS && P)
                         Pl[(int64_t)m * N + n] = sum;
                     else
                         Y[(int64_t)m * N + n] = __float2half_rn(sum);
@@ -383,17 +423,32 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
     const int g8 = lane >> 2, c = lane & 3;
     const bool xlane = g8 < M;  // B column g8 holds activation row g8; other lanes use zeros
     const uint32_t xrow = xs_u + (uint32_t)(xlane ? g8 : 0) * (uint32_t)RS * 2u;
+    const bool xlane1 = MT == 16 && g8 + 8 < M;  // MT == 16: column g8 of block 1 is row g8 + 8
+    const uint32_t xrow1 = xs_u + (uint32_t)(xlane1 ? g8 + 8 : 0) * (uint32_t)RS * 2u;
     uint32_t xofs[4];  // swizzled byte offset of word j's chunk within a group, for this lane
 #pragma unroll
     for (int j = 0; j < 4; ++j) xofs[j] = (uint32_t)ds_swz(c * 4 + j) * 16u;
     const int ccol = 2 * c < MT ? 2 * c : 0;  // first activation column of this thread's C pair
     // metadata of the warp's groups is vector-aligned (always in split mode: rows of SG groups)
-    const bool mvec = KS || (G % GPW) == 0;
+    const bool mvec = GPW >= 2 && (KS || (G % GPW) == 0);
     // this thread's W bytes inside a stage: rows g8 and g8 + 8 of the warp's groups, 16 bytes at 16 c
     const uint32_t wlane = (uint32_t)(g8 * ROWB + warp * GPW * 64 + c * 16);
     int s = 0, kc = 0, ms = 0, rs = 0;
     uint32_t ph = 0, rph = 0;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};  // rows (g8, g8+8) x cols (2c, 2c+1)
+    constexpr int NACC = MT == 16 ? 8 : 4;
+    float acc[NACC];  // rows (g8, g8+8) x cols (2c, 2c+1) [of block 0, then block 1]
+#pragma unroll
+    for (int i = 0; i < NACC; ++i) acc[i] = 0.0f;
+    // one group e of the current stage
+    auto group = [&](uint32_t st, uint32_t xg, uint32_t xg1, int gle, float fsa, float fsb, float fza, float fzb) {
+        if constexpr (MT == 16) {
+            ds_group16(st, st + 8 * ROWB, xg, xg1, xofs, xlane, xlane1, corr_u + (uint32_t)(gle * 16 + 2 * c) * 8u,
+                       corr_u + (uint32_t)(gle * 16 + 8 + 2 * c) * 8u, fsa, fsb, fza, fzb, acc);
+        } else {
+            ds_group<MT>(st, st + 8 * ROWB, xg, xofs, xlane, corr_u + (uint32_t)(gle * MT + ccol) * 8u, fsa, fsb,
+                         fza, fzb, acc);
+        }
+    };
     bool dead = false;
     for (int u = 0; u < n_units; ++u) {
         // After a timeout every wait is skipped; the loop still runs to the end.
@@ -407,32 +462,33 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
         const int ng = g0 >= G ? 0 : min(GPW, G - g0);
         if (!dead && ng > 0) {
             const uint32_t st = sbase + L.ring + (uint32_t)s * STAGE_BYTES + wlane;
-            const uint32_t xg = xrow + (uint32_t)gl0 * 256u;
+            const uint32_t xg = xrow + (uint32_t)gl0 * 256u, xg1 = xrow1 + (uint32_t)gl0 * 256u;
             // scales [16][mG] fp16, then zeros [16][mG] u8: the tile's (mG = K/128) or the stage's (mG = SG)
             const uint32_t mG = KS ? (uint32_t)SG : (uint32_t)G;
             const uint32_t msa = sbase + L.meta + (uint32_t)(KS ? s : ms) * L.mslot;
             const uint32_t mza = msa + 32u * mG;
             const uint32_t ia = g8 * mG + (uint32_t)(KS ? warp * GPW : g0), ib = ia + 8u * mG;
             if (ng == GPW && mvec) {
-                // the scales and zero points of the warp's groups, packed: GPW fp16 and GPW bytes per row
-                uint32_t sa[GPW / 2], sb[GPW / 2], za, zb;
-                if constexpr (GPW == 4) {
-                    const uint2 va = lds64(msa + 2u * ia), vb = lds64(msa + 2u * ib);
-                    sa[0] = va.x; sa[1] = va.y; sb[0] = vb.x; sb[1] = vb.y;
-                    za = lds32(mza + ia);
-                    zb = lds32(mza + ib);
-                } else {
-                    sa[0] = lds32(msa + 2u * ia);
-                    sb[0] = lds32(msa + 2u * ib);
-                    za = lds_u16(mza + ia);
-                    zb = lds_u16(mza + ib);
-                }
+                if constexpr (GPW >= 2) {
+                    // the scales and zero points of the warp's groups, packed: GPW fp16 and GPW bytes per row
+                    uint32_t sa[GPW / 2], sb[GPW / 2], za, zb;
+                    if constexpr (GPW == 4) {
+                        const uint2 va = lds64(msa + 2u * ia), vb = lds64(msa + 2u * ib);
+                        sa[0] = va.x; sa[1] = va.y; sb[0] = vb.x; sb[1] = vb.y;
+                        za = lds32(mza + ia);
+                        zb = lds32(mza + ib);
+                    } else {
+                        sa[0] = lds32(msa + 2u * ia);
+                        sb[0] = lds32(msa + 2u * ib);
+                        za = lds_u16(mza + ia);
+                        zb = lds_u16(mza + ib);
+                    }
 #pragma unroll
-                for (int e = 0; e < GPW; ++e) {
-                    const float fsa = ds_half(sa[e >> 1], e & 1), fsb = ds_half(sb[e >> 1], e & 1);
-                    const float fza = (float)((za >> (8 * e)) & 0xFFu), fzb = (float)((zb >> (8 * e)) & 0xFFu);
-                    ds_group<MT>(st + e * 64, st + e * 64 + 8 * ROWB, xg + e * 256, xofs, xlane,
-                                 corr_u + (uint32_t)((gl0 + e) * MT + ccol) * 8u, fsa, fsb, fza, fzb, acc);
+                    for (int e = 0; e < GPW; ++e) {
+                        const float fsa = ds_half(sa[e >> 1], e & 1), fsb = ds_half(sb[e >> 1], e & 1);
+                        const float fza = (float)((za >> (8 * e)) & 0xFFu), fzb = (float)((zb >> (8 * e)) & 0xFFu);
+                        group(st + e * 64, xg + e * 256, xg1 + e * 256, gl0 + e, fsa, fsb, fza, fzb);
+                    }
                 }
             } else {
                 for (int e = 0; e < ng; ++e) {
@@ -440,8 +496,7 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
                     const float fsb = __half2float(__ushort_as_half(lds_u16(msa + 2u * (ib + e))));
                     const float fza = (float)lds_u8(mza + ia + e);
                     const float fzb = (float)lds_u8(mza + ib + e);
-                    ds_group<MT>(st + e * 64, st + e * 64 + 8 * ROWB, xg + e * 256, xofs, xlane,
-                                 corr_u + (uint32_t)((gl0 + e) * MT + ccol) * 8u, fsa, fsb, fza, fzb, acc);
+                    group(st + e * 64, xg + e * 256, xg1 + e * 256, gl0 + e, fsa, fsb, fza, fzb);
                 }
             }
         }
@@ -460,18 +515,28 @@ __global__ void __launch_bounds__(DS_THREADS, 1)
             float* mine = red + (size_t)rs * (DS_CW * 16 * MT) + warp * (16 * MT);
             if (2 * c < MT) { mine[g8 * MT + 2 * c] = acc[0]; mine[(g8 + 8) * MT + 2 * c] = acc[2]; }
             if (2 * c + 1 < MT) { mine[g8 * MT + 2 * c + 1] = acc[1]; mine[(g8 + 8) * MT + 2 * c + 1] = acc[3]; }
+            if constexpr (MT == 16) {
+                mine[g8 * 16 + 8 + 2 * c] = acc[4];
+                mine[g8 * 16 + 9 + 2 * c] = acc[5];
+                mine[(g8 + 8) * 16 + 8 + 2 * c] = acc[6];
+                mine[(g8 + 8) * 16 + 9 + 2 * c] = acc[7];
+            }
             mbar_arrive(tile_full(rs));  // every lane: its own stores are released with it
             if (++rs == DS_RSLOTS) { rs = 0; rph ^= 1; }
-            acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < NACC; ++i) acc[i] = 0.0f;
             kc = 0;
         }
     }
 }
 
 // ------------------------------------------------------------------------------------ host side
-static int ds_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
+static int ds_mt(int64_t M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16; }
 
-constexpr int DS_SG = 32;       // groups per stage (32 KB stages: every consumer warp takes two groups)
+// Groups per stage: 32 (32 KB stages, two groups per consumer warp); 16 for the 16-row
+// instantiation, whose 16 staged activation rows take twice the shared memory per k.
+static int ds_sg(int mt) { return mt == 16 ? 16 : 32; }
+
 constexpr int DS_GOOD_NS = 4;   // ring depth below which the plan cuts K into slices (when it may)
 
 // Metadata slots of the unsplit kernel: enough to run two tiles ahead of the consumers.
@@ -482,45 +547,66 @@ static int ds_nms(int64_t tpc, int NC) {
 // Ring stages that fit in one SM's shared memory with `ncs` stages of k staged per activation row
 // (split mode) or the whole K (ncs == 0, with nms metadata slots); 0 when not even DS_MINNS fit.
 static int ds_fit(int64_t M, int64_t K, int ncs, int nms) {
-    const int mt = ds_mt(M);
+    const int mt = ds_mt(M), sg = ds_sg(mt);
     const bool ks = ncs > 0;
-    const int KL = ks ? ncs * DS_SG * 128 : (int)K;
-    const uint32_t fixed = ds_layout(DS_SG, mt, (int)M, KL, 0, 0, ks).total + (ks ? 0u : (uint32_t)nms * 48u * (uint32_t)(K / 128)) +
-                           1024;  // alignment slack
-    const uint32_t per = ds_stage_bytes(DS_SG) + (ks ? ds_stage_meta_bytes(DS_SG) : 0u);
+    const int KL = ks ? ncs * sg * 128 : (int)K;
+    const uint32_t fixed = ds_layout(sg, mt, (int)M, KL, 0, 0, ks).total +
+                           (ks ? 0u : (uint32_t)nms * 48u * (uint32_t)(K / 128)) + 1024;  // alignment slack
+    const uint32_t per = ds_stage_bytes(sg) + (ks ? ds_stage_meta_bytes(sg) : 0u);
     if (fixed + (uint32_t)DS_MINNS * per > DS_FULL_SMEM) return 0;
     return (int)std::min<uint32_t>((DS_FULL_SMEM - fixed) / per, DS_MAXNS);
 }
 
-// Stages per K slice (0: K is not cut).  A function of M and K alone, so the workspace query needs
-// no device.  K is cut when the whole K leaves fewer than DS_GOOD_NS ring stages (or does not fit
-// at all) and the metadata rows allow 2-D TMA boxes (K/128 a multiple of 16: 16-byte row strides
-// of the zero points); the slices are equal (their count divides the stages of K), the longest
-// that leave DS_GOOD_NS stages, else one stage each.
+// Stages per K slice: 0 when K is not cut, -1 when the shape is not served.  A function of M and K
+// alone, so the workspace query needs no device.  Split mode needs 2-D TMA boxes of the metadata
+// rows (K/128 a multiple of 16: 16-byte row strides of the zero points); the slices are equal
+// (their count divides the stages of K), the longest that leave DS_GOOD_NS ring stages, else one
+// stage each.  Up to 8 rows, K is cut only when the whole K leaves fewer than DS_GOOD_NS stages;
+// the 16-row instantiation always runs in split mode (with a single slice where K fits whole).
 static int ds_split_stages(int64_t M, int64_t K) {
+    const int mt = ds_mt(M), sg = ds_sg(mt);
     const int G = (int)(K / 128);
-    const int NC = (G + DS_SG - 1) / DS_SG;
-    if (ds_fit(M, K, 0, ds_nms(DS_MAXMS, NC)) >= DS_GOOD_NS || G % 16 != 0 || NC < 2) return 0;
+    const int NC = (G + sg - 1) / sg;
+    if (mt == 16) {
+        if (G % 16 != 0) return -1;
+        for (int ncs = NC; ncs >= 1; --ncs)
+            if (NC % ncs == 0 && ds_fit(M, K, ncs, 0) >= DS_GOOD_NS) return ncs;
+        return ds_fit(M, K, 1, 0) > 0 ? 1 : -1;
+    }
+    const int whole = ds_fit(M, K, 0, ds_nms(DS_MAXMS, NC));
+    if (whole >= DS_GOOD_NS || G % 16 != 0 || NC < 2) return whole > 0 ? 0 : -1;
     for (int ncs = NC - 1; ncs >= 1; --ncs)
         if (NC % ncs == 0 && ds_fit(M, K, ncs, 0) >= DS_GOOD_NS) return ncs;
-    return ds_fit(M, K, 1, 0) > ds_fit(M, K, 0, ds_nms(DS_MAXMS, NC)) ? 1 : 0;
+    if (ds_fit(M, K, 1, 0) > whole) return 1;
+    return whole > 0 ? 0 : -1;
 }
 
 int decode_stream_slices(int64_t M, int64_t K) {
     const int ncs = ds_split_stages(M, K);
-    const int NC = (int)((K / 128 + DS_SG - 1) / DS_SG);
-    return ncs ? (NC + ncs - 1) / ncs : 1;
+    const int sg = ds_sg(ds_mt(M));
+    const int NC = (int)((K / 128 + sg - 1) / sg);
+    return ncs > 0 ? (NC + ncs - 1) / ncs : 1;
+}
+
+// 16-row launches where they measured faster than two 8-row launches on B200 (K = 8192,
+// N = 8192: 25.5 vs 28.0 us at M = 16, 49.2 vs 54.3 at M = 32; a tie at N = 28672); at K = 28672
+// the 16-row consumer's doubled per-byte work and 14 slices of partials make them slower (78.3 vs
+// 73.2 us at M = 16), so longer K stays with 8-row launches.
+int decode_stream_rows(int64_t M, int64_t K) {
+    return M > 8 && K >= 128 && K % 128 == 0 && K <= 8192 && ds_split_stages(16, K) > 0 ? 16 : 8;
 }
 
 // Launch plan: ring depth and metadata slots within one SM's shared memory; one CTA per SM (or
 // per tile when there are fewer tiles than SMs), the SMs shared out over the K slices.
 bool plan_decode_stream(int64_t M, int64_t N, int64_t K, DecodePlan* p) {
     if (M < 1 || M > DS_MAXM || N < 8 || K < 128 || K % 128 != 0 || K > 65536 || N % 8 != 0) return false;
+    const int mt = ds_mt(M), sg = ds_sg(mt);
     const int G = (int)(K / 128);
-    const int NC = (G + DS_SG - 1) / DS_SG;
+    const int NC = (G + sg - 1) / sg;
     const int64_t T = (N + 15) / 16;
     const int sms = device_sm_count();
     const int ncs = ds_split_stages(M, K);
+    if (ncs < 0) return false;
     const int ks = ncs ? (NC + ncs - 1) / ncs : 1;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>(T, sms / ks));
     const int64_t tpc = (T + grid - 1) / grid;  // tiles of the largest CTA
@@ -528,24 +614,26 @@ bool plan_decode_stream(int64_t M, int64_t N, int64_t K, DecodePlan* p) {
     const int nms = ncs ? 0 : ds_nms(tpc, NC);
     const int ns = std::min(ds_fit(M, K, ncs, nms), units);
     if (ns < std::min(DS_MINNS, units) || ns < 1) return false;
-    p->sg = DS_SG;
-    p->mt = ds_mt(M);
+    p->sg = sg;
+    p->mt = mt;
     p->ns = ns;
     p->nms = ncs ? ns : nms;
     p->ks = ks;
     p->ncs = ncs;
     p->n_tiles = (int)T;
     p->grid = grid;
-    const int KL = ncs ? ncs * DS_SG * 128 : (int)K;
-    p->smem = ds_layout(DS_SG, p->mt, (int)M, KL, ns, p->nms, ncs > 0).total + 1024;
+    const int KL = ncs ? ncs * sg * 128 : (int)K;
+    p->smem = ds_layout(sg, mt, (int)M, KL, ns, p->nms, ncs > 0).total + 1024;
     return true;
 }
 
 size_t decode_stream_workspace(int64_t M, int64_t N, int64_t K) {
     if (M < 1 || N < 1 || K < 128 || K % 128 != 0) return 0;
-    // launches of up to 8 rows; each takes its slices' fp32 partials from the start of the workspace
+    // launches of up to decode_stream_rows rows; each takes its slices' fp32 partials from the start
+    // of the workspace
+    const int64_t rows = decode_stream_rows(M, K);
     size_t need = 0;
-    for (int64_t mc : {std::min<int64_t>(M, DS_MAXM), M % DS_MAXM}) {
+    for (int64_t mc : {std::min<int64_t>(M, rows), M % rows}) {
         if (mc < 1) continue;
         const int ks = decode_stream_slices(mc, K);
         if (ks > 1) need = std::max(need, (size_t)ks * (size_t)mc * (size_t)N * 4);
@@ -553,7 +641,7 @@ size_t decode_stream_workspace(int64_t M, int64_t N, int64_t K) {
     return need;
 }
 
-template <int MT, bool KS>
+template <int MT, int SG, bool KS>
 static cudaError_t ds_launch(const CUtensorMap& tm, const CUtensorMap& tmS, const CUtensorMap& tmZ, const uint16_t* X,
                              int64_t M, int64_t N, int64_t K, const uint16_t* scales, const uint8_t* zeros, uint16_t* Y,
                              float* P, const DecodePlan& p, bool weights_static, int* status, cudaStream_t stream) {
@@ -564,7 +652,7 @@ static cudaError_t ds_launch(const CUtensorMap& tm, const CUtensorMap& tmS, cons
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&]() {
-        attr_err[dev] = cudaFuncSetAttribute(decode_stream_kernel<MT, DS_SG, KS>,
+        attr_err[dev] = cudaFuncSetAttribute(decode_stream_kernel<MT, SG, KS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DS_FULL_SMEM);
     });
     if (attr_err[dev] != cudaSuccess) return attr_err[dev];
@@ -578,7 +666,7 @@ static cudaError_t ds_launch(const CUtensorMap& tm, const CUtensorMap& tmS, cons
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = weights_static ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<MT, DS_SG, KS>, tm, tmS, tmZ,
+    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<MT, SG, KS>, tm, tmS, tmZ,
                               reinterpret_cast<const __half*>(X), reinterpret_cast<const unsigned short*>(scales),
                               zeros, reinterpret_cast<__half*>(Y), P, (int)M, (int)N, (int)K, p.n_tiles, p.ns, p.nms,
                               p.ncs, weights_static ? 1 : 0, status);
@@ -587,13 +675,18 @@ static cudaError_t ds_launch(const CUtensorMap& tm, const CUtensorMap& tmS, cons
 template <bool KS>
 static cudaError_t ds_launch_mt(const CUtensorMap& tm, const CUtensorMap& tmS, const CUtensorMap& tmZ,
                                 const uint16_t* X, int64_t M, int64_t N, int64_t K, const uint16_t* scales,
-                                const uint8_t* zeros, uint16_t* Y, float* P, const DecodePlan& p, bool weights_static,
+                                const uint8_t* zeros, uint16_t* Y, float* P, const DecodePlan& p, bool ws_,
                                 int* status, cudaStream_t stream) {
     switch (p.mt) {
-        case 1: return ds_launch<1, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
-        case 2: return ds_launch<2, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
-        case 4: return ds_launch<4, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
-        default: return ds_launch<8, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
+        case 1: return ds_launch<1, 32, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, ws_, status, stream);
+        case 2: return ds_launch<2, 32, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, ws_, status, stream);
+        case 4: return ds_launch<4, 32, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, ws_, status, stream);
+        case 8: return ds_launch<8, 32, KS>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, ws_, status, stream);
+        default:
+            if constexpr (KS)
+                return ds_launch<16, 16, true>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, ws_, status, stream);
+            else
+                return cudaErrorInvalidValue;  // the 16-row instantiation runs in split mode only
     }
 }
 
@@ -606,10 +699,10 @@ cudaError_t launch_decode_stream(const uint16_t* X, int64_t M, int64_t N, int64_
     if (!make_tensor_map_2d(&tm, packed, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, (uint64_t)(K / 16), (uint64_t)N,
                             (uint32_t)(8 * p.sg), 16, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    if (p.ks == 1) return ds_launch_mt<false>(tm, tm, tm, X, M, N, K, scales, zeros, Y, nullptr, p, weights_static,
-                                              status, stream);
-    // split mode: [16][SG] boxes of the scales and zero points, fp32 partials in ws, then their sum
-    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15)) return cudaErrorInvalidValue;
+    if (p.ncs == 0) return ds_launch_mt<false>(tm, tm, tm, X, M, N, K, scales, zeros, Y, nullptr, p, weights_static,
+                                               status, stream);
+    // split mode: [16][SG] boxes of the scales and zero points; with several slices fp32 partials
+    // in ws, then their sum
     CUtensorMap tmS, tmZ;
     const uint64_t G = (uint64_t)(K / 128);
     if (!make_tensor_map_2d(&tmS, scales, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, G, (uint64_t)N, (uint32_t)p.sg, 16,
@@ -617,6 +710,10 @@ cudaError_t launch_decode_stream(const uint16_t* X, int64_t M, int64_t N, int64_
         !make_tensor_map_2d(&tmZ, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, G, (uint64_t)N, (uint32_t)p.sg, 16,
                             CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
+    if (p.ks == 1)
+        return ds_launch_mt<true>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, nullptr, p, weights_static, status,
+                                  stream);
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15)) return cudaErrorInvalidValue;
     float* P = static_cast<float*>(ws);
     cudaError_t e = ds_launch_mt<true>(tm, tmS, tmZ, X, M, N, K, scales, zeros, Y, P, p, weights_static, status, stream);
     if (e != cudaSuccess) return e;

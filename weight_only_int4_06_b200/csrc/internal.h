@@ -35,10 +35,10 @@ cudaError_t launch_skinny(const uint16_t* X, int64_t M, int64_t N, int64_t K,
                           uint16_t* Y, const SkinnyPlan& plan, bool weights_static,
                           cudaStream_t stream);
 
-// Decode GEMV for M <= 8, one TMA-fed CTA per SM (decode_stream.cu).
+// Decode GEMV for M <= 16, one TMA-fed CTA per SM (decode_stream.cu).
 struct DecodePlan {
-    int sg;             // groups of 128 k per 16-row stage (32: 32 KB)
-    int mt;             // activation-row bound of the instantiation: 1, 2, 4 or 8
+    int sg;             // groups of 128 k per 16-row stage (32: 32 KB; 16 for mt = 16)
+    int mt;             // activation-row bound of the instantiation: 1, 2, 4, 8 or 16
     int ns;             // ring stages
     int nms;            // metadata slots (split mode: one per ring stage)
     int ks;             // K slices (1: K is not cut)
@@ -48,8 +48,11 @@ struct DecodePlan {
     uint32_t smem;      // dynamic shared memory per CTA
 };
 bool plan_decode_stream(int64_t M, int64_t N, int64_t K, DecodePlan* plan);  // false: shape not served
-// K slices of one launch of M <= 8 rows (1: K is not cut; then a second, reducing launch follows).
+// K slices of one launch of M <= 16 rows (> 1: a second, reducing launch follows).
 int decode_stream_slices(int64_t M, int64_t K);
+// Activation rows per launch of this path for a call of M rows: 16 where the 16-row
+// instantiation serves K, else 8.
+int decode_stream_rows(int64_t M, int64_t K);
 // Bytes of fp32 partials a w4_gemm call of M rows on this path needs (0 when K is never cut); the
 // function of M, N and K alone.
 size_t decode_stream_workspace(int64_t M, int64_t N, int64_t K);
@@ -146,6 +149,14 @@ cudaError_t launch_wb_gemm(const uint16_t* X, int64_t M, int64_t N, int64_t K, c
                            void* ws, int* status, cudaStream_t stream);
 cudaError_t launch_act_prepare(const uint16_t* X, int64_t M, int64_t K, const int32_t* perm, const float* s,
                                uint16_t* Xo, int* status, cudaStream_t stream);
+
+// SM-driven copies between pinned host memory and the device (host_copy.cu).
+// Device address of a pinned, mapped host buffer, or null (pageable, unknown or managed memory).
+void* mapped_host_address(const void* p);
+// bytes (a multiple of 16, both addresses 16-byte aligned) from src to dst, either of them a mapped
+// host address; after_prior: launched as a programmatic dependent of the preceding kernel, whose
+// end it awaits before reading.  The kernel lets its own dependent launch at once.
+cudaError_t launch_host_copy(const void* src, void* dst, size_t bytes, bool after_prior, cudaStream_t stream);
 
 // Self-test of the bounded waits (selftest.cu).
 cudaError_t launch_selftest_wait(uint64_t limit_ns, int* status, cudaStream_t stream);
