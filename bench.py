@@ -265,7 +265,8 @@ class GemmWorkload:
         every Y in one device-to-host copy), prepared once per weight set as a serving loop over
         fixed buffers would and captured as a CUDA graph (HostGemmBatch.capture) that each step
         replays; the copies move the host buffers' current contents at every replay.  The step
-        ends when the stream has drained (the results are then readable on the host)."""
+        ends when the stream has drained (the results are then readable on the host, in the
+        batch's pinned result buffer: `HostGemmBatch.y(i)` views it)."""
         import torch
         if self.host_calls is None:
             try:
@@ -286,7 +287,7 @@ class GemmWorkload:
             b = self.host_calls[c]
             self.host_graphs[c].replay()
             torch.cuda.current_stream().synchronize()
-            return [b.y(i) for i in range(len(self.layers))]
+            return b
         s = step % self.n_sets
         for L in self.layers:
             p, sc, z = L["copies"][s]

@@ -401,6 +401,7 @@ __global__ void __launch_bounds__(256) transpose_pad_kernel(const unsigned short
 // lower = 0: every entry).  One block row of the grid per row of G.
 __global__ void gram_accumulate_kernel(const float* __restrict__ Gc, int K, bool first, int lower,
                                        double* __restrict__ G64) {
+    pdl_launch_dependents();  // the next chunk's product (other Gc buffer) may start beside this
     for (int i = blockIdx.x; i < K; i += gridDim.x) {
         const int jn = lower ? i + 1 : K;
         const int64_t r = (int64_t)i * K;
@@ -488,6 +489,9 @@ __global__ void __launch_bounds__(256) awq_fakequant_scaled_kernel(const uint4* 
             if ((l16 == 0 && p.overflow) || bad) record_status(status, W4_ERR_RANGE);
         }
     }
+    // Launched as a programmatic dependent of the previous alpha's contraction (which reads the
+    // other E buffer): end only after it, so that the next contraction follows both.
+    pdl_wait();
 }
 
 AwqGramLayout awq_gram_layout(int64_t T, int64_t N, int64_t K, int n_alpha) {
@@ -499,10 +503,10 @@ AwqGramLayout awq_gram_layout(int64_t T, int64_t N, int64_t K, int n_alpha) {
     size_t off = 0;
     L.colsum = off; off = align256(off + (size_t)K * 8);
     L.s_all = off; off = align256(off + (size_t)n_alpha * K * 4);
-    L.E = off; off = align256(off + (size_t)N * K * 2);
+    L.E = off; off = align256(off + 2 * (size_t)N * K * 2);  // two buffers: alpha i writes E[i % 2]
     L.part = off; off = align256(off + (size_t)n_alpha * L.n_part * 8);
     L.XT = off; off = align256(off + (size_t)K * (size_t)L.Tp * 2);
-    L.G = off; off = align256(off + (size_t)K * K * 4);
+    L.G = off; off = align256(off + 2 * (size_t)K * K * 4);  // two buffers: chunk c writes G[c % 2]
     L.G64 = off; off = align256(off + (size_t)K * K * 8);
     L.Gp = off; off = align256(off + (size_t)K * K * 2);
     L.d = off; off = align256(off + (size_t)K * 4);
@@ -544,12 +548,17 @@ cudaError_t launch_awq_gram(const uint16_t* X, int64_t T, const uint16_t* W, int
     // G is symmetric: for K > 128 only the 256 x 256 tiles on and below the diagonal are formed
     // (half the tensor-core work, one wave at K = 4096), accumulated and read back mirrored.
     const int lower = K > 128 ? 1 : 0;
-    for (int64_t c = 0; c < L.n_chunks; ++c) {  // G = sum over chunks of X_c^T X_c
+    // G = sum over chunks of X_c^T X_c.  Chunk c's product goes to Gc[c % 2]; from c = 1 on it is
+    // launched as a programmatic dependent of chunk c - 1's fp64 accumulation, so the tensor-core
+    // product and the memory-bound accumulation of the previous chunk overlap; the product's grid
+    // ends after that accumulation, so chunk c's accumulation (a plain launch) follows both.
+    for (int64_t c = 0; c < L.n_chunks; ++c) {
         const uint16_t* XTc = XT + c * K * L.chunk;
-        e = lower ? launch_tc_f32_lower(XTc, K, L.chunk, Gc, status, stream)
-                  : launch_tc_f32(XTc, K, XTc, K, L.chunk, Gc, status, stream);
+        float* Gcc = Gc + (c & 1) * K * K;
+        e = lower ? launch_tc_f32_lower(XTc, K, L.chunk, Gcc, status, stream, c > 0)
+                  : launch_tc_f32(XTc, K, XTc, K, L.chunk, Gcc, status, stream, c > 0);
         if (e != cudaSuccess) return e;
-        gram_accumulate_kernel<<<(unsigned)(K < 4096 ? K : 4096), 256, 0, stream>>>(Gc, (int)K, c == 0, lower, G64);
+        gram_accumulate_kernel<<<(unsigned)(K < 4096 ? K : 4096), 256, 0, stream>>>(Gcc, (int)K, c == 0, lower, G64);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     gram_diag_kernel<<<(unsigned)((K + 255) / 256), 256, 0, stream>>>(G64, (int)K, d, rd);
@@ -561,12 +570,24 @@ cudaError_t launch_awq_gram(const uint16_t* X, int64_t T, const uint16_t* W, int
     const int64_t want = ((n_groups + 1) / 2 + 7) / 8;
     const int64_t cap = (int64_t)device_sm_count() * 8;
     const int fq_blocks = (int)(want < cap ? want : cap);
+    // alpha i's errors go to E[i % 2]; from i = 1 on the fake-quantiser is a programmatic
+    // dependent of alpha i - 1's contraction (which reads the other buffer), so it runs beside it.
     for (int i = 0; i < n_alpha; ++i) {
-        awq_fakequant_scaled_kernel<<<fq_blocks, 256, 0, stream>>>(
-            reinterpret_cast<const uint4*>(W), s_all + (int64_t)i * K, d, n_groups, (int)G, reinterpret_cast<uint4*>(E),
-            status);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        e = launch_tc_dot(E, N, reinterpret_cast<const uint16_t*>(Gp), K, K, part + (int64_t)i * L.n_part, status,
+        uint16_t* Ei = E + (int64_t)(i & 1) * N * K;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)fq_blocks, 1, 1);
+        cfg.blockDim = dim3(256, 1, 1);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = i > 0 ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, awq_fakequant_scaled_kernel, reinterpret_cast<const uint4*>(W),
+                               (const float*)(s_all + (int64_t)i * K), (const float*)d, n_groups, (int)G,
+                               reinterpret_cast<uint4*>(Ei), status);
+        if (e != cudaSuccess) return e;
+        e = launch_tc_dot(Ei, N, reinterpret_cast<const uint16_t*>(Gp), K, K, part + (int64_t)i * L.n_part, status,
                           stream);
         if (e != cudaSuccess) return e;
     }

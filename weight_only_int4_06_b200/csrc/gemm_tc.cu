@@ -132,6 +132,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // A programmatically dependent successor may launch now (it waits for this grid before it
+    // reads anything this grid writes).
+    pdl_launch_dependents();
     const uint32_t tmem_d = *tmem_slot;
 
     auto fail = [&]() {
@@ -363,6 +366,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem_d, C::kTmemCols);
     }
+    // Launched as a programmatic dependent (pdl), this grid ends only after its predecessor has:
+    // a plain launch after it then also follows the predecessor.  A no-op otherwise.
+    pdl_wait();
 }
 
 // ------------------------------------------------------------------------------------ host side
@@ -423,7 +429,7 @@ template <bool DEQ, int EPI, int MT, int BN = TC_BN>
 static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int64_t N, int64_t K,
                              const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, double* sse_part,
                              int* status, cudaStream_t stream, float* Cf = nullptr, bool lower = false,
-                             int ksplit = 1) {
+                             int ksplit = 1, bool pdl = false) {
     using C = TcCfg<DEQ, MT, BN>;
     CUtensorMap ta, tb;
     if (!make_tensor_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, TC_BK, C::kBM,
@@ -441,10 +447,21 @@ static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int6
     const int n_tiles = (int)((N + BN - 1) / BN);
     if (lower && (M != N || C::kBM != BN)) return cudaErrorInvalidValue;  // square tiles of a square product
     const int grid = (lower ? m_tiles * (m_tiles + 1) / 2 : m_tiles * n_tiles) * ksplit;
-    tc_gemm_kernel<DEQ, EPI, MT, BN><<<grid, TC_THREADS, C::kBytes, stream>>>(
-        ta, tb, reinterpret_cast<const __half*>(scales), zeros, reinterpret_cast<__half*>(Y), sse_part, Cf,
-        reinterpret_cast<const __half*>(X), (int)M, (int)N, (int)K, m_tiles, n_tiles, lower ? 1 : 0, ksplit, status);
-    return cudaGetLastError();
+    // pdl: may start while the preceding kernel runs; only for operands that kernel does not
+    // write (the grid still ends after it: see the kernel's last statement)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
+    cfg.blockDim = dim3(TC_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::kBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<DEQ, EPI, MT, BN>, ta, tb, reinterpret_cast<const __half*>(scales),
+                              zeros, reinterpret_cast<__half*>(Y), sse_part, Cf, reinterpret_cast<const __half*>(X),
+                              (int)M, (int)N, (int)K, m_tiles, n_tiles, lower ? 1 : 0, ksplit, status);
 }
 
 // 256-row tiles once M is large enough to fill them; 128-row tiles otherwise.
@@ -562,15 +579,17 @@ cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64
 }
 
 cudaError_t launch_tc_f32(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, float* C,
-                          int* status, cudaStream_t stream) {
+                          int* status, cudaStream_t stream, bool pdl) {
     if (tc_mt(M) == 2)
-        return launch_tc<false, 2, 2>(A, M, B, N, K, nullptr, nullptr, nullptr, nullptr, status, stream, C);
-    return launch_tc<false, 2, 1>(A, M, B, N, K, nullptr, nullptr, nullptr, nullptr, status, stream, C);
+        return launch_tc<false, 2, 2>(A, M, B, N, K, nullptr, nullptr, nullptr, nullptr, status, stream, C, false, 1,
+                                      pdl);
+    return launch_tc<false, 2, 1>(A, M, B, N, K, nullptr, nullptr, nullptr, nullptr, status, stream, C, false, 1, pdl);
 }
 
-cudaError_t launch_tc_f32_lower(const uint16_t* A, int64_t M, int64_t K, float* C, int* status, cudaStream_t stream) {
+cudaError_t launch_tc_f32_lower(const uint16_t* A, int64_t M, int64_t K, float* C, int* status, cudaStream_t stream,
+                                bool pdl) {
     if (tc_mt(M) != 2) return cudaErrorInvalidValue;
-    return launch_tc<false, 2, 2>(A, M, A, M, K, nullptr, nullptr, nullptr, nullptr, status, stream, C, true);
+    return launch_tc<false, 2, 2>(A, M, A, M, K, nullptr, nullptr, nullptr, nullptr, status, stream, C, true, 1, pdl);
 }
 
 cudaError_t launch_tc_f16(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, uint16_t* Y,

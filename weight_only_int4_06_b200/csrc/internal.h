@@ -89,11 +89,14 @@ int tc_sse_partials(int64_t T, int64_t N);  // tiles of an M = T x N launch (par
 // Y [M, N] fp16 = A B^T with an fp16 B [N, K] (no dequantisation).
 cudaError_t launch_tc_f16(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, uint16_t* Y,
                           int* status, cudaStream_t stream);
+// pdl: launched as a programmatic dependent of the preceding kernel, which must not write A or B
+// (the grid still ends only after that kernel has).
 cudaError_t launch_tc_f32(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, float* C,
-                          int* status, cudaStream_t stream);
+                          int* status, cudaStream_t stream, bool pdl = false);
 // C [M, M] fp32 = A A^T on and below the diagonal only (256 x 256 tiles; M > 128): entries above the
 // diagonal are not written.
-cudaError_t launch_tc_f32_lower(const uint16_t* A, int64_t M, int64_t K, float* C, int* status, cudaStream_t stream);
+cudaError_t launch_tc_f32_lower(const uint16_t* A, int64_t M, int64_t K, float* C, int* status, cudaStream_t stream,
+                                bool pdl = false);
 // Per-tile sum over (m, n) of (A . B^T)[m, n] * A[m, n] into part[tile] (requires N == K).
 cudaError_t launch_tc_dot(const uint16_t* A, int64_t M, const uint16_t* B, int64_t N, int64_t K, double* part,
                           int* status, cudaStream_t stream);
