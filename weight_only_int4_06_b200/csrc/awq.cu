@@ -25,14 +25,18 @@
 
 namespace w4 {
 
-// |x| of an fp16 value as an integer number of 2^-24 units (exact; at most 2^41).
-__device__ __forceinline__ uint64_t abs_units(uint32_t h) {
-    const uint32_t b = h & 0x7FFFu;
-    const uint32_t e = b >> 10, m = b & 0x3FFu;
-    return e == 0 ? (uint64_t)m : ((uint64_t)(m | 0x400u) << (e - 1));
-}
-
 constexpr int CA_ROWS = 256;  // rows of X per CTA
+
+// Column sums of |x| as integer numbers of 2^-24 units (exact).  A thread adds its column's
+// |x| over CA_ROWS rows in fp64: every |x| is an exact multiple of 2^-24 below 2^16, so the sum of
+// 256 of them stays below 2^24 and needs at most 48 significant bits — every fp64 addition is
+// exact.  The sum times 2^24 is then an exact integer, added to the column's u64 total.
+__device__ __forceinline__ void colabs_add(uint32_t w, double& lo, double& hi) {
+    const uint32_t a = w & 0x7FFF7FFFu;  // |x| of both halves
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&a));
+    lo += (double)f.x;
+    hi += (double)f.y;
+}
 
 __global__ void __launch_bounds__(256) colabs_kernel(const uint4* __restrict__ X, int64_t T, int K,
                                                      unsigned long long* __restrict__ colsum) {
@@ -41,7 +45,7 @@ __global__ void __launch_bounds__(256) colabs_kernel(const uint4* __restrict__ X
     if (ch >= chunks) return;
     const int64_t r0 = (int64_t)blockIdx.y * CA_ROWS;
     const int64_t r1 = min(T, r0 + CA_ROWS);
-    uint64_t acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
     int64_t r = r0;
     for (; r + 4 <= r1; r += 4) {
         uint4 v[4];
@@ -49,25 +53,22 @@ __global__ void __launch_bounds__(256) colabs_kernel(const uint4* __restrict__ X
         for (int u = 0; u < 4; ++u) v[u] = ldg_stream(X + (r + u) * chunks + ch);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                acc[2 * i] += abs_units(w[i] & 0xFFFFu);
-                acc[2 * i + 1] += abs_units(w[i] >> 16);
-            }
+            colabs_add(v[u].x, acc[0], acc[1]);
+            colabs_add(v[u].y, acc[2], acc[3]);
+            colabs_add(v[u].z, acc[4], acc[5]);
+            colabs_add(v[u].w, acc[6], acc[7]);
         }
     }
     for (; r < r1; ++r) {
         const uint4 v = ldg_stream(X + r * chunks + ch);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            acc[2 * i] += abs_units(w[i] & 0xFFFFu);
-            acc[2 * i + 1] += abs_units(w[i] >> 16);
-        }
+        colabs_add(v.x, acc[0], acc[1]);
+        colabs_add(v.y, acc[2], acc[3]);
+        colabs_add(v.z, acc[4], acc[5]);
+        colabs_add(v.w, acc[6], acc[7]);
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) atomicAdd(colsum + ch * 8 + i, (unsigned long long)acc[i]);  // exact
+    for (int i = 0; i < 8; ++i)  // exact: an integer below 2^48
+        atomicAdd(colsum + ch * 8 + i, (unsigned long long)__double2ull_rn(acc[i] * 16777216.0));
 }
 
 // One CTA per alpha.  Block-wide max/min with a fixed reduction tree.
@@ -369,7 +370,6 @@ cudaError_t launch_awq_select(const double* sse, int n_parts, int n_alpha, int64
 // e^T G e = e'^T G' e'.  The per-alpha GEMM E' G'^T has an epilogue that sums (E' G'^T)[n, k] E'[n, k]
 // per tile; MSE_i = (fixed-order sum of the tile partials) / (T N), exactly as in the direct form.
 
-constexpr int TP_TILE = 32;
 constexpr int64_t GRAM_CHUNK = 4096;
 
 // Rows per chunk: all of T (padded to a multiple of 64) when T fits one chunk.
@@ -379,22 +379,41 @@ static int64_t gram_chunk_rows(int64_t T) {
 }
 
 // XT holds X^T chunk by chunk: chunk c is a [K, L] row-major block of rows t in [cL, cL + L), rows
-// t >= T zero (L % 64 == 0: whole K-steps for the GEMM).
-__global__ void __launch_bounds__(256) transpose_pad_kernel(const unsigned short* __restrict__ X, int64_t T,
-                                                            int K, int64_t L, int64_t Tp,
-                                                            unsigned short* __restrict__ XT) {
-    __shared__ unsigned short tile[TP_TILE][TP_TILE + 1];
+// t >= T zero (L % 64 == 0: whole K-steps for the GEMM).  A CTA moves one 64 (t) x 64 (k) tile
+// with 16-byte loads and stores: each thread loads 8 consecutive k of one t, scatters them into a
+// [k][t] shared tile whose 16-byte chunks are XOR-swizzled by k / 8 (the 2-byte stores of a warp
+// and the 16-byte loads of a quarter warp both hit distinct banks), then stores 8 consecutive t of
+// one k.
+constexpr int TP_TILE = 64;
+__global__ void __launch_bounds__(256) transpose_pad_kernel(const uint4* __restrict__ X, int64_t T, int K,
+                                                            int64_t L, int64_t Tp, uint4* __restrict__ XT) {
+    __shared__ __align__(16) unsigned short tile[TP_TILE * TP_TILE];
     const int64_t t0 = (int64_t)blockIdx.x * TP_TILE;
     const int k0 = blockIdx.y * TP_TILE;
-    for (int r = threadIdx.y; r < TP_TILE; r += blockDim.y) {
-        const int64_t t = t0 + r;
-        tile[r][threadIdx.x] = t < T ? X[t * K + k0 + threadIdx.x] : (unsigned short)0;
+    const int64_t kc8 = K / 8;  // 16-byte chunks per row of X
+#pragma unroll
+    for (int rep = 0; rep < 2; ++rep) {
+        const int idx = threadIdx.x + rep * 256;
+        const int tl = idx >> 3, kq = idx & 7;  // tile row (t) and its 8-k chunk
+        const int64_t t = t0 + tl;
+        const uint4 v = t < T ? ldg_stream(X + t * kc8 + (k0 >> 3) + kq) : make_uint4(0u, 0u, 0u, 0u);
+        const unsigned short* h = reinterpret_cast<const unsigned short*>(&v);
+        const int chunk = (tl >> 3) ^ kq;  // k / 8 == kq for all eight k of this chunk
+#pragma unroll
+        for (int j = 0; j < 8; ++j) tile[(kq * 8 + j) * TP_TILE + chunk * 8 + (tl & 7)] = h[j];
     }
     __syncthreads();
-    const int64_t t = t0 + threadIdx.x;
-    const int64_t c = t / L, tt = t - c * L;
-    for (int r = threadIdx.y; r < TP_TILE; r += blockDim.y)
-        if (t < Tp) XT[(c * K + k0 + r) * L + tt] = tile[threadIdx.x][r];
+#pragma unroll
+    for (int rep = 0; rep < 2; ++rep) {
+        const int idx = threadIdx.x + rep * 256;
+        const int kr = idx >> 3, tq = idx & 7;  // tile row (k) and its 8-t chunk
+        const uint4 v = *reinterpret_cast<const uint4*>(tile + kr * TP_TILE + ((tq ^ (kr >> 3)) * 8));
+        const int64_t t = t0 + tq * 8;  // eight consecutive t, all in one chunk (L % 64 == 0)
+        if (t < Tp) {
+            const int64_t c = t / L, tt = t - c * L;
+            XT[((c * K + k0 + kr) * L + tt) / 8] = v;
+        }
+    }
 }
 
 // G64 = Gc (first chunk) or G64 += Gc in fp64, on and below the diagonal (row i, columns j <= i;
@@ -541,8 +560,8 @@ cudaError_t launch_awq_gram(const uint16_t* X, int64_t T, const uint16_t* W, int
     }
     awq_scales_kernel<<<n_alpha, 1024, 0, stream>>>(colsum, T, (int)K, n_alpha, s_all);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    transpose_pad_kernel<<<dim3((unsigned)(L.Tp / TP_TILE), (unsigned)(K / TP_TILE)), dim3(TP_TILE, 8), 0, stream>>>(
-        reinterpret_cast<const unsigned short*>(X), T, (int)K, L.chunk, L.Tp, reinterpret_cast<unsigned short*>(XT));
+    transpose_pad_kernel<<<dim3((unsigned)(L.Tp / TP_TILE), (unsigned)(K / TP_TILE)), 256, 0, stream>>>(
+        reinterpret_cast<const uint4*>(X), T, (int)K, L.chunk, L.Tp, reinterpret_cast<uint4*>(XT));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const unsigned ew_blocks = (unsigned)device_sm_count() * 8;
     // G is symmetric: for K > 128 only the 256 x 256 tiles on and below the diagonal are formed
