@@ -330,6 +330,17 @@ def test_gemm_weights_static_flag_same_bits(M, K, N):
     assert np.array_equal(Y0.view(np.uint16), Y1.view(np.uint16))
 
 
+def test_gemm_tc_tail_split_ragged():
+    """Full waves of 256 x 256 tiles in one launch, the last partial wave's tiles cut along K (4
+    slices here) with their partials summed per tile: ragged M and N tiles included."""
+    M, K, N = 2000, 2048, 5000  # 8 x 20 = 160 tiles on 148 SMs: 12 tail tiles
+    assert B.w4_gemm_plan(M, N, K) == (B.VARIANT_TC, 3)
+    X, p, s, z = oracle_case(32, M, K, N)
+    Y1 = gpu_gemm(X, p, s, z)
+    assert_close(Y1, oracle.gemm(X, p, s, z), f"tail split {M}x{K}x{N}")
+    assert np.array_equal(Y1.view(np.uint16), gpu_gemm(X, p, s, z).view(np.uint16))  # deterministic
+
+
 def test_gemm_tc_deterministic():
     X, p, s, z = oracle_case(27, 1024, 4096, 2048)
     Y1 = gpu_gemm(X, p, s, z, B.VARIANT_TC)

@@ -74,7 +74,7 @@ w4_status gemm_plan(int64_t M, int64_t N, int64_t K, int family, bool meta_align
     const bool tc_fills = (N + 127) / 128 >= device_sm_count();
     if (family == W4_VARIANT_TC || (family == W4_VARIANT_AUTO && (M > 32 || (M > 16 && K <= 8192 && tc_fills)))) {
         *chosen = W4_VARIANT_TC;
-        *launches = tc_w4_split(M, N, K) > 1 ? 2 : 1;  // K slices, then their fixed-order sum
+        *launches = tc_w4_launches(M, N, K);  // with K slices: + their fixed-order sum
         return W4_OK;
     }
     if (family == W4_VARIANT_GEMV_TC) {
@@ -168,7 +168,7 @@ w4_status w4_gemm_ex(const uint16_t* X, int64_t M, int64_t N, int64_t K, const u
     st = gemm_plan(M, N, K, family, aligned16(scales) && aligned16(zeros), &chosen, &launches);
     if (st != W4_OK) return st;
     if (chosen == W4_VARIANT_TC) {
-        if (tc_w4_split(M, N, K) > 1 && (ws_bytes < tc_w4_workspace(M, N, K) || !ws)) return W4_ERR_WORKSPACE;
+        if (tc_w4_workspace(M, N, K) > 0 && (ws_bytes < tc_w4_workspace(M, N, K) || !ws)) return W4_ERR_WORKSPACE;
         return launch_tc_w4(X, M, N, K, packed, scales, zeros, Y, ws, status, s) == cudaSuccess ? W4_OK
                                                                                                 : W4_ERR_CUDA;
     }

@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                    const __half* __restrict__ scales, const uint8_t* __restrict__ zeros,
                    __half* __restrict__ Y, double* __restrict__ sse_part, float* __restrict__ Cf,
                    const __half* __restrict__ Adot, int M, int N, int K, int m_tiles, int n_tiles,
-                   int lower, int ksplit, int* status) {
+                   int lower, int ksplit, int tile_base, int n_compact, int* status) {
     constexpr bool SSE = EPI == 1 || EPI == 3;  // modes that reduce the tile to one fp64 partial
     using C = TcCfg<DEQ, MT, BN>;
     constexpr int S = C::kStages;
@@ -92,10 +92,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     int mt, nt;
-    // ksplit > 1: CTA b computes K slice b % ksplit of tile b / ksplit (whole groups of 128 k) and
-    // stores its fp32 partial tile into slice (b % ksplit) of Cf
+    // ksplit > 1: CTA b computes K slice b % ksplit of tile tile_base + b / ksplit (whole groups of
+    // 128 k) and stores its fp32 partial tile into slice (b % ksplit) of Cf: [slice][M][N], or with
+    // n_compact > 0 [slice][n_compact tiles][kBM][BN] (the tiles of this launch only)
     const int slice = ksplit > 1 ? (int)(blockIdx.x % ksplit) : 0;
-    const int tile_id = ksplit > 1 ? (int)(blockIdx.x / ksplit) : (int)blockIdx.x;
+    const int tile_id = (ksplit > 1 ? (int)(blockIdx.x / ksplit) : (int)blockIdx.x) + tile_base;
     if (lower) {  // only the tiles on or below the diagonal of a square product (one per CTA)
         const int t = tile_id;
         mt = (int)((sqrt(8.0 * (double)t + 1.0) - 1.0) * 0.5);
@@ -111,7 +112,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // 128) two per group of 128, a slice starting on a group
     const int kb0 = ksplit > 1 ? 2 * (int)(((int64_t)slice * G) / ksplit) : 0;
     const int nk = ksplit > 1 ? 2 * (int)(((int64_t)(slice + 1) * G) / ksplit) - kb0 : K / TC_BK;
-    if (ksplit > 1 && EPI == 2) Cf += (int64_t)slice * M * N;
+    if (ksplit > 1 && EPI == 2)
+        Cf += n_compact ? ((int64_t)slice * n_compact + (tile_id - tile_base)) * C::kBM * BN : (int64_t)slice * M * N;
 
     if (tid == 0) {
         for (int s = 0; s < S; ++s) {
@@ -310,6 +312,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                         }
                         sq += (double)a;
                     }
+                } else if (EPI == 2 && n_compact) {  // the tile's own [kBM][BN] block: no bounds
+                    float* crow = Cf + (int64_t)(m - m0) * BN + col;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(crow + i) =
+                            make_float4(__uint_as_float(v[i]), __uint_as_float(v[i + 1]),
+                                        __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
                 } else if (EPI == 2) {
                     if (m < M) {
                         const int nb = n0 + col;
@@ -429,7 +438,8 @@ template <bool DEQ, int EPI, int MT, int BN = TC_BN>
 static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int64_t N, int64_t K,
                              const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, double* sse_part,
                              int* status, cudaStream_t stream, float* Cf = nullptr, bool lower = false,
-                             int ksplit = 1, bool pdl = false) {
+                             int ksplit = 1, bool pdl = false, int tile_base = 0, int n_tiles_launch = -1,
+                             int n_compact = 0) {
     using C = TcCfg<DEQ, MT, BN>;
     CUtensorMap ta, tb;
     if (!make_tensor_map_2d(&ta, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M, TC_BK, C::kBM,
@@ -446,7 +456,9 @@ static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int6
     const int m_tiles = (int)((M + C::kBM - 1) / C::kBM);
     const int n_tiles = (int)((N + BN - 1) / BN);
     if (lower && (M != N || C::kBM != BN)) return cudaErrorInvalidValue;  // square tiles of a square product
-    const int grid = (lower ? m_tiles * (m_tiles + 1) / 2 : m_tiles * n_tiles) * ksplit;
+    const int all_tiles = lower ? m_tiles * (m_tiles + 1) / 2 : m_tiles * n_tiles;
+    const int grid = (n_tiles_launch >= 0 ? n_tiles_launch : all_tiles) * ksplit;
+    if (grid == 0) return cudaSuccess;
     // pdl: may start while the preceding kernel runs; only for operands that kernel does not
     // write (the grid still ends after it: see the kernel's last statement)
     cudaLaunchConfig_t cfg = {};
@@ -461,7 +473,8 @@ static cudaError_t launch_tc(const uint16_t* X, int64_t M, const void* Bop, int6
     cfg.numAttrs = pdl ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<DEQ, EPI, MT, BN>, ta, tb, reinterpret_cast<const __half*>(scales),
                               zeros, reinterpret_cast<__half*>(Y), sse_part, Cf, reinterpret_cast<const __half*>(X),
-                              (int)M, (int)N, (int)K, m_tiles, n_tiles, lower ? 1 : 0, ksplit, status);
+                              (int)M, (int)N, (int)K, m_tiles, n_tiles, lower ? 1 : 0, ksplit, tile_base, n_compact,
+                              status);
 }
 
 // 256-row tiles once M is large enough to fill them; 128-row tiles otherwise.
@@ -506,9 +519,71 @@ int tc_w4_split(int64_t M, int64_t N, int64_t K) {
     return s >= 2 ? (int)s : 1;
 }
 
+// Tail split of w4_gemm's tensor-core path: when the 256 x 256 tiles (the picked shape) fill whole
+// waves of one CTA per SM and then at most half of one more, the full waves run as one launch and
+// the last wave's `tail` tiles are cut along K into ks slices (whole groups, at least 8 k-blocks
+// each, ks <= 8) that fill the SMs; their fp32 partials are added per tile in slice order.  False:
+// no tail split.
+bool tc_w4_tail(int64_t M, int64_t N, int64_t K, int* full, int* tail, int* ks) {
+    if (M <= 128 || tc_w4_split(M, N, K) > 1) return false;
+    int mt = 2, bn = 256;
+    tc_w4_pick(M, N, &mt, &bn);
+    if (mt != 2 || bn != 256) return false;
+    const int64_t sms = device_sm_count();
+    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int64_t t = tiles % sms;
+    if (tiles < sms || t == 0 || 2 * t > sms) return false;
+    int64_t s = sms / t;
+    const int64_t max_by_k = (K / TC_BK) / 8;
+    if (s > max_by_k) s = max_by_k;
+    if (s > 8) s = 8;
+    if (s < 2) return false;
+    *full = (int)(tiles - t);
+    *tail = (int)t;
+    *ks = (int)s;
+    return true;
+}
+
 size_t tc_w4_workspace(int64_t M, int64_t N, int64_t K) {
     const int s = tc_w4_split(M, N, K);
-    return s > 1 ? (size_t)s * (size_t)M * (size_t)N * 4 : 0;
+    if (s > 1) return (size_t)s * (size_t)M * (size_t)N * 4;
+    int full = 0, tail = 0, ks = 0;
+    if (tc_w4_tail(M, N, K, &full, &tail, &ks)) return (size_t)ks * (size_t)tail * 256 * 256 * 4;
+    return 0;
+}
+
+int tc_w4_launches(int64_t M, int64_t N, int64_t K) {
+    if (tc_w4_split(M, N, K) > 1) return 2;  // the K slices, then their sum
+    int full = 0, tail = 0, ks = 0;
+    return tc_w4_tail(M, N, K, &full, &tail, &ks) ? 3 : 1;  // full waves, tail slices, their sum
+}
+
+// Y at the tail tiles = fp16(sum over the slices of the compact fp32 partial tiles
+// P [slice][tile][256][256], in slice order): deterministic.  A programmatic dependent of the
+// launch that writes the partials (it waits for that launch before reading them).
+__global__ void tail_reduce_kernel(const float* __restrict__ P, int slices, int n_tail, int tile_base, int m_tiles,
+                                   int n_tiles, int M, int N, __half* __restrict__ Y) {
+    pdl_launch_dependents();
+    pdl_wait();
+    constexpr int64_t TILE = 256 * 256;
+    const int64_t n4 = (int64_t)n_tail * (TILE / 4);
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n4; e += (int64_t)gridDim.x * blockDim.x) {
+        const int tl = (int)(e / (TILE / 4));
+        const int local = (int)(e - (int64_t)tl * (TILE / 4)) * 4;
+        int mt, nt;
+        tc_tile_coords(tile_base + tl, m_tiles, n_tiles, mt, nt);
+        const int m = mt * 256 + (local >> 8), n = nt * 256 + (local & 255);
+        if (m >= M || n >= N) continue;  // N % 8 == 0: n < N covers all four columns
+        float4 a = *reinterpret_cast<const float4*>(P + (int64_t)tl * TILE + local);
+        for (int s = 1; s < slices; ++s) {
+            const float4 b = *reinterpret_cast<const float4*>(P + ((int64_t)s * n_tail + tl) * TILE + local);
+            a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+        }
+        uint2 o;
+        o.x = pack_half2(a.x, a.y);
+        o.y = pack_half2(a.z, a.w);
+        *reinterpret_cast<uint2*>(Y + (int64_t)m * N + n) = o;
+    }
 }
 
 // Y = fp16(sum over the slices of the fp32 partials, in slice order): deterministic.  Launched as a
@@ -559,6 +634,34 @@ cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, con
                                                     stream, P, false, ks);
         if (e != cudaSuccess) return e;
         return launch_splitk_reduce(P, ks, M * N, Y, stream);
+    }
+    int full = 0, tail = 0, tks = 0;
+    if (tc_w4_tail(M, N, K, &full, &tail, &tks)) {
+        if (!ws) return cudaErrorInvalidValue;
+        float* P = static_cast<float*>(ws);
+        // the full waves, with their plain epilogue
+        cudaError_t e = launch_tc<true, 0, 2, 256>(X, M, packed, N, K, scales, zeros, Y, nullptr, status, stream,
+                                                   nullptr, false, 1, false, 0, full, 0);
+        if (e != cudaSuccess) return e;
+        // the last wave's tiles in K slices, compact partials: nothing the full waves write is read
+        // here, so its CTAs start on the SMs the full waves free (programmatic dependent launch)
+        e = launch_tc<true, 2, 2, 256>(X, M, packed, N, K, scales, zeros, nullptr, nullptr, status, stream, P, false,
+                                       tks, true, full, tail, tail);
+        if (e != cudaSuccess) return e;
+        const int m_tiles = (int)((M + 255) / 256), n_tiles = (int)((N + 255) / 256);
+        const int64_t want = ((int64_t)tail * 256 * 256 / 4 + 255) / 256;
+        const int64_t cap = (int64_t)device_sm_count() * 8;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(want < cap ? want : cap), 1, 1);
+        cfg.blockDim = dim3(256, 1, 1);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, tail_reduce_kernel, (const float*)P, tks, tail, full, m_tiles, n_tiles,
+                                  (int)M, (int)N, reinterpret_cast<__half*>(Y));
     }
     int mt = 2, bn = 256;
     tc_w4_pick(M, N, &mt, &bn);

@@ -81,7 +81,11 @@ cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, con
                          const uint16_t* scales, const uint8_t* zeros, uint16_t* Y, void* ws, int* status,
                          cudaStream_t stream);
 int tc_w4_split(int64_t M, int64_t N, int64_t K);         // K slices of the tensor-core path (1: none)
+// Tail split: full waves of 256 x 256 tiles in one launch, the last partial wave's `tail` tiles in
+// ks K slices with compact fp32 partials, summed per tile by a third launch.
+bool tc_w4_tail(int64_t M, int64_t N, int64_t K, int* full, int* tail, int* ks);
 size_t tc_w4_workspace(int64_t M, int64_t N, int64_t K);  // bytes of fp32 partials when split
+int tc_w4_launches(int64_t M, int64_t N, int64_t K);      // kernel launches of one call
 cudaError_t launch_tc_sse(const uint16_t* X, int64_t T, const uint16_t* E, int64_t N, int64_t K,
                           double* sse_part, int* status, cudaStream_t stream);
 int tc_sse_partials(int64_t T, int64_t N);  // tiles of an M = T x N launch (partials of EPI 1 and 3)
