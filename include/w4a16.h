@@ -120,9 +120,10 @@ w4_status w4_quantize_pack(const uint16_t* W, int64_t N, int64_t K, int group,
                            uint8_t* zeros, void* stream);
 
 /* Bytes of device workspace w4_gemm / w4_gemm_ex need for this shape (may be 0): fp32 partial
- * sums when the tensor-core GEMM (M > 128 with few output tiles) or the GEMV (activation rows too
- * long to stage whole next to a deep enough ring, K/128 a multiple of 16) cut K into slices.  A
- * function of M, N, K and group only; no device is touched. */
+ * sums when the tensor-core GEMM (M > 16 with few output tiles, or a last wave at most half full)
+ * or the GEMV (activation rows too long to stage whole next to a deep enough ring, K/128 a
+ * multiple of 16) cut K into slices.  A function of M, N, K and group (and the device's SM count,
+ * cached). */
 w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, size_t* bytes);
 
 /*
@@ -137,11 +138,12 @@ w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, siz
  *   ws / ws_bytes: device workspace of at least w4_gemm_workspace_size bytes, 16-byte aligned
  *   (may be NULL when that size is 0; misaligned: W4_ERR_ALIGN).  M == 0 or N == 0 is a no-op;
  *   K == 0 writes Y = 0.
- * Families (w4_gemm picks by M: GEMV, in launches of up to 8 activation rows, for M <= 32 when
- * scales/zeros are 16-byte aligned and 8 staged activation rows fit shared memory or K/128 is a
- * multiple of 16 (then K is cut into slices of 4096, their fp32 partials summed in slice order by
- * a second launch); skinny for the other M <= 32; TC above, or from M = 17 when its 128-row
- * weight tiles alone fill the SMs at K <= 8192):
+ * Families (w4_gemm picks by M: GEMV, in launches of up to 8 activation rows (16 at K <= 8192),
+ * for M <= 16 when scales/zeros are 16-byte aligned and the staged activation rows fit shared
+ * memory or K/128 is a multiple of 16 (then K is cut into slices, their fp32 partials summed in
+ * slice order by a second launch); skinny for the other M <= 16; TC above 16 rows, with K cut
+ * into slices when its tiles fill fewer than half the SMs, or its last wave's tiles when that wave
+ * is at most half full, the partials summed in slice order by a further launch):
  *   - GEMV: tensor-core sums of x with the raw operands 1024+q / 1024+16q, offsets and z removed
  *     per group with fp32 activation sums (fixed order), times s16 in fp32;
  *   - skinny: sum_k x_k (q_k - z) exactly per group on tensor cores in fp32, times s16 in fp32;

@@ -106,10 +106,12 @@ def test_workspace_queries(L):
     assert L.w4_gemm_workspace_size(4, 8192, 8192, 128, ctypes.byref(n)) == 0 and n.value == 0
     assert L.w4_gemm_workspace_size(8, 8192, 28672, 128, ctypes.byref(n)) == 0
     assert n.value == 7 * 8 * 8192 * 4
-    assert L.w4_gemm_workspace_size(32, 8192, 28672, 128, ctypes.byref(n)) == 0
+    assert L.w4_gemm_workspace_size(16, 8192, 28672, 128, ctypes.byref(n)) == 0
     assert n.value == 7 * 8 * 8192 * 4  # 8-row launches (7 slices of 4096) reuse it in turn
+    assert L.w4_gemm_workspace_size(16, 8192, 8192, 128, ctypes.byref(n)) == 0
+    assert n.value == 4 * 16 * 8192 * 4  # one 16-row launch (4 slices of 2048) at K = 8192
     assert L.w4_gemm_workspace_size(32, 8192, 8192, 128, ctypes.byref(n)) == 0
-    assert n.value == 4 * 16 * 8192 * 4  # 16-row launches (4 slices of 2048) at K = 8192
+    assert n.value == 4 * 32 * 8192 * 4  # the tensor cores' 4 K slices
     assert L.w4_gemm_workspace_size(12, 4096, 11008, 128, ctypes.byref(n)) == 0 and n.value == 0
     assert L.awq_workspace_size(256, 64, 512, 128, 0, ctypes.byref(n)) == 4
     assert L.awq_workspace_size(256, 64, 500, 128, 20, ctypes.byref(n)) == 2
@@ -275,18 +277,21 @@ def test_gemm_plan_query(L):
     """The dispatch query (CPU: no device work) agrees with the documented rule."""
     assert B.w4_gemm_plan(1, 4096, 4096) == (B.VARIANT_GEMV, 1)
     # 8 rows of K = 8192 leave 2 ring stages whole: K is cut in two, + 1 reducing launch; 9-16 rows
-    # run as one 16-row launch over slices of 2048 (+ 1 reducing launch), 32 rows as two of them
+    # run as one 16-row launch over slices of 2048 (+ 1 reducing launch); above 16 rows the tensor
+    # cores, their 32 tiles cut along K into 4 slices (+ 1 reducing launch)
     assert B.w4_gemm_plan(4, 8192, 8192) == (B.VARIANT_GEMV, 1)
     assert B.w4_gemm_plan(8, 8192, 8192) == (B.VARIANT_GEMV, 2)
     assert B.w4_gemm_plan(16, 8192, 8192) == (B.VARIANT_GEMV, 2)
-    assert B.w4_gemm_plan(32, 8192, 8192) == (B.VARIANT_GEMV, 4)
+    assert B.w4_gemm_plan(32, 8192, 8192) == (B.VARIANT_TC, 2)
     assert B.w4_gemm_plan(16, 520, 2048) == (B.VARIANT_GEMV, 1)  # one slice: no reducing launch
     assert B.w4_gemm_plan(12, 136, 1536) == (B.VARIANT_GEMV, 2)  # K/128 = 12: two 8-row launches
     # K = 28672 is cut into slices (4 rows of it do not fit whole): the GEMV, then the slice sum
     assert B.w4_gemm_plan(4, 8192, 28672) == (B.VARIANT_GEMV, 2)
-    assert B.w4_gemm_plan(32, 8192, 28672) == (B.VARIANT_GEMV, 8)  # 8-row launches at K = 28672
+    assert B.w4_gemm_plan(16, 8192, 28672) == (B.VARIANT_GEMV, 4)  # 8-row launches at K = 28672
+    assert B.w4_gemm_plan(32, 8192, 28672) == (B.VARIANT_TC, 2)
     assert B.w4_gemm_plan(4, 8192, 28800) == (B.VARIANT_SKINNY, 1)  # K/128 = 225: no slices, no fit
-    assert B.w4_gemm_plan(33, 4096, 4096) == (B.VARIANT_TC, 1)
+    assert B.w4_gemm_plan(33, 4096, 4096) == (B.VARIANT_TC, 2)  # 16 tiles: K in 8 slices + their sum
+    assert B.w4_gemm_plan(2048, 11008, 4096) == (B.VARIANT_TC, 3)  # 344 tiles: full waves + tail slices + sum
     assert B.w4_gemm_plan(0, 4096, 4096) == (B.VARIANT_AUTO, 0)
     assert B.w4_gemm_plan(64, 4096, 4096, variant=B.VARIANT_SKINNY) == (B.VARIANT_SKINNY, 2)
     fam, n = ctypes.c_int(0), ctypes.c_int(0)

@@ -58,21 +58,18 @@ int* device_status_ptr() {
 }
 
 // The kernel family and number of launches of one w4_gemm_ex call (shape already validated).
-// AUTO: the tensor-core GEMM above 32 activation rows; up to 32 rows the TMA-fed GEMV in
-// launches of up to 8 rows where its metadata is 16-byte aligned (it bulk-copies scales and zero
-// points) and either 8 staged activation rows fit its shared memory or K/128 is a multiple of 16
-// (K then cut into slices of 4096, + 1 reducing launch), else the skinny kernel in launches of up
-// to 32 rows; from 17 rows on, the tensor-core GEMM instead when its 128-row W tiles alone fill
-// the SMs.  Measured per shape on B200 (bench.py --workload dispatch, cold L2, us): decode M = 1
-// GEMV 4.7 / 9.5 / 8.6 / 8.8 vs skinny 6.2 / 19.5 / 18.8 / 14.2; at K = 8192 the GEMV beats the
-// skinny kernel at M = 4 .. 32 (12.9 / 15.4 / 28.0 / 54.3 vs 29.7 / 29.8 / 46.7 / 68.7 at
-// N = 8192, cutting K in two at M = 8: 15.4 vs 17.4 whole); at M = 32, N = 28672 the tensor-core
-// GEMM (90.8) beats four GEMV launches (146.3), at M = 16 it does not (89.7 vs 74.0); at
-// K = 28672 the sliced GEMV beats the skinny kernel at every M (31.9 / 37.6 / 73.2 / 145.2 vs
-// 90.7 / 91.6 / 144.0 / 220.5) and the tensor-core GEMM (224).
+// AUTO: the tensor-core GEMM above 16 activation rows (with its K split when its tiles fill fewer
+// than half the SMs); up to 16 rows the TMA-fed GEMV in launches of up to 8 rows (16 at
+// K <= 8192) where its metadata is 16-byte aligned (it bulk-copies scales and zero points) and
+// either 8 staged activation rows fit its shared memory or K/128 is a multiple of 16 (K then cut
+// into slices, + 1 reducing launch), else the skinny kernel in launches of up to 32 rows.
+// Measured per shape on B200 (bench.py --workload dispatch, cold L2, us): decode M = 1 GEMV
+// 4.7 / 9.5 / 8.8 / 8.8 vs skinny 6.2 / 19.7 / 19.2 / 14.3; M = 4 / 8 the GEMV everywhere (12.9 /
+// 15.3 at K = N = 8192, 31.8 / 37.9 at N = 28672, 32.2 / 38.5 at K = 28672; skinny 30-93, tensor
+// cores 64-222); M = 16 the GEMV (25.5 / 74.6 / 75.4 vs tensor cores 30.3 / 90.2 / 83.2); M = 32
+// the tensor cores (31.0 / 90.9 / 83.9 vs the GEMV's 16- or 8-row launches 49.3 / 146.5 / 147.9).
 w4_status gemm_plan(int64_t M, int64_t N, int64_t K, int family, bool meta_aligned, int* chosen, int* launches) {
-    const bool tc_fills = (N + 127) / 128 >= device_sm_count();
-    if (family == W4_VARIANT_TC || (family == W4_VARIANT_AUTO && (M > 32 || (M > 16 && K <= 8192 && tc_fills)))) {
+    if (family == W4_VARIANT_TC || (family == W4_VARIANT_AUTO && M > 16)) {
         *chosen = W4_VARIANT_TC;
         *launches = tc_w4_launches(M, N, K);  // with K slices: + their fixed-order sum
         return W4_OK;
@@ -131,7 +128,7 @@ w4_status w4_gemm_workspace_size(int64_t M, int64_t N, int64_t K, int group, siz
         return W4_ERR_SHAPE;
     // fp32 partials when the tensor-core path splits K (prefill shapes with few tiles) or the
     // GEMV cuts K into slices (activation rows too long to stage whole next to a deep ring)
-    const size_t tc = M > 32 && K > 0 && N > 0 ? tc_w4_workspace(M, N, K) : 0;
+    const size_t tc = M > 16 && K > 0 && N > 0 ? tc_w4_workspace(M, N, K) : 0;
     const size_t gv = K > 0 && N > 0 ? decode_stream_workspace(M, N, K) : 0;
     *bytes = tc > gv ? tc : gv;
     return W4_OK;

@@ -504,13 +504,15 @@ void tc_w4_pick(int64_t M, int64_t N, int* mt_out, int* bn_out) {
     }
 }
 
-// K slices of w4_gemm's tensor-core path: 256 x 256 tiles that fill fewer than half the SMs (M >
-// 128) are split along K into up to 8 slices of whole groups, at least 8 k-blocks of 64 each,
-// so that tiles x slices fill the SMs; 1 = no split.
+// K slices of w4_gemm's tensor-core path: (128 or 256) x 256 tiles (128 rows of X up to M = 128)
+// that fill fewer than half the SMs are split along K into up to 8 slices of whole groups, at
+// least 8 k-blocks of 64 each, so that tiles x slices fill the SMs; 1 = no split (always for
+// M <= 16, which the GEMV serves).
 int tc_w4_split(int64_t M, int64_t N, int64_t K) {
-    if (M <= 128) return 1;
+    if (M <= 16) return 1;
     const int64_t sms = device_sm_count();
-    const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    const int64_t bm = M > 128 ? 256 : 128;
+    const int64_t tiles = ((M + bm - 1) / bm) * ((N + 255) / 256);
     if (2 * tiles >= sms) return 1;
     int64_t s = sms / tiles;
     const int64_t max_by_k = (K / TC_BK) / 8;
@@ -630,8 +632,10 @@ cudaError_t launch_tc_w4(const uint16_t* X, int64_t M, int64_t N, int64_t K, con
     if (ks > 1) {  // M * N is a multiple of 8 (N % 8 == 0): whole float4s
         if (!ws) return cudaErrorInvalidValue;
         float* P = static_cast<float*>(ws);
-        cudaError_t e = launch_tc<true, 2, 2, 256>(X, M, packed, N, K, scales, zeros, nullptr, nullptr, status,
-                                                    stream, P, false, ks);
+        cudaError_t e = M > 128 ? launch_tc<true, 2, 2, 256>(X, M, packed, N, K, scales, zeros, nullptr, nullptr, status,
+                                                             stream, P, false, ks)
+                                : launch_tc<true, 2, 1, 256>(X, M, packed, N, K, scales, zeros, nullptr, nullptr, status,
+                                                             stream, P, false, ks);
         if (e != cudaSuccess) return e;
         return launch_splitk_reduce(P, ks, M * N, Y, stream);
     }
