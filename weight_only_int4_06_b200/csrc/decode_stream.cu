@@ -1,4 +1,4 @@
-// Decode GEMV / skinny GEMM for M <= 8: Y = X dequant(W)^T, streamed at HBM rate.
+// Decode GEMV / skinny GEMM for M <= 16: Y = X dequant(W)^T, streamed at HBM rate.
 //
 // "AutoAWQ vs The Stack v2" (WQLinear blurb): the GEMV kernel serves token-by-token generation,
 // where the layer is bound by memory traffic and weight reuse is minimal.  The traffic is the
@@ -7,7 +7,11 @@
 // Design (sm_100a):
 //  * One CTA per SM (or per tile when there are fewer tiles than SMs).  CTA c owns a contiguous,
 //    balanced range of 16-row tiles over the whole K (CTA sizes differ by at most one tile), so
-//    every output is finished inside one CTA: no split-K workspace, no cluster barrier.
+//    every output is finished inside one CTA: no split-K workspace, no cluster barrier.  Where
+//    the staged activation rows of the whole K would leave a shallow ring (split mode, KS), K is
+//    cut into slices of whole stages instead: blockIdx.y is the slice, each CTA stages its slice's
+//    activations only, every stage brings its own scales and zero points as two 2-D TMA boxes,
+//    and the slices' fp32 partials are summed in slice order by a second launch.
 //  * A producer warp streams each tile through a shared-memory ring of 32 KB stages with TMA: one
 //    stage is 16 rows x 32 groups (4096 k, 2 KB of each row).  A tile's scales and zero points are
 //    one contiguous block of each array and ride on the tile's first stage as two bulk copies.
@@ -37,7 +41,8 @@
 //    on; a reducer warp adds the warps' partials in warp order (deterministic) and writes Y, so
 //    the ring never waits for a reduction.
 //  * The kernel is instantiated per activation-row bound MT (1, 2, 4, 8): columns >= MT of the
-//    MMA fragments are never folded or parked.
+//    MMA fragments are never folded or parked.  MT = 16 (split mode, 16-group stages) feeds every
+//    dequantised A fragment to two MMAs, for activation rows 0-7 and 8-15.
 #include <algorithm>
 #include <mutex>
 

@@ -19,6 +19,10 @@
 // Other modes (for the AWQ search) load an fp16 B operand with TMA instead of dequantising and
 // replace the fp16 store (EPI 0) by a per-tile sum of squares (EPI 1), an fp32 store (EPI 2), or a
 // per-tile sum of D[m, n] * A[m, n] (EPI 3, for N == K: A read back from global memory).
+// w4_gemm also runs the dequantising GEMM with K cut into slices of whole groups (EPI 2 fp32
+// partial tiles, summed in slice order by splitk_reduce_kernel) when its tiles fill fewer than
+// half the SMs, and with a tail split (the full waves as one launch, the last, at most half full
+// wave's tiles in K slices with compact partials summed by tail_reduce_kernel).
 //
 // Every mbarrier wait is bounded; on timeout the kernel records W4_ERR_DEVICE_TIMEOUT, stops
 // issuing work, drains what it issued and frees TMEM before it exits.
