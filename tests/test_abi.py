@@ -299,3 +299,25 @@ def test_gemm_plan_query(L):
                           ctypes.byref(n)) == 3  # explicit GEMV with misaligned scales: W4_ERR_ALIGN
     assert L.w4_gemm_plan(1, 4096, 4096, 128, 0, BAD_ALIGN, GOOD, ctypes.byref(fam), ctypes.byref(n)) == 0
     assert (fam.value, n.value) == (B.VARIANT_SKINNY, 1)  # AUTO falls back to the skinny kernel
+
+
+def test_plan_and_workspace_agree():
+    """Every shape whose plan sums K slices in a further launch (the GEMV in split mode, the
+    tensor-core K split or tail split) gets a non-zero workspace from w4_gemm_workspace_size, for
+    AUTO and for each explicit family."""
+    shapes = [(M, N, K) for M in (1, 4, 8, 9, 16, 17, 32, 33, 64, 130, 512, 2048)
+              for (N, K) in ((8192, 8192), (8192, 28672), (28672, 8192), (4096, 4096), (11008, 4096),
+                             (4096, 11008), (520, 2048), (5000, 2048))]
+    n = ctypes.c_size_t(0)
+    for (M, N, K) in shapes:
+        assert B.lib().w4_gemm_workspace_size(M, N, K, 128, ctypes.byref(n)) == 0
+        need = n.value
+        for variant in (B.VARIANT_AUTO, B.VARIANT_GEMV, B.VARIANT_TC):
+            try:
+                fam, launches = B.w4_gemm_plan(M, N, K, variant=variant)
+            except B.W4Error:
+                continue  # the explicit family cannot serve this shape
+            if fam == B.VARIANT_TC and launches > 1:  # K slices or a tail split: fp32 partials
+                assert need > 0, (M, N, K, variant)
+            if fam == B.VARIANT_GEMV and M <= 8 and launches > 1:  # one GEMV launch + its slice sum
+                assert need > 0, (M, N, K, variant)
